@@ -1,0 +1,293 @@
+"""Fused residual-add + RMSNorm / LayerNorm + activation quantization for B200.
+
+A thin ctypes binding over ``libnq.so`` (see ``include/nq.h`` for the
+contract of every call).  This module only marshals arguments: it checks
+tensor dtypes / devices / layouts, allocates outputs with torch when the
+caller does not pass them, and forwards raw device pointers, strides and the
+current CUDA stream.  Every arithmetic step runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and importing fails loudly when
+the library has not been built (``python -m fp4_activation_quantization_b200.build``).
+
+Functions carry the C names:
+``nq_fused_add_rmsnorm_quant_fp8``, ``nq_rmsnorm_quant_fp8_static``,
+``nq_layernorm_quant_fp8``, ``nq_per_token_group_quant_fp8``,
+``nq_rmsnorm_quant_nvfp4``; plus ``nq_query_schedule``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
+    "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND",
+    "flag_schedule", "NQError", "lib", "library_path", "version",
+    "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
+    "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
+    "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4",
+]
+
+NQ_OK, NQ_ERR_INVALID_ARGUMENT, NQ_ERR_UNSUPPORTED, NQ_ERR_CUDA = 0, 1, 2, 3
+NQ_MAX_D = 16384
+FLAG_PDL = 1 << 0
+FLAG_SCALE_DIV = 1 << 1
+FLAG_SCALE_RECIP = 1 << 2
+FLAG_UE8M0 = 1 << 3
+FLAG_NORM_BF16_ROUND = 1 << 4
+OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4 = 0, 1, 2, 3
+
+
+def flag_schedule(log2_threads: int, log2_chunks: int) -> int:
+    """NQ_FLAG_SCHEDULE(t, k): force 2^t threads per row and 2^k chunks per thread."""
+    return (((log2_threads - 4) & 0xF) << 16) | (((log2_chunks + 1) & 0x7) << 20)
+
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libnq.so")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m fp4_activation_quantization_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I64, I32, U32, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_float
+    st = ctypes.c_int
+    L.nq_version.argtypes, L.nq_version.restype = [], ctypes.c_int
+    L.nq_status_string.argtypes, L.nq_status_string.restype = [st], ctypes.c_char_p
+    L.nq_last_error.argtypes, L.nq_last_error.restype = [], ctypes.c_char_p
+    L.nq_query_schedule.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.POINTER(ctypes.c_int),
+                                    ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    L.nq_query_schedule.restype = st
+    L.nq_fused_add_rmsnorm_quant_fp8.argtypes = [P, I64, P, P, I64, P, P, I64, P, P, I64, I64, I64, F, U32, P]
+    L.nq_rmsnorm_quant_fp8_static.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, I64, I64, F, U32, P]
+    L.nq_layernorm_quant_fp8.argtypes = [P, I64, P, P, P, P, I64, I64, I64, F, U32, P]
+    L.nq_per_token_group_quant_fp8.argtypes = [P, I64, P, I64, P, I64, I64, I64, I32, U32, P]
+    L.nq_rmsnorm_quant_nvfp4.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, P, I64, I64, I64, F, U32, P]
+    for name in ("nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
+                 "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4"):
+        getattr(L, name).restype = st
+    return L
+
+
+lib = _load()
+
+
+def version() -> int:
+    return lib.nq_version()
+
+
+class NQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.nq_last_error().decode()
+        super().__init__(f"{where}: {lib.nq_status_string(status).decode()}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != NQ_OK:
+        raise NQError(status, where)
+
+
+# ----------------------------------------------------------- marshalling ----
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def _rows(t: torch.Tensor, name: str, dtype, cols: int | None = None):
+    """2-D tensor on CUDA with a contiguous last dimension; returns (M, ncols, row stride)."""
+    _need(isinstance(t, torch.Tensor), f"{name} must be a torch.Tensor")
+    _need(t.is_cuda, f"{name} must be a CUDA tensor")
+    _need(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")
+    _need(t.dim() == 2, f"{name} must be 2-D [M, d], got shape {tuple(t.shape)}")
+    _need(t.stride(1) == 1 or t.shape[1] <= 1, f"{name} must have a contiguous last dimension")
+    if cols is not None:
+        _need(t.shape[1] == cols, f"{name} must have {cols} columns, got {t.shape[1]}")
+    ld = t.stride(0) if t.shape[0] > 1 else max(t.stride(0), t.shape[1])
+    return t.shape[0], t.shape[1], ld
+
+
+def _vec(t: torch.Tensor, name: str, dtype, n: int):
+    _need(isinstance(t, torch.Tensor) and t.is_cuda, f"{name} must be a CUDA tensor")
+    _need(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")
+    _need(t.dim() == 1 and t.shape[0] == n and t.stride(0) == 1, f"{name} must be contiguous [{n}]")
+
+
+def _scalar(t: torch.Tensor, name: str):
+    _need(isinstance(t, torch.Tensor) and t.is_cuda, f"{name} must be a one-element float32 CUDA tensor")
+    _need(t.dtype == torch.float32 and t.numel() == 1, f"{name} must be a one-element float32 CUDA tensor")
+
+
+def _same_device(*ts):
+    devs = {t.device for t in ts if t is not None}
+    _need(len(devs) == 1, f"all tensors must be on one device, got {devs}")
+
+
+def _out(t, shape, dtype, like: torch.Tensor, name: str):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=like.device)
+    _need(t.dtype == dtype and tuple(t.shape) == tuple(shape), f"{name} must be {dtype} {tuple(shape)}")
+    return t
+
+
+# ------------------------------------------------------------ the calls ----
+def nq_query_schedule(op: int, M: int, d: int, flags: int = 0):
+    """(threads per row, 16-byte chunks per thread, rows per CTA) the planner picks."""
+    t, k, r = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib.nq_query_schedule(op, M, d, flags, ctypes.byref(t), ctypes.byref(k), ctypes.byref(r)),
+           "nq_query_schedule")
+    return t.value, k.value, r.value
+
+
+def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, residual_out=None,
+                                   q_out=None, scale_out=None, norm_out=None, want_norm: bool = False,
+                                   flags: int = 0, stream=None):
+    """Residual-add + RMSNorm + dynamic per-token e4m3.
+
+    ``x`` bf16 [M, d] (may be a column slice), ``residual`` bf16 [M, d],
+    ``gamma`` bf16 [d].  ``residual_out`` defaults to a new tensor; pass
+    ``residual_out=residual`` for the in-place update.  Returns
+    ``(q float8_e4m3fn [M, d], scale float32 [M], residual_out, norm_out or None)``.
+    """
+    M, d, ld_x = _rows(x, "x", torch.bfloat16)
+    _, _, ld_r = _rows(residual, "residual", torch.bfloat16, d)
+    _need(residual.shape[0] == M, "residual must have M rows")
+    _vec(gamma, "gamma", torch.bfloat16, d)
+    residual_out = _out(residual_out, (M, d), torch.bfloat16, x, "residual_out")
+    _, _, ld_ro = _rows(residual_out, "residual_out", torch.bfloat16, d)
+    _need(ld_ro == ld_r, "residual_out must have the row stride of residual")
+    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    scale_out = _out(scale_out, (M,), torch.float32, x, "scale_out")
+    _vec(scale_out, "scale_out", torch.float32, M)
+    if want_norm and norm_out is None:
+        norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
+    _same_device(x, residual, gamma, residual_out, q_out, scale_out, norm_out)
+    with torch.cuda.device(x.device):
+        _check(lib.nq_fused_add_rmsnorm_quant_fp8(
+            _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(q_out), ld_q,
+            _ptr(scale_out), _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)),
+            "nq_fused_add_rmsnorm_quant_fp8")
+    return q_out, scale_out, residual_out, norm_out
+
+
+def nq_rmsnorm_quant_fp8_static(x, gamma, scale, eps: float = 1e-6, *, residual=None, residual_out=None,
+                                q_out=None, norm_out=None, want_norm: bool = False, flags: int = 0,
+                                stream=None):
+    """RMSNorm (optional residual-add) + e4m3 with a one-element device scale.
+
+    Returns ``(q float8_e4m3fn [M, d], residual_out or None, norm_out or None)``.
+    """
+    M, d, ld_x = _rows(x, "x", torch.bfloat16)
+    _vec(gamma, "gamma", torch.bfloat16, d)
+    _scalar(scale, "scale")
+    ld_r = d
+    if residual is not None:
+        _, _, ld_r = _rows(residual, "residual", torch.bfloat16, d)
+        _need(residual.shape[0] == M, "residual must have M rows")
+        residual_out = _out(residual_out, (M, d), torch.bfloat16, x, "residual_out")
+        _need(_rows(residual_out, "residual_out", torch.bfloat16, d)[2] == ld_r,
+              "residual_out must have the row stride of residual")
+    else:
+        _need(residual_out is None, "residual_out needs residual")
+    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    if want_norm and norm_out is None:
+        norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
+    _same_device(x, gamma, scale, residual, residual_out, q_out, norm_out)
+    with torch.cuda.device(x.device):
+        _check(lib.nq_rmsnorm_quant_fp8_static(
+            _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(scale), _ptr(q_out),
+            ld_q, _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)), "nq_rmsnorm_quant_fp8_static")
+    return q_out, residual_out, norm_out
+
+
+def nq_layernorm_quant_fp8(x, gamma, beta, scale, eps: float = 1e-5, *, q_out=None, flags: int = 0,
+                           stream=None):
+    """LayerNorm (float32 gamma, beta) + e4m3 with a one-element device scale. Returns q."""
+    M, d, ld_x = _rows(x, "x", torch.bfloat16)
+    _vec(gamma, "gamma", torch.float32, d)
+    _vec(beta, "beta", torch.float32, d)
+    _scalar(scale, "scale")
+    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    _same_device(x, gamma, beta, scale, q_out)
+    with torch.cuda.device(x.device):
+        _check(lib.nq_layernorm_quant_fp8(_ptr(x), ld_x, _ptr(gamma), _ptr(beta), _ptr(scale), _ptr(q_out),
+                                          ld_q, M, d, eps, flags, _stream(stream)), "nq_layernorm_quant_fp8")
+    return q_out
+
+
+def nq_per_token_group_quant_fp8(x, group: int = 128, *, q_out=None, scales_out=None, flags: int = 0,
+                                 stream=None):
+    """Per-token-group e4m3. Returns ``(q float8_e4m3fn [M, K], scales float32 [M, K/group])``."""
+    M, K, ld_x = _rows(x, "x", torch.bfloat16)
+    _need(group > 0 and K % group == 0, f"K = {K} must be a multiple of group = {group}")
+    q_out = _out(q_out, (M, K), torch.float8_e4m3fn, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, K)
+    scales_out = _out(scales_out, (M, K // group), torch.float32, x, "scales_out")
+    _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, K // group)
+    _same_device(x, q_out, scales_out)
+    with torch.cuda.device(x.device):
+        _check(lib.nq_per_token_group_quant_fp8(_ptr(x), ld_x, _ptr(q_out), ld_q, _ptr(scales_out), ld_s, M, K,
+                                                group, flags, _stream(stream)), "nq_per_token_group_quant_fp8")
+    return q_out, scales_out
+
+
+def nq_rmsnorm_quant_nvfp4(x, gamma, global_scale, eps: float = 1e-6, *, residual=None, residual_out=None,
+                           q_out=None, sf_out=None, norm_out=None, want_norm: bool = False, flags: int = 0,
+                           stream=None):
+    """RMSNorm (optional residual-add) + NVFP4.
+
+    Returns ``(q uint8 [M, d/2] packed e2m1, sf float8_e4m3fn [M, d/16],
+    residual_out or None, norm_out or None)``.
+    """
+    M, d, ld_x = _rows(x, "x", torch.bfloat16)
+    _need(d % 16 == 0, f"d = {d} must be a multiple of 16")
+    _vec(gamma, "gamma", torch.bfloat16, d)
+    _scalar(global_scale, "global_scale")
+    ld_r = d
+    if residual is not None:
+        _, _, ld_r = _rows(residual, "residual", torch.bfloat16, d)
+        _need(residual.shape[0] == M, "residual must have M rows")
+        residual_out = _out(residual_out, (M, d), torch.bfloat16, x, "residual_out")
+        _need(_rows(residual_out, "residual_out", torch.bfloat16, d)[2] == ld_r,
+              "residual_out must have the row stride of residual")
+    else:
+        _need(residual_out is None, "residual_out needs residual")
+    q_out = _out(q_out, (M, d // 2), torch.uint8, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", torch.uint8, d // 2)
+    sf_out = _out(sf_out, (M, d // 16), torch.float8_e4m3fn, x, "sf_out")
+    _, _, ld_sf = _rows(sf_out, "sf_out", torch.float8_e4m3fn, d // 16)
+    if want_norm and norm_out is None:
+        norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
+    _same_device(x, gamma, global_scale, residual, residual_out, q_out, sf_out, norm_out)
+    with torch.cuda.device(x.device):
+        _check(lib.nq_rmsnorm_quant_nvfp4(
+            _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(global_scale), _ptr(q_out),
+            ld_q, _ptr(sf_out), ld_sf, _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)),
+            "nq_rmsnorm_quant_nvfp4")
+    return q_out, sf_out, residual_out, norm_out

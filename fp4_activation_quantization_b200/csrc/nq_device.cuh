@@ -1,0 +1,154 @@
+// nq_device.cuh — device helpers shared by the sm_100a kernels of libnq.
+//
+// Format conversions use the hardware's packed converters
+// (cvt.rn.satfinite.e4m3x2.f32, cvt.rn.satfinite.e2m1x2.f32, cvt.rn.bf16x2.f32):
+// round to nearest even, saturate to the largest finite value.  Every other
+// float operation is written with an explicit IEEE intrinsic (__fadd_rn,
+// __fmul_rn, __fmaf_rn, __fdiv_rn, __frcp_rn, __fsqrt_rn) so that contraction
+// or approximation can never change a rounding: results are identical on
+// every schedule and reproducible on the CPU.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace nq {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kE4M3Max = 448.0f;
+constexpr float kE2M1Max = 6.0f;
+
+// ---------------------------------------------------------------- PDL -----
+// Programmatic dependent launch: both are no-ops when the grid was launched
+// without the programmatic-serialization attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- bf16 ----
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&v)[8]) {
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
+  v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z);
+  v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+
+// Two floats -> two bf16 (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<const uint16_t*>(&h);
+}
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&v)[8]) {
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
+}
+__device__ __forceinline__ float round_bf16(float f) { return bf16_to_f32(f32_to_bf16(f)); }
+
+// ---------------------------------------------------------------- e4m3 ----
+// Four floats -> four e4m3 bytes, a0 in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(out)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return out;
+}
+__device__ __forceinline__ uint32_t f32_to_e4m3(float a) { return pack_e4m3x4(a, 0.f, 0.f, 0.f) & 0xFFu; }
+
+// e4m3 code (never the NaN code here) -> float, exact.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
+  const float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))  // (1 + m/8) 2^(e-7)
+                      : __fmul_rn(float(m), 0.001953125f);                 // m 2^-9
+  return (c & 0x80u) ? -mag : mag;
+}
+
+// ---------------------------------------------------------------- e2m1 ----
+// Eight floats -> eight e2m1 nibbles packed in 4 bytes; element 2i in the low
+// nibble of byte i.
+__device__ __forceinline__ uint32_t pack_e2m1x8(const float (&v)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+// --------------------------------------------------------------- UE8M0 ----
+// Smallest power of two >= s, clamped to [2^-127, 2^127]; s <= 0 -> 2^-127.
+__device__ __forceinline__ float ue8m0_ceil(float s) {
+  if (!(s > 0.0f)) return __uint_as_float(0x00400000u);
+  const uint32_t b = __float_as_uint(s);
+  const int e = int((b >> 23) & 0xFFu);
+  const uint32_t m = b & 0x7FFFFFu;
+  int p;
+  if (e == 0) p = -149 + (m == 1u ? 0 : 32 - __clz(int(m - 1u)));  // subnormal input
+  else p = e - 127 + (m ? 1 : 0);
+  p = p < -127 ? -127 : (p > 127 ? 127 : p);
+  return p >= -126 ? __uint_as_float(uint32_t(p + 127) << 23) : __uint_as_float(1u << (p + 149));
+}
+
+// ---------------------------------------------------------- reductions ----
+// Canonical row sum.  Thread t of a row group of T threads holds chunk
+// partials for chunks t, t+T, t+2T, ... already combined (highest index bit
+// first) into `v`.  The remaining levels of the pairwise tree over the chunk
+// index are: across warps (warp w absorbs warp w + W/2, lane by lane, highest
+// bit first), then inside the warp (xor butterfly 16, 8, 4, 2, 1; IEEE
+// addition is commutative, so lane l and l^o compute the same value).  Every
+// thread returns the row total.  `red` holds W*32 floats (unused for T == 32).
+// For T > 32 the row is the whole CTA and this contains one __syncthreads().
+template <int T>
+__device__ __forceinline__ float row_sum(float v, float* red, int tid) {
+  if constexpr (T > 32) {
+    constexpr int W = T / 32;
+    const int lane = tid & 31, w = tid >> 5;
+    red[w * 32 + lane] = v;
+    __syncthreads();
+    float p[W];
+#pragma unroll
+    for (int i = 0; i < W; ++i) p[i] = red[i * 32 + lane];
+#pragma unroll
+    for (int h = W / 2; h >= 1; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) p[i] = __fadd_rn(p[i], p[i + h]);
+    v = p[0];
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+// Row maximum of non-negative floats (order-free; exact).  `red` holds W words.
+template <int T>
+__device__ __forceinline__ float row_max_nonneg(float v, uint32_t* red, int tid) {
+  uint32_t u = __reduce_max_sync(kFull, __float_as_uint(v));
+  if constexpr (T > 32) {
+    constexpr int W = T / 32;
+    if ((tid & 31) == 0) red[tid >> 5] = u;
+    __syncthreads();
+    u = 0;
+#pragma unroll
+    for (int i = 0; i < W; ++i) u = max(u, red[i]);
+  }
+  return __uint_as_float(u);
+}
+
+}  // namespace nq

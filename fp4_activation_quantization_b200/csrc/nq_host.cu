@@ -1,0 +1,375 @@
+// nq_host.cu — the C ABI of libnq: argument validation, schedule planning and
+// kernel launch.  Declarations and the contract of every entry point are in
+// include/nq.h.  Nothing here allocates, synchronizes or reads device memory.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "nq.h"
+#include "nq_internal.h"
+
+namespace {
+
+using nq::RowArgs;
+using nq::GroupArgs;
+
+thread_local std::string g_last_error;
+
+nq_status fail(nq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
+                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK;
+
+nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
+                      bool allow_bf16_round) {
+  if (flags & ~kKnownFlags) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: unknown flag bits 0x%x", fn, flags & ~kKnownFlags);
+  if ((flags & NQ_FLAG_SCALE_DIV) && (flags & NQ_FLAG_SCALE_RECIP))
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
+  if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_UE8M0 applies to group quantization only", fn);
+  if ((flags & NQ_FLAG_SCHEDULE_MASK) && !allow_schedule)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE applies to the norm calls only", fn);
+  if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
+  return NQ_OK;
+}
+
+uint32_t kernel_flags(uint32_t flags, bool default_div) {
+  const bool div = (flags & NQ_FLAG_SCALE_DIV) ? true : (flags & NQ_FLAG_SCALE_RECIP) ? false : default_div;
+  uint32_t k = 0;
+  if (div) k |= nq::kFlagDiv;
+  if (flags & NQ_FLAG_UE8M0) k |= nq::kFlagUe8m0;
+  if (flags & NQ_FLAG_NORM_BF16_ROUND) k |= nq::kFlagNormBf16;
+  return k;
+}
+
+struct Schedule {
+  int log_t, log_k;
+};
+
+// Row -> thread mapping.  C = ceil(d / 8) chunks of 16 bytes, P = the next
+// power of two.  Rows of <= 1024 elements: one warp per row (eight rows per
+// CTA), 2^max(0, log P - 5) chunks per thread.  Wider rows: one CTA per row
+// with four chunks per thread, so each thread keeps 64 bytes of the row (128
+// with a residual) in flight.  Few rows (M < 148, fewer than one per SM):
+// spread the row over up to 1024 threads with one or two chunks each, which
+// shortens the per-row critical path.  Every mapping gives identical bits.
+nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedule* s) {
+  const int64_t C = (d + 7) / 8;
+  int lp = 0;
+  while ((int64_t(1) << lp) < C) ++lp;
+  const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
+  if (ft || fk) {
+    if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
+    const int lt = int(ft) + 4, lk = int(fk) - 1;
+    if (!nq::schedule_built(lt, lk))
+      return fail(NQ_ERR_UNSUPPORTED, "%s: schedule of 2^%d threads x 2^%d chunks is not built", fn, lt, lk);
+    if ((int64_t(1) << (lt + lk)) < C)
+      return fail(NQ_ERR_INVALID_ARGUMENT, "%s: schedule covers %lld chunks, a row has %lld", fn,
+                  (long long)(int64_t(1) << (lt + lk)), (long long)C);
+    *s = {lt, lk};
+    return NQ_OK;
+  }
+  if (lp <= 7) {
+    s->log_t = 5;
+    s->log_k = lp > 5 ? lp - 5 : 0;
+  } else if (M < 148) {
+    s->log_t = lp < 10 ? lp : 10;
+    s->log_k = lp - s->log_t;
+  } else {
+    s->log_t = lp - 2 < 10 ? lp - 2 : 10;
+    s->log_k = lp - s->log_t;
+  }
+  if (!nq::schedule_built(s->log_t, s->log_k))
+    return fail(NQ_ERR_UNSUPPORTED, "%s: no built schedule for d = %lld", fn, (long long)d);
+  return NQ_OK;
+}
+
+nq_status launch(const char* fn, const void* kernel, unsigned grid, unsigned block, void** args,
+                 bool pdl, cudaStream_t stream) {
+  if (kernel == nullptr) return fail(NQ_ERR_UNSUPPORTED, "%s: kernel variant not built", fn);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  const cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, args);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();  // launch errors are not sticky: clear so later callers do not see them
+    return fail(NQ_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  }
+  return NQ_OK;
+}
+
+nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
+  if (M < 0) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: M = %lld < 0", fn, (long long)M);
+  if (d < 1) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: d = %lld < 1", fn, (long long)d);
+  if (d > NQ_MAX_D) return fail(NQ_ERR_UNSUPPORTED, "%s: d = %lld > NQ_MAX_D (%d)", fn, (long long)d, NQ_MAX_D);
+  if (!(eps >= 0.0f) || !std::isfinite(eps))
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: eps must be finite and >= 0", fn);
+  if (M > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: M = %lld too large", fn, (long long)M);
+  return NQ_OK;
+}
+
+#define NQ_REQUIRE(cond, ...)                                   \
+  do {                                                          \
+    if (!(cond)) return fail(NQ_ERR_INVALID_ARGUMENT, __VA_ARGS__); \
+  } while (0)
+
+const nq::KernelTable& table_of(int op) {
+  switch (op) {
+    case nq::kOpRmsDynFp8: return nq::row_kernels_rms_dyn();
+    case nq::kOpRmsStaticFp8: return nq::row_kernels_rms_static();
+    case nq::kOpLnStaticFp8: return nq::row_kernels_ln_static();
+    default: return nq::row_kernels_rms_nvfp4();
+  }
+}
+
+// Shared tail of the four norm calls.
+nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
+  Schedule s;
+  nq_status st = plan_rows(fn, a.M, a.d, flags, &s);
+  if (st != NQ_OK) return st;
+  const int threads = 1 << s.log_t;
+  const int rows = nq::rows_per_cta(threads);
+  const int64_t grid = (a.M + rows - 1) / rows;
+  const void* k = table_of(op)[s.log_t - nq::kMinLogT][s.log_k][vec ? 1 : 0];
+  void* args[] = {&a};
+  return launch(fn, k, unsigned(grid), unsigned(threads * rows), args, (flags & NQ_FLAG_PDL) != 0, stream);
+}
+
+bool vec_bf16(const void* p, int64_t ld) { return p == nullptr || (aligned(p, 16) && ld % 8 == 0); }
+
+}  // namespace
+
+extern "C" {
+
+int nq_version(void) { return 100; }
+
+const char* nq_status_string(nq_status status) {
+  switch (status) {
+    case NQ_OK: return "NQ_OK";
+    case NQ_ERR_INVALID_ARGUMENT: return "NQ_ERR_INVALID_ARGUMENT";
+    case NQ_ERR_UNSUPPORTED: return "NQ_ERR_UNSUPPORTED";
+    case NQ_ERR_CUDA: return "NQ_ERR_CUDA";
+  }
+  return "unknown nq_status";
+}
+
+const char* nq_last_error(void) { return g_last_error.c_str(); }
+
+nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
+                            int* chunks_per_thread, int* rows_per_cta) {
+  const char* fn = "nq_query_schedule";
+  NQ_REQUIRE(op >= 0 && op < nq::kNumRowOps, "%s: op %d out of range", fn, op);
+  NQ_REQUIRE(threads_per_row && chunks_per_thread && rows_per_cta, "%s: null output pointer", fn);
+  nq_status st = check_common(fn, M, d, 1.0f);
+  if (st != NQ_OK) return st;
+  Schedule s;
+  st = plan_rows(fn, M, d, flags, &s);
+  if (st != NQ_OK) return st;
+  *threads_per_row = 1 << s.log_t;
+  *chunks_per_thread = 1 << s.log_k;
+  *rows_per_cta = nq::rows_per_cta(1 << s.log_t);
+  return NQ_OK;
+}
+
+nq_status nq_fused_add_rmsnorm_quant_fp8(const void* x, int64_t ld_x, const void* residual_in,
+                                         void* residual_out, int64_t ld_res, const void* gamma,
+                                         void* q_out, int64_t ld_q, float* scale_out,
+                                         void* norm_out, int64_t ld_norm, int64_t M, int64_t d,
+                                         float eps, uint32_t flags, nq_stream_t stream) {
+  const char* fn = "nq_fused_add_rmsnorm_quant_fp8";
+  nq_status st = check_common(fn, M, d, eps);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
+  NQ_REQUIRE(ld_x >= d && ld_res >= d && ld_q >= d && (!norm_out || ld_norm >= d),
+             "%s: every row stride must be >= d", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && residual_in && residual_out && gamma && q_out && scale_out,
+             "%s: x, residual_in, residual_out, gamma, q_out and scale_out are required", fn);
+  RowArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.res_in = static_cast<const uint16_t*>(residual_in);
+  a.res_out = static_cast<uint16_t*>(residual_out);
+  a.ld_res = ld_res;
+  a.gamma = gamma;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.scale_out = scale_out;
+  a.norm_out = static_cast<uint16_t*>(norm_out);
+  a.ld_norm = ld_norm;
+  a.M = M;
+  a.d = int32_t(d);
+  a.eps = eps;
+  a.flags = kernel_flags(flags, /*default_div=*/true);
+  const bool vec = d % 8 == 0 && vec_bf16(x, ld_x) && vec_bf16(residual_in, ld_res) &&
+                   vec_bf16(residual_out, ld_res) && aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) &&
+                   aligned(q_out, 8) && ld_q % 8 == 0;
+  return run_rows(fn, nq::kOpRmsDynFp8, a, vec, flags, stream);
+}
+
+nq_status nq_rmsnorm_quant_fp8_static(const void* x, int64_t ld_x, const void* residual_in,
+                                      void* residual_out, int64_t ld_res, const void* gamma,
+                                      const float* scale, void* q_out, int64_t ld_q,
+                                      void* norm_out, int64_t ld_norm, int64_t M, int64_t d,
+                                      float eps, uint32_t flags, nq_stream_t stream) {
+  const char* fn = "nq_rmsnorm_quant_fp8_static";
+  nq_status st = check_common(fn, M, d, eps);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
+  NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
+             "%s: residual_in and residual_out must both be given or both be NULL", fn);
+  NQ_REQUIRE(ld_x >= d && ld_q >= d && (!residual_in || ld_res >= d) && (!norm_out || ld_norm >= d),
+             "%s: every row stride must be >= d", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && gamma && scale && q_out, "%s: x, gamma, scale and q_out are required", fn);
+  RowArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.res_in = static_cast<const uint16_t*>(residual_in);
+  a.res_out = static_cast<uint16_t*>(residual_out);
+  a.ld_res = ld_res;
+  a.gamma = gamma;
+  a.scale = scale;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.norm_out = static_cast<uint16_t*>(norm_out);
+  a.ld_norm = ld_norm;
+  a.M = M;
+  a.d = int32_t(d);
+  a.eps = eps;
+  a.flags = kernel_flags(flags, /*default_div=*/false);
+  const bool vec = d % 8 == 0 && vec_bf16(x, ld_x) && vec_bf16(residual_in, ld_res) &&
+                   vec_bf16(residual_out, ld_res) && aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) &&
+                   aligned(q_out, 8) && ld_q % 8 == 0;
+  return run_rows(fn, nq::kOpRmsStaticFp8, a, vec, flags, stream);
+}
+
+nq_status nq_layernorm_quant_fp8(const void* x, int64_t ld_x, const float* gamma,
+                                 const float* beta, const float* scale, void* q_out, int64_t ld_q,
+                                 int64_t M, int64_t d, float eps, uint32_t flags,
+                                 nq_stream_t stream) {
+  const char* fn = "nq_layernorm_quant_fp8";
+  nq_status st = check_common(fn, M, d, eps);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
+  NQ_REQUIRE(ld_x >= d && ld_q >= d, "%s: every row stride must be >= d", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && gamma && beta && scale && q_out, "%s: x, gamma, beta, scale and q_out are required", fn);
+  RowArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.gamma = gamma;
+  a.beta = beta;
+  a.scale = scale;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.M = M;
+  a.d = int32_t(d);
+  a.eps = eps;
+  a.flags = kernel_flags(flags, /*default_div=*/false);
+  const bool vec = d % 8 == 0 && vec_bf16(x, ld_x) && aligned(gamma, 16) && aligned(beta, 16) &&
+                   aligned(q_out, 8) && ld_q % 8 == 0;
+  return run_rows(fn, nq::kOpLnStaticFp8, a, vec, flags, stream);
+}
+
+nq_status nq_rmsnorm_quant_nvfp4(const void* x, int64_t ld_x, const void* residual_in,
+                                 void* residual_out, int64_t ld_res, const void* gamma,
+                                 const float* global_scale, void* q_out, int64_t ld_q,
+                                 void* sf_out, int64_t ld_sf, void* norm_out, int64_t ld_norm,
+                                 int64_t M, int64_t d, float eps, uint32_t flags,
+                                 nq_stream_t stream) {
+  const char* fn = "nq_rmsnorm_quant_nvfp4";
+  nq_status st = check_common(fn, M, d, eps);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
+  NQ_REQUIRE(d % 16 == 0, "%s: d = %lld is not a multiple of 16", fn, (long long)d);
+  NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
+             "%s: residual_in and residual_out must both be given or both be NULL", fn);
+  NQ_REQUIRE(ld_x >= d && ld_q >= d / 2 && ld_sf >= d / 16 && (!residual_in || ld_res >= d) &&
+                 (!norm_out || ld_norm >= d),
+             "%s: row strides too small (ld_x >= d, ld_q >= d/2, ld_sf >= d/16)", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && gamma && global_scale && q_out && sf_out,
+             "%s: x, gamma, global_scale, q_out and sf_out are required", fn);
+  RowArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.res_in = static_cast<const uint16_t*>(residual_in);
+  a.res_out = static_cast<uint16_t*>(residual_out);
+  a.ld_res = ld_res;
+  a.gamma = gamma;
+  a.scale = global_scale;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.sf = static_cast<uint8_t*>(sf_out);
+  a.ld_sf = ld_sf;
+  a.norm_out = static_cast<uint16_t*>(norm_out);
+  a.ld_norm = ld_norm;
+  a.M = M;
+  a.d = int32_t(d);
+  a.eps = eps;
+  a.flags = kernel_flags(flags, /*default_div=*/false);
+  const bool vec = vec_bf16(x, ld_x) && vec_bf16(residual_in, ld_res) && vec_bf16(residual_out, ld_res) &&
+                   aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) && aligned(q_out, 4) && ld_q % 4 == 0;
+  return run_rows(fn, nq::kOpRmsNvfp4, a, vec, flags, stream);
+}
+
+nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out, int64_t ld_q,
+                                       float* scales_out, int64_t ld_s, int64_t M, int64_t K,
+                                       int32_t group, uint32_t flags, nq_stream_t stream) {
+  const char* fn = "nq_per_token_group_quant_fp8";
+  nq_status st = check_flags(fn, flags, true, false, false);
+  if (st != NQ_OK) return st;
+  NQ_REQUIRE(M >= 0 && K >= 1, "%s: need M >= 0 and K >= 1", fn);
+  if (group != 64 && group != 128) return fail(NQ_ERR_UNSUPPORTED, "%s: group %d not in {64, 128}", fn, group);
+  NQ_REQUIRE(K % group == 0, "%s: K = %lld is not a multiple of group %d", fn, (long long)K, group);
+  NQ_REQUIRE(ld_x >= K && ld_q >= K && ld_s >= K / group, "%s: row strides too small", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && q_out && scales_out, "%s: x, q_out and scales_out are required", fn);
+  GroupArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.s = scales_out;
+  a.ld_s = ld_s;
+  a.groups_per_row = K / group;
+  a.G = M * (K / group);
+  a.flags = kernel_flags(flags, /*default_div=*/false);
+  const bool vec = vec_bf16(x, ld_x) && aligned(q_out, 8) && ld_q % 8 == 0;
+  const int slot = nq::kGroupThreads / (group / 8);
+  // Four groups in flight per thread once there are enough groups to give
+  // every SM several CTAs that way; otherwise one, for more CTAs.
+  const int units = a.G >= int64_t(148) * slot * 4 * 2 ? 4 : 1;
+  const int64_t grid = (a.G + int64_t(slot) * units - 1) / (int64_t(slot) * units);
+  if (grid > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: too many groups", fn);
+  const void* k = nq::group_kernels()[group == 128 ? 1 : 0][units == 4 ? 1 : 0][vec ? 1 : 0];
+  void* args[] = {&a};
+  return launch(fn, k, unsigned(grid), nq::kGroupThreads, args, (flags & NQ_FLAG_PDL) != 0, stream);
+}
+
+}  // extern "C"

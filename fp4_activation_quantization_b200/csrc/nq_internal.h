@@ -1,0 +1,80 @@
+// nq_internal.h — argument blocks and kernel tables shared by the host
+// launcher (nq_host.cu) and the kernel translation units.  Not installed.
+#pragma once
+
+#include <cstdint>
+
+namespace nq {
+
+// Operations served by the row kernel (one token = one row of d elements).
+enum RowOp : int {
+  kOpRmsDynFp8 = 0,     // residual-add + RMSNorm + dynamic per-token e4m3
+  kOpRmsStaticFp8 = 1,  // RMSNorm (+residual) + static-scale e4m3
+  kOpLnStaticFp8 = 2,   // LayerNorm + static-scale e4m3
+  kOpRmsNvfp4 = 3,      // RMSNorm (+residual) + NVFP4
+  kNumRowOps = 4
+};
+
+// Kernel-side flag bits (the public NQ_FLAG_* values, repeated for the
+// device code, which does not include the public header).
+constexpr uint32_t kFlagDiv = 1u << 1;
+constexpr uint32_t kFlagUe8m0 = 1u << 3;
+constexpr uint32_t kFlagNormBf16 = 1u << 4;
+
+struct RowArgs {
+  const uint16_t* x;  // bf16 [M, ld_x]
+  int64_t ld_x;
+  const uint16_t* res_in;  // bf16 [M, ld_res] or null
+  uint16_t* res_out;       // bf16 [M, ld_res] or null (may equal res_in)
+  int64_t ld_res;
+  const void* gamma;   // bf16 [d] (RMSNorm) or float [d] (LayerNorm)
+  const float* beta;   // float [d] (LayerNorm)
+  const float* scale;  // device scalar: static scale or NVFP4 global scale
+  uint8_t* q;          // e4m3 [M, ld_q] or packed e2m1 [M, ld_q]
+  int64_t ld_q;
+  float* scale_out;  // float [M] (dynamic per-token)
+  uint8_t* sf;       // e4m3 block scales [M, ld_sf] (NVFP4)
+  int64_t ld_sf;
+  uint16_t* norm_out;  // bf16 [M, ld_norm] or null
+  int64_t ld_norm;
+  int64_t M;
+  int32_t d;
+  float eps;
+  uint32_t flags;  // kFlag* bits; kFlagDiv set means divide, clear means reciprocal
+};
+
+struct GroupArgs {
+  const uint16_t* x;  // bf16 [M, ld_x]
+  int64_t ld_x;
+  uint8_t* q;  // e4m3 [M, ld_q]
+  int64_t ld_q;
+  float* s;  // float [M, ld_s]
+  int64_t ld_s;
+  int64_t groups_per_row;
+  int64_t G;  // M * groups_per_row
+  uint32_t flags;
+};
+
+// Schedules: 2^t threads per row (t = 5..10), 2^k chunks of 8 elements per
+// thread (k = 0..2).  Rows per CTA: 8 when t == 5 (one warp per row), else 1.
+constexpr int kMinLogT = 5, kMaxLogT = 10, kMaxLogK = 2;
+inline int rows_per_cta(int threads) { return threads == 32 ? 8 : 1; }
+inline bool schedule_built(int log_t, int log_k) {
+  return log_t >= kMinLogT && log_t <= kMaxLogT && log_k >= 0 && log_k <= kMaxLogK &&
+         !(log_t == 10 && log_k == 2);
+}
+
+// Host-side kernel tables (pointer to the __global__ stub), one per
+// translation unit.  Index: [log_t - 5][log_k][vec].
+using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
+const KernelTable& row_kernels_rms_dyn();
+const KernelTable& row_kernels_rms_static();
+const KernelTable& row_kernels_ln_static();
+const KernelTable& row_kernels_rms_nvfp4();
+
+// Group kernel: [group == 128][units per thread: 0 -> 1, 1 -> 4][vec]
+using GroupTable = const void* [2][2][2];
+const GroupTable& group_kernels();
+constexpr int kGroupThreads = 256;
+
+}  // namespace nq

@@ -1,0 +1,11 @@
+// nq_row_ln_static.cu — instantiates the row kernel for LayerNorm + static-scale e4m3
+// (every built schedule, vector and scalar paths).  One file per operation so
+// that the kernels compile in parallel.
+#include "nq_row_kernel.cuh"
+
+namespace nq {
+const KernelTable& row_kernels_ln_static() {
+  static const RowTable<kOpLnStaticFp8> table;
+  return table.t;
+}
+}  // namespace nq

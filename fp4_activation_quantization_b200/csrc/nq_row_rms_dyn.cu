@@ -1,0 +1,11 @@
+// nq_row_rms_dyn.cu — instantiates the row kernel for residual-add + RMSNorm + dynamic per-token e4m3
+// (every built schedule, vector and scalar paths).  One file per operation so
+// that the kernels compile in parallel.
+#include "nq_row_kernel.cuh"
+
+namespace nq {
+const KernelTable& row_kernels_rms_dyn() {
+  static const RowTable<kOpRmsDynFp8> table;
+  return table.t;
+}
+}  // namespace nq

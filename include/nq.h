@@ -1,0 +1,211 @@
+/*
+ * nq.h — C ABI of the fused norm + activation-quantization library (libnq.so)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * One call = one kernel launch that, per token (row of d elements), adds the
+ * residual, normalizes (RMSNorm or LayerNorm) in float32 registers and
+ * quantizes the float32 result once, to e4m3 (FP8) or to NVFP4 (packed e2m1 +
+ * e4m3 block scales).  A fifth call quantizes raw bf16 activations per group
+ * of 128 (or 64) elements.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Status. Every call returns an nq_status. NQ_OK = 0. On any other value
+ *   nothing was launched and nq_last_error() (thread-local) says why. No call
+ *   throws across the ABI, traps on the device, synchronizes the stream or the
+ *   device, or allocates memory.
+ * Memory. Every pointer is caller-owned DEVICE memory on the current CUDA
+ *   device (the "scale" arguments too: they are read by the kernel at execution
+ *   time, so a captured CUDA graph sees scale updates made between replays).
+ *   bf16 tensors are row-major with a row stride ("ld_*") in ELEMENTS of that
+ *   tensor; e4m3 / packed-e2m1 / block-scale outputs have row strides in BYTES
+ *   (= elements); float32 scale arrays in elements.  The last dimension is
+ *   contiguous.  A column slice of a wider tensor is passed as a pointer to its
+ *   first column plus the wide tensor's row stride.
+ * Aliasing. residual_out may equal residual_in (in-place update, same stride);
+ *   no other output may overlap any input or another output.
+ * Asynchrony. Work is enqueued on `stream` (NULL = legacy default stream).
+ * Alignment. Any alignment is accepted. When every pointer is 16-byte aligned
+ *   (8-byte for e4m3 outputs, 4-byte for packed e2m1), every row stride keeps
+ *   rows so aligned and d % 8 == 0, the 16-byte vector path runs; otherwise a
+ *   scalar path with identical results runs.
+ * Sizes. M == 0 returns NQ_OK without a launch. 1 <= d <= NQ_MAX_D for the
+ *   norm calls; row strides must be >= d.
+ * Numerics (identical on every schedule, reproduced exactly by the oracle):
+ *   r = RN(x + residual) in float32; the bf16 residual_out is RN_bf16(r);
+ *   row sums use a fixed chunked pairwise order (8 consecutive elements per
+ *   chunk summed left to right from +0, then a pairwise tree over chunk index,
+ *   highest index bit first);
+ *   rstd = RN(1 / RN(sqrt(RN(mean + eps)))) with mean = RN(sum / d);
+ *   RMSNorm y = RN(RN(r * rstd) * gamma); LayerNorm y = fma(RN((r - mu) * rstd),
+ *   gamma, beta); e4m3 / e2m1 conversion rounds to nearest even and saturates
+ *   to +-448 / +-6.
+ *
+ * Sources (web pages, by title and section):
+ *  - "Fusing RMSNorm and FP8 Quantization Under torch.compile" (netraruntime
+ *    blog): TL;DR and "Where norm+quant sits" (residual add + RMSNorm +
+ *    per-token e4m3, quantized once from float32 registers); FAQ (residual
+ *    update exact, bf16 normed output written identically).
+ *  - FlashInfer PR #3962 "feat: fused FP8 quantization output for LayerNorm":
+ *    Description (layernorm_quant(out, input, gamma, beta, scale, eps); scale
+ *    applied as a division; float32 gamma/beta).
+ *  - TensorRT-LLM PR #14848 "RMSNorm nvfp4 quant fusion for DS V3.2 /
+ *    Kimi-K2.5": Description and commit notes (RMSNorm with or without
+ *    residual -> packed E2M1 + per-16 E4M3 block scales; row-strided column
+ *    slice input; hidden % 16 == 0; mandatory outputs non-null; residual sum
+ *    returned as a separate tensor).
+ *  - vLLM PR #61343 "per_token_group_quant_8bit: multiply by reciprocal
+ *    instead of dividing per element": Overview and Details (groups of 128,
+ *    one reciprocal per group, UE8M0 power-of-two scales).
+ *  - FlashInfer PR #2459 "RMSNorm/FusedRMSNorm + Quant kernels cuda graph
+ *    fixes": Description and Changes (scale passed as a one-element float32
+ *    device tensor, read as scale[0], inverse computed in the kernel).
+ */
+#ifndef NQ_H_
+#define NQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* nq_stream_t;
+
+typedef enum nq_status {
+  NQ_OK = 0,
+  NQ_ERR_INVALID_ARGUMENT = 1, /* null mandatory pointer, bad size/stride/flag */
+  NQ_ERR_UNSUPPORTED = 2,      /* valid request outside what is built (d > NQ_MAX_D, group) */
+  NQ_ERR_CUDA = 3              /* the CUDA runtime refused the launch */
+} nq_status;
+
+/* Widest row the norm calls accept (elements). */
+#define NQ_MAX_D 16384
+
+/* ---- flags (bitwise OR) ---- */
+/* Launch with programmatic dependent launch: the kernel's prologue may
+ * overlap the tail of the previous kernel on the stream. */
+#define NQ_FLAG_PDL (1u << 0)
+/* Quantize by exact per-element division RN(y / s). */
+#define NQ_FLAG_SCALE_DIV (1u << 1)
+/* Quantize by multiplying with the rounded reciprocal RN(y * RN(1 / s)).
+ * At most one of DIV / RECIP; with neither, each call's documented default. */
+#define NQ_FLAG_SCALE_RECIP (1u << 2)
+/* Group quantization: round every group scale up to a power of two (UE8M0). */
+#define NQ_FLAG_UE8M0 (1u << 3)
+/* Round y to bf16 before quantizing: reproduces the two-kernel (norm -> bf16
+ * -> quant) numerics for A/B comparisons.  Not for production use. */
+#define NQ_FLAG_NORM_BF16_ROUND (1u << 4)
+/* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
+ * thread (k = 0..2), with 2^(t+k) * 8 >= d.  Every schedule gives bitwise
+ * identical results; this exists for tests and tuning.  0 = automatic. */
+#define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
+#define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int nq_version(void);
+/* Static text of a status code. */
+const char* nq_status_string(nq_status status);
+/* Message of the last failing call on this thread ("" if none). */
+const char* nq_last_error(void);
+
+/*
+ * Schedule the planner picks for a norm call (op: 0 = fused add+RMSNorm+
+ * dynamic FP8, 1 = RMSNorm static FP8, 2 = LayerNorm static FP8, 3 = RMSNorm
+ * NVFP4) at (M, d, flags): threads per row, 16-byte chunks per thread and rows
+ * per CTA.  Pure host function; launches nothing.
+ */
+nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
+                            int* chunks_per_thread, int* rows_per_cta);
+
+/*
+ * Fused residual-add + RMSNorm + dynamic per-token e4m3.
+ * ("Fusing RMSNorm and FP8 Quantization Under torch.compile": TL;DR, "Where
+ * norm+quant sits"; per-token scale s = absmax(y) / 448.)
+ *   x            bf16 [M, ld_x]   input (first d columns used)          required
+ *   residual_in  bf16 [M, ld_res] residual stream                        required
+ *   residual_out bf16 [M, ld_res] RN_bf16(x + residual); may == residual_in  required
+ *   gamma        bf16 [d]         RMSNorm weight                         required
+ *   q_out        e4m3 [M, ld_q]   codes of y / s                         required
+ *   scale_out    f32  [M]         s = RN(max|y| / 448) (dequant: y ~ q * s)  required
+ *   norm_out     bf16 [M, ld_norm] RN_bf16(y), or NULL to skip
+ * Default quantization: exact division (NQ_FLAG_SCALE_DIV); NQ_FLAG_SCALE_RECIP
+ * multiplies by RN(1 / s).  A row with s == 0 stores the signed zeros of y.
+ */
+nq_status nq_fused_add_rmsnorm_quant_fp8(const void* x, int64_t ld_x, const void* residual_in,
+                                         void* residual_out, int64_t ld_res, const void* gamma,
+                                         void* q_out, int64_t ld_q, float* scale_out,
+                                         void* norm_out, int64_t ld_norm, int64_t M, int64_t d,
+                                         float eps, uint32_t flags, nq_stream_t stream);
+
+/*
+ * RMSNorm (residual-add optional) + e4m3 with a static scale held in device
+ * memory ("RMSNorm/FusedRMSNorm + Quant kernels cuda graph fixes": Changes;
+ * scale is a dequantization multiplier, q = e4m3(y / scale[0])).
+ *   residual_in / residual_out: both NULL (no residual) or both non-NULL.
+ *   scale: float32 device pointer, 1 element, read at kernel execution.
+ * Default quantization: NQ_FLAG_SCALE_RECIP (y * RN(1 / scale[0])).
+ * scale[0] must be positive and finite; 0 follows IEEE (1/0 = inf: nonzero y
+ * saturate to +-448, y = 0 gives a NaN code); it is never trapped.
+ */
+nq_status nq_rmsnorm_quant_fp8_static(const void* x, int64_t ld_x, const void* residual_in,
+                                      void* residual_out, int64_t ld_res, const void* gamma,
+                                      const float* scale, void* q_out, int64_t ld_q,
+                                      void* norm_out, int64_t ld_norm, int64_t M, int64_t d,
+                                      float eps, uint32_t flags, nq_stream_t stream);
+
+/*
+ * LayerNorm + e4m3 with a static device scale ("feat: fused FP8 quantization
+ * output for LayerNorm": Description; out = normed / scale).
+ *   x bf16 [M, ld_x]; gamma, beta float32 [d]; scale float32 device [1];
+ *   q_out e4m3 [M, ld_q].  mean and biased variance (two-pass) of each row.
+ * Default quantization: NQ_FLAG_SCALE_RECIP, as the RMSNorm static call.
+ */
+nq_status nq_layernorm_quant_fp8(const void* x, int64_t ld_x, const float* gamma,
+                                 const float* beta, const float* scale, void* q_out, int64_t ld_q,
+                                 int64_t M, int64_t d, float eps, uint32_t flags,
+                                 nq_stream_t stream);
+
+/*
+ * Per-token-group e4m3 of raw bf16 activations ("per_token_group_quant_8bit:
+ * multiply by reciprocal instead of dividing per element": Overview, Details).
+ *   x bf16 [M, ld_x] (first K columns); q_out e4m3 [M, ld_q];
+ *   scales_out float32 [M, ld_s] row-major, K / group scales per row:
+ *   s = RN(absmax / 448), or with NQ_FLAG_UE8M0 the smallest power of two
+ *   >= s (a zero group gives 2^-127).  group in {64, 128}; K % group == 0.
+ * Default quantization: NQ_FLAG_SCALE_RECIP; a zero fp32 scale stores the
+ * signed zeros of x.
+ */
+nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out, int64_t ld_q,
+                                       float* scales_out, int64_t ld_s, int64_t M, int64_t K,
+                                       int32_t group, uint32_t flags, nq_stream_t stream);
+
+/*
+ * RMSNorm (residual-add optional) + NVFP4 ("RMSNorm nvfp4 quant fusion for
+ * DS V3.2 / Kimi-K2.5": Description, commit notes).
+ *   x bf16 [M, ld_x] (may be a column slice of a wider tensor);
+ *   residual_in / residual_out: both NULL or both non-NULL;
+ *   global_scale float32 device [1]: dequantization multiplier g (x ~ e2m1 *
+ *     block_scale * g), read at kernel execution, positive and finite;
+ *   q_out uint8 [M, ld_q] packed e2m1, element 2i in the low nibble of byte i
+ *     (d / 2 bytes per row);
+ *   sf_out uint8 [M, ld_sf] e4m3 block scales, one per 16 elements, row-major:
+ *     sf = e4m3(RN(RN(absmax / 6) / g)); element multiplier RN(1 / RN(sf * g));
+ *   norm_out bf16 [M, ld_norm] or NULL.
+ *   d % 16 == 0.
+ * Default quantization: NQ_FLAG_SCALE_RECIP; NQ_FLAG_SCALE_DIV divides by
+ * RN(sf * g).  A block whose scale decodes to 0 stores zero codes.
+ */
+nq_status nq_rmsnorm_quant_nvfp4(const void* x, int64_t ld_x, const void* residual_in,
+                                 void* residual_out, int64_t ld_res, const void* gamma,
+                                 const float* global_scale, void* q_out, int64_t ld_q,
+                                 void* sf_out, int64_t ld_sf, void* norm_out, int64_t ld_norm,
+                                 int64_t M, int64_t d, float eps, uint32_t flags,
+                                 nq_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* NQ_H_ */

@@ -25,6 +25,9 @@ Workload recipes (shapes and distributions of the pages' configurations):
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
+import os
+
 import numpy as np
 
 __all__ = [
@@ -80,16 +83,32 @@ def uniform01(seed: int, stream_id: int, n: int, offset: int = 0) -> np.ndarray:
     return ((z >> np.uint64(11)).astype(np.float64) + 1.0) * (2.0 ** -53)
 
 
-def normal_f64(seed: int, stream_id: int, n: int) -> np.ndarray:
-    """Standard normals by Box–Muller, both branches used (cos for even, sin for odd)."""
-    half = (n + 1) // 2
-    u = uniform01(seed, stream_id, 2 * half)
+def _normal_block(seed: int, stream_id: int, lo: int, hi: int, out: np.ndarray) -> None:
+    u = uniform01(seed, stream_id, 2 * (hi - lo), offset=2 * lo)
     u1, u2 = u[0::2], u[1::2]
     rad = np.sqrt(-2.0 * np.log(u1))
     ang = 2.0 * np.pi * u2
+    out[2 * lo:2 * hi:2] = rad * np.cos(ang)
+    out[2 * lo + 1:2 * hi:2] = rad * np.sin(ang)
+
+
+def normal_f64(seed: int, stream_id: int, n: int) -> np.ndarray:
+    """Standard normals by Box–Muller, both branches used (cos for even, sin for odd).
+
+    Pair ``i`` uses uniforms ``2i`` and ``2i + 1`` of the stream, so blocks of
+    pairs are independent and are generated on a few threads (numpy releases
+    the GIL); the result does not depend on the blocking.
+    """
+    half = (n + 1) // 2
     out = np.empty(2 * half, dtype=np.float64)
-    out[0::2] = rad * np.cos(ang)
-    out[1::2] = rad * np.sin(ang)
+    block = 1 << 20
+    spans = [(lo, min(half, lo + block)) for lo in range(0, half, block)]
+    if len(spans) <= 1:
+        for lo, hi in spans:
+            _normal_block(seed, stream_id, lo, hi, out)
+    else:
+        with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda sp: _normal_block(seed, stream_id, sp[0], sp[1], out), spans))
     return out[:n]
 
 

@@ -1,0 +1,124 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+and its host-side validation and planner answer without touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nq.h")
+
+
+@pytest.fixture(scope="module")
+def nq():
+    from fp4_activation_quantization_b200 import build as b
+    b.build()
+    import fp4_activation_quantization_b200 as nq
+    return nq
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(nq):
+    names = declared_functions()
+    assert {"nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
+            "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4"} <= set(names)
+    raw = ctypes.CDLL(nq.library_path())
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_version_and_strings(nq):
+    assert nq.version() >= 100
+    assert nq.lib.nq_status_string(0) == b"NQ_OK"
+    assert nq.lib.nq_status_string(1) == b"NQ_ERR_INVALID_ARGUMENT"
+    assert nq.lib.nq_status_string(2) == b"NQ_ERR_UNSUPPORTED"
+    assert nq.lib.nq_status_string(3) == b"NQ_ERR_CUDA"
+
+
+def test_flag_values_match_header(nq):
+    text = open(HEADER).read()
+    assert "#define NQ_MAX_D 16384" in text and nq.NQ_MAX_D == 16384
+    for name, val in [("NQ_FLAG_PDL", nq.FLAG_PDL), ("NQ_FLAG_SCALE_DIV", nq.FLAG_SCALE_DIV),
+                      ("NQ_FLAG_SCALE_RECIP", nq.FLAG_SCALE_RECIP), ("NQ_FLAG_UE8M0", nq.FLAG_UE8M0),
+                      ("NQ_FLAG_NORM_BF16_ROUND", nq.FLAG_NORM_BF16_ROUND)]:
+        m = re.search(rf"#define {name} \(1u << (\d+)\)", text)
+        assert m and (1 << int(m.group(1))) == val, name
+
+
+FAKE = 0x10000  # a non-null address that validation rejects before any CUDA use
+
+
+def call_fused(nq, M=4, d=64, x=FAKE, res=FAKE, res_out=FAKE, gamma=FAKE, q=FAKE, s=FAKE, ld_x=None,
+               eps=1e-6, flags=0):
+    ld_x = d if ld_x is None else ld_x
+    return nq.lib.nq_fused_add_rmsnorm_quant_fp8(x, ld_x, res, res_out, d, gamma, q, d, s, None, d, M, d,
+                                                 eps, flags, None)
+
+
+def test_validation_without_gpu(nq):
+    INV, UNS = nq.NQ_ERR_INVALID_ARGUMENT, nq.NQ_ERR_UNSUPPORTED
+    assert call_fused(nq, x=None) == INV
+    assert b"required" in nq.lib.nq_last_error()
+    assert call_fused(nq, q=None) == INV
+    assert call_fused(nq, s=None) == INV
+    assert call_fused(nq, M=-1) == INV
+    assert call_fused(nq, d=0) == INV
+    assert call_fused(nq, d=16385) == UNS
+    assert call_fused(nq, ld_x=32) == INV
+    assert call_fused(nq, eps=float("nan")) == INV
+    assert call_fused(nq, eps=-1.0) == INV
+    assert call_fused(nq, flags=nq.FLAG_SCALE_DIV | nq.FLAG_SCALE_RECIP) == INV
+    assert call_fused(nq, flags=nq.FLAG_UE8M0) == INV
+    assert call_fused(nq, flags=1 << 30) == INV
+    # M == 0 is a no-op, even with null pointers
+    assert call_fused(nq, M=0, x=None, res=None, res_out=None, gamma=None, q=None, s=None) == nq.NQ_OK
+    # schedule too small for the row
+    assert call_fused(nq, d=1024, flags=nq.flag_schedule(5, 0)) == INV
+    # static: residual pair must be both or neither
+    L = nq.lib
+    assert L.nq_rmsnorm_quant_fp8_static(FAKE, 64, FAKE, None, 64, FAKE, FAKE, FAKE, 64, None, 64, 4, 64,
+                                         1e-6, 0, None) == INV
+    # NVFP4 needs d % 16 == 0
+    assert L.nq_rmsnorm_quant_nvfp4(FAKE, 24, None, None, 24, FAKE, FAKE, FAKE, 12, FAKE, 1, None, 24, 4, 24,
+                                    1e-6, 0, None) == INV
+    # group: K % group, group size, schedule flag not allowed
+    assert L.nq_per_token_group_quant_fp8(FAKE, 200, FAKE, 200, FAKE, 2, 4, 200, 128, 0, None) == INV
+    assert L.nq_per_token_group_quant_fp8(FAKE, 96, FAKE, 96, FAKE, 3, 4, 96, 32, 0, None) == UNS
+    assert L.nq_per_token_group_quant_fp8(FAKE, 256, FAKE, 256, FAKE, 2, 4, 256, 128,
+                                          nq.flag_schedule(5, 0), None) == INV
+    assert L.nq_per_token_group_quant_fp8(None, 256, None, 256, None, 2, 0, 256, 128, 0, None) == nq.NQ_OK
+    # LayerNorm rejects the bf16 double-rounding flag only when there is no norm: it has one, so fine;
+    # it rejects UE8M0
+    assert L.nq_layernorm_quant_fp8(FAKE, 64, FAKE, FAKE, FAKE, FAKE, 64, 4, 64, 1e-5, nq.FLAG_UE8M0,
+                                    None) == INV
+
+
+@pytest.mark.parametrize("M,d,exp", [
+    (64, 2816, (512, 1, 1)),      # fewer rows than SMs: one chunk per thread
+    (4096, 2816, (128, 4, 1)),    # rows > 1024 elements: one CTA per row, 4 chunks per thread
+    (4096, 4096, (128, 4, 1)),
+    (65536, 8192, (256, 4, 1)),
+    (8192, 7168, (256, 4, 1)),
+    (8192, 512, (32, 2, 8)),      # narrow rows: one warp per row, 8 rows per CTA
+    (8192, 1536, (64, 4, 1)),
+    (1, 8192, (1024, 1, 1)),      # a single row spreads over 1024 threads
+    (16, 16384, (1024, 2, 1)),
+    (1, 100, (32, 1, 8)),
+])
+def test_planner(nq, M, d, exp):
+    assert nq.nq_query_schedule(0, M, d) == exp
+
+
+def test_planner_forced_schedules(nq):
+    assert nq.nq_query_schedule(0, 100, 4096, nq.flag_schedule(9, 0)) == (512, 1, 1)
+    assert nq.nq_query_schedule(3, 100, 1024, nq.flag_schedule(5, 2)) == (32, 4, 8)
+    with pytest.raises(nq.NQError):
+        nq.nq_query_schedule(0, 100, 4096, nq.flag_schedule(5, 2))   # 32 * 4 * 8 < 4096
+    with pytest.raises(nq.NQError):
+        nq.nq_query_schedule(0, 100, 64, nq.flag_schedule(10, 2))    # not built

@@ -1,0 +1,402 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs (needs a B200).
+
+Bar (stated per test):
+* canonical mode: bit-exact for residual_out, norm_out, scales and codes;
+* against the oracle's plain float64-order mode: scales within 1e-6
+  relative, codes at most 1 ulp apart on at most 0.1% of elements;
+* every schedule the planner can pick gives identical bits;
+* outputs never write outside their rows (sentinel guard bands).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+from gpu_helpers import (Guarded, dev_bf16, dev_f32, e2m1_rank, e4m3_rank, host_u8, host_u16,
+                         same_codes_e4m3)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import fp4_activation_quantization_b200 as nq
+    return nq
+
+
+def all_schedules(d):
+    C = (d + 7) // 8
+    out = []
+    for lt in range(5, 11):
+        for lk in range(0, 3):
+            if lt == 10 and lk == 2:
+                continue
+            if (1 << (lt + lk)) >= C:
+                out.append((lt, lk))
+    return out
+
+
+# ------------------------------------------------ dynamic per-token FP8 ----
+def run_fused(nq, w, d=None, flags=0, eps=1e-6, want_norm=False, inplace=False, guarded=False):
+    x = dev_bf16(w["x"])
+    d = x.shape[1] if d is None else d
+    xs = x[:, :d]
+    res = dev_bf16(w["residual"])
+    g = dev_bf16(w["gamma"])
+    M = xs.shape[0]
+    kw = {}
+    guards = []
+    if guarded:
+        gq = Guarded(M, d, torch.float8_e4m3fn)
+        gr = Guarded(M, d, torch.bfloat16)
+        gr.view.copy_(res)
+        res = gr.view
+        kw.update(q_out=gq.view, residual_out=gr.view)
+        guards = [gq, gr]
+    if inplace:
+        kw["residual_out"] = res
+    q, s, ro, no = nq.nq_fused_add_rmsnorm_quant_fp8(xs, res, g, eps, flags=flags, want_norm=want_norm, **kw)
+    torch.cuda.synchronize()
+    for gd in guards:
+        assert gd.guards_intact()
+    return host_u8(q), s.cpu().numpy(), host_u16(ro), (host_u16(no) if no is not None else None)
+
+
+def oracle_fused(w, d=None, flags=0, eps=1e-6, want_norm=False):
+    return oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"], eps=eps, flags=flags, d=d,
+                                              want_norm=want_norm)
+
+
+def assert_fused_equal(got, exp):
+    assert np.array_equal(got[2], exp[2]), "residual_out"
+    assert np.array_equal(got[1].view(np.uint32), exp[1].view(np.uint32)), "scales"
+    assert np.array_equal(got[0], exp[0]), f"codes differ at {np.argwhere(got[0] != exp[0])[:5]}"
+    if exp[3] is not None:
+        assert np.array_equal(got[3], exp[3]), "norm_out"
+
+
+@pytest.mark.parametrize("flags_name", ["default", "div", "recip"])
+def test_fused_dynamic_small_config_bit_exact(nq, flags_name):
+    """64 tokens x 2816, seed 0, eps 1e-6: bit-exact codes, scales, residual and bf16 norm output."""
+    flags = {"default": 0, "div": nq.FLAG_SCALE_DIV, "recip": nq.FLAG_SCALE_RECIP}[flags_name]
+    oflags = {"default": 0, "div": oracle.DIV, "recip": oracle.RECIP}[flags_name]
+    w = S.make_rms_inputs(64, 2816, seed=0)
+    got = run_fused(nq, w, flags=flags, want_norm=True, guarded=True)
+    assert_fused_equal(got, oracle_fused(w, flags=oflags, want_norm=True))
+
+
+@pytest.mark.parametrize("d", [1, 7, 8, 32, 111, 128, 1000, 1024, 2816, 4104, 8192, 8208, 16384])
+def test_fused_dynamic_every_schedule(nq, d):
+    """Every built schedule covering the row gives the oracle's bits (ragged d included)."""
+    M = 19
+    w = S.make_rms_inputs(M, d, seed=d, x_outlier_channels=d >= 8)
+    exp = oracle_fused(w)
+    for lt, lk in all_schedules(d):
+        got = run_fused(nq, w, flags=nq.flag_schedule(lt, lk))
+        assert_fused_equal(got, exp)
+    assert_fused_equal(run_fused(nq, w), exp)
+
+
+@pytest.mark.parametrize("M", [1, 16, 256, 4096])
+@pytest.mark.parametrize("d", [2816, 4096, 7168, 8192])
+def test_sweep_cells_bit_exact(nq, M, d):
+    """Sweep cells (x with four x100 outlier channels) at the planner's schedule, M <= 4096."""
+    w = S.make_rms_inputs(M, d, seed=0, x_outlier_channels=True)
+    assert_fused_equal(run_fused(nq, w), oracle_fused(w))
+
+
+@pytest.mark.parametrize("d", [2816, 8192])
+def test_sweep_largest_m_sampled_rows(nq, d):
+    """M = 65536 sweep cells: device-generated inputs, sampled rows checked one by one."""
+    M = 65536
+    gen = torch.Generator(device="cuda").manual_seed(1234 + d)
+    x = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+    for c in S.outlier_channels(d):
+        x[:, c] *= 100
+    res = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+    g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(torch.bfloat16)
+    rows = np.unique(np.concatenate([[0, 1, M // 2, M - 2, M - 1],
+                                     np.random.default_rng(d).integers(0, M, 59)]))
+    res_rows = host_u16(res[rows])
+    q, s, ro, _ = nq.nq_fused_add_rmsnorm_quant_fp8(x, res, g, 1e-6)
+    torch.cuda.synchronize()
+    w = {"x": host_u16(x[rows]), "residual": res_rows, "gamma": host_u16(g)}
+    exp = oracle_fused(w)
+    got = (host_u8(q[rows]), s[rows].cpu().numpy(), host_u16(ro[rows]), None)
+    assert_fused_equal(got, exp)
+
+
+def test_fused_inplace_residual(nq):
+    w = S.make_rms_inputs(33, 4096, seed=3)
+    got = run_fused(nq, w, inplace=True)
+    assert_fused_equal(got, oracle_fused(w))
+
+
+def test_fused_plain_order_tolerance(nq):
+    """GPU vs the oracle's float64-order sums: scales within 1e-6 relative; codes <= 1 ulp on <= 0.1%."""
+    w = S.make_rms_inputs(512, 4096, seed=9, x_outlier_channels=True)
+    q, s, ro, _ = run_fused(nq, w)
+    eq, es, er, _ = oracle_fused(w, flags=oracle.SUM_PLAIN)
+    assert np.array_equal(ro, er)
+    assert np.all(np.abs(s.astype(np.float64) / es - 1) <= 1e-6)
+    diff = np.abs(e4m3_rank(q) - e4m3_rank(eq))
+    assert diff.max() <= 1 and (diff > 0).mean() <= 1e-3
+
+
+def test_fused_vs_unfused_on_gpu(nq):
+    """The bf16 double-rounding emulation matches the oracle's, and differs from fused on ~2-3% of codes."""
+    w = S.make_rms_inputs(128, 2816, seed=5)
+    fused = run_fused(nq, w)
+    unf = run_fused(nq, w, flags=nq.FLAG_NORM_BF16_ROUND)
+    assert_fused_equal(unf, oracle_fused(w, flags=oracle.NORM_BF16_ROUND))
+    frac = (fused[0] != unf[0]).mean()
+    assert 0.015 <= frac <= 0.045
+
+
+def test_fused_misaligned_column_slice(nq):
+    """x starting one element into a wider tensor takes the scalar path; same bits as the oracle."""
+    M, d = 40, 1024
+    w = S.make_rms_inputs(M, d, seed=4, ld_x=d + 8)
+    xfull = dev_bf16(w["x"])
+    xs = xfull[:, 1:1 + d]
+    res = dev_bf16(w["residual"])
+    g = dev_bf16(w["gamma"])
+    q, s, ro, _ = nq.nq_fused_add_rmsnorm_quant_fp8(xs, res, g, 1e-6)
+    exp = oracle.fused_add_rmsnorm_quant_fp8(w["x"][:, 1:1 + d], w["residual"], w["gamma"])
+    assert_fused_equal((host_u8(q), s.cpu().numpy(), host_u16(ro), None), exp)
+
+
+def test_zero_rows_and_m0(nq):
+    d = 256
+    x = torch.zeros(9, d, dtype=torch.bfloat16, device="cuda")
+    res = torch.zeros_like(x)
+    g = torch.ones(d, dtype=torch.bfloat16, device="cuda")
+    q, s, ro, _ = nq.nq_fused_add_rmsnorm_quant_fp8(x, res, g, 1e-6)
+    assert (s == 0).all() and (host_u8(q) == 0).all()
+    e = torch.empty(0, d, dtype=torch.bfloat16, device="cuda")
+    q0, s0, r0, _ = nq.nq_fused_add_rmsnorm_quant_fp8(e, torch.empty_like(e), g, 1e-6)
+    assert q0.shape == (0, d)
+
+
+def test_pdl_flag_same_bits(nq):
+    w = S.make_rms_inputs(300, 4096, seed=8)
+    a = run_fused(nq, w)
+    b = run_fused(nq, w, flags=nq.FLAG_PDL)
+    assert_fused_equal(b, a)
+
+
+# ---------------------------------------------------- static-scale FP8 ----
+@pytest.mark.parametrize("residual", [False, True])
+@pytest.mark.parametrize("flags_name", ["default", "div"])
+def test_rms_static_config_bit_exact(nq, residual, flags_name):
+    """4096 x 4096, scale 0.05 in device memory, eps 1e-5: bit-exact."""
+    M, d = 4096, 4096
+    w = S.make_rms_inputs(M, d, seed=0, residual=residual)
+    flags = nq.FLAG_SCALE_DIV if flags_name == "div" else 0
+    oflags = oracle.DIV if flags_name == "div" else 0
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    gq = Guarded(M, d, torch.float8_e4m3fn)
+    q, ro, no = nq.nq_rmsnorm_quant_fp8_static(dev_bf16(w["x"]), dev_bf16(w["gamma"]), sc, 1e-5,
+                                               residual=dev_bf16(w["residual"]) if residual else None,
+                                               q_out=gq.view, want_norm=True, flags=flags)
+    torch.cuda.synchronize()
+    assert gq.guards_intact()
+    eq, er, en = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, residual=w.get("residual"),
+                                                 eps=1e-5, flags=oflags, want_norm=True)
+    assert np.array_equal(host_u8(q), eq)
+    assert np.array_equal(host_u16(no), en)
+    if residual:
+        assert np.array_equal(host_u16(ro), er)
+
+
+@pytest.mark.parametrize("flags_name", ["default", "div"])
+def test_layernorm_static_config_bit_exact(nq, flags_name):
+    M, d = 4096, 4096
+    w = S.make_ln_inputs(M, d, seed=0)
+    flags = nq.FLAG_SCALE_DIV if flags_name == "div" else 0
+    oflags = oracle.DIV if flags_name == "div" else 0
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    q = nq.nq_layernorm_quant_fp8(dev_bf16(w["x"]), dev_f32(w["gamma"]), dev_f32(w["beta"]), sc, 1e-5, flags=flags)
+    eq = oracle.layernorm_quant_fp8(w["x"], w["gamma"], w["beta"], 0.05, eps=1e-5, flags=oflags)
+    assert np.array_equal(host_u8(q), eq)
+
+
+@pytest.mark.parametrize("d", [1, 7, 111, 128, 989, 2816, 8208, 16384])
+def test_static_paths_every_schedule(nq, d):
+    """Odd and wide hidden sizes, every schedule, RMSNorm and LayerNorm, three scales."""
+    M = 13
+    w = S.make_rms_inputs(M, d, seed=d, residual=True)
+    lw = S.make_ln_inputs(M, d, seed=d)
+    for scale in (0.01, 1.0, 10.0):
+        sc = torch.tensor([scale], dtype=torch.float32, device="cuda")
+        eq, er, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], scale, residual=w["residual"])
+        el = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], scale, eps=1e-6)
+        for sched in [None, *all_schedules(d)]:
+            f = 0 if sched is None else nq.flag_schedule(*sched)
+            q, ro, _ = nq.nq_rmsnorm_quant_fp8_static(dev_bf16(w["x"]), dev_bf16(w["gamma"]), sc, 1e-6,
+                                                      residual=dev_bf16(w["residual"]), flags=f)
+            assert np.array_equal(host_u8(q), eq) and np.array_equal(host_u16(ro), er), (scale, sched)
+            ql = nq.nq_layernorm_quant_fp8(dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"]), sc,
+                                           1e-6, flags=f)
+            assert np.array_equal(host_u8(ql), el), (scale, sched)
+
+
+def test_static_zero_scale_ieee(nq):
+    w = S.make_rms_inputs(4, 64, seed=1, residual=False)
+    x = w["x"].copy()
+    x[0, :8] = 0  # zeros give 0 * inf = NaN codes
+    sc = torch.zeros(1, dtype=torch.float32, device="cuda")
+    q, _, _ = nq.nq_rmsnorm_quant_fp8_static(dev_bf16(x), dev_bf16(w["gamma"]), sc, 1e-6)
+    eq, _, _ = oracle.rmsnorm_quant_fp8_static(x, w["gamma"], 0.0)
+    assert same_codes_e4m3(host_u8(q), eq)
+
+
+def test_static_scale_graph_replay(nq):
+    """The scale is read at execution time: a captured graph follows scale updates."""
+    w = S.make_rms_inputs(256, 4096, seed=2, residual=False)
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    q = torch.empty(256, 4096, dtype=torch.float8_e4m3fn, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, q_out=q)  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, q_out=q)
+    for scale in (0.05, 0.5, 0.013):
+        sc.fill_(scale)
+        graph.replay()
+        torch.cuda.synchronize()
+        eq, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], scale)
+        assert np.array_equal(host_u8(q), eq), scale
+
+
+# ------------------------------------------------------- group FP8 ----
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("M", [1, 32768])
+def test_group_config_bit_exact(nq, M, ue8m0):
+    """bf16 [M, 4096] with 0.1% x50 outliers, group 128, fp32 or UE8M0 scales, x * (1/s)."""
+    K = 4096
+    w = S.make_group_inputs(M, K, seed=0)
+    flags = nq.FLAG_UE8M0 if ue8m0 else 0
+    q, s = nq.nq_per_token_group_quant_fp8(dev_bf16(w["x"]), 128, flags=flags)
+    torch.cuda.synchronize()
+    eq, es = oracle.per_token_group_quant_fp8(w["x"], 128, oracle.UE8M0 if ue8m0 else 0)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32))
+    assert np.array_equal(host_u8(q), eq)
+
+
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("flags_name", ["div", "recip", "ue8m0"])
+def test_group_variants_and_strides(nq, group, flags_name):
+    M, K = 77, 1024
+    w = S.make_group_inputs(M, K + 64, seed=group)
+    f = {"div": nq.FLAG_SCALE_DIV, "recip": 0, "ue8m0": nq.FLAG_UE8M0}[flags_name]
+    of = {"div": oracle.DIV, "recip": 0, "ue8m0": oracle.UE8M0}[flags_name]
+    xfull = dev_bf16(w["x"])
+    for off in (0, 8, 1):  # aligned slice, 16-byte-aligned offset, misaligned (scalar path)
+        xs = xfull[:, off:off + K]
+        gq = Guarded(M, K, torch.float8_e4m3fn)
+        gs = Guarded(M, K // group, torch.float32)
+        q, s = nq.nq_per_token_group_quant_fp8(xs, group, q_out=gq.view, scales_out=gs.view, flags=f)
+        torch.cuda.synchronize()
+        assert gq.guards_intact() and gs.guards_intact()
+        eq, es = oracle.per_token_group_quant_fp8(w["x"][:, off:off + K], group, of)
+        assert np.array_equal(host_u8(q), eq), off
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32)), off
+
+
+def test_group_cvt_over_all_bf16_values(nq):
+    """Groups whose absmax is 448 have scale 1, so their codes are the hardware
+    e4m3 conversion of every finite bf16 value in [-448, 448]: compare with the oracle."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f = oracle.bf16_to_f32(bits)
+    vals = bits[np.isfinite(f) & (np.abs(f) <= 448)]
+    n_per = 127
+    G = (len(vals) + n_per - 1) // n_per
+    rows = np.zeros((G, 128), np.uint16)
+    rows[:, 0] = 0x43E0  # 448.0 in bf16
+    flat = np.zeros(G * n_per, np.uint16)
+    flat[: len(vals)] = vals
+    rows[:, 1:] = flat.reshape(G, n_per)
+    q, s = nq.nq_per_token_group_quant_fp8(dev_bf16(rows), 128)
+    eq, es = oracle.per_token_group_quant_fp8(rows, 128)
+    assert np.all(es == 1.0)
+    assert np.array_equal(host_u8(q), eq)
+
+
+# ------------------------------------------------------------ NVFP4 ----
+def run_nvfp4(nq, w, d, g, residual, flags=0, want_norm=False, xoff=0):
+    xfull = dev_bf16(w["x"])
+    xs = xfull[:, xoff:xoff + d]
+    M = xs.shape[0]
+    gs = torch.tensor([g], dtype=torch.float32, device="cuda")
+    gq = Guarded(M, d // 2, torch.uint8)
+    gsf = Guarded(M, d // 16, torch.float8_e4m3fn)
+    q, sf, ro, no = nq.nq_rmsnorm_quant_nvfp4(xs, dev_bf16(w["gamma"]), gs, 1e-6,
+                                              residual=dev_bf16(w["residual"]) if residual else None,
+                                              q_out=gq.view, sf_out=gsf.view, want_norm=want_norm, flags=flags)
+    torch.cuda.synchronize()
+    assert gq.guards_intact() and gsf.guards_intact()
+    return (host_u8(q), host_u8(sf), host_u16(ro) if ro is not None else None,
+            host_u16(no) if no is not None else None)
+
+
+@pytest.mark.parametrize("residual", [False, True])
+@pytest.mark.parametrize("M", [1, 64, 8192])
+@pytest.mark.parametrize("d", [7168, 1536, 512])
+def test_nvfp4_configs_bit_exact(nq, d, M, residual):
+    """d in {7168, 1536 (column slice of a [M, 2112] tensor), 512}, M in {1, 64, 8192}."""
+    ld = 2112 if d == 1536 else d
+    w = S.make_rms_inputs(M, d, seed=0, residual=residual, ld_x=ld)
+    g = oracle.nvfp4_global_scale(w["x"], w["gamma"], w.get("residual"), d=d)
+    got = run_nvfp4(nq, w, d, g, residual, want_norm=True)
+    eq, esf, er, en = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], g, residual=w.get("residual"), d=d,
+                                                 want_norm=True)
+    assert np.array_equal(got[1], esf), "block scales"
+    assert np.array_equal(got[0], eq), "codes"
+    assert np.array_equal(got[3], en), "norm_out"
+    if residual:
+        assert np.array_equal(got[2], er), "residual_out"
+
+
+@pytest.mark.parametrize("d", [16, 32, 128, 8208, 16384])
+def test_nvfp4_every_schedule_and_partial_warps(nq, d):
+    """Hidden sizes that leave warps partially active (32, 128, 8208) on every schedule."""
+    M = 11
+    w = S.make_rms_inputs(M, d, seed=d)
+    g = oracle.nvfp4_global_scale(w["x"], w["gamma"], w["residual"])
+    exp = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], g, residual=w["residual"])
+    for sched in [None, *all_schedules(d)]:
+        f = 0 if sched is None else nq.flag_schedule(*sched)
+        got = run_nvfp4(nq, w, d, g, True, flags=f)
+        assert np.array_equal(got[0], exp[0]) and np.array_equal(got[1], exp[1]), sched
+        assert np.array_equal(got[2], exp[2]), sched
+
+
+def test_nvfp4_div_misaligned_and_bf16_round(nq):
+    M, d = 21, 1536
+    w = S.make_rms_inputs(M, d, seed=6, residual=False, ld_x=2112)
+    g = oracle.nvfp4_global_scale(w["x"][:, 1:1 + d], w["gamma"])
+    for flags, oflags in [(nq.FLAG_SCALE_DIV, oracle.DIV), (nq.FLAG_NORM_BF16_ROUND, oracle.NORM_BF16_ROUND)]:
+        got = run_nvfp4(nq, w, d, g, False, flags=flags, xoff=1)
+        eq, esf, _, _ = oracle.rmsnorm_quant_nvfp4(w["x"][:, 1:1 + d], w["gamma"], g, flags=oflags)
+        assert np.array_equal(got[1], esf) and np.array_equal(got[0], eq)
+
+
+def test_nvfp4_zero_blocks(nq):
+    M, d = 3, 64
+    w = S.make_rms_inputs(M, d, seed=2, residual=False)
+    x = w["x"].copy()
+    x[1] = 0
+    x[2, :16] = 0
+    w["x"] = x
+    got = run_nvfp4(nq, w, d, 0.01, False)
+    eq, esf, _, _ = oracle.rmsnorm_quant_nvfp4(x, w["gamma"], 0.01)
+    assert np.array_equal(got[0], eq) and np.array_equal(got[1], esf)
+    assert not got[0][1].any() and not got[1][1].any()
