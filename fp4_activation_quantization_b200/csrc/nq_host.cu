@@ -7,7 +7,9 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "nq.h"
 #include "nq_internal.h"
@@ -32,7 +34,8 @@ nq_status fail(nq_status st, const char* fmt, ...) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
-                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK;
+                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK |
+                                 NQ_FLAG_PIPELINE_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
                       bool allow_bf16_round) {
@@ -41,8 +44,13 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
   if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_UE8M0 applies to group quantization only", fn);
-  if ((flags & NQ_FLAG_SCHEDULE_MASK) && !allow_schedule)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE applies to the norm calls only", fn);
+  if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_PIPELINE_MASK)) && !allow_schedule)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_PIPELINE apply to the norm calls only", fn);
+  {
+    const uint32_t pl = (flags & NQ_FLAG_PIPELINE_MASK) >> 24;
+    if (pl > uint32_t(nq::kMaxStages))
+      return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_PIPELINE(%u): at most %d stages", fn, pl, nq::kMaxStages);
+  }
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -99,13 +107,13 @@ nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedu
   return NQ_OK;
 }
 
-nq_status launch(const char* fn, const void* kernel, unsigned grid, unsigned block, void** args,
-                 bool pdl, cudaStream_t stream) {
+nq_status launch(const char* fn, const void* kernel, unsigned grid, unsigned block, size_t smem,
+                 void** args, bool pdl, cudaStream_t stream) {
   if (kernel == nullptr) return fail(NQ_ERR_UNSUPPORTED, "%s: kernel variant not built", fn);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(block, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   if (pdl) {
@@ -119,6 +127,71 @@ nq_status launch(const char* fn, const void* kernel, unsigned grid, unsigned blo
     (void)cudaGetLastError();  // launch errors are not sticky: clear so later callers do not see them
     return fail(NQ_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
   }
+  return NQ_OK;
+}
+
+// ---- device facts used by the staged (persistent) kernel's launch shape ----
+constexpr size_t kMaxDynSmem = 200 * 1024;  // dynamic shared memory opted into per staged kernel
+
+struct OccKey {
+  const void* k;
+  int dev;
+  size_t smem;
+  int occ;
+};
+std::mutex g_mu;
+std::vector<OccKey> g_occ;
+std::vector<std::pair<const void*, int>> g_attr_set;  // (kernel, device) with the smem attribute raised
+int g_sms[64] = {0};
+
+nq_status device_sms(const char* fn, int* dev, int* sms) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(NQ_ERR_CUDA, "%s: no current CUDA device: %s", fn, cudaGetErrorString(e));
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (*dev < 0 || *dev >= 64) return fail(NQ_ERR_UNSUPPORTED, "%s: device ordinal %d", fn, *dev);
+  if (g_sms[*dev] == 0) {
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, *dev);
+    if (e != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      return fail(NQ_ERR_CUDA, "%s: cannot read the SM count", fn);
+    }
+    g_sms[*dev] = n;
+  }
+  *sms = g_sms[*dev];
+  return NQ_OK;
+}
+
+// Resident CTAs per SM of `kernel` with `block` threads and `smem` dynamic bytes.
+nq_status occupancy(const char* fn, const void* kernel, int dev, int block, size_t smem, int* occ) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  bool attr_done = false;
+  for (auto& p : g_attr_set)
+    if (p.first == kernel && p.second == dev) attr_done = true;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxDynSmem));
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return fail(NQ_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", fn, cudaGetErrorString(e));
+    }
+    g_attr_set.push_back({kernel, dev});
+  }
+  for (auto& o : g_occ)
+    if (o.k == kernel && o.dev == dev && o.smem == smem) {
+      *occ = o.occ;
+      return NQ_OK;
+    }
+  int n = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(NQ_ERR_CUDA, "%s: occupancy query: %s", fn, cudaGetErrorString(e));
+  }
+  g_occ.push_back({kernel, dev, smem, n});
+  *occ = n;
   return NQ_OK;
 }
 
@@ -137,7 +210,7 @@ nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
     if (!(cond)) return fail(NQ_ERR_INVALID_ARGUMENT, __VA_ARGS__); \
   } while (0)
 
-const nq::KernelTable& table_of(int op) {
+const nq::RowKernels& table_of(int op) {
   switch (op) {
     case nq::kOpRmsDynFp8: return nq::row_kernels_rms_dyn();
     case nq::kOpRmsStaticFp8: return nq::row_kernels_rms_static();
@@ -146,17 +219,105 @@ const nq::KernelTable& table_of(int op) {
   }
 }
 
+// Full launch plan of a norm call.
+struct LaunchPlan {
+  Schedule s;
+  bool staged;
+  int stages;
+  int64_t grid;
+  int block;
+  size_t smem;
+  const void* kernel;
+};
+
+// The staged kernel's own mapping: rows of <= 1024 elements keep one warp per
+// row; wider rows use 2^min(9, log P - 1) threads with two (or four) chunks
+// each, so a CTA of 256-512 threads holds one row.
+Schedule staged_schedule(int64_t d) {
+  const int64_t C = (d + 7) / 8;
+  int lp = 0;
+  while ((int64_t(1) << lp) < C) ++lp;
+  Schedule s;
+  if (lp <= 7) {
+    s.log_t = 5;
+    s.log_k = lp > 5 ? lp - 5 : 0;
+  } else {
+    s.log_t = lp - 1 < 9 ? lp - 1 : 9;
+    s.log_k = lp - s.log_t;
+  }
+  return s;
+}
+
+// Direct kernel for few rows, unaligned rows or NQ_FLAG_PIPELINE(1); else the
+// staged persistent kernel with a ring deep enough that each SM keeps about
+// 64 KiB of row loads in flight, and one CTA per resident slot.
+nq_status plan_launch(const char* fn, int op, int64_t M, int64_t d, bool vec, bool has_res, uint32_t flags,
+                      LaunchPlan* p) {
+  const uint32_t pipe = (flags & NQ_FLAG_PIPELINE_MASK) >> 24;
+  const bool forced_sched = (flags & NQ_FLAG_SCHEDULE_MASK) != 0;
+  nq_status st = plan_rows(fn, M, d, flags, &p->s);
+  if (st != NQ_OK) return st;
+  p->staged = false;
+  p->stages = 0;
+  p->smem = 0;
+  {
+    const int threads = 1 << p->s.log_t;
+    const int rows = nq::rows_per_cta(threads);
+    p->block = threads * rows;
+    p->grid = (M + rows - 1) / rows;
+    p->kernel = table_of(op).direct[p->s.log_t - nq::kMinLogT][p->s.log_k][vec ? 1 : 0];
+  }
+  if (!vec || pipe == 1) return NQ_OK;
+
+  const Schedule ss = forced_sched ? p->s : staged_schedule(d);
+  if (!nq::schedule_built(ss.log_t, ss.log_k)) return NQ_OK;
+  const int threads = 1 << ss.log_t;
+  const int rows = nq::rows_per_cta(threads);
+  const int block = threads * rows;
+  const void* kernel = table_of(op).staged[ss.log_t - nq::kMinLogT][ss.log_k];
+  if (kernel == nullptr) return NQ_OK;
+  int dev = 0, sms = 0, occ0 = 0;
+  if ((st = device_sms(fn, &dev, &sms)) != NQ_OK) return st;
+  if ((st = occupancy(fn, kernel, dev, block, 0, &occ0)) != NQ_OK) return st;
+  if (occ0 <= 0) return NQ_OK;
+  const size_t stage_bytes = size_t(has_res ? 2 : 1) * (size_t(1) << ss.log_k) * size_t(block) * 16;
+  int stages = int(pipe);
+  if (stages < 2) {
+    const size_t want = 64 * 1024;
+    stages = 1 + int((want + size_t(occ0) * stage_bytes - 1) / (size_t(occ0) * stage_bytes));
+    stages = stages < 3 ? 3 : (stages > nq::kMaxStages ? nq::kMaxStages : stages);
+  }
+  while (stages > 2 && size_t(stages) * stage_bytes > kMaxDynSmem) --stages;
+  const size_t smem = size_t(stages) * stage_bytes;
+  if (smem > kMaxDynSmem) return NQ_OK;
+  int occ = 0;
+  if ((st = occupancy(fn, kernel, dev, block, smem, &occ)) != NQ_OK) return st;
+  if (occ <= 0) return NQ_OK;
+  const int64_t groups = (M + rows - 1) / rows;
+  const int64_t slots = int64_t(sms) * occ;
+  // Staging pays once each resident thread group walks at least two rows.
+  if (pipe < 2 && groups < 2 * slots) return NQ_OK;
+  p->s = ss;
+  p->staged = true;
+  p->stages = stages;
+  p->smem = smem;
+  p->block = block;
+  p->grid = groups < slots ? groups : slots;
+  p->kernel = kernel;
+  return NQ_OK;
+}
+
 // Shared tail of the four norm calls.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
-  Schedule s;
-  nq_status st = plan_rows(fn, a.M, a.d, flags, &s);
+  LaunchPlan p;
+  const bool has_res = (op != nq::kOpLnStaticFp8) && a.res_in != nullptr;
+  nq_status st = plan_launch(fn, op, a.M, a.d, vec, has_res, flags, &p);
   if (st != NQ_OK) return st;
-  const int threads = 1 << s.log_t;
-  const int rows = nq::rows_per_cta(threads);
-  const int64_t grid = (a.M + rows - 1) / rows;
-  const void* k = table_of(op)[s.log_t - nq::kMinLogT][s.log_k][vec ? 1 : 0];
-  void* args[] = {&a};
-  return launch(fn, k, unsigned(grid), unsigned(threads * rows), args, (flags & NQ_FLAG_PDL) != 0, stream);
+  int stages = p.stages;
+  void* args_direct[] = {&a};
+  void* args_staged[] = {&a, &stages};
+  return launch(fn, p.kernel, unsigned(p.grid), unsigned(p.block), p.smem, p.staged ? args_staged : args_direct,
+                (flags & NQ_FLAG_PDL) != 0, stream);
 }
 
 bool vec_bf16(const void* p, int64_t ld) { return p == nullptr || (aligned(p, 16) && ld % 8 == 0); }
@@ -192,6 +353,28 @@ nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* t
   *threads_per_row = 1 << s.log_t;
   *chunks_per_thread = 1 << s.log_k;
   *rows_per_cta = nq::rows_per_cta(1 << s.log_t);
+  return NQ_OK;
+}
+
+nq_status nq_query_launch(int op, int64_t M, int64_t d, uint32_t flags, int has_residual, int aligned16,
+                          int64_t* info) {
+  const char* fn = "nq_query_launch";
+  NQ_REQUIRE(op >= 0 && op < nq::kNumRowOps, "%s: op %d out of range", fn, op);
+  NQ_REQUIRE(info != nullptr, "%s: null output pointer", fn);
+  nq_status st = check_common(fn, M, d, 1.0f);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
+  LaunchPlan p;
+  const bool vec = aligned16 && d % 8 == 0;
+  if ((st = plan_launch(fn, op, M, d, vec, has_residual && op != nq::kOpLnStaticFp8, flags, &p)) != NQ_OK)
+    return st;
+  info[0] = 1 << p.s.log_t;
+  info[1] = 1 << p.s.log_k;
+  info[2] = nq::rows_per_cta(1 << p.s.log_t);
+  info[3] = p.staged ? 1 : 0;
+  info[4] = p.stages;
+  info[5] = p.grid;
+  info[6] = int64_t(p.smem);
   return NQ_OK;
 }
 
@@ -369,7 +552,7 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   if (grid > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: too many groups", fn);
   const void* k = nq::group_kernels()[group == 128 ? 1 : 0][units == 4 ? 1 : 0][vec ? 1 : 0];
   void* args[] = {&a};
-  return launch(fn, k, unsigned(grid), nq::kGroupThreads, args, (flags & NQ_FLAG_PDL) != 0, stream);
+  return launch(fn, k, unsigned(grid), nq::kGroupThreads, 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }
 
 }  // extern "C"

@@ -65,12 +65,19 @@ inline bool schedule_built(int log_t, int log_k) {
 }
 
 // Host-side kernel tables (pointer to the __global__ stub), one per
-// translation unit.  Index: [log_t - 5][log_k][vec].
+// translation unit.  Direct kernel: [log_t - 5][log_k][vec]; staged
+// (persistent, cp.async ring, 16-byte-aligned rows only): [log_t - 5][log_k].
 using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
-const KernelTable& row_kernels_rms_dyn();
-const KernelTable& row_kernels_rms_static();
-const KernelTable& row_kernels_ln_static();
-const KernelTable& row_kernels_rms_nvfp4();
+using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1];
+struct RowKernels {
+  KernelTable direct;
+  StagedTable staged;
+};
+const RowKernels& row_kernels_rms_dyn();
+const RowKernels& row_kernels_rms_static();
+const RowKernels& row_kernels_ln_static();
+const RowKernels& row_kernels_rms_nvfp4();
+constexpr int kMaxStages = 8;
 
 // Group kernel: [group == 128][units per thread: 0 -> 1, 1 -> 4][vec]
 using GroupTable = const void* [2][2][2];

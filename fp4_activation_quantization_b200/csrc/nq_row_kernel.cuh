@@ -1,11 +1,11 @@
-// nq_row_kernel.cuh — the fused residual-add + norm + quantize row kernel.
+// nq_row_kernel.cuh — the fused residual-add + norm + quantize row kernels.
 //
 // One row (token) is owned by a group of T threads: a single warp (T = 32,
 // eight rows per CTA) or the whole CTA (T = 64..1024).  Thread t of the group
 // owns the 16-byte chunks c = t + k*T, k = 0..K-1, of the row (8 bf16 values
 // each), so every load and store instruction of a warp touches one contiguous
-// 512-byte span.  The whole row stays in float32 registers from load to
-// quantized store: the row is read once, and each output is written once.
+// 512-byte span.  The row stays in float32 registers from load to quantized
+// store: the row is read once, and each output is written once.
 //
 // Steps, per row (netraruntime blog "Fusing RMSNorm and FP8 Quantization
 // Under torch.compile", TL;DR and FAQ; FlashInfer PR #3962 Description;
@@ -19,6 +19,17 @@
 //   a5 scale: dynamic s = RN(max|y| / 448), static RN(1 / scale[0]), or the
 //      NVFP4 per-16 block scale e4m3(RN(RN(amax / 6) / g));
 //   a6 quantize, pack (cvt.rn.satfinite e4m3x2 / e2m1x2) and store.
+//
+// Two kernels share that per-row body:
+//   row_kernel        one row per thread group, loads straight to registers;
+//                     the choice for few rows (latency) and unaligned rows;
+//   row_kernel_staged persistent thread groups that walk rows with a stride
+//                     and keep the next STAGES-1 rows in flight through a
+//                     per-thread cp.async ring in shared memory, so HBM
+//                     traffic never stalls on the row's reductions.  Each
+//                     thread copies and later reads only its own chunks, so
+//                     the ring needs no barrier and no flag: cp.async.wait_group
+//                     is the only wait.
 #pragma once
 
 #include "nq_device.cuh"
@@ -26,52 +37,17 @@
 
 namespace nq {
 
+// Per-thread copies of gamma (and beta) for the chunks the thread owns.
+template <int K>
+struct GammaRegs {
+  uint4 g16[K];     // bf16 gamma (RMSNorm)
+  float gf[K][8];   // float gamma (LayerNorm)
+  float bf[K][8];   // float beta (LayerNorm)
+};
+
 template <int OP, int T, int K, bool VEC>
-__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
-  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
-  constexpr int W = T / 32;             // warps per row
-  static_assert(K == 1 || K == 2 || K == 4, "chunks per thread");
-  static_assert(R * T <= 1024, "CTA size");
-
-  __shared__ float s_sum[2][W > 1 ? W * 32 : 1];
-  __shared__ uint32_t s_max[W > 1 ? W : 1];
-
-  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
-  const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5)
-                                : int64_t(blockIdx.x);
-  // Rows past M (only possible with eight rows per CTA) run every step with
-  // zeros so that warp-wide shuffles stay converged, and store nothing.
-  const bool live = row < a.M;
+__device__ __forceinline__ void load_gamma(const RowArgs& a, int tid, int C, GammaRegs<K>& G) {
   const int d = a.d;
-  const int C = (d + 7) >> 3;
-  const bool div = (a.flags & kFlagDiv) != 0;
-  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
-
-  griddep_wait();
-
-  // ---- a1: loads (all issued before any store, for memory-level parallelism)
-  float v[K][8];
-  uint4 graw[K];     // bf16 gamma chunks (RMSNorm)
-  float gf[K][8];    // float gamma (LayerNorm)
-  float bf[K][8];    // float beta (LayerNorm)
-  const uint16_t* xrow = a.x + row * a.ld_x;
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
-    const bool ok = live && c < C;
-    if constexpr (VEC) {
-      uint4 u = make_uint4(0u, 0u, 0u, 0u);
-      if (ok) u = __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c));
-      unpack_bf16x8(u, v[k]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = 8 * c + j;
-        v[k][j] = (live && c < C && e < d) ? bf16_to_f32(xrow[e]) : 0.0f;
-      }
-    }
-  }
-  // gamma / beta: shared by every row, served from L1/L2.
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
@@ -86,22 +62,22 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
           b0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
           b1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
         }
-        gf[k][0] = g0.x; gf[k][1] = g0.y; gf[k][2] = g0.z; gf[k][3] = g0.w;
-        gf[k][4] = g1.x; gf[k][5] = g1.y; gf[k][6] = g1.z; gf[k][7] = g1.w;
-        bf[k][0] = b0.x; bf[k][1] = b0.y; bf[k][2] = b0.z; bf[k][3] = b0.w;
-        bf[k][4] = b1.x; bf[k][5] = b1.y; bf[k][6] = b1.z; bf[k][7] = b1.w;
+        G.gf[k][0] = g0.x; G.gf[k][1] = g0.y; G.gf[k][2] = g0.z; G.gf[k][3] = g0.w;
+        G.gf[k][4] = g1.x; G.gf[k][5] = g1.y; G.gf[k][6] = g1.z; G.gf[k][7] = g1.w;
+        G.bf[k][0] = b0.x; G.bf[k][1] = b0.y; G.bf[k][2] = b0.z; G.bf[k][3] = b0.w;
+        G.bf[k][4] = b1.x; G.bf[k][5] = b1.y; G.bf[k][6] = b1.z; G.bf[k][7] = b1.w;
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int e = 8 * c + j;
-          gf[k][j] = (ok && e < d) ? __ldg(g + e) : 0.0f;
-          bf[k][j] = (ok && e < d) ? __ldg(a.beta + e) : 0.0f;
+          G.gf[k][j] = (ok && e < d) ? __ldg(g + e) : 0.0f;
+          G.bf[k][j] = (ok && e < d) ? __ldg(a.beta + e) : 0.0f;
         }
       }
     } else {
       const uint16_t* g = static_cast<const uint16_t*>(a.gamma);
       if constexpr (VEC) {
-        graw[k] = ok ? __ldg(reinterpret_cast<const uint4*>(g + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+        G.g16[k] = ok ? __ldg(reinterpret_cast<const uint4*>(g + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
       } else {
         uint32_t w[4];
 #pragma unroll
@@ -111,39 +87,54 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
           const uint32_t hi = (ok && e + 1 < d) ? uint32_t(__ldg(g + e + 1)) : 0u;
           w[j] = lo | (hi << 16);
         }
-        graw[k] = make_uint4(w[0], w[1], w[2], w[3]);
+        G.g16[k] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
+}
+
+// Row chunks of a bf16 row straight from global memory (zeros past the row).
+template <int T, int K, bool VEC>
+__device__ __forceinline__ void load_row(const uint16_t* rowp, int d, int C, int tid, bool live,
+                                         float (&v)[K][8]) {
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const bool ok = live && c < C;
+    if constexpr (VEC) {
+      uint4 u = make_uint4(0u, 0u, 0u, 0u);
+      if (ok) u = __ldcs(reinterpret_cast<const uint4*>(rowp + 8 * c));
+      unpack_bf16x8(u, v[k]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = 8 * c + j;
+        v[k][j] = (ok && e < d) ? bf16_to_f32(rowp[e]) : 0.0f;
+      }
+    }
+  }
+}
+
+// Steps a2..a6 of one row whose x (v) and residual (rv, when has_res) chunks
+// are in registers.  Contains the row group's barriers (T > 32).
+template <int OP, int T, int K, bool VEC>
+__device__ __forceinline__ void row_finish(const RowArgs& a, int64_t row, bool live, int tid,
+                                           float (&v)[K][8], const float (&rv)[K][8], bool has_res,
+                                           const GammaRegs<K>& G, float* s_sum0, float* s_sum1,
+                                           uint32_t* s_max) {
+  const int d = a.d;
+  const int C = (d + 7) >> 3;
+  const bool div = (a.flags & kFlagDiv) != 0;
 
   // ---- a2: residual add and residual write
   if (has_res) {
-    const uint16_t* rrow = a.res_in + row * a.ld_res;
-    float rv[K][8];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      const bool ok = live && c < C;
-      if constexpr (VEC) {
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (ok) u = __ldcs(reinterpret_cast<const uint4*>(rrow + 8 * c));
-        unpack_bf16x8(u, rv[k]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int e = 8 * c + j;
-          rv[k][j] = (ok && e < d) ? bf16_to_f32(rrow[e]) : 0.0f;
-        }
-      }
-    }
     uint16_t* orow = a.res_out + row * a.ld_res;
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
-      const bool ok = live && c < C;
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[k][j] = __fadd_rn(v[k][j], rv[k][j]);
-      if (ok) {
+      if (live && c < C) {
         if constexpr (VEC) {
           *reinterpret_cast<uint4*>(orow + 8 * c) = pack_bf16x8(v[k]);
         } else {
@@ -171,10 +162,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   for (int h = K / 2; h >= 1; h >>= 1)
 #pragma unroll
     for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-  const float total = row_sum<T>(part[0], s_sum[0], tid);
-
-  // The next kernel on the stream may start its prologue now.
-  griddep_launch_dependents();
+  const float total = row_sum<T>(part[0], s_sum0, tid);
 
   const float fd = float(d);
   float rstd;
@@ -201,7 +189,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
     for (int h = K / 2; h >= 1; h >>= 1)
 #pragma unroll
       for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-    const float sq = row_sum<T>(part[0], s_sum[1], tid);
+    const float sq = row_sum<T>(part[0], s_sum1, tid);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
   } else {
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
@@ -213,10 +201,10 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   for (int k = 0; k < K; ++k) {
     if constexpr (OP == kOpLnStaticFp8) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[k][j] = __fmaf_rn(__fmul_rn(v[k][j], rstd), gf[k][j], bf[k][j]);
+      for (int j = 0; j < 8; ++j) v[k][j] = __fmaf_rn(__fmul_rn(v[k][j], rstd), G.gf[k][j], G.bf[k][j]);
     } else {
       float g[8];
-      unpack_bf16x8(graw[k], g);
+      unpack_bf16x8(G.g16[k], g);
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[k][j] = __fmul_rn(__fmul_rn(v[k][j], rstd), g[j]);
     }
@@ -318,17 +306,149 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   }
 }
 
-// Kernel table of one operation: every built (threads, chunks, vec) schedule.
+// ------------------------------------------------------------- direct ----
+template <int OP, int T, int K, bool VEC>
+__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
+  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
+  constexpr int W = T / 32;             // warps per row
+  static_assert(K == 1 || K == 2 || K == 4, "chunks per thread");
+  static_assert(R * T <= 1024, "CTA size");
+
+  __shared__ float s_sum[2][W > 1 ? W * 32 : 1];
+  __shared__ uint32_t s_max[W > 1 ? W : 1];
+
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5)
+                                : int64_t(blockIdx.x);
+  // Rows past M (only possible with eight rows per CTA) run every step with
+  // zeros so that warp-wide shuffles stay converged, and store nothing.
+  const bool live = row < a.M;
+  const int C = (a.d + 7) >> 3;
+  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
+
+  griddep_wait();
+
+  // All loads are issued before any store, for memory-level parallelism.
+  float v[K][8], rv[K][8];
+  load_row<T, K, VEC>(a.x + row * a.ld_x, a.d, C, tid, live, v);
+  GammaRegs<K> G;
+  load_gamma<OP, T, K, VEC>(a, tid, C, G);
+  if (has_res) load_row<T, K, VEC>(a.res_in + row * a.ld_res, a.d, C, tid, live, rv);
+  // The next kernel on the stream may start its prologue now.
+  griddep_launch_dependents();
+  row_finish<OP, T, K, VEC>(a, row, live, tid, v, rv, has_res, G, s_sum[0], s_sum[1], s_max);
+}
+
+// ------------------------------------------------------------- staged ----
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+               "l"(gmem), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// Wait until at most n of this thread's committed groups are pending (n in 0..7).
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;\n" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;\n" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;\n" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;\n" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;\n" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;\n" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;\n" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;\n" ::: "memory"); break;
+  }
+}
+
+// Persistent, 16-byte-aligned rows only.  Thread group g (of G = gridDim.x * R
+// groups) handles rows g, g + G, g + 2G, ...  Dynamic shared memory holds
+// `stages` ring slots of NT (1 or 2: x, residual) x K chunks per thread.
+template <int OP, int T, int K>
+__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel_staged(const RowArgs a, int stages) {
+  constexpr int R = (T == 32) ? 8 : 1;
+  constexpr int W = T / 32;
+  constexpr int NTHR = R * T;
+  __shared__ float s_sum[2][W > 1 ? W * 32 : 1];
+  __shared__ uint32_t s_max[W > 1 ? W : 1];
+  extern __shared__ uint4 ring[];
+
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
+  const int64_t n_groups = int64_t(gridDim.x) * R;
+  const int64_t nrows = group < a.M ? (a.M - group + n_groups - 1) / n_groups : 0;
+  const int C = (a.d + 7) >> 3;
+  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
+  const int NT = has_res ? 2 : 1;
+
+  griddep_wait();
+
+  // Slot s, tensor tt, chunk k of this thread.
+  auto slot = [&](int s, int tt, int k) -> uint4* {
+    return ring + (size_t(s * NT + tt) * K + k) * NTHR + threadIdx.x;
+  };
+  auto issue = [&](int64_t j) {  // prefetch row j of this group into slot j % stages
+    if (j < nrows) {
+      const int64_t row = group + j * n_groups;
+      const int s = int(j % stages);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int c = tid + k * T;
+        const bool ok = c < C;
+        cp_async16(slot(s, 0, k), ok ? a.x + row * a.ld_x + 8 * c : a.x, ok ? 16u : 0u);
+        if (has_res) cp_async16(slot(s, 1, k), ok ? a.res_in + row * a.ld_res + 8 * c : a.res_in, ok ? 16u : 0u);
+      }
+    }
+    cp_async_commit();  // one group per row index, empty past the end, so the counting stays uniform
+  };
+
+  for (int j = 0; j < stages - 1; ++j) issue(j);
+  GammaRegs<K> G;
+  load_gamma<OP, T, K, true>(a, tid, C, G);
+  // Once every remaining row of this group is in flight, the next kernel on
+  // the stream may start its prologue.
+  const int64_t trigger = nrows > stages - 1 ? nrows - (stages - 1) : 0;
+  if (nrows == 0) griddep_launch_dependents();
+
+  for (int64_t j = 0; j < nrows; ++j) {
+    issue(j + stages - 1);  // refills the slot consumed in iteration j - 1
+    cp_async_wait_pending(stages - 1);
+    const int s = int(j % stages);
+    float v[K][8], rv[K][8];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      unpack_bf16x8(*slot(s, 0, k), v[k]);
+      if (has_res) unpack_bf16x8(*slot(s, 1, k), rv[k]);
+    }
+    if (j == trigger) griddep_launch_dependents();
+    // The reduction buffers are reused row after row.  LayerNorm's two sums
+    // use both buffers, each separated from its next use by the other sum's
+    // barrier; single-sum operations alternate buffers by row parity, so a
+    // buffer is rewritten only after every thread has passed the barrier of
+    // the row in between.
+    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
+    row_finish<OP, T, K, true>(a, group + j * n_groups, true, tid, v, rv, has_res, G, b0, s_sum[1], s_max);
+  }
+  cp_async_wait_pending(0);
+}
+
+// Kernel tables of one operation: every built (threads, chunks, vec) schedule
+// of the direct kernel, and every (threads, chunks) of the staged kernel.
 template <int OP>
 struct RowTable {
-  KernelTable t;
+  RowKernels k;
+  KernelTable& t = k.direct;
+  StagedTable& st = k.staged;
   RowTable() {
-    for (auto& a : t)
-      for (auto& b : a)
-        for (auto& c : b) c = nullptr;
-#define NQ_ROW_ENTRY(LT, LK)                                                            \
+    for (auto& x : t)
+      for (auto& y : x)
+        for (auto& z : y) z = nullptr;
+    for (auto& x : st)
+      for (auto& y : x) y = nullptr;
+#define NQ_ROW_ENTRY(LT, LK)                                                                            \
   t[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
-  t[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);
+  t[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);  \
+  st[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK)>);
     NQ_ROW_ENTRY(5, 0) NQ_ROW_ENTRY(5, 1) NQ_ROW_ENTRY(5, 2)
     NQ_ROW_ENTRY(6, 0) NQ_ROW_ENTRY(6, 1) NQ_ROW_ENTRY(6, 2)
     NQ_ROW_ENTRY(7, 0) NQ_ROW_ENTRY(7, 1) NQ_ROW_ENTRY(7, 2)

@@ -4,8 +4,8 @@
 #include "nq_row_kernel.cuh"
 
 namespace nq {
-const KernelTable& row_kernels_ln_static() {
+const RowKernels& row_kernels_ln_static() {
   static const RowTable<kOpLnStaticFp8> table;
-  return table.t;
+  return table.k;
 }
 }  // namespace nq

@@ -4,8 +4,8 @@
 #include "nq_row_kernel.cuh"
 
 namespace nq {
-const KernelTable& row_kernels_rms_dyn() {
+const RowKernels& row_kernels_rms_dyn() {
   static const RowTable<kOpRmsDynFp8> table;
-  return table.t;
+  return table.k;
 }
 }  // namespace nq

@@ -4,8 +4,8 @@
 #include "nq_row_kernel.cuh"
 
 namespace nq {
-const KernelTable& row_kernels_rms_nvfp4() {
+const RowKernels& row_kernels_rms_nvfp4() {
   static const RowTable<kOpRmsNvfp4> table;
-  return table.t;
+  return table.k;
 }
 }  // namespace nq

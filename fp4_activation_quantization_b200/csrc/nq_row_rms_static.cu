@@ -4,8 +4,8 @@
 #include "nq_row_kernel.cuh"
 
 namespace nq {
-const KernelTable& row_kernels_rms_static() {
+const RowKernels& row_kernels_rms_static() {
   static const RowTable<kOpRmsStaticFp8> table;
-  return table.t;
+  return table.k;
 }
 }  // namespace nq

@@ -102,6 +102,12 @@ typedef enum nq_status {
  * identical results; this exists for tests and tuning.  0 = automatic. */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
+/* Force the row pipeline: n = 1 runs the direct kernel (one row per thread
+ * group, loads straight to registers); n = 2..8 runs the persistent staged
+ * kernel with an n-slot cp.async ring (16-byte-aligned rows only; otherwise
+ * the direct kernel runs).  Same bits either way.  0 = automatic. */
+#define NQ_FLAG_PIPELINE(n) ((((uint32_t)(n)) & 0xFu) << 24)
+#define NQ_FLAG_PIPELINE_MASK (0xFu << 24)
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int nq_version(void);
@@ -118,6 +124,16 @@ const char* nq_last_error(void);
  */
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
                             int* chunks_per_thread, int* rows_per_cta);
+
+/*
+ * Launch the library would make for a norm call (same op codes as
+ * nq_query_schedule) over M rows of d elements, with or without a residual,
+ * with 16-byte-aligned rows or not.  info[0..6] = threads per row, chunks per
+ * thread, rows per CTA, staged (0/1), ring slots, grid size, dynamic shared
+ * bytes.  Needs a current CUDA device (occupancy queries); launches nothing.
+ */
+nq_status nq_query_launch(int op, int64_t M, int64_t d, uint32_t flags, int has_residual, int aligned16,
+                          int64_t* info);
 
 /*
  * Fused residual-add + RMSNorm + dynamic per-token e4m3.
