@@ -230,9 +230,10 @@ struct LaunchPlan {
   const void* kernel;
 };
 
-// The staged kernel's own mapping: rows of <= 1024 elements keep one warp per
-// row; wider rows use 2^min(9, log P - 1) threads with two (or four) chunks
-// each, so a CTA of 256-512 threads holds one row.
+// The staged kernel's own mapping.  Its registers do not grow with the
+// chunks per thread (rows are streamed from shared memory), so rows of <= 1024
+// elements keep one warp per row and wider rows use 128 threads per row with
+// up to 16 chunks each: small CTAs, many rows in flight per SM.
 Schedule staged_schedule(int64_t d) {
   const int64_t C = (d + 7) / 8;
   int lp = 0;
@@ -242,68 +243,96 @@ Schedule staged_schedule(int64_t d) {
     s.log_t = 5;
     s.log_k = lp > 5 ? lp - 5 : 0;
   } else {
-    s.log_t = lp - 1 < 9 ? lp - 1 : 9;
+    s.log_t = lp - 4 > 7 ? lp - 4 : 7;
     s.log_k = lp - s.log_t;
   }
   return s;
 }
 
 // Direct kernel for few rows, unaligned rows or NQ_FLAG_PIPELINE(1); else the
-// staged persistent kernel with a ring deep enough that each SM keeps about
-// 64 KiB of row loads in flight, and one CTA per resident slot.
+// staged persistent kernel.  Its ring depth is the one (2..8 slots) that puts
+// the most row bytes in flight per SM, counted up to 128 KiB, given how many
+// CTAs then fit; ties go to more resident CTAs.  One CTA per resident slot.
 nq_status plan_launch(const char* fn, int op, int64_t M, int64_t d, bool vec, bool has_res, uint32_t flags,
                       LaunchPlan* p) {
   const uint32_t pipe = (flags & NQ_FLAG_PIPELINE_MASK) >> 24;
-  const bool forced_sched = (flags & NQ_FLAG_SCHEDULE_MASK) != 0;
-  nq_status st = plan_rows(fn, M, d, flags, &p->s);
-  if (st != NQ_OK) return st;
+  const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
+  const bool forced_sched = ft || fk;
+  const int64_t C = (d + 7) / 8;
   p->staged = false;
   p->stages = 0;
   p->smem = 0;
-  {
-    const int threads = 1 << p->s.log_t;
-    const int rows = nq::rows_per_cta(threads);
-    p->block = threads * rows;
-    p->grid = (M + rows - 1) / rows;
-    p->kernel = table_of(op).direct[p->s.log_t - nq::kMinLogT][p->s.log_k][vec ? 1 : 0];
-  }
-  if (!vec || pipe == 1) return NQ_OK;
+  nq_status st;
 
-  const Schedule ss = forced_sched ? p->s : staged_schedule(d);
-  if (!nq::schedule_built(ss.log_t, ss.log_k)) return NQ_OK;
-  const int threads = 1 << ss.log_t;
-  const int rows = nq::rows_per_cta(threads);
-  const int block = threads * rows;
-  const void* kernel = table_of(op).staged[ss.log_t - nq::kMinLogT][ss.log_k];
-  if (kernel == nullptr) return NQ_OK;
-  int dev = 0, sms = 0, occ0 = 0;
-  if ((st = device_sms(fn, &dev, &sms)) != NQ_OK) return st;
-  if ((st = occupancy(fn, kernel, dev, block, 0, &occ0)) != NQ_OK) return st;
-  if (occ0 <= 0) return NQ_OK;
-  const size_t stage_bytes = size_t(has_res ? 2 : 1) * (size_t(1) << ss.log_k) * size_t(block) * 16;
-  int stages = int(pipe);
-  if (stages < 2) {
-    const size_t want = 64 * 1024;
-    stages = 1 + int((want + size_t(occ0) * stage_bytes - 1) / (size_t(occ0) * stage_bytes));
-    stages = stages < 3 ? 3 : (stages > nq::kMaxStages ? nq::kMaxStages : stages);
+  if (vec && pipe != 1) {
+    Schedule ss = staged_schedule(d);
+    bool ok = true;
+    if (forced_sched) {
+      if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
+      ss = {int(ft) + 4, int(fk) - 1};
+      ok = nq::staged_built(ss.log_t, ss.log_k) && (int64_t(1) << (ss.log_t + ss.log_k)) >= C;
+      if (!ok && pipe >= 2)
+        return fail(NQ_ERR_UNSUPPORTED, "%s: staged schedule 2^%d threads x 2^%d chunks is not built for d = %lld",
+                    fn, ss.log_t, ss.log_k, (long long)d);
+    }
+    const void* kernel = ok ? table_of(op).staged[ss.log_t - nq::kMinLogT][ss.log_k] : nullptr;
+    if (kernel != nullptr) {
+      const int threads = 1 << ss.log_t;
+      const int rows = nq::rows_per_cta(threads);
+      const int block = threads * rows;
+      int dev = 0, sms = 0;
+      if ((st = device_sms(fn, &dev, &sms)) != NQ_OK) return st;
+      const size_t stage_bytes = size_t(has_res ? 2 : 1) * (size_t(1) << ss.log_k) * size_t(block) * 16;
+      const size_t row_bytes = size_t(has_res ? 2 : 1) * size_t(d) * 2 * size_t(rows);  // useful bytes per slot
+      int best_stages = 0, best_occ = 0;
+      double best_score = -1.0;
+      const int lo = pipe >= 2 ? int(pipe) : 2, hi = pipe >= 2 ? int(pipe) : nq::kMaxStages;
+      for (int n = lo; n <= hi; ++n) {
+        if (size_t(n) * stage_bytes > kMaxDynSmem) break;
+        int occ = 0;
+        if ((st = occupancy(fn, kernel, dev, block, size_t(n) * stage_bytes, &occ)) != NQ_OK) return st;
+        if (occ <= 0) continue;
+        double inflight = double(occ) * double(n - 1) * double(row_bytes);
+        const double score = (inflight < 131072.0 ? inflight : 131072.0) + occ;  // + occ breaks ties
+        if (score > best_score) {
+          best_score = score;
+          best_stages = n;
+          best_occ = occ;
+        }
+      }
+      if (best_stages == 0 && pipe >= 2) {
+        // the forced depth does not fit: take the deepest that does
+        for (int n = int(pipe) - 1; n >= 2 && best_stages == 0; --n) {
+          int occ = 0;
+          if (size_t(n) * stage_bytes > kMaxDynSmem) continue;
+          if ((st = occupancy(fn, kernel, dev, block, size_t(n) * stage_bytes, &occ)) != NQ_OK) return st;
+          if (occ > 0) {
+            best_stages = n;
+            best_occ = occ;
+          }
+        }
+      }
+      const int64_t groups = (M + rows - 1) / rows;
+      const int64_t slots = int64_t(sms) * best_occ;
+      // Staging pays once each resident thread group walks at least two rows.
+      if (best_stages > 0 && (pipe >= 2 || groups >= 2 * slots)) {
+        p->s = ss;
+        p->staged = true;
+        p->stages = best_stages;
+        p->smem = size_t(best_stages) * stage_bytes;
+        p->block = block;
+        p->grid = groups < slots ? groups : slots;
+        p->kernel = kernel;
+        return NQ_OK;
+      }
+    }
   }
-  while (stages > 2 && size_t(stages) * stage_bytes > kMaxDynSmem) --stages;
-  const size_t smem = size_t(stages) * stage_bytes;
-  if (smem > kMaxDynSmem) return NQ_OK;
-  int occ = 0;
-  if ((st = occupancy(fn, kernel, dev, block, smem, &occ)) != NQ_OK) return st;
-  if (occ <= 0) return NQ_OK;
-  const int64_t groups = (M + rows - 1) / rows;
-  const int64_t slots = int64_t(sms) * occ;
-  // Staging pays once each resident thread group walks at least two rows.
-  if (pipe < 2 && groups < 2 * slots) return NQ_OK;
-  p->s = ss;
-  p->staged = true;
-  p->stages = stages;
-  p->smem = smem;
-  p->block = block;
-  p->grid = groups < slots ? groups : slots;
-  p->kernel = kernel;
+  if ((st = plan_rows(fn, M, d, flags, &p->s)) != NQ_OK) return st;
+  const int threads = 1 << p->s.log_t;
+  const int rows = nq::rows_per_cta(threads);
+  p->block = threads * rows;
+  p->grid = (M + rows - 1) / rows;
+  p->kernel = table_of(op).direct[p->s.log_t - nq::kMinLogT][p->s.log_k][vec ? 1 : 0];
   return NQ_OK;
 }
 

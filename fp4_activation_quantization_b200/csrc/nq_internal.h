@@ -68,7 +68,12 @@ inline bool schedule_built(int log_t, int log_k) {
 // translation unit.  Direct kernel: [log_t - 5][log_k][vec]; staged
 // (persistent, cp.async ring, 16-byte-aligned rows only): [log_t - 5][log_k].
 using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
-using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1];
+constexpr int kMaxLogKStaged = 4;
+inline bool staged_built(int log_t, int log_k) {
+  return log_t >= 5 && log_t <= 9 && log_k >= 0 && log_k <= kMaxLogKStaged && log_t + log_k <= 11 &&
+         !(log_t == 8 && log_k == 4);
+}
+using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogKStaged + 1];
 struct RowKernels {
   KernelTable direct;
   StagedTable staged;

@@ -363,9 +363,15 @@ __device__ __forceinline__ void cp_async_wait_pending(int n) {
 
 // Persistent, 16-byte-aligned rows only.  Thread group g (of G = gridDim.x * R
 // groups) handles rows g, g + G, g + 2G, ...  Dynamic shared memory holds
-// `stages` ring slots of NT (1 or 2: x, residual) x K chunks per thread.
+// `stages` ring slots of NT (1 or 2: x, residual) x K chunks per thread.  The
+// row being processed stays in its slot and is streamed through registers one
+// chunk at a time, once per pass (sum; LayerNorm variance; absmax; quantize):
+// r = x + residual is recomputed from the slot in each pass (same bits), so
+// the register count does not grow with the row width and many rows can be
+// in flight per SM.  gamma / beta are re-read per chunk through L1.
 template <int OP, int T, int K>
-__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel_staged(const RowArgs a, int stages) {
+__global__ void __launch_bounds__(T == 32 ? 256 : T, 1024 / (T == 32 ? 256 : T))
+    row_kernel_staged(const RowArgs a, int stages) {  // <= 64 registers: >= 1024 threads per SM
   constexpr int R = (T == 32) ? 8 : 1;
   constexpr int W = T / 32;
   constexpr int NTHR = R * T;
@@ -377,57 +383,206 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel_staged(const Row
   const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
   const int64_t n_groups = int64_t(gridDim.x) * R;
   const int64_t nrows = group < a.M ? (a.M - group + n_groups - 1) / n_groups : 0;
-  const int C = (a.d + 7) >> 3;
+  const int d = a.d;
+  const int C = d >> 3;  // 16-byte rows: d % 8 == 0
   const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
   const int NT = has_res ? 2 : 1;
+  const bool div = (a.flags & kFlagDiv) != 0;
+  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
+  const float fd = float(d);
 
   griddep_wait();
 
-  // Slot s, tensor tt, chunk k of this thread.
-  auto slot = [&](int s, int tt, int k) -> uint4* {
-    return ring + (size_t(s * NT + tt) * K + k) * NTHR + threadIdx.x;
-  };
   auto issue = [&](int64_t j) {  // prefetch row j of this group into slot j % stages
     if (j < nrows) {
       const int64_t row = group + j * n_groups;
-      const int s = int(j % stages);
+      uint4* base = ring + size_t(j % stages) * NT * K * NTHR + threadIdx.x;
+      const uint16_t* xr = a.x + row * a.ld_x;
+      const uint16_t* rr = a.res_in + row * a.ld_res;
 #pragma unroll
       for (int k = 0; k < K; ++k) {
         const int c = tid + k * T;
         const bool ok = c < C;
-        cp_async16(slot(s, 0, k), ok ? a.x + row * a.ld_x + 8 * c : a.x, ok ? 16u : 0u);
-        if (has_res) cp_async16(slot(s, 1, k), ok ? a.res_in + row * a.ld_res + 8 * c : a.res_in, ok ? 16u : 0u);
+        cp_async16(base + k * NTHR, ok ? xr + 8 * c : a.x, ok ? 16u : 0u);
+        if (has_res) cp_async16(base + (K + k) * NTHR, ok ? rr + 8 * c : a.res_in, ok ? 16u : 0u);
       }
     }
     cp_async_commit();  // one group per row index, empty past the end, so the counting stays uniform
   };
-
   for (int j = 0; j < stages - 1; ++j) issue(j);
-  GammaRegs<K> G;
-  load_gamma<OP, T, K, true>(a, tid, C, G);
-  // Once every remaining row of this group is in flight, the next kernel on
-  // the stream may start its prologue.
+
   const int64_t trigger = nrows > stages - 1 ? nrows - (stages - 1) : 0;
   if (nrows == 0) griddep_launch_dependents();
+  const float scale_static = (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8 || OP == kOpRmsNvfp4)
+                                 ? __ldg(a.scale) : 1.0f;
 
   for (int64_t j = 0; j < nrows; ++j) {
     issue(j + stages - 1);  // refills the slot consumed in iteration j - 1
     cp_async_wait_pending(stages - 1);
-    const int s = int(j % stages);
-    float v[K][8], rv[K][8];
+    if (j == trigger) griddep_launch_dependents();  // every remaining row is in flight
+    const int64_t row = group + j * n_groups;
+    const uint4* xs = ring + size_t(j % stages) * NT * K * NTHR + threadIdx.x;
+    const uint4* rs = xs + K * NTHR;
+    // r (8 values of chunk k): x, plus the residual when there is one.
+    auto load_r = [&](int k, float (&r)[8]) {
+      unpack_bf16x8(xs[k * NTHR], r);
+      if (has_res) {
+        float t[8];
+        unpack_bf16x8(rs[k * NTHR], t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = __fadd_rn(r[e], t[e]);
+      }
+    };
+    // Reduction buffers are reused row after row.  LayerNorm's two sums use
+    // both buffers, each separated from its next use by the other sum's
+    // barrier; single-sum operations alternate by row parity.
+    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
+
+    // ---- pass A: residual write and first row sum
+    float part[K];
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-      unpack_bf16x8(*slot(s, 0, k), v[k]);
-      if (has_res) unpack_bf16x8(*slot(s, 1, k), rv[k]);
+      const int c = tid + k * T;
+      float r[8];
+      load_r(k, r);
+      if (has_res && c < C) *reinterpret_cast<uint4*>(a.res_out + row * a.ld_res + 8 * c) = pack_bf16x8(r);
+      float p = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if constexpr (OP == kOpLnStaticFp8) p = __fadd_rn(p, r[e]);
+        else p = __fmaf_rn(r[e], r[e], p);
+      }
+      part[k] = p;
     }
-    if (j == trigger) griddep_launch_dependents();
-    // The reduction buffers are reused row after row.  LayerNorm's two sums
-    // use both buffers, each separated from its next use by the other sum's
-    // barrier; single-sum operations alternate buffers by row parity, so a
-    // buffer is rewritten only after every thread has passed the barrier of
-    // the row in between.
-    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
-    row_finish<OP, T, K, true>(a, group + j * n_groups, true, tid, v, rv, has_res, G, b0, s_sum[1], s_max);
+#pragma unroll
+    for (int h = K / 2; h >= 1; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
+    const float total = row_sum<T>(part[0], b0, tid);
+
+    float rstd, mean = 0.0f;
+    if constexpr (OP == kOpLnStaticFp8) {
+      mean = __fdiv_rn(total, fd);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int c = tid + k * T;
+        float r[8];
+        load_r(k, r);
+        float p = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float ce = (c < C) ? __fsub_rn(r[e], mean) : 0.0f;
+          p = __fmaf_rn(ce, ce, p);
+        }
+        part[k] = p;
+      }
+#pragma unroll
+      for (int h = K / 2; h >= 1; h >>= 1)
+#pragma unroll
+        for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
+      const float sq = row_sum<T>(part[0], s_sum[1], tid);
+      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
+    } else {
+      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
+    }
+
+    // y (8 values of chunk k) from the slot.
+    auto make_y = [&](int k, float (&y)[8]) {
+      const int c = tid + k * T;
+      float r[8];
+      load_r(k, r);
+      if constexpr (OP == kOpLnStaticFp8) {
+        float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
+        if (c < C) {
+          const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
+          g0 = __ldg(reinterpret_cast<const float4*>(gp));
+          g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
+          e0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
+          e1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
+        }
+        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float bb[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float ce = (c < C) ? __fsub_rn(r[e], mean) : 0.0f;
+          y[e] = __fmaf_rn(__fmul_rn(ce, rstd), gg[e], bb[e]);
+        }
+      } else {
+        uint4 gu = make_uint4(0u, 0u, 0u, 0u);
+        if (c < C) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
+        float g[8];
+        unpack_bf16x8(gu, g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(__fmul_rn(r[e], rstd), g[e]);
+      }
+      if (bf16_round) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = round_bf16(y[e]);
+      }
+    };
+    auto store_e4m3 = [&](int k, const float (&t)[8]) {
+      const int c = tid + k * T;
+      const uint32_t lo = pack_e4m3x4(t[0], t[1], t[2], t[3]);
+      const uint32_t hi = pack_e4m3x4(t[4], t[5], t[6], t[7]);
+      if (c < C) *reinterpret_cast<uint2*>(a.q + row * a.ld_q + 8 * c) = make_uint2(lo, hi);
+    };
+
+    // ---- pass B: normalize; static scales and NVFP4 quantize here
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      float y[8];
+      make_y(k, y);
+      if constexpr (OP != kOpLnStaticFp8) {
+        if (a.norm_out != nullptr && c < C)
+          *reinterpret_cast<uint4*>(a.norm_out + row * a.ld_norm + 8 * c) = pack_bf16x8(y);
+      }
+      if constexpr (OP == kOpRmsDynFp8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(y[e]));
+      } else if constexpr (OP == kOpRmsNvfp4) {
+        float m8 = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8 = fmaxf(m8, fabsf(y[e]));
+        const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));  // chunks c, c^1 form a block
+        const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), scale_static));
+        const float S = __fmul_rn(e4m3_to_f32(sfc), scale_static);
+        const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = (div && S != 0.0f) ? __fdiv_rn(y[e], S) : __fmul_rn(y[e], mult);
+        const uint32_t packed = pack_e2m1x8(t);
+        if (c < C) {
+          *reinterpret_cast<uint32_t*>(a.q + row * a.ld_q + 4 * c) = packed;
+          if ((c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
+        }
+      } else {
+        const float inv = __frcp_rn(scale_static);
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = div ? __fdiv_rn(y[e], scale_static) : __fmul_rn(y[e], inv);
+        store_e4m3(k, t);
+      }
+    }
+
+    // ---- pass C (dynamic per-token scale): quantize with the row's scale
+    if constexpr (OP == kOpRmsDynFp8) {
+      const float amax = row_max_nonneg<T>(m, s_max, tid);
+      const float sc = __fdiv_rn(amax, kE4M3Max);
+      if (tid == 0) a.scale_out[row] = sc;
+      const float inv = __frcp_rn(sc);
+      const bool passthrough = (sc == 0.0f);  // zero row: store the signed zeros of y
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        float y[8], t[8];
+        make_y(k, y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          t[e] = passthrough ? y[e] : (div ? __fdiv_rn(y[e], sc) : __fmul_rn(y[e], inv));
+        store_e4m3(k, t);
+      }
+    }
   }
   cp_async_wait_pending(0);
 }
@@ -437,25 +592,30 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel_staged(const Row
 template <int OP>
 struct RowTable {
   RowKernels k;
-  KernelTable& t = k.direct;
-  StagedTable& st = k.staged;
   RowTable() {
-    for (auto& x : t)
+    for (auto& x : k.direct)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
-    for (auto& x : st)
+    for (auto& x : k.staged)
       for (auto& y : x) y = nullptr;
-#define NQ_ROW_ENTRY(LT, LK)                                                                            \
-  t[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
-  t[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);  \
-  st[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK)>);
-    NQ_ROW_ENTRY(5, 0) NQ_ROW_ENTRY(5, 1) NQ_ROW_ENTRY(5, 2)
-    NQ_ROW_ENTRY(6, 0) NQ_ROW_ENTRY(6, 1) NQ_ROW_ENTRY(6, 2)
-    NQ_ROW_ENTRY(7, 0) NQ_ROW_ENTRY(7, 1) NQ_ROW_ENTRY(7, 2)
-    NQ_ROW_ENTRY(8, 0) NQ_ROW_ENTRY(8, 1) NQ_ROW_ENTRY(8, 2)
-    NQ_ROW_ENTRY(9, 0) NQ_ROW_ENTRY(9, 1) NQ_ROW_ENTRY(9, 2)
-    NQ_ROW_ENTRY(10, 0) NQ_ROW_ENTRY(10, 1)
-#undef NQ_ROW_ENTRY
+#define NQ_DIRECT(LT, LK)                                                                                     \
+  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);
+#define NQ_STAGED(LT, LK) \
+  k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK)>);
+    NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2)
+    NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2)
+    NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2)
+    NQ_DIRECT(8, 0) NQ_DIRECT(8, 1) NQ_DIRECT(8, 2)
+    NQ_DIRECT(9, 0) NQ_DIRECT(9, 1) NQ_DIRECT(9, 2)
+    NQ_DIRECT(10, 0) NQ_DIRECT(10, 1)
+    NQ_STAGED(5, 0) NQ_STAGED(5, 1) NQ_STAGED(5, 2) NQ_STAGED(5, 3) NQ_STAGED(5, 4)
+    NQ_STAGED(6, 0) NQ_STAGED(6, 1) NQ_STAGED(6, 2) NQ_STAGED(6, 3) NQ_STAGED(6, 4)
+    NQ_STAGED(7, 0) NQ_STAGED(7, 1) NQ_STAGED(7, 2) NQ_STAGED(7, 3) NQ_STAGED(7, 4)
+    NQ_STAGED(8, 0) NQ_STAGED(8, 1) NQ_STAGED(8, 2) NQ_STAGED(8, 3)
+    NQ_STAGED(9, 0) NQ_STAGED(9, 1) NQ_STAGED(9, 2)
+#undef NQ_DIRECT
+#undef NQ_STAGED
   }
 };
 

@@ -97,9 +97,11 @@ typedef enum nq_status {
 /* Round y to bf16 before quantizing: reproduces the two-kernel (norm -> bf16
  * -> quant) numerics for A/B comparisons.  Not for production use. */
 #define NQ_FLAG_NORM_BF16_ROUND (1u << 4)
-/* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
- * thread (k = 0..2), with 2^(t+k) * 8 >= d.  Every schedule gives bitwise
- * identical results; this exists for tests and tuning.  0 = automatic. */
+/* Force a schedule: 2^t threads per row and 2^k 16-byte chunks per thread,
+ * with 2^(t+k) * 8 >= d.  The direct kernel is built for t = 5..10, k = 0..2
+ * (not t = 10 with k = 2); the staged kernel for t = 5..9, k = 0..4 with
+ * t + k <= 11.  Every schedule gives bitwise identical results; this exists
+ * for tests and tuning.  0 = automatic. */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
 /* Force the row pipeline: n = 1 runs the direct kernel (one row per thread

@@ -410,7 +410,16 @@ STAGED_CASES = [  # (d, M, ld_x): M large enough that every thread group walks s
 
 
 def staged_schedules(d):
-    return [(lt, lk) for (lt, lk) in all_schedules(d) if (1 << (lt + lk)) < 4 * ((d + 7) // 8) or lt == 5]
+    """Staged-kernel schedules (2^lt threads x 2^lk chunks) that cover a row of d without 4x waste."""
+    C = (d + 7) // 8
+    out = []
+    for lt in range(5, 10):
+        for lk in range(0, 5):
+            if lt + lk > 11:
+                continue
+            if C <= (1 << (lt + lk)) < 4 * C:
+                out.append((lt, lk))
+    return out
 
 
 @pytest.mark.parametrize("d,M,ld", STAGED_CASES)
@@ -429,7 +438,8 @@ def test_staged_all_ops_bit_exact(nq, d, M, ld):
     e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
     e_fp4 = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn, residual=w["residual"], d=d)
     variants = [nq.flag_pipeline(n) for n in (2, 3, 5, 8)]
-    variants += [nq.flag_pipeline(3) | nq.flag_schedule(*s) for s in staged_schedules(d)[:3]]
+    sch = staged_schedules(d)
+    variants += [nq.flag_pipeline(3) | nq.flag_schedule(*s) for s in sch[:2] + sch[-2:]]
     for f in variants:
         info = nq.nq_query_launch(nq.OP_RMS_DYN_FP8, M, d, f, True)
         assert info["staged"] == 1, info
