@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
     "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND",
-    "flag_schedule", "flag_pipeline", "nq_query_launch", "NQError", "lib", "library_path", "version",
+    "flag_schedule", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4",
@@ -42,11 +42,6 @@ OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4 = 0, 1, 2, 3
 def flag_schedule(log2_threads: int, log2_chunks: int) -> int:
     """NQ_FLAG_SCHEDULE(t, k): force 2^t threads per row and 2^k chunks per thread."""
     return (((log2_threads - 4) & 0xF) << 16) | (((log2_chunks + 1) & 0x7) << 20)
-
-
-def flag_pipeline(stages: int) -> int:
-    """NQ_FLAG_PIPELINE(n): 1 = direct kernel, 2..8 = staged kernel with an n-slot ring."""
-    return (stages & 0xF) << 24
 
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,9 +66,6 @@ def _load() -> ctypes.CDLL:
     L.nq_query_schedule.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     L.nq_query_schedule.restype = st
-    L.nq_query_launch.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.c_int, ctypes.c_int,
-                                  ctypes.POINTER(ctypes.c_int64)]
-    L.nq_query_launch.restype = st
     L.nq_fused_add_rmsnorm_quant_fp8.argtypes = [P, I64, P, P, I64, P, P, I64, P, P, I64, I64, I64, F, U32, P]
     L.nq_rmsnorm_quant_fp8_static.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, I64, I64, F, U32, P]
     L.nq_layernorm_quant_fp8.argtypes = [P, I64, P, P, P, P, I64, I64, I64, F, U32, P]
@@ -165,15 +157,6 @@ def nq_query_schedule(op: int, M: int, d: int, flags: int = 0):
     _check(lib.nq_query_schedule(op, M, d, flags, ctypes.byref(t), ctypes.byref(k), ctypes.byref(r)),
            "nq_query_schedule")
     return t.value, k.value, r.value
-
-
-def nq_query_launch(op: int, M: int, d: int, flags: int = 0, has_residual: bool = False,
-                    aligned16: bool = True) -> dict:
-    """The launch a norm call would make (needs a CUDA device)."""
-    info = (ctypes.c_int64 * 7)()
-    _check(lib.nq_query_launch(op, M, d, flags, int(has_residual), int(aligned16), info), "nq_query_launch")
-    keys = ("threads_per_row", "chunks_per_thread", "rows_per_cta", "staged", "stages", "grid", "smem_bytes")
-    return dict(zip(keys, [int(v) for v in info]))
 
 
 def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, residual_out=None,

@@ -7,9 +7,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
-#include <mutex>
 #include <string>
-#include <vector>
 
 #include "nq.h"
 #include "nq_internal.h"
@@ -34,8 +32,7 @@ nq_status fail(nq_status st, const char* fmt, ...) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
-                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK |
-                                 NQ_FLAG_PIPELINE_MASK;
+                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
                       bool allow_bf16_round) {
@@ -44,13 +41,8 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
   if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_UE8M0 applies to group quantization only", fn);
-  if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_PIPELINE_MASK)) && !allow_schedule)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_PIPELINE apply to the norm calls only", fn);
-  {
-    const uint32_t pl = (flags & NQ_FLAG_PIPELINE_MASK) >> 24;
-    if (pl > uint32_t(nq::kMaxStages))
-      return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_PIPELINE(%u): at most %d stages", fn, pl, nq::kMaxStages);
-  }
+  if ((flags & NQ_FLAG_SCHEDULE_MASK) && !allow_schedule)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE applies to the norm calls only", fn);
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -72,8 +64,8 @@ struct Schedule {
 // Row -> thread mapping.  C = ceil(d / 8) chunks of 16 bytes, P = the next
 // power of two.  Rows of <= 1024 elements: one warp per row (eight rows per
 // CTA), 2^max(0, log P - 5) chunks per thread.  Wider rows: one CTA per row
-// with four chunks per thread, so each thread keeps 64 bytes of the row (128
-// with a residual) in flight.  Few rows (M < 148, fewer than one per SM):
+// with four chunks per thread (64 bytes of the row per thread, 128 with a
+// residual, in flight at once).  Few rows (M < 148, fewer than one per SM):
 // spread the row over up to 1024 threads with one or two chunks each, which
 // shortens the per-row critical path.  Every mapping gives identical bits.
 nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedule* s) {
@@ -130,71 +122,6 @@ nq_status launch(const char* fn, const void* kernel, unsigned grid, unsigned blo
   return NQ_OK;
 }
 
-// ---- device facts used by the staged (persistent) kernel's launch shape ----
-constexpr size_t kMaxDynSmem = 200 * 1024;  // dynamic shared memory opted into per staged kernel
-
-struct OccKey {
-  const void* k;
-  int dev;
-  size_t smem;
-  int occ;
-};
-std::mutex g_mu;
-std::vector<OccKey> g_occ;
-std::vector<std::pair<const void*, int>> g_attr_set;  // (kernel, device) with the smem attribute raised
-int g_sms[64] = {0};
-
-nq_status device_sms(const char* fn, int* dev, int* sms) {
-  cudaError_t e = cudaGetDevice(dev);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return fail(NQ_ERR_CUDA, "%s: no current CUDA device: %s", fn, cudaGetErrorString(e));
-  }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (*dev < 0 || *dev >= 64) return fail(NQ_ERR_UNSUPPORTED, "%s: device ordinal %d", fn, *dev);
-  if (g_sms[*dev] == 0) {
-    int n = 0;
-    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, *dev);
-    if (e != cudaSuccess || n <= 0) {
-      (void)cudaGetLastError();
-      return fail(NQ_ERR_CUDA, "%s: cannot read the SM count", fn);
-    }
-    g_sms[*dev] = n;
-  }
-  *sms = g_sms[*dev];
-  return NQ_OK;
-}
-
-// Resident CTAs per SM of `kernel` with `block` threads and `smem` dynamic bytes.
-nq_status occupancy(const char* fn, const void* kernel, int dev, int block, size_t smem, int* occ) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  bool attr_done = false;
-  for (auto& p : g_attr_set)
-    if (p.first == kernel && p.second == dev) attr_done = true;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxDynSmem));
-    if (e != cudaSuccess) {
-      (void)cudaGetLastError();
-      return fail(NQ_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", fn, cudaGetErrorString(e));
-    }
-    g_attr_set.push_back({kernel, dev});
-  }
-  for (auto& o : g_occ)
-    if (o.k == kernel && o.dev == dev && o.smem == smem) {
-      *occ = o.occ;
-      return NQ_OK;
-    }
-  int n = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return fail(NQ_ERR_CUDA, "%s: occupancy query: %s", fn, cudaGetErrorString(e));
-  }
-  g_occ.push_back({kernel, dev, smem, n});
-  *occ = n;
-  return NQ_OK;
-}
-
 nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
   if (M < 0) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: M = %lld < 0", fn, (long long)M);
   if (d < 1) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: d = %lld < 1", fn, (long long)d);
@@ -219,134 +146,17 @@ const nq::RowKernels& table_of(int op) {
   }
 }
 
-// Full launch plan of a norm call.
-struct LaunchPlan {
-  Schedule s;
-  bool staged;
-  int stages;
-  int64_t grid;
-  int block;
-  size_t smem;
-  const void* kernel;
-};
-
-// The staged kernel's own mapping.  Its registers do not grow with the
-// chunks per thread (rows are streamed from shared memory), so rows of <= 1024
-// elements keep one warp per row and wider rows use 128 threads per row with
-// up to 16 chunks each: small CTAs, many rows in flight per SM.
-Schedule staged_schedule(int64_t d) {
-  const int64_t C = (d + 7) / 8;
-  int lp = 0;
-  while ((int64_t(1) << lp) < C) ++lp;
-  Schedule s;
-  if (lp <= 7) {
-    s.log_t = 5;
-    s.log_k = lp > 5 ? lp - 5 : 0;
-  } else {
-    s.log_t = lp - 4 > 7 ? lp - 4 : 7;
-    s.log_k = lp - s.log_t;
-  }
-  return s;
-}
-
-// Direct kernel for few rows, unaligned rows or NQ_FLAG_PIPELINE(1); else the
-// staged persistent kernel.  Its ring depth is the one (2..8 slots) that puts
-// the most row bytes in flight per SM, counted up to 128 KiB, given how many
-// CTAs then fit; ties go to more resident CTAs.  One CTA per resident slot.
-nq_status plan_launch(const char* fn, int op, int64_t M, int64_t d, bool vec, bool has_res, uint32_t flags,
-                      LaunchPlan* p) {
-  const uint32_t pipe = (flags & NQ_FLAG_PIPELINE_MASK) >> 24;
-  const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
-  const bool forced_sched = ft || fk;
-  const int64_t C = (d + 7) / 8;
-  p->staged = false;
-  p->stages = 0;
-  p->smem = 0;
-  nq_status st;
-
-  if (vec && pipe != 1) {
-    Schedule ss = staged_schedule(d);
-    bool ok = true;
-    if (forced_sched) {
-      if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
-      ss = {int(ft) + 4, int(fk) - 1};
-      ok = nq::staged_built(ss.log_t, ss.log_k) && (int64_t(1) << (ss.log_t + ss.log_k)) >= C;
-      if (!ok && pipe >= 2)
-        return fail(NQ_ERR_UNSUPPORTED, "%s: staged schedule 2^%d threads x 2^%d chunks is not built for d = %lld",
-                    fn, ss.log_t, ss.log_k, (long long)d);
-    }
-    const void* kernel = ok ? table_of(op).staged[ss.log_t - nq::kMinLogT][ss.log_k] : nullptr;
-    if (kernel != nullptr) {
-      const int threads = 1 << ss.log_t;
-      const int rows = nq::rows_per_cta(threads);
-      const int block = threads * rows;
-      int dev = 0, sms = 0;
-      if ((st = device_sms(fn, &dev, &sms)) != NQ_OK) return st;
-      const size_t stage_bytes = size_t(has_res ? 2 : 1) * (size_t(1) << ss.log_k) * size_t(block) * 16;
-      const size_t row_bytes = size_t(has_res ? 2 : 1) * size_t(d) * 2 * size_t(rows);  // useful bytes per slot
-      int best_stages = 0, best_occ = 0;
-      double best_score = -1.0;
-      const int lo = pipe >= 2 ? int(pipe) : 2, hi = pipe >= 2 ? int(pipe) : nq::kMaxStages;
-      for (int n = lo; n <= hi; ++n) {
-        if (size_t(n) * stage_bytes > kMaxDynSmem) break;
-        int occ = 0;
-        if ((st = occupancy(fn, kernel, dev, block, size_t(n) * stage_bytes, &occ)) != NQ_OK) return st;
-        if (occ <= 0) continue;
-        double inflight = double(occ) * double(n - 1) * double(row_bytes);
-        const double score = (inflight < 131072.0 ? inflight : 131072.0) + occ;  // + occ breaks ties
-        if (score > best_score) {
-          best_score = score;
-          best_stages = n;
-          best_occ = occ;
-        }
-      }
-      if (best_stages == 0 && pipe >= 2) {
-        // the forced depth does not fit: take the deepest that does
-        for (int n = int(pipe) - 1; n >= 2 && best_stages == 0; --n) {
-          int occ = 0;
-          if (size_t(n) * stage_bytes > kMaxDynSmem) continue;
-          if ((st = occupancy(fn, kernel, dev, block, size_t(n) * stage_bytes, &occ)) != NQ_OK) return st;
-          if (occ > 0) {
-            best_stages = n;
-            best_occ = occ;
-          }
-        }
-      }
-      const int64_t groups = (M + rows - 1) / rows;
-      const int64_t slots = int64_t(sms) * best_occ;
-      // Staging pays once each resident thread group walks at least two rows.
-      if (best_stages > 0 && (pipe >= 2 || groups >= 2 * slots)) {
-        p->s = ss;
-        p->staged = true;
-        p->stages = best_stages;
-        p->smem = size_t(best_stages) * stage_bytes;
-        p->block = block;
-        p->grid = groups < slots ? groups : slots;
-        p->kernel = kernel;
-        return NQ_OK;
-      }
-    }
-  }
-  if ((st = plan_rows(fn, M, d, flags, &p->s)) != NQ_OK) return st;
-  const int threads = 1 << p->s.log_t;
-  const int rows = nq::rows_per_cta(threads);
-  p->block = threads * rows;
-  p->grid = (M + rows - 1) / rows;
-  p->kernel = table_of(op).direct[p->s.log_t - nq::kMinLogT][p->s.log_k][vec ? 1 : 0];
-  return NQ_OK;
-}
-
 // Shared tail of the four norm calls.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
-  LaunchPlan p;
-  const bool has_res = (op != nq::kOpLnStaticFp8) && a.res_in != nullptr;
-  nq_status st = plan_launch(fn, op, a.M, a.d, vec, has_res, flags, &p);
+  Schedule s;
+  nq_status st = plan_rows(fn, a.M, a.d, flags, &s);
   if (st != NQ_OK) return st;
-  int stages = p.stages;
-  void* args_direct[] = {&a};
-  void* args_staged[] = {&a, &stages};
-  return launch(fn, p.kernel, unsigned(p.grid), unsigned(p.block), p.smem, p.staged ? args_staged : args_direct,
-                (flags & NQ_FLAG_PDL) != 0, stream);
+  const int threads = 1 << s.log_t;
+  const int rows = nq::rows_per_cta(threads);
+  const int64_t grid = (a.M + rows - 1) / rows;
+  const void* k = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k][vec ? 1 : 0];
+  void* args[] = {&a};
+  return launch(fn, k, unsigned(grid), unsigned(threads * rows), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }
 
 bool vec_bf16(const void* p, int64_t ld) { return p == nullptr || (aligned(p, 16) && ld % 8 == 0); }
@@ -382,28 +192,6 @@ nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* t
   *threads_per_row = 1 << s.log_t;
   *chunks_per_thread = 1 << s.log_k;
   *rows_per_cta = nq::rows_per_cta(1 << s.log_t);
-  return NQ_OK;
-}
-
-nq_status nq_query_launch(int op, int64_t M, int64_t d, uint32_t flags, int has_residual, int aligned16,
-                          int64_t* info) {
-  const char* fn = "nq_query_launch";
-  NQ_REQUIRE(op >= 0 && op < nq::kNumRowOps, "%s: op %d out of range", fn, op);
-  NQ_REQUIRE(info != nullptr, "%s: null output pointer", fn);
-  nq_status st = check_common(fn, M, d, 1.0f);
-  if (st != NQ_OK) return st;
-  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
-  LaunchPlan p;
-  const bool vec = aligned16 && d % 8 == 0;
-  if ((st = plan_launch(fn, op, M, d, vec, has_residual && op != nq::kOpLnStaticFp8, flags, &p)) != NQ_OK)
-    return st;
-  info[0] = 1 << p.s.log_t;
-  info[1] = 1 << p.s.log_k;
-  info[2] = nq::rows_per_cta(1 << p.s.log_t);
-  info[3] = p.staged ? 1 : 0;
-  info[4] = p.stages;
-  info[5] = p.grid;
-  info[6] = int64_t(p.smem);
   return NQ_OK;
 }
 

@@ -56,33 +56,24 @@ struct GroupArgs {
 };
 
 // Schedules: 2^t threads per row (t = 5..10), 2^k chunks of 8 elements per
-// thread (k = 0..2).  Rows per CTA: 8 when t == 5 (one warp per row), else 1.
-constexpr int kMinLogT = 5, kMaxLogT = 10, kMaxLogK = 2;
+// thread (k = 0..3, with t + k <= 11, i.e. up to 2048 chunks = 16384
+// elements).  Rows per CTA: 8 when t == 5 (one warp per row), else 1.
+constexpr int kMinLogT = 5, kMaxLogT = 10, kMaxLogK = 3;
 inline int rows_per_cta(int threads) { return threads == 32 ? 8 : 1; }
 inline bool schedule_built(int log_t, int log_k) {
-  return log_t >= kMinLogT && log_t <= kMaxLogT && log_k >= 0 && log_k <= kMaxLogK &&
-         !(log_t == 10 && log_k == 2);
+  return log_t >= kMinLogT && log_t <= kMaxLogT && log_k >= 0 && log_k <= kMaxLogK && log_t + log_k <= 11;
 }
 
 // Host-side kernel tables (pointer to the __global__ stub), one per
-// translation unit.  Direct kernel: [log_t - 5][log_k][vec]; staged
-// (persistent, cp.async ring, 16-byte-aligned rows only): [log_t - 5][log_k].
+// translation unit: [log_t - 5][log_k][vec].
 using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
-constexpr int kMaxLogKStaged = 4;
-inline bool staged_built(int log_t, int log_k) {
-  return log_t >= 5 && log_t <= 9 && log_k >= 0 && log_k <= kMaxLogKStaged && log_t + log_k <= 11 &&
-         !(log_t == 8 && log_k == 4);
-}
-using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogKStaged + 1];
 struct RowKernels {
   KernelTable direct;
-  StagedTable staged;
 };
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();
 const RowKernels& row_kernels_rms_nvfp4();
-constexpr int kMaxStages = 8;
 
 // Group kernel: [group == 128][units per thread: 0 -> 1, 1 -> 4][vec]
 using GroupTable = const void* [2][2][2];

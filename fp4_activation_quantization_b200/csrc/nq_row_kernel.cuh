@@ -1,4 +1,4 @@
-// nq_row_kernel.cuh — the fused residual-add + norm + quantize row kernels.
+// nq_row_kernel.cuh — the fused residual-add + norm + quantize row kernel.
 //
 // One row (token) is owned by a group of T threads: a single warp (T = 32,
 // eight rows per CTA) or the whole CTA (T = 64..1024).  Thread t of the group
@@ -20,16 +20,11 @@
 //      NVFP4 per-16 block scale e4m3(RN(RN(amax / 6) / g));
 //   a6 quantize, pack (cvt.rn.satfinite e4m3x2 / e2m1x2) and store.
 //
-// Two kernels share that per-row body:
-//   row_kernel        one row per thread group, loads straight to registers;
-//                     the choice for few rows (latency) and unaligned rows;
-//   row_kernel_staged persistent thread groups that walk rows with a stride
-//                     and keep the next STAGES-1 rows in flight through a
-//                     per-thread cp.async ring in shared memory, so HBM
-//                     traffic never stalls on the row's reductions.  Each
-//                     thread copies and later reads only its own chunks, so
-//                     the ring needs no barrier and no flag: cp.async.wait_group
-//                     is the only wait.
+// The kernel is bound by instruction issue as much as by HBM, so every
+// per-element float operation is a packed two-lane one (add / mul / fma
+// .f32x2: each lane rounds exactly like its scalar form), the chunk sums use
+// an even and an odd accumulator so that they too run two lanes wide, and
+// gamma / beta are fetched only after the row's reductions.
 #pragma once
 
 #include "nq_device.cuh"
@@ -37,180 +32,212 @@
 
 namespace nq {
 
-// Per-thread copies of gamma (and beta) for the chunks the thread owns.
-template <int K>
-struct GammaRegs {
-  uint4 g16[K];     // bf16 gamma (RMSNorm)
-  float gf[K][8];   // float gamma (LayerNorm)
-  float bf[K][8];   // float beta (LayerNorm)
-};
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-template <int OP, int T, int K, bool VEC>
-__device__ __forceinline__ void load_gamma(const RowArgs& a, int tid, int C, GammaRegs<K>& G) {
-  const int d = a.d;
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
-    const bool ok = c < C;
-    if constexpr (OP == kOpLnStaticFp8) {
-      const float* g = static_cast<const float*>(a.gamma);
-      if constexpr (VEC) {
-        float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, b0 = g0, b1 = g0;
-        if (ok) {
-          g0 = __ldg(reinterpret_cast<const float4*>(g + 8 * c));
-          g1 = __ldg(reinterpret_cast<const float4*>(g + 8 * c + 4));
-          b0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
-          b1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
-        }
-        G.gf[k][0] = g0.x; G.gf[k][1] = g0.y; G.gf[k][2] = g0.z; G.gf[k][3] = g0.w;
-        G.gf[k][4] = g1.x; G.gf[k][5] = g1.y; G.gf[k][6] = g1.z; G.gf[k][7] = g1.w;
-        G.bf[k][0] = b0.x; G.bf[k][1] = b0.y; G.bf[k][2] = b0.z; G.bf[k][3] = b0.w;
-        G.bf[k][4] = b1.x; G.bf[k][5] = b1.y; G.bf[k][6] = b1.z; G.bf[k][7] = b1.w;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int e = 8 * c + j;
-          G.gf[k][j] = (ok && e < d) ? __ldg(g + e) : 0.0f;
-          G.bf[k][j] = (ok && e < d) ? __ldg(a.beta + e) : 0.0f;
-        }
-      }
-    } else {
-      const uint16_t* g = static_cast<const uint16_t*>(a.gamma);
-      if constexpr (VEC) {
-        G.g16[k] = ok ? __ldg(reinterpret_cast<const uint4*>(g + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
-      } else {
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = 8 * c + 2 * j;
-          const uint32_t lo = (ok && e < d) ? uint32_t(__ldg(g + e)) : 0u;
-          const uint32_t hi = (ok && e + 1 < d) ? uint32_t(__ldg(g + e + 1)) : 0u;
-          w[j] = lo | (hi << 16);
-        }
-        G.g16[k] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-  }
+// 8 bf16 (one 16-byte chunk) -> 4 float pairs, element 2i in .x of pair i.
+__device__ __forceinline__ void unpack_pairs(const uint4& u, float2 (&v)[4]) {
+  v[0] = make_float2(bf16_lo(u.x), bf16_hi(u.x));
+  v[1] = make_float2(bf16_lo(u.y), bf16_hi(u.y));
+  v[2] = make_float2(bf16_lo(u.z), bf16_hi(u.z));
+  v[3] = make_float2(bf16_lo(u.w), bf16_hi(u.w));
+}
+__device__ __forceinline__ uint4 pack_pairs_bf16(const float2 (&v)[4]) {
+  return make_uint4(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y), pack_bf16x2(v[2].x, v[2].y),
+                    pack_bf16x2(v[3].x, v[3].y));
+}
+__device__ __forceinline__ uint2 pack_pairs_e4m3(const float2 (&t)[4]) {
+  return make_uint2(pack_e4m3x4(t[0].x, t[0].y, t[1].x, t[1].y), pack_e4m3x4(t[2].x, t[2].y, t[3].x, t[3].y));
 }
 
-// Row chunks of a bf16 row straight from global memory (zeros past the row).
-template <int T, int K, bool VEC>
-__device__ __forceinline__ void load_row(const uint16_t* rowp, int d, int C, int tid, bool live,
-                                         float (&v)[K][8]) {
+// Chunk partial of the canonical order: even / odd accumulators from +0,
+// then RN(even + odd).
+template <bool SQUARES>
+__device__ __forceinline__ float chunk_partial(const float2 (&v)[4]) {
+  float2 acc = f2(0.0f);
 #pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
-    const bool ok = live && c < C;
-    if constexpr (VEC) {
-      uint4 u = make_uint4(0u, 0u, 0u, 0u);
-      if (ok) u = __ldcs(reinterpret_cast<const uint4*>(rowp + 8 * c));
-      unpack_bf16x8(u, v[k]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = 8 * c + j;
-        v[k][j] = (ok && e < d) ? bf16_to_f32(rowp[e]) : 0.0f;
-      }
-    }
-  }
+  for (int i = 0; i < 4; ++i) acc = SQUARES ? fma2(v[i], v[i], acc) : add2(acc, v[i]);
+  return __fadd_rn(acc.x, acc.y);
 }
 
-// Steps a2..a6 of one row whose x (v) and residual (rv, when has_res) chunks
-// are in registers.  Contains the row group's barriers (T > 32).
-template <int OP, int T, int K, bool VEC>
-__device__ __forceinline__ void row_finish(const RowArgs& a, int64_t row, bool live, int tid,
-                                           float (&v)[K][8], const float (&rv)[K][8], bool has_res,
-                                           const GammaRegs<K>& G, float* s_sum0, float* s_sum1,
-                                           uint32_t* s_max) {
-  const int d = a.d;
-  const int C = (d + 7) >> 3;
-  const bool div = (a.flags & kFlagDiv) != 0;
-
-  // ---- a2: residual add and residual write
-  if (has_res) {
-    uint16_t* orow = a.res_out + row * a.ld_res;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[k][j] = __fadd_rn(v[k][j], rv[k][j]);
-      if (live && c < C) {
-        if constexpr (VEC) {
-          *reinterpret_cast<uint4*>(orow + 8 * c) = pack_bf16x8(v[k]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (8 * c + j < d) orow[8 * c + j] = f32_to_bf16(v[k][j]);
-        }
-      }
-    }
-  }
-
-  // ---- a3: first row sum (sum of squares, or plain sum for LayerNorm)
-  float part[K];
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    float p = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if constexpr (OP == kOpLnStaticFp8) p = __fadd_rn(p, v[k][j]);
-      else p = __fmaf_rn(v[k][j], v[k][j], p);
-    }
-    part[k] = p;
-  }
+// Row sum of the K chunk partials held by each thread of the group (highest
+// chunk-index bit first: the thread's own chunks, then across threads).
+template <int T, int K>
+__device__ __forceinline__ float row_total(float (&part)[K], float* red, int tid) {
 #pragma unroll
   for (int h = K / 2; h >= 1; h >>= 1)
 #pragma unroll
     for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-  const float total = row_sum<T>(part[0], s_sum0, tid);
+  return row_sum<T>(part[0], red, tid);
+}
+
+template <int OP, int T, int K, bool VEC>
+__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
+  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
+  constexpr int W = T / 32;             // warps per row
+  static_assert(K == 1 || K == 2 || K == 4 || K == 8, "chunks per thread");
+  static_assert(R * T <= 1024, "CTA size");
+
+  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
+  __shared__ uint32_t s_max[W > 1 ? W : 1];
+
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5)
+                                : int64_t(blockIdx.x);
+  // Rows past M (only possible with eight rows per CTA) run every step with
+  // zeros so that warp-wide shuffles stay converged, and store nothing.
+  const bool live = row < a.M;
+  const int d = a.d;
+  const int C = (d + 7) >> 3;
+  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
+  const bool div = (a.flags & kFlagDiv) != 0;
+
+  griddep_wait();
+
+  // ---- a1: loads, all issued before any use
+  uint4 xr[K], rr[K];
+  {
+    const uint16_t* xrow = a.x + row * a.ld_x;
+    const uint16_t* rrow = a.res_in + row * a.ld_res;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      const bool ok = live && c < C;
+      if constexpr (VEC) {
+        xr[k] = ok ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+        rr[k] = (has_res && ok) ? __ldcs(reinterpret_cast<const uint4*>(rrow + 8 * c))
+                                : make_uint4(0u, 0u, 0u, 0u);
+      } else {
+        uint32_t w[4], z[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 8 * c + 2 * j;
+          w[j] = ((ok && e < d) ? uint32_t(xrow[e]) : 0u) | ((ok && e + 1 < d) ? uint32_t(xrow[e + 1]) << 16 : 0u);
+          z[j] = 0u;
+          if (has_res)
+            z[j] = ((ok && e < d) ? uint32_t(rrow[e]) : 0u) | ((ok && e + 1 < d) ? uint32_t(rrow[e + 1]) << 16 : 0u);
+        }
+        xr[k] = make_uint4(w[0], w[1], w[2], w[3]);
+        rr[k] = make_uint4(z[0], z[1], z[2], z[3]);
+      }
+    }
+  }
+  griddep_launch_dependents();  // the next kernel on the stream may start its prologue
+
+  // ---- a2: r = x + residual, residual_out; a3: chunk partials
+  float2 v[K][4];
+  float part[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    unpack_pairs(xr[k], v[k]);
+    if (has_res) {
+      float2 t[4];
+      unpack_pairs(rr[k], t);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = add2(v[k][i], t[i]);
+      if (live && c < C) {
+        uint16_t* orow = a.res_out + row * a.ld_res;
+        if constexpr (VEC) {
+          *reinterpret_cast<uint4*>(orow + 8 * c) = pack_pairs_bf16(v[k]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (8 * c + 2 * i < d) orow[8 * c + 2 * i] = f32_to_bf16(v[k][i].x);
+            if (8 * c + 2 * i + 1 < d) orow[8 * c + 2 * i + 1] = f32_to_bf16(v[k][i].y);
+          }
+        }
+      }
+    }
+    part[k] = chunk_partial<OP != kOpLnStaticFp8>(v[k]);
+  }
+  const float total = row_total<T, K>(part, s_sum[0], tid);
 
   const float fd = float(d);
   float rstd;
   if constexpr (OP == kOpLnStaticFp8) {
-    // Centre on the row mean, then the biased variance (second pass, in registers).
-    const float mean = __fdiv_rn(total, fd);
+    // Centre on the row mean (RN(r - mean) == RN(r + (-mean))), then the
+    // biased variance; padding elements stay exactly zero.
+    const float2 nm = f2(-__fdiv_rn(total, fd));
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
+      const bool ok = live && c < C;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const bool in = live && c < C && (VEC || 8 * c + j < d);
-        v[k][j] = in ? __fsub_rn(v[k][j], mean) : 0.0f;
+      for (int i = 0; i < 4; ++i) {
+        float2 t = add2(v[k][i], nm);
+        if constexpr (!VEC) {
+          if (8 * c + 2 * i >= d) t.x = 0.0f;
+          if (8 * c + 2 * i + 1 >= d) t.y = 0.0f;
+        }
+        v[k][i] = ok ? t : f2(0.0f);
       }
+      part[k] = chunk_partial<true>(v[k]);
     }
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      float p = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) p = __fmaf_rn(v[k][j], v[k][j], p);
-      part[k] = p;
-    }
-#pragma unroll
-    for (int h = K / 2; h >= 1; h >>= 1)
-#pragma unroll
-      for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-    const float sq = row_sum<T>(part[0], s_sum1, tid);
+    const float sq = row_total<T, K>(part, s_sum[1], tid);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
   } else {
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
   }
 
-  // ---- a4: normalize (y overwrites v)
+  // ---- a4: normalize (y overwrites v); gamma / beta fetched now, through L1
+  const float2 rs2 = f2(rstd);
   const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
 #pragma unroll
   for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const bool gok = c < C;
     if constexpr (OP == kOpLnStaticFp8) {
+      const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
+      const float* bp = a.beta + 8 * c;
+      float2 g[4], b[4];
+      if constexpr (VEC) {
+        float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, b0 = g0, b1 = g0;
+        if (gok) {
+          g0 = __ldg(reinterpret_cast<const float4*>(gp));
+          g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
+          b0 = __ldg(reinterpret_cast<const float4*>(bp));
+          b1 = __ldg(reinterpret_cast<const float4*>(bp + 4));
+        }
+        g[0] = make_float2(g0.x, g0.y); g[1] = make_float2(g0.z, g0.w);
+        g[2] = make_float2(g1.x, g1.y); g[3] = make_float2(g1.z, g1.w);
+        b[0] = make_float2(b0.x, b0.y); b[1] = make_float2(b0.z, b0.w);
+        b[2] = make_float2(b1.x, b1.y); b[3] = make_float2(b1.z, b1.w);
+      } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[k][j] = __fmaf_rn(__fmul_rn(v[k][j], rstd), G.gf[k][j], G.bf[k][j]);
+        for (int i = 0; i < 4; ++i) {
+          const int e = 8 * c + 2 * i;
+          g[i] = make_float2((gok && e < d) ? __ldg(gp + 2 * i) : 0.f, (gok && e + 1 < d) ? __ldg(gp + 2 * i + 1) : 0.f);
+          b[i] = make_float2((gok && e < d) ? __ldg(bp + 2 * i) : 0.f, (gok && e + 1 < d) ? __ldg(bp + 2 * i + 1) : 0.f);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = fma2(mul2(v[k][i], rs2), g[i], b[i]);
     } else {
-      float g[8];
-      unpack_bf16x8(G.g16[k], g);
+      const uint16_t* gp = static_cast<const uint16_t*>(a.gamma) + 8 * c;
+      uint4 gu = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (VEC) {
+        if (gok) gu = __ldg(reinterpret_cast<const uint4*>(gp));
+      } else {
+        uint32_t w[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[k][j] = __fmul_rn(__fmul_rn(v[k][j], rstd), g[j]);
+        for (int j = 0; j < 4; ++j) {
+          const int e = 8 * c + 2 * j;
+          w[j] = ((gok && e < d) ? uint32_t(__ldg(gp + 2 * j)) : 0u) |
+                 ((gok && e + 1 < d) ? uint32_t(__ldg(gp + 2 * j + 1)) << 16 : 0u);
+        }
+        gu = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      float2 g[4];
+      unpack_pairs(gu, g);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = mul2(mul2(v[k][i], rs2), g[i]);
     }
     if (bf16_round) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[k][j] = round_bf16(v[k][j]);
+      for (int i = 0; i < 4; ++i) v[k][i] = make_float2(round_bf16(v[k][i].x), round_bf16(v[k][i].y));
     }
   }
   if constexpr (OP != kOpLnStaticFp8) {
@@ -221,11 +248,13 @@ __device__ __forceinline__ void row_finish(const RowArgs& a, int64_t row, bool l
         const int c = tid + k * T;
         if (live && c < C) {
           if constexpr (VEC) {
-            *reinterpret_cast<uint4*>(nrow + 8 * c) = pack_bf16x8(v[k]);
+            *reinterpret_cast<uint4*>(nrow + 8 * c) = pack_pairs_bf16(v[k]);
           } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (8 * c + j < d) nrow[8 * c + j] = f32_to_bf16(v[k][j]);
+            for (int i = 0; i < 4; ++i) {
+              if (8 * c + 2 * i < d) nrow[8 * c + 2 * i] = f32_to_bf16(v[k][i].x);
+              if (8 * c + 2 * i + 1 < d) nrow[8 * c + 2 * i + 1] = f32_to_bf16(v[k][i].y);
+            }
           }
         }
       }
@@ -243,15 +272,27 @@ __device__ __forceinline__ void row_finish(const RowArgs& a, int64_t row, bool l
       const bool ok = live && c < C;
       float m8 = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) m8 = fmaxf(m8, fabsf(v[k][j]));
+      for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
       // A 16-element block is chunks (c, c^1), held by lanes (t, t^1).
       const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
       const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), g));
       const float S = __fmul_rn(e4m3_to_f32(sfc), g);
       const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
       float t[8];
+      if (div && S != 0.0f) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) t[j] = (div && S != 0.0f) ? __fdiv_rn(v[k][j], S) : __fmul_rn(v[k][j], mult);
+        for (int i = 0; i < 4; ++i) {
+          t[2 * i] = __fdiv_rn(v[k][i].x, S);
+          t[2 * i + 1] = __fdiv_rn(v[k][i].y, S);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 q = mul2(v[k][i], f2(mult));
+          t[2 * i] = q.x;
+          t[2 * i + 1] = q.y;
+        }
+      }
       const uint32_t packed = pack_e2m1x8(t);
       if (ok) {
         if constexpr (VEC) {
@@ -264,14 +305,14 @@ __device__ __forceinline__ void row_finish(const RowArgs& a, int64_t row, bool l
       }
     }
   } else {
-    float s_div = 1.0f, s_inv = 1.0f;
+    float s_div, s_inv;
     bool passthrough = false;
     if constexpr (OP == kOpRmsDynFp8) {
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < K; ++k)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[k][j]));
+        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
       const float amax = row_max_nonneg<T>(m, s_max, tid);
       const float s = __fdiv_rn(amax, kE4M3Max);
       if (live && tid == 0) a.scale_out[row] = s;
@@ -279,316 +320,40 @@ __device__ __forceinline__ void row_finish(const RowArgs& a, int64_t row, bool l
       s_inv = __frcp_rn(s);
       passthrough = (s == 0.0f);  // zero row: store the signed zeros of y
     } else {
-      const float sc = __ldg(a.scale);
-      s_div = sc;
-      s_inv = __frcp_rn(sc);
+      s_div = __ldg(a.scale);
+      s_inv = __frcp_rn(s_div);
     }
     uint8_t* qrow = a.q + row * a.ld_q;
+    const float2 inv2 = f2(s_inv);
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
-      float t[8];
+      float2 t[4];
+      if (passthrough) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        t[j] = passthrough ? v[k][j] : (div ? __fdiv_rn(v[k][j], s_div) : __fmul_rn(v[k][j], s_inv));
-      const uint32_t lo = pack_e4m3x4(t[0], t[1], t[2], t[3]);
-      const uint32_t hi = pack_e4m3x4(t[4], t[5], t[6], t[7]);
+        for (int i = 0; i < 4; ++i) t[i] = v[k][i];
+      } else if (div) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = make_float2(__fdiv_rn(v[k][i].x, s_div), __fdiv_rn(v[k][i].y, s_div));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = mul2(v[k][i], inv2);
+      }
+      const uint2 codes = pack_pairs_e4m3(t);
       if (live && c < C) {
         if constexpr (VEC) {
-          *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(lo, hi);
+          *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            if (8 * c + j < d) qrow[8 * c + j] = uint8_t((j < 4 ? lo : hi) >> (8 * (j & 3)));
+            if (8 * c + j < d) qrow[8 * c + j] = uint8_t((j < 4 ? codes.x : codes.y) >> (8 * (j & 3)));
         }
       }
     }
   }
 }
 
-// ------------------------------------------------------------- direct ----
-template <int OP, int T, int K, bool VEC>
-__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
-  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
-  constexpr int W = T / 32;             // warps per row
-  static_assert(K == 1 || K == 2 || K == 4, "chunks per thread");
-  static_assert(R * T <= 1024, "CTA size");
-
-  __shared__ float s_sum[2][W > 1 ? W * 32 : 1];
-  __shared__ uint32_t s_max[W > 1 ? W : 1];
-
-  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
-  const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5)
-                                : int64_t(blockIdx.x);
-  // Rows past M (only possible with eight rows per CTA) run every step with
-  // zeros so that warp-wide shuffles stay converged, and store nothing.
-  const bool live = row < a.M;
-  const int C = (a.d + 7) >> 3;
-  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
-
-  griddep_wait();
-
-  // All loads are issued before any store, for memory-level parallelism.
-  float v[K][8], rv[K][8];
-  load_row<T, K, VEC>(a.x + row * a.ld_x, a.d, C, tid, live, v);
-  GammaRegs<K> G;
-  load_gamma<OP, T, K, VEC>(a, tid, C, G);
-  if (has_res) load_row<T, K, VEC>(a.res_in + row * a.ld_res, a.d, C, tid, live, rv);
-  // The next kernel on the stream may start its prologue now.
-  griddep_launch_dependents();
-  row_finish<OP, T, K, VEC>(a, row, live, tid, v, rv, has_res, G, s_sum[0], s_sum[1], s_max);
-}
-
-// ------------------------------------------------------------- staged ----
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
-               "l"(gmem), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-// Wait until at most n of this thread's committed groups are pending (n in 0..7).
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-  switch (n) {
-    case 0: asm volatile("cp.async.wait_group 0;\n" ::: "memory"); break;
-    case 1: asm volatile("cp.async.wait_group 1;\n" ::: "memory"); break;
-    case 2: asm volatile("cp.async.wait_group 2;\n" ::: "memory"); break;
-    case 3: asm volatile("cp.async.wait_group 3;\n" ::: "memory"); break;
-    case 4: asm volatile("cp.async.wait_group 4;\n" ::: "memory"); break;
-    case 5: asm volatile("cp.async.wait_group 5;\n" ::: "memory"); break;
-    case 6: asm volatile("cp.async.wait_group 6;\n" ::: "memory"); break;
-    default: asm volatile("cp.async.wait_group 7;\n" ::: "memory"); break;
-  }
-}
-
-// Persistent, 16-byte-aligned rows only.  Thread group g (of G = gridDim.x * R
-// groups) handles rows g, g + G, g + 2G, ...  Dynamic shared memory holds
-// `stages` ring slots of NT (1 or 2: x, residual) x K chunks per thread.  The
-// row being processed stays in its slot and is streamed through registers one
-// chunk at a time, once per pass (sum; LayerNorm variance; absmax; quantize):
-// r = x + residual is recomputed from the slot in each pass (same bits), so
-// the register count does not grow with the row width and many rows can be
-// in flight per SM.  gamma / beta are re-read per chunk through L1.
-template <int OP, int T, int K>
-__global__ void __launch_bounds__(T == 32 ? 256 : T, 1024 / (T == 32 ? 256 : T))
-    row_kernel_staged(const RowArgs a, int stages) {  // <= 64 registers: >= 1024 threads per SM
-  constexpr int R = (T == 32) ? 8 : 1;
-  constexpr int W = T / 32;
-  constexpr int NTHR = R * T;
-  __shared__ float s_sum[2][W > 1 ? W * 32 : 1];
-  __shared__ uint32_t s_max[W > 1 ? W : 1];
-  extern __shared__ uint4 ring[];
-
-  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
-  const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
-  const int64_t n_groups = int64_t(gridDim.x) * R;
-  const int64_t nrows = group < a.M ? (a.M - group + n_groups - 1) / n_groups : 0;
-  const int d = a.d;
-  const int C = d >> 3;  // 16-byte rows: d % 8 == 0
-  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
-  const int NT = has_res ? 2 : 1;
-  const bool div = (a.flags & kFlagDiv) != 0;
-  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
-  const float fd = float(d);
-
-  griddep_wait();
-
-  auto issue = [&](int64_t j) {  // prefetch row j of this group into slot j % stages
-    if (j < nrows) {
-      const int64_t row = group + j * n_groups;
-      uint4* base = ring + size_t(j % stages) * NT * K * NTHR + threadIdx.x;
-      const uint16_t* xr = a.x + row * a.ld_x;
-      const uint16_t* rr = a.res_in + row * a.ld_res;
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int c = tid + k * T;
-        const bool ok = c < C;
-        cp_async16(base + k * NTHR, ok ? xr + 8 * c : a.x, ok ? 16u : 0u);
-        if (has_res) cp_async16(base + (K + k) * NTHR, ok ? rr + 8 * c : a.res_in, ok ? 16u : 0u);
-      }
-    }
-    cp_async_commit();  // one group per row index, empty past the end, so the counting stays uniform
-  };
-  for (int j = 0; j < stages - 1; ++j) issue(j);
-
-  const int64_t trigger = nrows > stages - 1 ? nrows - (stages - 1) : 0;
-  if (nrows == 0) griddep_launch_dependents();
-  const float scale_static = (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8 || OP == kOpRmsNvfp4)
-                                 ? __ldg(a.scale) : 1.0f;
-
-  for (int64_t j = 0; j < nrows; ++j) {
-    issue(j + stages - 1);  // refills the slot consumed in iteration j - 1
-    cp_async_wait_pending(stages - 1);
-    if (j == trigger) griddep_launch_dependents();  // every remaining row is in flight
-    const int64_t row = group + j * n_groups;
-    const uint4* xs = ring + size_t(j % stages) * NT * K * NTHR + threadIdx.x;
-    const uint4* rs = xs + K * NTHR;
-    // r (8 values of chunk k): x, plus the residual when there is one.
-    auto load_r = [&](int k, float (&r)[8]) {
-      unpack_bf16x8(xs[k * NTHR], r);
-      if (has_res) {
-        float t[8];
-        unpack_bf16x8(rs[k * NTHR], t);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) r[e] = __fadd_rn(r[e], t[e]);
-      }
-    };
-    // Reduction buffers are reused row after row.  LayerNorm's two sums use
-    // both buffers, each separated from its next use by the other sum's
-    // barrier; single-sum operations alternate by row parity.
-    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
-
-    // ---- pass A: residual write and first row sum
-    float part[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      float r[8];
-      load_r(k, r);
-      if (has_res && c < C) *reinterpret_cast<uint4*>(a.res_out + row * a.ld_res + 8 * c) = pack_bf16x8(r);
-      float p = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if constexpr (OP == kOpLnStaticFp8) p = __fadd_rn(p, r[e]);
-        else p = __fmaf_rn(r[e], r[e], p);
-      }
-      part[k] = p;
-    }
-#pragma unroll
-    for (int h = K / 2; h >= 1; h >>= 1)
-#pragma unroll
-      for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-    const float total = row_sum<T>(part[0], b0, tid);
-
-    float rstd, mean = 0.0f;
-    if constexpr (OP == kOpLnStaticFp8) {
-      mean = __fdiv_rn(total, fd);
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int c = tid + k * T;
-        float r[8];
-        load_r(k, r);
-        float p = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float ce = (c < C) ? __fsub_rn(r[e], mean) : 0.0f;
-          p = __fmaf_rn(ce, ce, p);
-        }
-        part[k] = p;
-      }
-#pragma unroll
-      for (int h = K / 2; h >= 1; h >>= 1)
-#pragma unroll
-        for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-      const float sq = row_sum<T>(part[0], s_sum[1], tid);
-      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
-    } else {
-      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
-    }
-
-    // y (8 values of chunk k) from the slot.
-    auto make_y = [&](int k, float (&y)[8]) {
-      const int c = tid + k * T;
-      float r[8];
-      load_r(k, r);
-      if constexpr (OP == kOpLnStaticFp8) {
-        float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
-        if (c < C) {
-          const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
-          g0 = __ldg(reinterpret_cast<const float4*>(gp));
-          g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
-          e0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
-          e1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
-        }
-        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        const float bb[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float ce = (c < C) ? __fsub_rn(r[e], mean) : 0.0f;
-          y[e] = __fmaf_rn(__fmul_rn(ce, rstd), gg[e], bb[e]);
-        }
-      } else {
-        uint4 gu = make_uint4(0u, 0u, 0u, 0u);
-        if (c < C) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
-        float g[8];
-        unpack_bf16x8(gu, g);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(__fmul_rn(r[e], rstd), g[e]);
-      }
-      if (bf16_round) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = round_bf16(y[e]);
-      }
-    };
-    auto store_e4m3 = [&](int k, const float (&t)[8]) {
-      const int c = tid + k * T;
-      const uint32_t lo = pack_e4m3x4(t[0], t[1], t[2], t[3]);
-      const uint32_t hi = pack_e4m3x4(t[4], t[5], t[6], t[7]);
-      if (c < C) *reinterpret_cast<uint2*>(a.q + row * a.ld_q + 8 * c) = make_uint2(lo, hi);
-    };
-
-    // ---- pass B: normalize; static scales and NVFP4 quantize here
-    float m = 0.0f;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      float y[8];
-      make_y(k, y);
-      if constexpr (OP != kOpLnStaticFp8) {
-        if (a.norm_out != nullptr && c < C)
-          *reinterpret_cast<uint4*>(a.norm_out + row * a.ld_norm + 8 * c) = pack_bf16x8(y);
-      }
-      if constexpr (OP == kOpRmsDynFp8) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(y[e]));
-      } else if constexpr (OP == kOpRmsNvfp4) {
-        float m8 = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m8 = fmaxf(m8, fabsf(y[e]));
-        const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));  // chunks c, c^1 form a block
-        const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), scale_static));
-        const float S = __fmul_rn(e4m3_to_f32(sfc), scale_static);
-        const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
-        float t[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = (div && S != 0.0f) ? __fdiv_rn(y[e], S) : __fmul_rn(y[e], mult);
-        const uint32_t packed = pack_e2m1x8(t);
-        if (c < C) {
-          *reinterpret_cast<uint32_t*>(a.q + row * a.ld_q + 4 * c) = packed;
-          if ((c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
-        }
-      } else {
-        const float inv = __frcp_rn(scale_static);
-        float t[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = div ? __fdiv_rn(y[e], scale_static) : __fmul_rn(y[e], inv);
-        store_e4m3(k, t);
-      }
-    }
-
-    // ---- pass C (dynamic per-token scale): quantize with the row's scale
-    if constexpr (OP == kOpRmsDynFp8) {
-      const float amax = row_max_nonneg<T>(m, s_max, tid);
-      const float sc = __fdiv_rn(amax, kE4M3Max);
-      if (tid == 0) a.scale_out[row] = sc;
-      const float inv = __frcp_rn(sc);
-      const bool passthrough = (sc == 0.0f);  // zero row: store the signed zeros of y
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        float y[8], t[8];
-        make_y(k, y);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          t[e] = passthrough ? y[e] : (div ? __fdiv_rn(y[e], sc) : __fmul_rn(y[e], inv));
-        store_e4m3(k, t);
-      }
-    }
-  }
-  cp_async_wait_pending(0);
-}
-
-// Kernel tables of one operation: every built (threads, chunks, vec) schedule
-// of the direct kernel, and every (threads, chunks) of the staged kernel.
+// Kernel table of one operation: every built (threads, chunks, vec) schedule.
 template <int OP>
 struct RowTable {
   RowKernels k;
@@ -596,26 +361,16 @@ struct RowTable {
     for (auto& x : k.direct)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
-    for (auto& x : k.staged)
-      for (auto& y : x) y = nullptr;
 #define NQ_DIRECT(LT, LK)                                                                                     \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
   k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);
-#define NQ_STAGED(LT, LK) \
-  k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK)>);
-    NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2)
-    NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2)
-    NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2)
-    NQ_DIRECT(8, 0) NQ_DIRECT(8, 1) NQ_DIRECT(8, 2)
+    NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
+    NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)
+    NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2) NQ_DIRECT(7, 3)
+    NQ_DIRECT(8, 0) NQ_DIRECT(8, 1) NQ_DIRECT(8, 2) NQ_DIRECT(8, 3)
     NQ_DIRECT(9, 0) NQ_DIRECT(9, 1) NQ_DIRECT(9, 2)
     NQ_DIRECT(10, 0) NQ_DIRECT(10, 1)
-    NQ_STAGED(5, 0) NQ_STAGED(5, 1) NQ_STAGED(5, 2) NQ_STAGED(5, 3) NQ_STAGED(5, 4)
-    NQ_STAGED(6, 0) NQ_STAGED(6, 1) NQ_STAGED(6, 2) NQ_STAGED(6, 3) NQ_STAGED(6, 4)
-    NQ_STAGED(7, 0) NQ_STAGED(7, 1) NQ_STAGED(7, 2) NQ_STAGED(7, 3) NQ_STAGED(7, 4)
-    NQ_STAGED(8, 0) NQ_STAGED(8, 1) NQ_STAGED(8, 2) NQ_STAGED(8, 3)
-    NQ_STAGED(9, 0) NQ_STAGED(9, 1) NQ_STAGED(9, 2)
 #undef NQ_DIRECT
-#undef NQ_STAGED
   }
 };
 

@@ -97,20 +97,11 @@ typedef enum nq_status {
 /* Round y to bf16 before quantizing: reproduces the two-kernel (norm -> bf16
  * -> quant) numerics for A/B comparisons.  Not for production use. */
 #define NQ_FLAG_NORM_BF16_ROUND (1u << 4)
-/* Force a schedule: 2^t threads per row and 2^k 16-byte chunks per thread,
- * with 2^(t+k) * 8 >= d.  The direct kernel is built for t = 5..10, k = 0..2
- * (not t = 10 with k = 2); the staged kernel for t = 5..9, k = 0..4 with
- * t + k <= 11.  Every schedule gives bitwise identical results; this exists
- * for tests and tuning.  0 = automatic. */
+/* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
+ * thread (k = 0..3, t + k <= 11), with 2^(t+k) * 8 >= d.  Every schedule gives
+ * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
-/* Force the row pipeline: n = 1 runs the direct kernel (one row per thread
- * group, loads straight to registers); n = 2..8 runs the persistent staged
- * kernel with an n-slot cp.async ring (16-byte-aligned rows only; otherwise
- * the direct kernel runs).  Same bits either way.  0 = automatic. */
-#define NQ_FLAG_PIPELINE(n) ((((uint32_t)(n)) & 0xFu) << 24)
-#define NQ_FLAG_PIPELINE_MASK (0xFu << 24)
-
 /* Library version (major * 10000 + minor * 100 + patch). */
 int nq_version(void);
 /* Static text of a status code. */
@@ -126,16 +117,6 @@ const char* nq_last_error(void);
  */
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
                             int* chunks_per_thread, int* rows_per_cta);
-
-/*
- * Launch the library would make for a norm call (same op codes as
- * nq_query_schedule) over M rows of d elements, with or without a residual,
- * with 16-byte-aligned rows or not.  info[0..6] = threads per row, chunks per
- * thread, rows per CTA, staged (0/1), ring slots, grid size, dynamic shared
- * bytes.  Needs a current CUDA device (occupancy queries); launches nothing.
- */
-nq_status nq_query_launch(int op, int64_t M, int64_t d, uint32_t flags, int has_residual, int aligned16,
-                          int64_t* info);
 
 /*
  * Fused residual-add + RMSNorm + dynamic per-token e4m3.

@@ -37,8 +37,9 @@
 //    and reciprocal; eps inside the square root; mean divides by d;
 //  * y = RN(RN(r * rstd) * gamma) for RMSNorm and
 //    y = fma(RN((r - mean) * rstd), gamma, beta) for LayerNorm;
-//  * canonical sum order (see canonical_sum) so that a parallel reduction can
-//    reproduce it exactly; OR_SUM_PLAIN switches to float64 sequential sums;
+//  * canonical sum order (see canonical_sum) so that a parallel reduction with
+//    packed two-lane arithmetic can reproduce it exactly; OR_SUM_PLAIN
+//    switches to float64 sequential sums;
 //  * e4m3 / e2m1 encoders round to nearest, ties to even, and saturate to the
 //    largest finite magnitude (448 / 6);
 //  * NVFP4 global scale g is a dequantization multiplier (x ~ q * sf * g),
@@ -146,23 +147,27 @@ float ue8m0_ceil(float s) {
 
 // ---- canonical sum of a row ----
 // The pages fix no summation order.  The oracle fixes one that a parallel
-// reduction can reproduce bit for bit: elements are cut into chunks of 8
-// consecutive values; chunk partial p_c starts at +0 and accumulates the
-// chunk's values in index order (p = RN(p + v) for a sum, p = fma(v, v, p) for
-// a sum of squares); chunk count is padded with +0 partials to a power of two
-// P; then for half = P/2, P/4, ..., 1: p[c] = RN(p[c] + p[c + half]) for every
-// c < half.  Starting partials at +0 keeps every partial away from -0, so
-// extra +0 padding levels never change the result.
+// reduction with packed two-lane float arithmetic can reproduce bit for bit:
+// elements are cut into chunks of 8 consecutive values (the last one padded
+// with +0); inside a chunk two accumulators, one for the even positions
+// (0, 2, 4, 6) and one for the odd positions (1, 3, 5, 7), start at +0 and take
+// their four values in order (acc = RN(acc + v) for a sum, acc = fma(v, v, acc)
+// for a sum of squares); the chunk partial is RN(even + odd).  Chunk count is
+// padded with +0 partials to a power of two P; then for half = P/2, P/4, ...,
+// 1: p[c] = RN(p[c] + p[c + half]) for every c < half.  No partial is ever -0
+// (they start at +0), so extra +0 padding never changes the result.
 float canonical_sum(const float* v, int64_t n, bool squares) {
   const int64_t C = (n + 7) / 8;
   int64_t P = 1;
   while (P < C) P *= 2;
   std::vector<float> p(size_t(P), 0.0f);
   for (int64_t c = 0; c < C; ++c) {
-    float acc = 0.0f;
-    for (int64_t i = 8 * c; i < 8 * c + 8 && i < n; ++i)
-      acc = squares ? std::fma(v[i], v[i], acc) : acc + v[i];
-    p[size_t(c)] = acc;
+    float acc[2] = {0.0f, 0.0f};
+    for (int64_t i = 8 * c; i < 8 * c + 8 && i < n; ++i) {
+      float& a = acc[(i - 8 * c) & 1];
+      a = squares ? std::fma(v[i], v[i], a) : a + v[i];
+    }
+    p[size_t(c)] = acc[0] + acc[1];
   }
   for (int64_t half = P / 2; half >= 1; half /= 2)
     for (int64_t c = 0; c < half; ++c) p[size_t(c)] = p[size_t(c)] + p[size_t(c + half)];

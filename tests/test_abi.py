@@ -121,4 +121,5 @@ def test_planner_forced_schedules(nq):
     with pytest.raises(nq.NQError):
         nq.nq_query_schedule(0, 100, 4096, nq.flag_schedule(5, 2))   # 32 * 4 * 8 < 4096
     with pytest.raises(nq.NQError):
-        nq.nq_query_schedule(0, 100, 64, nq.flag_schedule(10, 2))    # not built
+        nq.nq_query_schedule(0, 100, 64, nq.flag_schedule(10, 2))    # not built (t + k > 11)
+    assert nq.nq_query_schedule(0, 100, 8192, nq.flag_schedule(7, 3)) == (128, 8, 1)
