@@ -5,8 +5,9 @@ contract of every call).  This module only marshals arguments: it checks
 tensor dtypes / devices / layouts, allocates outputs with torch when the
 caller does not pass them, and forwards raw device pointers, strides and the
 current CUDA stream.  Every arithmetic step runs in the library's CUDA
-kernels; there is no CPU or PyTorch fallback, and importing fails loudly when
-the library has not been built (``python -m fp4_activation_quantization_b200.build``).
+kernels; there is no CPU or PyTorch fallback.  The library is loaded on first
+use, and that use raises ImportError when it has not been built
+(``python -m fp4_activation_quantization_b200.build``).
 
 Functions carry the C names:
 ``nq_fused_add_rmsnorm_quant_fp8``, ``nq_rmsnorm_quant_fp8_static``,
@@ -23,7 +24,7 @@ import torch
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
     "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND",
-    "flag_schedule", "NQError", "lib", "library_path", "version",
+    "FLAG_PERSISTENT", "FLAG_ONE_ROW", "flag_schedule", "nq_query_launch", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4",
@@ -36,6 +37,8 @@ FLAG_SCALE_DIV = 1 << 1
 FLAG_SCALE_RECIP = 1 << 2
 FLAG_UE8M0 = 1 << 3
 FLAG_NORM_BF16_ROUND = 1 << 4
+FLAG_PERSISTENT = 1 << 24
+FLAG_ONE_ROW = 1 << 25
 OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4 = 0, 1, 2, 3
 
 
@@ -66,6 +69,8 @@ def _load() -> ctypes.CDLL:
     L.nq_query_schedule.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     L.nq_query_schedule.restype = st
+    L.nq_query_launch.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
+    L.nq_query_launch.restype = st
     L.nq_fused_add_rmsnorm_quant_fp8.argtypes = [P, I64, P, P, I64, P, P, I64, P, P, I64, I64, I64, F, U32, P]
     L.nq_rmsnorm_quant_fp8_static.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, I64, I64, F, U32, P]
     L.nq_layernorm_quant_fp8.argtypes = [P, I64, P, P, P, P, I64, I64, I64, F, U32, P]
@@ -77,18 +82,32 @@ def _load() -> ctypes.CDLL:
     return L
 
 
-lib = _load()
+_lib = None
+
+
+def _get_lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def __getattr__(name):  # module attribute `lib`, loaded on first access
+    if name == "lib":
+        return _get_lib()
+    raise AttributeError(name)
 
 
 def version() -> int:
-    return lib.nq_version()
+    return _get_lib().nq_version()
 
 
 class NQError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        msg = lib.nq_last_error().decode()
-        super().__init__(f"{where}: {lib.nq_status_string(status).decode()}: {msg}")
+        L = _get_lib()
+        msg = L.nq_last_error().decode()
+        super().__init__(f"{where}: {L.nq_status_string(status).decode()}: {msg}")
 
 
 def _check(status: int, where: str) -> None:
@@ -154,9 +173,17 @@ def _out(t, shape, dtype, like: torch.Tensor, name: str):
 def nq_query_schedule(op: int, M: int, d: int, flags: int = 0):
     """(threads per row, 16-byte chunks per thread, rows per CTA) the planner picks."""
     t, k, r = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(lib.nq_query_schedule(op, M, d, flags, ctypes.byref(t), ctypes.byref(k), ctypes.byref(r)),
+    _check(_get_lib().nq_query_schedule(op, M, d, flags, ctypes.byref(t), ctypes.byref(k), ctypes.byref(r)),
            "nq_query_schedule")
     return t.value, k.value, r.value
+
+
+def nq_query_launch(op: int, M: int, d: int, flags: int = 0, aligned16: bool = True) -> dict:
+    """The launch a norm call would make (needs a CUDA device)."""
+    info = (ctypes.c_int64 * 5)()
+    _check(_get_lib().nq_query_launch(op, M, d, flags, int(aligned16), info), "nq_query_launch")
+    keys = ("threads_per_row", "chunks_per_thread", "rows_per_cta", "persistent", "grid")
+    return dict(zip(keys, [int(v) for v in info]))
 
 
 def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, residual_out=None,
@@ -185,7 +212,7 @@ def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, res
     ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
     _same_device(x, residual, gamma, residual_out, q_out, scale_out, norm_out)
     with torch.cuda.device(x.device):
-        _check(lib.nq_fused_add_rmsnorm_quant_fp8(
+        _check(_get_lib().nq_fused_add_rmsnorm_quant_fp8(
             _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(q_out), ld_q,
             _ptr(scale_out), _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)),
             "nq_fused_add_rmsnorm_quant_fp8")
@@ -218,7 +245,7 @@ def nq_rmsnorm_quant_fp8_static(x, gamma, scale, eps: float = 1e-6, *, residual=
     ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
     _same_device(x, gamma, scale, residual, residual_out, q_out, norm_out)
     with torch.cuda.device(x.device):
-        _check(lib.nq_rmsnorm_quant_fp8_static(
+        _check(_get_lib().nq_rmsnorm_quant_fp8_static(
             _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(scale), _ptr(q_out),
             ld_q, _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)), "nq_rmsnorm_quant_fp8_static")
     return q_out, residual_out, norm_out
@@ -235,7 +262,7 @@ def nq_layernorm_quant_fp8(x, gamma, beta, scale, eps: float = 1e-5, *, q_out=No
     _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
     _same_device(x, gamma, beta, scale, q_out)
     with torch.cuda.device(x.device):
-        _check(lib.nq_layernorm_quant_fp8(_ptr(x), ld_x, _ptr(gamma), _ptr(beta), _ptr(scale), _ptr(q_out),
+        _check(_get_lib().nq_layernorm_quant_fp8(_ptr(x), ld_x, _ptr(gamma), _ptr(beta), _ptr(scale), _ptr(q_out),
                                           ld_q, M, d, eps, flags, _stream(stream)), "nq_layernorm_quant_fp8")
     return q_out
 
@@ -251,7 +278,7 @@ def nq_per_token_group_quant_fp8(x, group: int = 128, *, q_out=None, scales_out=
     _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, K // group)
     _same_device(x, q_out, scales_out)
     with torch.cuda.device(x.device):
-        _check(lib.nq_per_token_group_quant_fp8(_ptr(x), ld_x, _ptr(q_out), ld_q, _ptr(scales_out), ld_s, M, K,
+        _check(_get_lib().nq_per_token_group_quant_fp8(_ptr(x), ld_x, _ptr(q_out), ld_q, _ptr(scales_out), ld_s, M, K,
                                                 group, flags, _stream(stream)), "nq_per_token_group_quant_fp8")
     return q_out, scales_out
 
@@ -286,7 +313,7 @@ def nq_rmsnorm_quant_nvfp4(x, gamma, global_scale, eps: float = 1e-6, *, residua
     ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
     _same_device(x, gamma, global_scale, residual, residual_out, q_out, sf_out, norm_out)
     with torch.cuda.device(x.device):
-        _check(lib.nq_rmsnorm_quant_nvfp4(
+        _check(_get_lib().nq_rmsnorm_quant_nvfp4(
             _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(global_scale), _ptr(q_out),
             ld_q, _ptr(sf_out), ld_sf, _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)),
             "nq_rmsnorm_quant_nvfp4")

@@ -73,59 +73,47 @@ __device__ __forceinline__ float row_total(float (&part)[K], float* red, int tid
   return row_sum<T>(part[0], red, tid);
 }
 
-template <int OP, int T, int K, bool VEC>
-__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
-  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
-  constexpr int W = T / 32;             // warps per row
-  static_assert(K == 1 || K == 2 || K == 4 || K == 8, "chunks per thread");
-  static_assert(R * T <= 1024, "CTA size");
-
-  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
-  __shared__ uint32_t s_max[W > 1 ? W : 1];
-
-  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
-  const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5)
-                                : int64_t(blockIdx.x);
-  // Rows past M (only possible with eight rows per CTA) run every step with
-  // zeros so that warp-wide shuffles stay converged, and store nothing.
-  const bool live = row < a.M;
+// a1: raw bf16 chunks of one row (zeros past the row or for dead rows).
+template <int T, int K, bool VEC>
+__device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
+                                         uint4 (&xr)[K], uint4 (&rr)[K]) {
   const int d = a.d;
   const int C = (d + 7) >> 3;
-  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
-  const bool div = (a.flags & kFlagDiv) != 0;
-
-  griddep_wait();
-
-  // ---- a1: loads, all issued before any use
-  uint4 xr[K], rr[K];
-  {
-    const uint16_t* xrow = a.x + row * a.ld_x;
-    const uint16_t* rrow = a.res_in + row * a.ld_res;
+  const uint16_t* xrow = a.x + row * a.ld_x;
+  const uint16_t* rrow = a.res_in + row * a.ld_res;
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      const bool ok = live && c < C;
-      if constexpr (VEC) {
-        xr[k] = ok ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
-        rr[k] = (has_res && ok) ? __ldcs(reinterpret_cast<const uint4*>(rrow + 8 * c))
-                                : make_uint4(0u, 0u, 0u, 0u);
-      } else {
-        uint32_t w[4], z[4];
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const bool ok = live && c < C;
+    if constexpr (VEC) {
+      xr[k] = ok ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+      rr[k] = (has_res && ok) ? __ldcs(reinterpret_cast<const uint4*>(rrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      uint32_t w[4], z[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = 8 * c + 2 * j;
-          w[j] = ((ok && e < d) ? uint32_t(xrow[e]) : 0u) | ((ok && e + 1 < d) ? uint32_t(xrow[e + 1]) << 16 : 0u);
-          z[j] = 0u;
-          if (has_res)
-            z[j] = ((ok && e < d) ? uint32_t(rrow[e]) : 0u) | ((ok && e + 1 < d) ? uint32_t(rrow[e + 1]) << 16 : 0u);
-        }
-        xr[k] = make_uint4(w[0], w[1], w[2], w[3]);
-        rr[k] = make_uint4(z[0], z[1], z[2], z[3]);
+      for (int j = 0; j < 4; ++j) {
+        const int e = 8 * c + 2 * j;
+        w[j] = ((ok && e < d) ? uint32_t(xrow[e]) : 0u) | ((ok && e + 1 < d) ? uint32_t(xrow[e + 1]) << 16 : 0u);
+        z[j] = 0u;
+        if (has_res)
+          z[j] = ((ok && e < d) ? uint32_t(rrow[e]) : 0u) | ((ok && e + 1 < d) ? uint32_t(rrow[e + 1]) << 16 : 0u);
       }
+      xr[k] = make_uint4(w[0], w[1], w[2], w[3]);
+      rr[k] = make_uint4(z[0], z[1], z[2], z[3]);
     }
   }
-  griddep_launch_dependents();  // the next kernel on the stream may start its prologue
+}
 
+// a2..a6 of one row whose raw chunks are in registers.  Contains the row
+// group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
+// reduction buffers.
+template <int OP, int T, int K, bool VEC>
+__device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
+                                            const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
+                                            float* s_sum1, uint32_t* s_max) {
+  const int d = a.d;
+  const int C = (d + 7) >> 3;
+  const bool div = (a.flags & kFlagDiv) != 0;
   // ---- a2: r = x + residual, residual_out; a3: chunk partials
   float2 v[K][4];
   float part[K];
@@ -153,7 +141,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
     }
     part[k] = chunk_partial<OP != kOpLnStaticFp8>(v[k]);
   }
-  const float total = row_total<T, K>(part, s_sum[0], tid);
+  const float total = row_total<T, K>(part, s_sum0, tid);
 
   const float fd = float(d);
   float rstd;
@@ -176,7 +164,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
       }
       part[k] = chunk_partial<true>(v[k]);
     }
-    const float sq = row_total<T, K>(part, s_sum[1], tid);
+    const float sq = row_total<T, K>(part, s_sum1, tid);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
   } else {
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
@@ -353,7 +341,71 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   }
 }
 
-// Kernel table of one operation: every built (threads, chunks, vec) schedule.
+// One row per thread group: loads straight to registers.  The choice for few
+// rows (latency) and for unaligned rows.
+template <int OP, int T, int K, bool VEC>
+__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
+  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
+  constexpr int W = T / 32;             // warps per row
+  static_assert(K == 1 || K == 2 || K == 4 || K == 8, "chunks per thread");
+  static_assert(R * T <= 1024, "CTA size");
+  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
+  __shared__ uint32_t s_max[W > 1 ? W : 1];
+
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5) : int64_t(blockIdx.x);
+  // Rows past M (only possible with eight rows per CTA) run every step with
+  // zeros so that warp-wide shuffles stay converged, and store nothing.
+  const bool live = row < a.M;
+  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
+
+  griddep_wait();
+  uint4 xr[K], rr[K];
+  load_raw<T, K, VEC>(a, row, live, has_res, tid, xr, rr);
+  griddep_launch_dependents();  // the next kernel on the stream may start its prologue
+  process_row<OP, T, K, VEC>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+}
+
+// Persistent thread groups (16-byte rows only): group g of G = gridDim.x * R
+// walks rows g, g + G, g + 2G, ... and loads row j + 1 into a second set of
+// registers before it processes row j, so each thread always has the next
+// row's bytes in flight while the current row is reduced and stored.
+template <int OP, int T, int K>
+__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel_persistent(const RowArgs a) {
+  constexpr int R = (T == 32) ? 8 : 1;
+  constexpr int W = T / 32;
+  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
+  __shared__ uint32_t s_max[W > 1 ? W : 1];
+
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
+  const int64_t n_groups = int64_t(gridDim.x) * R;
+  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
+
+  griddep_wait();
+  uint4 xa[K], ra[K], xb[K], rb[K];
+  int64_t row = group;
+  load_raw<T, K, true>(a, row, row < a.M, has_res, tid, xa, ra);
+  // Reduction buffers are reused row after row.  LayerNorm's two sums use both
+  // buffers, each separated from its next use by the other sum's barrier;
+  // single-sum operations alternate by row parity.
+  for (int parity = 0; row < a.M; parity ^= 1) {
+    const int64_t next = row + n_groups;
+    if (next >= a.M) griddep_launch_dependents();  // nothing left to load
+    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[parity];
+    if (parity == 0) {
+      load_raw<T, K, true>(a, next, next < a.M, has_res, tid, xb, rb);
+      process_row<OP, T, K, true>(a, row, true, has_res, tid, xa, ra, b0, s_sum[1], s_max);
+    } else {
+      load_raw<T, K, true>(a, next, next < a.M, has_res, tid, xa, ra);
+      process_row<OP, T, K, true>(a, row, true, has_res, tid, xb, rb, b0, s_sum[1], s_max);
+    }
+    row = next;
+  }
+}
+
+// Kernel tables of one operation: every built (threads, chunks, vec) schedule
+// of the one-row kernel and every (threads, chunks) of the persistent one.
 template <int OP>
 struct RowTable {
   RowKernels k;
@@ -361,9 +413,12 @@ struct RowTable {
     for (auto& x : k.direct)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
+    for (auto& x : k.persistent)
+      for (auto& y : x) y = nullptr;
 #define NQ_DIRECT(LT, LK)                                                                                     \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
-  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);  \
+  k.persistent[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_persistent<OP, (1 << LT), (1 << LK)>);
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)
     NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2) NQ_DIRECT(7, 3)
