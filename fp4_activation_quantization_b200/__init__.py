@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
     "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND",
-    "FLAG_PERSISTENT", "FLAG_ONE_ROW", "flag_schedule", "nq_query_launch", "NQError", "lib", "library_path", "version",
+    "flag_schedule", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4",
@@ -37,8 +37,6 @@ FLAG_SCALE_DIV = 1 << 1
 FLAG_SCALE_RECIP = 1 << 2
 FLAG_UE8M0 = 1 << 3
 FLAG_NORM_BF16_ROUND = 1 << 4
-FLAG_PERSISTENT = 1 << 24
-FLAG_ONE_ROW = 1 << 25
 OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4 = 0, 1, 2, 3
 
 
@@ -69,8 +67,6 @@ def _load() -> ctypes.CDLL:
     L.nq_query_schedule.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     L.nq_query_schedule.restype = st
-    L.nq_query_launch.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
-    L.nq_query_launch.restype = st
     L.nq_fused_add_rmsnorm_quant_fp8.argtypes = [P, I64, P, P, I64, P, P, I64, P, P, I64, I64, I64, F, U32, P]
     L.nq_rmsnorm_quant_fp8_static.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, I64, I64, F, U32, P]
     L.nq_layernorm_quant_fp8.argtypes = [P, I64, P, P, P, P, I64, I64, I64, F, U32, P]
@@ -176,14 +172,6 @@ def nq_query_schedule(op: int, M: int, d: int, flags: int = 0):
     _check(_get_lib().nq_query_schedule(op, M, d, flags, ctypes.byref(t), ctypes.byref(k), ctypes.byref(r)),
            "nq_query_schedule")
     return t.value, k.value, r.value
-
-
-def nq_query_launch(op: int, M: int, d: int, flags: int = 0, aligned16: bool = True) -> dict:
-    """The launch a norm call would make (needs a CUDA device)."""
-    info = (ctypes.c_int64 * 5)()
-    _check(_get_lib().nq_query_launch(op, M, d, flags, int(aligned16), info), "nq_query_launch")
-    keys = ("threads_per_row", "chunks_per_thread", "rows_per_cta", "persistent", "grid")
-    return dict(zip(keys, [int(v) for v in info]))
 
 
 def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, residual_out=None,

@@ -7,9 +7,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
-#include <mutex>
 #include <string>
-#include <vector>
 
 #include "nq.h"
 #include "nq_internal.h"
@@ -34,8 +32,7 @@ nq_status fail(nq_status st, const char* fmt, ...) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
-                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK |
-                                 NQ_FLAG_PERSISTENT | NQ_FLAG_ONE_ROW;
+                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
                       bool allow_bf16_round) {
@@ -44,10 +41,8 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
   if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_UE8M0 applies to group quantization only", fn);
-  if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_PERSISTENT | NQ_FLAG_ONE_ROW)) && !allow_schedule)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: schedule and kernel flags apply to the norm calls only", fn);
-  if ((flags & NQ_FLAG_PERSISTENT) && (flags & NQ_FLAG_ONE_ROW))
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_PERSISTENT and NQ_FLAG_ONE_ROW are exclusive", fn);
+  if ((flags & NQ_FLAG_SCHEDULE_MASK) && !allow_schedule)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE applies to the norm calls only", fn);
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -151,89 +146,17 @@ const nq::RowKernels& table_of(int op) {
   }
 }
 
-// ---- device facts for the persistent kernel's grid (host queries, cached) ----
-struct OccEntry {
-  const void* kernel;
-  int dev;
-  int occ;
-};
-std::mutex g_mu;
-std::vector<OccEntry> g_occ;
-int g_sms[64] = {0};
-
-nq_status resident_slots(const char* fn, const void* kernel, int block, int64_t* slots) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= 64) {
-    (void)cudaGetLastError();
-    return fail(NQ_ERR_CUDA, "%s: no current CUDA device", fn);
-  }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_sms[dev] == 0) {
-    int n = 0;
-    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess || n <= 0) {
-      (void)cudaGetLastError();
-      return fail(NQ_ERR_CUDA, "%s: cannot read the SM count", fn);
-    }
-    g_sms[dev] = n;
-  }
-  int occ = -1;
-  for (const auto& o : g_occ)
-    if (o.kernel == kernel && o.dev == dev) occ = o.occ;
-  if (occ < 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, block, 0);
-    if (e != cudaSuccess) {
-      (void)cudaGetLastError();
-      return fail(NQ_ERR_CUDA, "%s: occupancy query: %s", fn, cudaGetErrorString(e));
-    }
-    g_occ.push_back({kernel, dev, occ});
-  }
-  *slots = int64_t(g_sms[dev]) * occ;
-  return NQ_OK;
-}
-
-struct LaunchPlan {
-  Schedule s;
-  bool persistent;
-  int64_t grid;
-  int block;
-  const void* kernel;
-};
-
-// One-row kernel unless the rows are 16-byte aligned and every resident
-// thread group would walk at least two rows (or NQ_FLAG_PERSISTENT): then the
-// persistent kernel with one CTA per resident slot.
-nq_status plan_launch(const char* fn, int op, int64_t M, int64_t d, bool vec, uint32_t flags, LaunchPlan* p) {
-  nq_status st = plan_rows(fn, M, d, flags, &p->s);
-  if (st != NQ_OK) return st;
-  const int threads = 1 << p->s.log_t;
-  const int rows = nq::rows_per_cta(threads);
-  const int64_t groups = (M + rows - 1) / rows;
-  p->block = threads * rows;
-  p->persistent = false;
-  p->grid = groups;
-  p->kernel = table_of(op).direct[p->s.log_t - nq::kMinLogT][p->s.log_k][vec ? 1 : 0];
-  if (!vec || (flags & NQ_FLAG_ONE_ROW)) return NQ_OK;
-  const void* pk = table_of(op).persistent[p->s.log_t - nq::kMinLogT][p->s.log_k];
-  if (pk == nullptr) return NQ_OK;
-  int64_t slots = 0;
-  if ((st = resident_slots(fn, pk, p->block, &slots)) != NQ_OK) return st;
-  if (slots <= 0) return NQ_OK;
-  if (!(flags & NQ_FLAG_PERSISTENT) && groups < 2 * slots) return NQ_OK;
-  p->persistent = true;
-  p->kernel = pk;
-  p->grid = groups < slots ? groups : slots;
-  return NQ_OK;
-}
-
 // Shared tail of the four norm calls.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
-  LaunchPlan p;
-  nq_status st = plan_launch(fn, op, a.M, a.d, vec, flags, &p);
+  Schedule s;
+  nq_status st = plan_rows(fn, a.M, a.d, flags, &s);
   if (st != NQ_OK) return st;
+  const int threads = 1 << s.log_t;
+  const int rows = nq::rows_per_cta(threads);
+  const int64_t grid = (a.M + rows - 1) / rows;
+  const void* k = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k][vec ? 1 : 0];
   void* args[] = {&a};
-  return launch(fn, p.kernel, unsigned(p.grid), unsigned(p.block), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
+  return launch(fn, k, unsigned(grid), unsigned(threads * rows), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }
 
 bool vec_bf16(const void* p, int64_t ld) { return p == nullptr || (aligned(p, 16) && ld % 8 == 0); }
@@ -269,23 +192,6 @@ nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* t
   *threads_per_row = 1 << s.log_t;
   *chunks_per_thread = 1 << s.log_k;
   *rows_per_cta = nq::rows_per_cta(1 << s.log_t);
-  return NQ_OK;
-}
-
-nq_status nq_query_launch(int op, int64_t M, int64_t d, uint32_t flags, int aligned16, int64_t* info) {
-  const char* fn = "nq_query_launch";
-  NQ_REQUIRE(op >= 0 && op < nq::kNumRowOps, "%s: op %d out of range", fn, op);
-  NQ_REQUIRE(info != nullptr, "%s: null output pointer", fn);
-  nq_status st = check_common(fn, M, d, 1.0f);
-  if (st != NQ_OK) return st;
-  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
-  LaunchPlan p;
-  if ((st = plan_launch(fn, op, M, d, aligned16 && d % 8 == 0, flags, &p)) != NQ_OK) return st;
-  info[0] = 1 << p.s.log_t;
-  info[1] = 1 << p.s.log_k;
-  info[2] = nq::rows_per_cta(1 << p.s.log_t);
-  info[3] = p.persistent ? 1 : 0;
-  info[4] = p.grid;
   return NQ_OK;
 }
 

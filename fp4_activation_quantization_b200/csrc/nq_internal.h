@@ -67,10 +67,8 @@ inline bool schedule_built(int log_t, int log_k) {
 // Host-side kernel tables (pointer to the __global__ stub), one per
 // translation unit: [log_t - 5][log_k][vec].
 using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
-using PersistentTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1];
 struct RowKernels {
-  KernelTable direct;          // one row per thread group
-  PersistentTable persistent;  // persistent groups with next-row prefetch (16-byte rows)
+  KernelTable direct;  // one row per thread group
 };
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();

@@ -341,8 +341,10 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   }
 }
 
-// One row per thread group: loads straight to registers.  The choice for few
-// rows (latency) and for unaligned rows.
+// One row per thread group: loads straight to registers.  Many small CTAs per
+// SM keep enough rows in flight; a persistent variant that prefetched the
+// next row into a second register set measured slower on B200 (the doubled
+// registers halve occupancy), and so did shared-memory cp.async staging.
 template <int OP, int T, int K, bool VEC>
 __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
@@ -366,46 +368,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   process_row<OP, T, K, VEC>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
-// Persistent thread groups (16-byte rows only): group g of G = gridDim.x * R
-// walks rows g, g + G, g + 2G, ... and loads row j + 1 into a second set of
-// registers before it processes row j, so each thread always has the next
-// row's bytes in flight while the current row is reduced and stored.
-template <int OP, int T, int K>
-__global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel_persistent(const RowArgs a) {
-  constexpr int R = (T == 32) ? 8 : 1;
-  constexpr int W = T / 32;
-  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
-  __shared__ uint32_t s_max[W > 1 ? W : 1];
-
-  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
-  const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
-  const int64_t n_groups = int64_t(gridDim.x) * R;
-  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
-
-  griddep_wait();
-  uint4 xa[K], ra[K], xb[K], rb[K];
-  int64_t row = group;
-  load_raw<T, K, true>(a, row, row < a.M, has_res, tid, xa, ra);
-  // Reduction buffers are reused row after row.  LayerNorm's two sums use both
-  // buffers, each separated from its next use by the other sum's barrier;
-  // single-sum operations alternate by row parity.
-  for (int parity = 0; row < a.M; parity ^= 1) {
-    const int64_t next = row + n_groups;
-    if (next >= a.M) griddep_launch_dependents();  // nothing left to load
-    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[parity];
-    if (parity == 0) {
-      load_raw<T, K, true>(a, next, next < a.M, has_res, tid, xb, rb);
-      process_row<OP, T, K, true>(a, row, true, has_res, tid, xa, ra, b0, s_sum[1], s_max);
-    } else {
-      load_raw<T, K, true>(a, next, next < a.M, has_res, tid, xa, ra);
-      process_row<OP, T, K, true>(a, row, true, has_res, tid, xb, rb, b0, s_sum[1], s_max);
-    }
-    row = next;
-  }
-}
-
-// Kernel tables of one operation: every built (threads, chunks, vec) schedule
-// of the one-row kernel and every (threads, chunks) of the persistent one.
+// Kernel table of one operation: every built (threads, chunks, vec) schedule.
 template <int OP>
 struct RowTable {
   RowKernels k;
@@ -413,12 +376,9 @@ struct RowTable {
     for (auto& x : k.direct)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
-    for (auto& x : k.persistent)
-      for (auto& y : x) y = nullptr;
 #define NQ_DIRECT(LT, LK)                                                                                     \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
-  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);  \
-  k.persistent[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_persistent<OP, (1 << LT), (1 << LK)>);
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)
     NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2) NQ_DIRECT(7, 3)

@@ -102,12 +102,6 @@ typedef enum nq_status {
  * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
-/* Force the persistent kernel (thread groups walk rows and prefetch the next
- * row while reducing the current one; 16-byte-aligned rows only, otherwise
- * ignored), or force the one-row-per-group kernel.  Same bits either way.
- * Neither: automatic (persistent once each resident group gets >= 2 rows). */
-#define NQ_FLAG_PERSISTENT (1u << 24)
-#define NQ_FLAG_ONE_ROW (1u << 25)
 /* Library version (major * 10000 + minor * 100 + patch). */
 int nq_version(void);
 /* Static text of a status code. */
@@ -123,14 +117,6 @@ const char* nq_last_error(void);
  */
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
                             int* chunks_per_thread, int* rows_per_cta);
-
-/*
- * Launch a norm call would make (op codes as nq_query_schedule) over M rows
- * of d elements, with 16-byte-aligned rows or not.  info[0..4] = threads per
- * row, chunks per thread, rows per CTA, persistent (0/1), grid size.  Needs a
- * current CUDA device (occupancy query); launches nothing.
- */
-nq_status nq_query_launch(int op, int64_t M, int64_t d, uint32_t flags, int aligned16, int64_t* info);
 
 /*
  * Fused residual-add + RMSNorm + dynamic per-token e4m3.

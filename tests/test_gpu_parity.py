@@ -394,57 +394,3 @@ def test_nvfp4_zero_blocks(nq):
     eq, esf, _, _ = oracle.rmsnorm_quant_nvfp4(x, w["gamma"], 0.01)
     assert np.array_equal(got[0], eq) and np.array_equal(got[1], esf)
     assert not got[0][1].any() and not got[1][1].any()
-
-
-# ------------------------------------------------ persistent kernel ----
-PERSIST_CASES = [  # (d, M, ld_x): M large enough that every thread group walks several rows
-    (512, 40000, 512), (1536, 6000, 2112), (2816, 4096, 2816), (4096, 4096, 4096), (8192, 2000, 8192),
-    (16384, 700, 16384),
-]
-
-
-@pytest.mark.parametrize("d,M,ld", PERSIST_CASES)
-def test_persistent_all_ops_bit_exact(nq, d, M, ld):
-    """Persistent prefetching kernel: every op, default and forced schedules, against the oracle."""
-    w = S.make_rms_inputs(M, d, seed=d + 1, ld_x=ld, x_outlier_channels=True)
-    lw = S.make_ln_inputs(M, d, seed=d + 2)
-    x = dev_bf16(w["x"])[:, :d]
-    res = dev_bf16(w["residual"])
-    g = dev_bf16(w["gamma"])
-    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
-    gn = oracle.nvfp4_global_scale(w["x"], w["gamma"], w["residual"], d=d)
-    gs = torch.tensor([gn], dtype=torch.float32, device="cuda")
-    e_dyn = oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"], d=d)
-    e_st, e_str, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, residual=w["residual"], d=d)
-    e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
-    e_fp4 = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn, residual=w["residual"], d=d)
-    sch = all_schedules(d)
-    variants = [nq.FLAG_PERSISTENT] + [nq.FLAG_PERSISTENT | nq.flag_schedule(*s) for s in (sch[:2] + sch[-2:])]
-    for f in variants:
-        info = nq.nq_query_launch(nq.OP_RMS_DYN_FP8, M, d, f)
-        assert info["persistent"] == 1, info
-        q, s, ro, _ = nq.nq_fused_add_rmsnorm_quant_fp8(x, res, g, 1e-6, flags=f)
-        assert_fused_equal((host_u8(q), s.cpu().numpy(), host_u16(ro), None), e_dyn)
-        q, ro, _ = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, residual=res, flags=f)
-        assert np.array_equal(host_u8(q), e_st) and np.array_equal(host_u16(ro), e_str), f
-        q = nq.nq_layernorm_quant_fp8(dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"]), sc, 1e-6,
-                                      flags=f)
-        assert np.array_equal(host_u8(q), e_ln), f
-        q, sf, ro, _ = nq.nq_rmsnorm_quant_nvfp4(x, g, gs, 1e-6, residual=res, flags=f)
-        assert np.array_equal(host_u8(q), e_fp4[0]) and np.array_equal(host_u8(sf), e_fp4[1]), f
-        assert np.array_equal(host_u16(ro), e_fp4[2]), f
-
-
-def test_launch_choice(nq):
-    big = nq.nq_query_launch(nq.OP_RMS_STATIC_FP8, 65536, 4096)
-    assert big["persistent"] == 1 and big["grid"] < 65536
-    assert nq.nq_query_launch(nq.OP_RMS_STATIC_FP8, 65536, 4096, aligned16=False)["persistent"] == 0
-    assert nq.nq_query_launch(nq.OP_RMS_DYN_FP8, 1, 8192)["persistent"] == 0
-    assert nq.nq_query_launch(nq.OP_RMS_STATIC_FP8, 65536, 4096, nq.FLAG_ONE_ROW)["persistent"] == 0
-
-
-def test_persistent_inplace_residual_and_guards(nq):
-    M, d = 5000, 2816
-    w = S.make_rms_inputs(M, d, seed=77)
-    got = run_fused(nq, w, flags=nq.FLAG_PERSISTENT, guarded=True)
-    assert_fused_equal(got, oracle_fused(w))
