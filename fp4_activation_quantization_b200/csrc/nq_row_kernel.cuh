@@ -73,72 +73,6 @@ __device__ __forceinline__ float row_total(float (&part)[K], float* red, int tid
   return row_sum<T>(part[0], red, tid);
 }
 
-// Row total in the canonical order, finished by warp 0 alone: the value is
-// meaningful in warp 0 (every lane) only.  For T > 32 this holds one barrier;
-// the other warps then wait at warp0_scalars' barrier instead of repeating
-// the cross-warp tree and the shuffles.
-template <int T, int K>
-__device__ __forceinline__ float row_total_w0(float (&part)[K], float* red, int tid) {
-#pragma unroll
-  for (int h = K / 2; h >= 1; h >>= 1)
-#pragma unroll
-    for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-  float v = part[0];
-  if constexpr (T > 32) {
-    constexpr int W = T / 32;
-    red[(tid >> 5) * 32 + (tid & 31)] = v;
-    __syncthreads();
-    if (tid >= 32) return v;
-    float p[W];
-#pragma unroll
-    for (int i = 0; i < W; ++i) p[i] = red[i * 32 + tid];
-#pragma unroll
-    for (int h = W / 2; h >= 1; h >>= 1)
-#pragma unroll
-      for (int i = 0; i < h; ++i) p[i] = __fadd_rn(p[i], p[i + h]);
-    v = p[0];
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, o));
-  return v;
-}
-
-// Row maximum of non-negative floats, meaningful in warp 0 only (T > 32).
-template <int T>
-__device__ __forceinline__ float row_max_w0(float v, uint32_t* red, int tid) {
-  uint32_t u = __reduce_max_sync(kFull, __float_as_uint(v));
-  if constexpr (T > 32) {
-    constexpr int W = T / 32;
-    if ((tid & 31) == 0) red[tid >> 5] = u;
-    __syncthreads();
-    if (tid >= 32) return 0.0f;
-    u = 0;
-#pragma unroll
-    for (int i = 0; i < W; ++i) u = max(u, red[i]);
-  }
-  return __uint_as_float(u);
-}
-
-// Two per-row scalars computed by warp 0 (f() is evaluated there only) and
-// handed to every thread of the group through shared memory (one barrier
-// when T > 32).
-template <int T, class F>
-__device__ __forceinline__ float2 warp0_scalars(int tid, float* s_bc, F f) {
-  if constexpr (T == 32) {
-    return f();
-  } else {
-    if (tid < 32) {
-      const float2 r = f();
-      if (tid == 0) {
-        s_bc[0] = r.x;
-        s_bc[1] = r.y;
-      }
-    }
-    __syncthreads();
-    return make_float2(s_bc[0], s_bc[1]);
-  }
-}
-
 // a1: raw bf16 chunks of one row (zeros past the row or for dead rows).
 template <int T, int K, bool VEC>
 __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
@@ -175,8 +109,8 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 // reduction buffers.
 template <int OP, int T, int K, bool VEC>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
-                                            const uint4 (&xr)[K], const uint4 (&rr)[K], float scale_in,
-                                            float* s_sum0, float* s_sum1, uint32_t* s_max, float* s_bc) {
+                                            const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
+                                            float* s_sum1, uint32_t* s_max) {
   const int d = a.d;
   const int C = (d + 7) >> 3;
   const bool div = (a.flags & kFlagDiv) != 0;
@@ -207,16 +141,14 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     }
     part[k] = chunk_partial<OP != kOpLnStaticFp8>(v[k]);
   }
-  const float total = row_total_w0<T, K>(part, s_sum0, tid);
+  const float total = row_total<T, K>(part, s_sum0, tid);
 
   const float fd = float(d);
-  // Per-row scalars: rstd and, for the static scales, RN(1 / scale).
-  float rstd, inv_static = 0.0f;
+  float rstd;
   if constexpr (OP == kOpLnStaticFp8) {
     // Centre on the row mean (RN(r - mean) == RN(r + (-mean))), then the
     // biased variance; padding elements stay exactly zero.
-    const float mean = warp0_scalars<T>(tid, s_bc, [&] { return make_float2(__fdiv_rn(total, fd), 0.0f); }).x;
-    const float2 nm = f2(-mean);
+    const float2 nm = f2(-__fdiv_rn(total, fd));
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
@@ -232,19 +164,10 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       }
       part[k] = chunk_partial<true>(v[k]);
     }
-    const float sq = row_total_w0<T, K>(part, s_sum1, tid);
-    const float2 sc = warp0_scalars<T>(tid, s_bc + 2, [&] {
-      return make_float2(__frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps))), __frcp_rn(scale_in));
-    });
-    rstd = sc.x;
-    inv_static = sc.y;
+    const float sq = row_total<T, K>(part, s_sum1, tid);
+    rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
   } else {
-    const float2 sc = warp0_scalars<T>(tid, s_bc, [&] {
-      const float r = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
-      return make_float2(r, OP == kOpRmsStaticFp8 ? __frcp_rn(scale_in) : 0.0f);
-    });
-    rstd = sc.x;
-    inv_static = sc.y;
+    rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
   }
 
   // ---- a4: normalize (y overwrites v); gamma / beta fetched now, through L1
@@ -328,7 +251,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 
   // ---- a5 + a6: scale, quantize, pack, store
   if constexpr (OP == kOpRmsNvfp4) {
-    const float g = scale_in;
+    const float g = __ldg(a.scale);
     uint8_t* qrow = a.q + row * a.ld_q;
     uint8_t* sfrow = a.sf + row * a.ld_sf;
 #pragma unroll
@@ -378,18 +301,15 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       for (int k = 0; k < K; ++k)
 #pragma unroll
         for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
-      const float amax = row_max_w0<T>(m, s_max, tid);
-      const float2 sc = warp0_scalars<T>(tid, s_bc + 2, [&] {
-        const float s = __fdiv_rn(amax, kE4M3Max);
-        return make_float2(s, __frcp_rn(s));
-      });
-      if (live && tid == 0) a.scale_out[row] = sc.x;
-      s_div = sc.x;
-      s_inv = sc.y;
-      passthrough = (sc.x == 0.0f);  // zero row: store the signed zeros of y
+      const float amax = row_max_nonneg<T>(m, s_max, tid);
+      const float s = __fdiv_rn(amax, kE4M3Max);
+      if (live && tid == 0) a.scale_out[row] = s;
+      s_div = s;
+      s_inv = __frcp_rn(s);
+      passthrough = (s == 0.0f);  // zero row: store the signed zeros of y
     } else {
-      s_div = scale_in;
-      s_inv = inv_static;
+      s_div = __ldg(a.scale);
+      s_inv = __frcp_rn(s_div);
     }
     uint8_t* qrow = a.q + row * a.ld_q;
     const float2 inv2 = f2(s_inv);
@@ -433,7 +353,6 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   static_assert(R * T <= 1024, "CTA size");
   __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
   __shared__ uint32_t s_max[W > 1 ? W : 1];
-  __shared__ float s_bc[4];
 
   const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
   const int64_t row = (T == 32) ? int64_t(blockIdx.x) * R + int64_t(threadIdx.x >> 5) : int64_t(blockIdx.x);
@@ -445,10 +364,8 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   griddep_wait();
   uint4 xr[K], rr[K];
   load_raw<T, K, VEC>(a, row, live, has_res, tid, xr, rr);
-  // Static scale / NVFP4 global scale, read at execution time (graph replays see updates).
-  const float scale_in = (OP == kOpRmsDynFp8) ? 0.0f : __ldg(a.scale);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
-  process_row<OP, T, K, VEC>(a, row, live, has_res, tid, xr, rr, scale_in, s_sum[0], s_sum[1], s_max, s_bc);
+  process_row<OP, T, K, VEC>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
 // Kernel table of one operation: every built (threads, chunks, vec) schedule.
