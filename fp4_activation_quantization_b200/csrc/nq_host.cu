@@ -154,7 +154,8 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   const int threads = 1 << s.log_t;
   const int rows = nq::rows_per_cta(threads);
   const int64_t grid = (a.M + rows - 1) / rows;
-  const void* k = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k][vec ? 1 : 0];
+  const bool full = vec && threads > 32 && a.d == 8 * int64_t(threads) << s.log_k;
+  const void* k = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k][full ? 2 : (vec ? 1 : 0)];
   void* args[] = {&a};
   return launch(fn, k, unsigned(grid), unsigned(threads * rows), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }

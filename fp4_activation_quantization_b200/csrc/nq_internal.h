@@ -65,8 +65,9 @@ inline bool schedule_built(int log_t, int log_k) {
 }
 
 // Host-side kernel tables (pointer to the __global__ stub), one per
-// translation unit: [log_t - 5][log_k][vec].
-using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
+// translation unit: [log_t - 5][log_k][mode], mode 0 = any alignment,
+// 1 = 16-byte rows, 2 = 16-byte rows with d == 8 * threads * chunks (t > 5).
+using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][3];
 struct RowKernels {
   KernelTable direct;  // one row per thread group
 };

@@ -74,7 +74,9 @@ __device__ __forceinline__ float row_total(float (&part)[K], float* red, int tid
 }
 
 // a1: raw bf16 chunks of one row (zeros past the row or for dead rows).
-template <int T, int K, bool VEC>
+// FULL: every chunk slot of the schedule is a real chunk of a live row (d ==
+// 8 * T * K, one row per CTA), so no predicate or zero fill is needed.
+template <int T, int K, bool VEC, bool FULL>
 __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
                                          uint4 (&xr)[K], uint4 (&rr)[K]) {
   const int d = a.d;
@@ -84,7 +86,7 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
-    const bool ok = live && c < C;
+    const bool ok = FULL || (live && c < C);
     if constexpr (VEC) {
       xr[k] = ok ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
       rr[k] = (has_res && ok) ? __ldcs(reinterpret_cast<const uint4*>(rrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
@@ -107,12 +109,13 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.
-template <int OP, int T, int K, bool VEC>
-__device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
+template <int OP, int T, int K, bool VEC, bool FULL>
+__device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
                                             float* s_sum1, uint32_t* s_max) {
   const int d = a.d;
-  const int C = (d + 7) >> 3;
+  const int C = FULL ? T * K : (d + 7) >> 3;
+  const bool live = FULL || live_in;
   const bool div = (a.flags & kFlagDiv) != 0;
   // ---- a2: r = x + residual, residual_out; a3: chunk partials
   float2 v[K][4];
@@ -126,7 +129,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       unpack_pairs(rr[k], t);
 #pragma unroll
       for (int i = 0; i < 4; ++i) v[k][i] = add2(v[k][i], t[i]);
-      if (live && c < C) {
+      if (FULL || (live && c < C)) {
         uint16_t* orow = a.res_out + row * a.ld_res;
         if constexpr (VEC) {
           *reinterpret_cast<uint4*>(orow + 8 * c) = pack_pairs_bf16(v[k]);
@@ -152,7 +155,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
-      const bool ok = live && c < C;
+      const bool ok = FULL || (live && c < C);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float2 t = add2(v[k][i], nm);
@@ -176,7 +179,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
-    const bool gok = c < C;
+    const bool gok = FULL || c < C;
     if constexpr (OP == kOpLnStaticFp8) {
       const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
       const float* bp = a.beta + 8 * c;
@@ -234,7 +237,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
       for (int k = 0; k < K; ++k) {
         const int c = tid + k * T;
-        if (live && c < C) {
+        if (FULL || (live && c < C)) {
           if constexpr (VEC) {
             *reinterpret_cast<uint4*>(nrow + 8 * c) = pack_pairs_bf16(v[k]);
           } else {
@@ -257,7 +260,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
-      const bool ok = live && c < C;
+      const bool ok = FULL || (live && c < C);
       float m8 = 0.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
@@ -328,7 +331,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
         for (int i = 0; i < 4; ++i) t[i] = mul2(v[k][i], inv2);
       }
       const uint2 codes = pack_pairs_e4m3(t);
-      if (live && c < C) {
+      if (FULL || (live && c < C)) {
         if constexpr (VEC) {
           *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
         } else {
@@ -345,8 +348,12 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 // SM keep enough rows in flight; a persistent variant that prefetched the
 // next row into a second register set measured slower on B200 (the doubled
 // registers halve occupancy), and so did shared-memory cp.async staging.
-template <int OP, int T, int K, bool VEC>
+// MODE 0: any alignment (scalar loads); 1: 16-byte rows; 2: 16-byte rows that
+// exactly fill the schedule (d == 8 * T * K, T > 32): no predicates at all.
+template <int OP, int T, int K, int MODE>
 __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
+  constexpr bool VEC = MODE >= 1;
+  constexpr bool FULL = MODE == 2;
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
   constexpr int W = T / 32;             // warps per row
   static_assert(K == 1 || K == 2 || K == 4 || K == 8, "chunks per thread");
@@ -363,9 +370,9 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
 
   griddep_wait();
   uint4 xr[K], rr[K];
-  load_raw<T, K, VEC>(a, row, live, has_res, tid, xr, rr);
+  load_raw<T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
-  process_row<OP, T, K, VEC>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+  process_row<OP, T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
 // Kernel table of one operation: every built (threads, chunks, vec) schedule.
@@ -376,9 +383,10 @@ struct RowTable {
     for (auto& x : k.direct)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
-#define NQ_DIRECT(LT, LK)                                                                                     \
-  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), false>); \
-  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), true>);
+#define NQ_DIRECT(LT, LK)                                                                                 \
+  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0>); \
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1>); \
+  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2>);
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)
     NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2) NQ_DIRECT(7, 3)
