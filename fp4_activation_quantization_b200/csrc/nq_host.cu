@@ -7,7 +7,9 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "nq.h"
 #include "nq_internal.h"
@@ -146,6 +148,21 @@ const nq::RowKernels& table_of(int op) {
   }
 }
 
+// Registers per thread of a kernel (host query, cached per kernel).
+std::mutex g_regs_mu;
+std::vector<std::pair<const void*, int>> g_regs;
+int kernel_regs(const void* k) {
+  std::lock_guard<std::mutex> lk(g_regs_mu);
+  for (const auto& p : g_regs)
+    if (p.first == k) return p.second;
+  cudaFuncAttributes attr;
+  int regs = -1;
+  if (cudaFuncGetAttributes(&attr, k) == cudaSuccess) regs = attr.numRegs;
+  else (void)cudaGetLastError();
+  g_regs.push_back({k, regs});
+  return regs;
+}
+
 // Shared tail of the four norm calls.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   Schedule s;
@@ -154,8 +171,14 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   const int threads = 1 << s.log_t;
   const int rows = nq::rows_per_cta(threads);
   const int64_t grid = (a.M + rows - 1) / rows;
-  const bool full = vec && threads > 32 && a.d == 8 * int64_t(threads) << s.log_k;
-  const void* k = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k][full ? 2 : (vec ? 1 : 0)];
+  const auto& tab = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k];
+  const void* k = tab[vec ? 1 : 0];
+  // The predicate-free variant for rows that exactly fill the schedule, when
+  // it does not need more registers (occupancy decides this kernel's speed).
+  if (vec && threads > 32 && a.d == (8 * int64_t(threads)) << s.log_k && tab[2] != nullptr) {
+    const int r_full = kernel_regs(tab[2]), r_vec = kernel_regs(tab[1]);
+    if (r_full > 0 && r_vec > 0 && r_full <= r_vec) k = tab[2];
+  }
   void* args[] = {&a};
   return launch(fn, k, unsigned(grid), unsigned(threads * rows), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }
