@@ -203,13 +203,21 @@ def barrier(world):
 
 
 def max_over_ranks(world, value: float) -> float:
+    """Largest value over the ranks (host plumbing: one float, on the process group's device)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, steps: int, step_bytes: int, elapsed_ms: float) -> float:
+    """Whole-job GB/s: every rank processed `steps` steps of `step_bytes` (weak scaling)
+    in at most `elapsed_ms` (the max over ranks)."""
+    return world * steps * step_bytes / (elapsed_ms * 1e-3) / 1e9
 
 
 # ------------------------------------------------------------ GPU arm ----
@@ -315,7 +323,7 @@ def run_gpu_arm(args):
     elapsed_ms = max_over_ranks(world, elapsed_ms)
 
     step_bytes = rms_static_bytes(M, d) + ln_static_bytes(M, d)
-    value = world * K * step_bytes / (elapsed_ms * 1e-3) / 1e9
+    value = job_throughput(world, K, step_bytes, elapsed_ms)
     peak, peak_src = measured_peak()
     rms_us, ln_us = rms_ms * 1e3 / K, ln_ms * 1e3 / K
     dom = ("nq_rmsnorm_quant_fp8_static", rms_us, rms_static_bytes(M, d)) if rms_us >= ln_us else \
@@ -354,7 +362,7 @@ def run_gpu_arm(args):
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(world, a.elapsed_time(b))
         barrier(world)
-        e2e = {"value": round(world * ke * step_bytes / (e2e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+        e2e = {"value": round(job_throughput(world, ke, step_bytes, e2e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": 2 * M * d * 2, "d2h_bytes_per_step": 2 * M * d, "steps": ke,
                "ms_per_step": round(e2e_ms / ke, 4)}
 
@@ -558,6 +566,35 @@ def run_reference_arm(args):
     }), flush=True)
 
 
+def run_case(args):
+    """Run one call a few times on a device-seeded input (for ncu captures of a
+    single kernel on a small case); prints nothing but 'ok'."""
+    import torch
+    import fp4_activation_quantization_b200 as nq
+    M, d, op = args.M, args.d, args.case
+    bf = torch.bfloat16
+    g = torch.Generator(device="cuda").manual_seed(0)
+    x = torch.randn(M, d, device="cuda", generator=g).to(bf)
+    res = torch.randn(M, d, device="cuda", generator=g).to(bf) if op in ("fused_add_rmsnorm_quant_fp8", "nvfp4_res") else None
+    gam = (1 + 0.1 * torch.randn(d, device="cuda", generator=g)).to(bf)
+    gl = 1 + 0.1 * torch.randn(d, device="cuda", generator=g)
+    bl = 0.02 * torch.randn(d, device="cuda", generator=g)
+    sc = torch.tensor([SCALE], device="cuda")
+    for _ in range(args.iters):
+        if op == "rmsnorm_quant_fp8_static":
+            nq.nq_rmsnorm_quant_fp8_static(x, gam, sc, EPS)
+        elif op == "layernorm_quant_fp8":
+            nq.nq_layernorm_quant_fp8(x, gl, bl, sc, EPS)
+        elif op == "fused_add_rmsnorm_quant_fp8":
+            nq.nq_fused_add_rmsnorm_quant_fp8(x, res, gam, 1e-6, residual_out=res)
+        elif op in ("nvfp4", "nvfp4_res"):
+            nq.nq_rmsnorm_quant_nvfp4(x, gam, sc, 1e-6, residual=res, residual_out=res)
+        elif op == "per_token_group_quant_fp8":
+            nq.nq_per_token_group_quant_fp8(x, 128)
+    torch.cuda.synchronize()
+    print("ok")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -571,8 +608,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--case", choices=["rmsnorm_quant_fp8_static", "layernorm_quant_fp8",
+                                       "fused_add_rmsnorm_quant_fp8", "nvfp4", "nvfp4_res",
+                                       "per_token_group_quant_fp8"],
+                    help="run one call --iters times on M x d and exit (for profiler captures)")
+    ap.add_argument("--M", type=int, default=16384)
+    ap.add_argument("--d", type=int, default=4096)
+    ap.add_argument("--iters", type=int, default=3)
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference_arm(args)
     else:
         run_gpu_arm(args)
