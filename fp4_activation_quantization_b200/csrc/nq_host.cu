@@ -34,7 +34,8 @@ nq_status fail(nq_status st, const char* fmt, ...) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
-                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK;
+                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK |
+                                 NQ_FLAG_VARIANT_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
                       bool allow_bf16_round) {
@@ -43,8 +44,10 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
   if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_UE8M0 applies to group quantization only", fn);
-  if ((flags & NQ_FLAG_SCHEDULE_MASK) && !allow_schedule)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE applies to the norm calls only", fn);
+  if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK)) && !allow_schedule)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_VARIANT apply to the norm calls only", fn);
+  if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 3)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT(n) takes n in 0..3", fn);
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -163,21 +166,68 @@ int kernel_regs(const void* k) {
   return regs;
 }
 
+// SM count and resident CTAs per SM of a kernel (host queries, cached).
+std::mutex g_occ_mu;
+std::vector<std::pair<const void*, int>> g_occ;
+int g_sms = 0;
+int64_t resident_ctas(const void* k, int block) {
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  if (g_sms == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return 0;
+    }
+    g_sms = n;
+  }
+  for (const auto& p : g_occ)
+    if (p.first == k) return int64_t(g_sms) * p.second;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, block, 0) != cudaSuccess) {
+    (void)cudaGetLastError();
+    occ = 0;
+  }
+  g_occ.push_back({k, occ});
+  return int64_t(g_sms) * occ;
+}
+
 // Shared tail of the four norm calls.
+//
+// Kernel variants (same bits): register rows (row_kernel: the row as float32
+// in registers; any op, any alignment), raw rows (row_kernel_raw: ops without
+// a residual, 16-byte rows, one CTA per row, raw bf16 kept and unpacked per
+// pass), and raw rows persistent (one CTA per resident slot, next row
+// prefetched).  NQ_FLAG_VARIANT forces one where it applies.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   Schedule s;
   nq_status st = plan_rows(fn, a.M, a.d, flags, &s);
   if (st != NQ_OK) return st;
   const int threads = 1 << s.log_t;
   const int rows = nq::rows_per_cta(threads);
-  const int64_t grid = (a.M + rows - 1) / rows;
-  const auto& tab = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k];
-  const void* k = tab[vec ? 1 : 0];
-  // The predicate-free variant for rows that exactly fill the schedule, when
-  // it does not need more registers (occupancy decides this kernel's speed).
-  if (vec && threads > 32 && a.d == (8 * int64_t(threads)) << s.log_k && tab[2] != nullptr) {
-    const int r_full = kernel_regs(tab[2]), r_vec = kernel_regs(tab[1]);
-    if (r_full > 0 && r_vec > 0 && r_full <= r_vec) k = tab[2];
+  int64_t grid = (a.M + rows - 1) / rows;
+  const bool has_res = a.res_in != nullptr;
+  const uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
+  const void* k = nullptr;
+  if (vec && threads > 32 && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
+    const auto& raw = table_of(op).raw[s.log_t - nq::kMinLogT][s.log_k];
+    if (variant == 3 && raw[1] != nullptr) {
+      const int64_t slots = resident_ctas(raw[1], threads);
+      if (slots > 0) {
+        k = raw[1];
+        grid = grid < slots ? grid : slots;
+      }
+    }
+    if (k == nullptr) k = raw[0];
+  }
+  if (k == nullptr) {
+    const auto& tab = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k];
+    k = tab[vec ? 1 : 0];
+    // The predicate-free variant for rows that exactly fill the schedule, when
+    // it does not need more registers (occupancy decides this kernel's speed).
+    if (vec && threads > 32 && a.d == (8 * int64_t(threads)) << s.log_k && tab[2] != nullptr) {
+      const int r_full = kernel_regs(tab[2]), r_vec = kernel_regs(tab[1]);
+      if (r_full > 0 && r_vec > 0 && r_full <= r_vec) k = tab[2];
+    }
   }
   void* args[] = {&a};
   return launch(fn, k, unsigned(grid), unsigned(threads * rows), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);

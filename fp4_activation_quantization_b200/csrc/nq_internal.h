@@ -68,8 +68,10 @@ inline bool schedule_built(int log_t, int log_k) {
 // translation unit: [log_t - 5][log_k][mode], mode 0 = any alignment,
 // 1 = 16-byte rows, 2 = 16-byte rows with d == 8 * threads * chunks (t > 5).
 using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][3];
+using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
 struct RowKernels {
   KernelTable direct;  // one row per thread group
+  RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent]
 };
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();

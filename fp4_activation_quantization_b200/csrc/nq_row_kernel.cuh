@@ -375,6 +375,165 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   process_row<OP, T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
+// Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
+// residual), 16-byte rows, T > 32.  Only the raw bf16 chunks are kept (half
+// the registers of float32); each pass unpacks them again.  With PERSIST the
+// CTA walks rows g, g + G, ... and loads the next row's raw chunks before it
+// processes the current one, so a load is always in flight; the static scale's
+// reciprocal is then computed once per CTA.
+template <int OP, int T, int K, bool PERSIST>
+__global__ void __launch_bounds__(T) row_kernel_raw(const RowArgs a) {
+  static_assert(T > 32 && OP != kOpRmsDynFp8, "raw rows: one row per CTA, no residual");
+  constexpr int W = T / 32;
+  __shared__ __align__(16) float s_sum[2][W * 32];
+  const int tid = int(threadIdx.x);
+  const int d = a.d;
+  const int C = d >> 3;
+  const float fd = float(d);
+  const bool div = (a.flags & kFlagDiv) != 0;
+  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
+
+  griddep_wait();
+  const float scale_in = __ldg(a.scale);
+  const float inv_static = __frcp_rn(scale_in);
+
+  auto load = [&](int64_t row, uint4 (&xr)[K]) {
+    const uint16_t* xrow = a.x + row * a.ld_x;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      xr[k] = (row < a.M && c < C) ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  auto process = [&](int64_t row, const uint4 (&xr)[K], float* b0, float* b1) {
+    float part[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      float2 v[4];
+      unpack_pairs(xr[k], v);
+      part[k] = chunk_partial<OP != kOpLnStaticFp8>(v);
+    }
+    const float total = row_total<T, K>(part, b0, tid);
+    float rstd, mean = 0.0f;
+    if constexpr (OP == kOpLnStaticFp8) {
+      mean = __fdiv_rn(total, fd);
+      const float2 nm = f2(-mean);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int c = tid + k * T;
+        float2 v[4];
+        unpack_pairs(xr[k], v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = (c < C) ? add2(v[i], nm) : f2(0.0f);
+        part[k] = chunk_partial<true>(v);
+      }
+      const float sq = row_total<T, K>(part, b1, tid);
+      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
+    } else {
+      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
+    }
+    const float2 rs2 = f2(rstd), nm = f2(-mean), inv2 = f2(inv_static);
+    uint8_t* qrow = a.q + row * a.ld_q;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      const bool ok = c < C;
+      float2 v[4];
+      unpack_pairs(xr[k], v);
+      if constexpr (OP == kOpLnStaticFp8) {
+        float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
+        if (ok) {
+          const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
+          g0 = __ldg(reinterpret_cast<const float4*>(gp));
+          g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
+          e0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
+          e1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
+        }
+        const float2 g[4] = {make_float2(g0.x, g0.y), make_float2(g0.z, g0.w), make_float2(g1.x, g1.y),
+                             make_float2(g1.z, g1.w)};
+        const float2 b[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w), make_float2(e1.x, e1.y),
+                             make_float2(e1.z, e1.w)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = fma2(mul2(add2(v[i], nm), rs2), g[i], b[i]);
+      } else {
+        uint4 gu = make_uint4(0u, 0u, 0u, 0u);
+        if (ok) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
+        float2 g[4];
+        unpack_pairs(gu, g);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = mul2(mul2(v[i], rs2), g[i]);
+      }
+      if (bf16_round) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = make_float2(round_bf16(v[i].x), round_bf16(v[i].y));
+      }
+      if constexpr (OP != kOpLnStaticFp8) {
+        if (a.norm_out != nullptr && ok)
+          *reinterpret_cast<uint4*>(a.norm_out + row * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
+      }
+      if constexpr (OP == kOpRmsNvfp4) {
+        float m8 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+        const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));  // chunks c, c^1 form a block
+        const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), scale_in));
+        const float S = __fmul_rn(e4m3_to_f32(sfc), scale_in);
+        const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+        float t[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (div && S != 0.0f) {
+            t[2 * i] = __fdiv_rn(v[i].x, S);
+            t[2 * i + 1] = __fdiv_rn(v[i].y, S);
+          } else {
+            const float2 q = mul2(v[i], f2(mult));
+            t[2 * i] = q.x;
+            t[2 * i + 1] = q.y;
+          }
+        }
+        const uint32_t packed = pack_e2m1x8(t);
+        if (ok) {
+          *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
+          if ((c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
+        }
+      } else {
+        float2 t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
+        if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_e4m3(t);
+      }
+    }
+  };
+
+  if constexpr (!PERSIST) {
+    uint4 xr[K];
+    load(blockIdx.x, xr);
+    griddep_launch_dependents();
+    process(blockIdx.x, xr, s_sum[0], s_sum[1]);
+  } else {
+    // Reduction buffers are reused row after row: LayerNorm's two sums use
+    // both buffers (each separated from its next use by the other sum's
+    // barrier); single-sum operations alternate by row parity.
+    uint4 xa[K], xb[K];
+    int64_t row = blockIdx.x;
+    load(row, xa);
+    for (int parity = 0; row < a.M; parity ^= 1) {
+      const int64_t next = row + gridDim.x;
+      if (next >= a.M) griddep_launch_dependents();  // nothing left to load
+      float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[parity];
+      if (parity == 0) {
+        load(next, xb);
+        process(row, xa, b0, s_sum[1]);
+      } else {
+        load(next, xa);
+        process(row, xb, b0, s_sum[1]);
+      }
+      row = next;
+    }
+  }
+}
+
 // Kernel table of one operation: every built (threads, chunks, vec) schedule.
 template <int OP>
 struct RowTable {
@@ -383,10 +542,17 @@ struct RowTable {
     for (auto& x : k.direct)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
+    for (auto& x : k.raw)
+      for (auto& y : x)
+        for (auto& z : y) z = nullptr;
 #define NQ_DIRECT(LT, LK)                                                                                 \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0>); \
   k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1>); \
-  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2>);
+  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2>); \
+  if constexpr (LT > 5 && OP != kOpRmsDynFp8) {                                                         \
+    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false>); \
+    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true>);  \
+  }
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)
     NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2) NQ_DIRECT(7, 3)

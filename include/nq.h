@@ -102,6 +102,13 @@ typedef enum nq_status {
  * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
+/* Force a kernel variant (tests and tuning; same bits either way): n = 1 keeps
+ * the row in float32 registers; n = 2 keeps only the raw bf16 row and unpacks
+ * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row.
+ * n = 2, 3 apply to 16-byte-aligned rows without a residual and more than 32
+ * threads per row, and are ignored otherwise.  0 = automatic. */
+#define NQ_FLAG_VARIANT(n) ((((uint32_t)(n)) & 0x7u) << 24)
+#define NQ_FLAG_VARIANT_MASK (0x7u << 24)
 /* Library version (major * 10000 + minor * 100 + patch). */
 int nq_version(void);
 /* Static text of a status code. */

@@ -394,3 +394,32 @@ def test_nvfp4_zero_blocks(nq):
     eq, esf, _, _ = oracle.rmsnorm_quant_nvfp4(x, w["gamma"], 0.01)
     assert np.array_equal(got[0], eq) and np.array_equal(got[1], esf)
     assert not got[0][1].any() and not got[1][1].any()
+
+
+# ------------------------------------------------ kernel variants ----
+@pytest.mark.parametrize("d,M,ld", [(512, 3000, 512), (1536, 2000, 2112), (2816, 1500, 2816), (4096, 4096, 4096),
+                                    (7168, 700, 7168), (16384, 300, 16384)])
+def test_variants_without_residual_bit_exact(nq, d, M, ld):
+    """Raw-row and persistent raw-row variants (static RMSNorm, LayerNorm, NVFP4 without residual)
+    give the oracle's bits for the default and forced schedules."""
+    w = S.make_rms_inputs(M, d, seed=d + 5, residual=False, ld_x=ld, x_outlier_channels=True)
+    lw = S.make_ln_inputs(M, d, seed=d + 6)
+    x = dev_bf16(w["x"])[:, :d]
+    g = dev_bf16(w["gamma"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    gn = oracle.nvfp4_global_scale(w["x"], w["gamma"], d=d)
+    gs = torch.tensor([gn], dtype=torch.float32, device="cuda")
+    e_st, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, d=d, eps=1e-6)
+    e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
+    e_fp4 = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn, d=d)
+    sch = [s for s in all_schedules(d) if s[0] > 5]
+    for var in (2, 3):
+        for sched in [None] + sch[:2] + sch[-1:]:
+            f = nq.flag_variant(var) | (0 if sched is None else nq.flag_schedule(*sched))
+            q, _, _ = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, flags=f)
+            assert np.array_equal(host_u8(q), e_st), (var, sched)
+            q = nq.nq_layernorm_quant_fp8(dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"]), sc, 1e-6,
+                                          flags=f)
+            assert np.array_equal(host_u8(q), e_ln), (var, sched)
+            q, sf, _, _ = nq.nq_rmsnorm_quant_nvfp4(x, g, gs, 1e-6, flags=f)
+            assert np.array_equal(host_u8(q), e_fp4[0]) and np.array_equal(host_u8(sf), e_fp4[1]), (var, sched)
