@@ -206,13 +206,24 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   const int rows = nq::rows_per_cta(threads);
   int64_t grid = (a.M + rows - 1) / rows;
   const bool has_res = a.res_in != nullptr;
-  const uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
+  uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
+  if (variant == 0 && !has_res) {
+    // Automatic choice, from measurements on B200: static RMSNorm gains from
+    // raw rows (fewer registers, more CTAs per SM) and, once every resident
+    // CTA gets two or more rows, from the persistent prefetching form; NVFP4
+    // gains from raw rows on wide rows; LayerNorm (two reductions in a row)
+    // does not, and keeps float32 rows.
+    if (op == nq::kOpRmsStaticFp8) variant = 3;
+    else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
+  }
   const void* k = nullptr;
   if (vec && threads > 32 && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
     const auto& raw = table_of(op).raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1] != nullptr) {
       const int64_t slots = resident_ctas(raw[1], threads);
-      if (slots > 0) {
+      // Persistent pays once each resident CTA walks two or more rows.
+      const bool forced = ((flags & NQ_FLAG_VARIANT_MASK) >> 24) == 3;
+      if (slots > 0 && (forced || grid >= 2 * slots)) {
         k = raw[1];
         grid = grid < slots ? grid : slots;
       }
