@@ -73,7 +73,7 @@ struct Schedule {
 // residual, in flight at once).  Few rows (M < 148, fewer than one per SM):
 // spread the row over up to 1024 threads with one or two chunks each, which
 // shortens the per-row critical path.  Every mapping gives identical bits.
-nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedule* s) {
+nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedule* s, bool raw = false) {
   const int64_t C = (d + 7) / 8;
   int lp = 0;
   while ((int64_t(1) << lp) < C) ++lp;
@@ -81,7 +81,7 @@ nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedu
   if (ft || fk) {
     if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
     const int lt = int(ft) + 4, lk = int(fk) - 1;
-    if (!nq::schedule_built(lt, lk))
+    if (!(raw ? nq::raw_schedule_built(lt, lk) : nq::schedule_built(lt, lk)))
       return fail(NQ_ERR_UNSUPPORTED, "%s: schedule of 2^%d threads x 2^%d chunks is not built", fn, lt, lk);
     if ((int64_t(1) << (lt + lk)) < C)
       return fail(NQ_ERR_INVALID_ARGUMENT, "%s: schedule covers %lld chunks, a row has %lld", fn,
@@ -199,14 +199,15 @@ int64_t resident_ctas(const void* k, int block) {
 // pass), and raw rows persistent (one CTA per resident slot, next row
 // prefetched).  NQ_FLAG_VARIANT forces one where it applies.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
+  const bool has_res = a.res_in != nullptr;
+  uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
+  const bool raw_forced = (variant == 2 || variant == 3) && vec && !has_res && op != nq::kOpRmsDynFp8;
   Schedule s;
-  nq_status st = plan_rows(fn, a.M, a.d, flags, &s);
+  nq_status st = plan_rows(fn, a.M, a.d, flags, &s, raw_forced);
   if (st != NQ_OK) return st;
   const int threads = 1 << s.log_t;
   const int rows = nq::rows_per_cta(threads);
   int64_t grid = (a.M + rows - 1) / rows;
-  const bool has_res = a.res_in != nullptr;
-  uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
   if (variant == 0 && !has_res) {
     // Automatic choice, from measurements on B200: static RMSNorm gains from
     // raw rows (fewer registers, more CTAs per SM) and, once every resident
@@ -217,7 +218,7 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
   }
   const void* k = nullptr;
-  if (vec && threads > 32 && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
+  if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
     const auto& raw = table_of(op).raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1] != nullptr) {
       const int64_t slots = resident_ctas(raw[1], threads);

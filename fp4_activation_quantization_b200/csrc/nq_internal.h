@@ -68,7 +68,12 @@ inline bool schedule_built(int log_t, int log_k) {
 // translation unit: [log_t - 5][log_k][mode], mode 0 = any alignment,
 // 1 = 16-byte rows, 2 = 16-byte rows with d == 8 * threads * chunks (t > 5).
 using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][3];
-using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][2];
+// Raw-row schedules: those of the direct kernel, plus one warp per row with 16
+// chunks per lane (t = 5, k = 4).
+inline bool raw_schedule_built(int log_t, int log_k) {
+  return schedule_built(log_t, log_k) || (log_t == 5 && log_k == 4);
+}
+using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
 struct RowKernels {
   KernelTable direct;  // one row per thread group
   RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent]

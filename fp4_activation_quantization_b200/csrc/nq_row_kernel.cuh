@@ -381,12 +381,28 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
 // CTA walks rows g, g + G, ... and loads the next row's raw chunks before it
 // processes the current one, so a load is always in flight; the static scale's
 // reciprocal is then computed once per CTA.
+// Register budget of the raw kernel: the raw row (4 registers per chunk, 8
+// when the next row is prefetched) plus ~48 working registers; the launch
+// bound asks ptxas to fit it, which stops it from hoisting every chunk's
+// gamma / beta loads at once (more CTAs per SM matter more here).
+template <int T, int K, bool PERSIST>
+constexpr int raw_min_blocks() {
+  constexpr int threads = (T == 32) ? 256 : T;
+  constexpr int cap = (PERSIST ? 8 * K : 4 * K) + 48;
+  constexpr int blocks = 65536 / (threads * (cap < 64 ? 64 : cap));
+  return blocks < 1 ? 1 : blocks;
+}
+
 template <int OP, int T, int K, bool PERSIST>
-__global__ void __launch_bounds__(T) row_kernel_raw(const RowArgs a) {
-  static_assert(T > 32 && OP != kOpRmsDynFp8, "raw rows: one row per CTA, no residual");
+__global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
+    row_kernel_raw(const RowArgs a) {
+  static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
+  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
   constexpr int W = T / 32;
-  __shared__ __align__(16) float s_sum[2][W * 32];
-  const int tid = int(threadIdx.x);
+  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
+  const int64_t n_groups = int64_t(gridDim.x) * R;
   const int d = a.d;
   const int C = d >> 3;
   const float fd = float(d);
@@ -406,6 +422,7 @@ __global__ void __launch_bounds__(T) row_kernel_raw(const RowArgs a) {
     }
   };
   auto process = [&](int64_t row, const uint4 (&xr)[K], float* b0, float* b1) {
+    const bool live = row < a.M;  // rows past M (warp rows only) compute on zeros and store nothing
     float part[K];
 #pragma unroll
     for (int k = 0; k < K; ++k) {
@@ -437,12 +454,12 @@ __global__ void __launch_bounds__(T) row_kernel_raw(const RowArgs a) {
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
-      const bool ok = c < C;
+      const bool ok = live && c < C;
       float2 v[4];
       unpack_pairs(xr[k], v);
       if constexpr (OP == kOpLnStaticFp8) {
         float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
-        if (ok) {
+        if (c < C) {
           const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
           g0 = __ldg(reinterpret_cast<const float4*>(gp));
           g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
@@ -457,7 +474,7 @@ __global__ void __launch_bounds__(T) row_kernel_raw(const RowArgs a) {
         for (int i = 0; i < 4; ++i) v[i] = fma2(mul2(add2(v[i], nm), rs2), g[i], b[i]);
       } else {
         uint4 gu = make_uint4(0u, 0u, 0u, 0u);
-        if (ok) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
+        if (c < C) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
         float2 g[4];
         unpack_pairs(gu, g);
 #pragma unroll
@@ -508,18 +525,18 @@ __global__ void __launch_bounds__(T) row_kernel_raw(const RowArgs a) {
 
   if constexpr (!PERSIST) {
     uint4 xr[K];
-    load(blockIdx.x, xr);
+    load(group, xr);
     griddep_launch_dependents();
-    process(blockIdx.x, xr, s_sum[0], s_sum[1]);
+    process(group, xr, s_sum[0], s_sum[1]);
   } else {
     // Reduction buffers are reused row after row: LayerNorm's two sums use
     // both buffers (each separated from its next use by the other sum's
     // barrier); single-sum operations alternate by row parity.
     uint4 xa[K], xb[K];
-    int64_t row = blockIdx.x;
+    int64_t row = group;
     load(row, xa);
     for (int parity = 0; row < a.M; parity ^= 1) {
-      const int64_t next = row + gridDim.x;
+      const int64_t next = row + n_groups;
       if (next >= a.M) griddep_launch_dependents();  // nothing left to load
       float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[parity];
       if (parity == 0) {
@@ -545,21 +562,25 @@ struct RowTable {
     for (auto& x : k.raw)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
+#define NQ_RAW(LT, LK)                                                                                         \
+  if constexpr (OP != kOpRmsDynFp8) {                                                                          \
+    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false>); \
+    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true>);  \
+  }
 #define NQ_DIRECT(LT, LK)                                                                                 \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0>); \
   k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1>); \
   if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2>); \
-  if constexpr (LT > 5 && OP != kOpRmsDynFp8) {                                                         \
-    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false>); \
-    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true>);  \
-  }
+  NQ_RAW(LT, LK)
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)
     NQ_DIRECT(7, 0) NQ_DIRECT(7, 1) NQ_DIRECT(7, 2) NQ_DIRECT(7, 3)
     NQ_DIRECT(8, 0) NQ_DIRECT(8, 1) NQ_DIRECT(8, 2) NQ_DIRECT(8, 3)
     NQ_DIRECT(9, 0) NQ_DIRECT(9, 1) NQ_DIRECT(9, 2)
     NQ_DIRECT(10, 0) NQ_DIRECT(10, 1)
+    NQ_RAW(5, 4)  // one warp per row, 16 chunks per lane (rows of up to 4096 elements)
 #undef NQ_DIRECT
+#undef NQ_RAW
   }
 };
 

@@ -105,8 +105,9 @@ typedef enum nq_status {
 /* Force a kernel variant (tests and tuning; same bits either way): n = 1 keeps
  * the row in float32 registers; n = 2 keeps only the raw bf16 row and unpacks
  * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row.
- * n = 2, 3 apply to 16-byte-aligned rows without a residual and more than 32
- * threads per row, and are ignored otherwise.  0 = automatic. */
+ * n = 2, 3 apply to 16-byte-aligned rows without a residual and are ignored
+ * otherwise; with them NQ_FLAG_SCHEDULE also accepts t = 5, k = 4 (one warp
+ * per row, 16 chunks per lane, rows of up to 4096 elements).  0 = automatic. */
 #define NQ_FLAG_VARIANT(n) ((((uint32_t)(n)) & 0x7u) << 24)
 #define NQ_FLAG_VARIANT_MASK (0x7u << 24)
 /* Library version (major * 10000 + minor * 100 + patch). */

@@ -413,6 +413,8 @@ def test_variants_without_residual_bit_exact(nq, d, M, ld):
     e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
     e_fp4 = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn, d=d)
     sch = [s for s in all_schedules(d) if s[0] > 5]
+    if (d + 7) // 8 <= 512:
+        sch.append((5, 4))  # one warp per row, 16 chunks per lane (raw variants only)
     for var in (2, 3):
         for sched in [None] + sch[:2] + sch[-1:]:
             f = nq.flag_variant(var) | (0 if sched is None else nq.flag_schedule(*sched))
