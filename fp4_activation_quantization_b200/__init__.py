@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
     "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND",
-    "flag_schedule", "flag_variant", "NQError", "lib", "library_path", "version",
+    "flag_schedule", "flag_group_schedule", "flag_variant", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4",
@@ -43,6 +43,11 @@ OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4 = 0, 1, 2, 3
 def flag_schedule(log2_threads: int, log2_chunks: int) -> int:
     """NQ_FLAG_SCHEDULE(t, k): force 2^t threads per row and 2^k chunks per thread."""
     return (((log2_threads - 4) & 0xF) << 16) | (((log2_chunks + 1) & 0x7) << 20)
+
+
+def flag_group_schedule(log2_lanes: int, log2_groups: int) -> int:
+    """NQ_FLAG_GROUP_SCHEDULE(t, k): 2^t lanes per group, 2^k groups per thread (group quantization)."""
+    return ((log2_lanes & 0xF) << 16) | (((log2_groups + 1) & 0x7) << 20)
 
 
 def flag_variant(n: int) -> int:

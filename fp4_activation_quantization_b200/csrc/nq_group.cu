@@ -7,19 +7,25 @@
 // per group, q = e4m3(RN(x * RN(1 / s))) (NQ_FLAG_SCALE_DIV: RN(x / s)).
 //
 // Mapping: the activations are a flat list of G = M * K / GROUP groups.  A
-// group is owned by GROUP / 8 consecutive lanes, one 16-byte chunk each, so a
-// warp reads two (GROUP = 128) or four (GROUP = 64) neighbouring groups as one
-// contiguous 512-byte span.  Each thread keeps U groups in flight; the group
-// absmax is an xor-butterfly max inside the lane group (exact, order-free).
+// group (GROUP / 8 chunks of 16 bytes) is owned by a team of TPG lanes; lane j
+// of the team takes chunks j, j + TPG, j + 2 TPG, ..., so at each load step a
+// team reads TPG consecutive chunks (TPG * 16 contiguous bytes, whole 32-byte
+// sectors for TPG >= 2) and a warp reads 32 / TPG such runs.  The group's
+// scale (a correctly rounded division and reciprocal) is paid once per lane
+// for GROUP / TPG elements, so small teams amortize it; the absmax is a max
+// over the lane's elements, then an xor-butterfly inside the team.  Each
+// thread handles U groups, all loads issued first.
 #include "nq_device.cuh"
 #include "nq_internal.h"
 
 namespace nq {
 
-template <int GROUP, int U, bool VEC>
+template <int GROUP, int TPG, int U, bool VEC>
 __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a) {
-  constexpr int TPG = GROUP / 8;                 // lanes per group
-  constexpr int SLOT = kGroupThreads / TPG;      // groups per CTA per unit
+  constexpr int CPG = GROUP / 8;             // chunks per group
+  constexpr int CPL = CPG / TPG;             // chunks per lane
+  constexpr int SLOT = kGroupThreads / TPG;  // groups per CTA per unit
+  static_assert(CPG % TPG == 0, "team size divides the group's chunks");
   const int lane_g = int(threadIdx.x) % TPG;
   const int slot = int(threadIdx.x) / TPG;
   const int64_t base = int64_t(blockIdx.x) * SLOT * U;
@@ -28,7 +34,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
 
   griddep_wait();
 
-  float v[U][8];
+  uint4 raw[U][CPL];
   int64_t row[U], cg[U];
   bool ok[U];
 #pragma unroll
@@ -37,14 +43,19 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
     ok[u] = g < a.G;
     row[u] = ok[u] ? g / a.groups_per_row : 0;
     cg[u] = ok[u] ? g - row[u] * a.groups_per_row : 0;
-    const uint16_t* src = a.x + row[u] * a.ld_x + cg[u] * GROUP + 8 * lane_g;
-    if constexpr (VEC) {
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (ok[u]) w = __ldcs(reinterpret_cast<const uint4*>(src));
-      unpack_bf16x8(w, v[u]);
-    } else {
+    const uint16_t* src = a.x + row[u] * a.ld_x + cg[u] * GROUP;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[u][j] = ok[u] ? bf16_to_f32(src[j]) : 0.0f;
+    for (int j = 0; j < CPL; ++j) {
+      const int c = lane_g + j * TPG;
+      if constexpr (VEC) {
+        raw[u][j] = ok[u] ? __ldcs(reinterpret_cast<const uint4*>(src + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] = ok[u] ? (uint32_t(src[8 * c + 2 * e]) | (uint32_t(src[8 * c + 2 * e + 1]) << 16)) : 0u;
+        raw[u][j] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
   }
   griddep_launch_dependents();
@@ -53,27 +64,49 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
   for (int u = 0; u < U; ++u) {
     float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[u][j]));
+    for (int j = 0; j < CPL; ++j) {
+      float v[8];
+      unpack_bf16x8(raw[u][j], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+    }
 #pragma unroll
     for (int o = TPG / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
     float s = __fdiv_rn(m, kE4M3Max);
     if (ue8m0) s = ue8m0_ceil(s);
     const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
-    float t[8];
+    const float2 inv2 = make_float2(inv, inv);
+    uint8_t* dst = a.q + row[u] * a.ld_q + cg[u] * GROUP;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) t[j] = (div && s != 0.0f) ? __fdiv_rn(v[u][j], s) : __fmul_rn(v[u][j], inv);
-    const uint32_t lo = pack_e4m3x4(t[0], t[1], t[2], t[3]);
-    const uint32_t hi = pack_e4m3x4(t[4], t[5], t[6], t[7]);
-    if (ok[u]) {
-      uint8_t* dst = a.q + row[u] * a.ld_q + cg[u] * GROUP + 8 * lane_g;
-      if constexpr (VEC) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
-      } else {
+    for (int j = 0; j < CPL; ++j) {
+      const int c = lane_g + j * TPG;
+      const uint4 w = raw[u][j];
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      float t[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dst[j] = uint8_t((j < 4 ? lo : hi) >> (8 * (j & 3)));
+      for (int e = 0; e < 4; ++e) {
+        const float2 x2 = make_float2(bf16_lo(ww[e]), bf16_hi(ww[e]));
+        if (div && s != 0.0f) {
+          t[2 * e] = __fdiv_rn(x2.x, s);
+          t[2 * e + 1] = __fdiv_rn(x2.y, s);
+        } else {
+          const float2 q2 = __fmul2_rn(x2, inv2);
+          t[2 * e] = q2.x;
+          t[2 * e + 1] = q2.y;
+        }
       }
-      if (lane_g == 0) a.s[row[u] * a.ld_s + cg[u]] = s;
+      const uint32_t lo = pack_e4m3x4(t[0], t[1], t[2], t[3]);
+      const uint32_t hi = pack_e4m3x4(t[4], t[5], t[6], t[7]);
+      if (ok[u]) {
+        if constexpr (VEC) {
+          *reinterpret_cast<uint2*>(dst + 8 * c) = make_uint2(lo, hi);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dst[8 * c + e] = uint8_t((e < 4 ? lo : hi) >> (8 * (e & 3)));
+        }
+      }
     }
+    if (ok[u] && lane_g == 0) a.s[row[u] * a.ld_s + cg[u]] = s;
   }
 }
 
@@ -81,14 +114,22 @@ namespace {
 struct GroupTableHolder {
   GroupTable t;
   GroupTableHolder() {
-    t[0][0][0] = reinterpret_cast<const void*>(&group_kernel<64, 1, false>);
-    t[0][0][1] = reinterpret_cast<const void*>(&group_kernel<64, 1, true>);
-    t[0][1][0] = reinterpret_cast<const void*>(&group_kernel<64, 4, false>);
-    t[0][1][1] = reinterpret_cast<const void*>(&group_kernel<64, 4, true>);
-    t[1][0][0] = reinterpret_cast<const void*>(&group_kernel<128, 1, false>);
-    t[1][0][1] = reinterpret_cast<const void*>(&group_kernel<128, 1, true>);
-    t[1][1][0] = reinterpret_cast<const void*>(&group_kernel<128, 4, false>);
-    t[1][1][1] = reinterpret_cast<const void*>(&group_kernel<128, 4, true>);
+    for (auto& x : t)
+      for (auto& y : x)
+        for (auto& z : y)
+          for (auto& w : z) w = nullptr;
+#define NQ_GROUP(GI, G, TI, TPG, UI, U)                                                  \
+  t[GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false>); \
+  t[GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true>);
+    // group 64 (8 chunks): teams of 2, 4, 8 lanes; group 128 (16 chunks): 2, 4, 8, 16
+    NQ_GROUP(0, 64, 0, 2, 0, 1) NQ_GROUP(0, 64, 0, 2, 1, 2) NQ_GROUP(0, 64, 0, 2, 2, 4)
+    NQ_GROUP(0, 64, 1, 4, 0, 1) NQ_GROUP(0, 64, 1, 4, 1, 2) NQ_GROUP(0, 64, 1, 4, 2, 4)
+    NQ_GROUP(0, 64, 2, 8, 0, 1) NQ_GROUP(0, 64, 2, 8, 1, 2) NQ_GROUP(0, 64, 2, 8, 2, 4)
+    NQ_GROUP(1, 128, 0, 2, 0, 1) NQ_GROUP(1, 128, 0, 2, 1, 2) NQ_GROUP(1, 128, 0, 2, 2, 4)
+    NQ_GROUP(1, 128, 1, 4, 0, 1) NQ_GROUP(1, 128, 1, 4, 1, 2) NQ_GROUP(1, 128, 1, 4, 2, 4)
+    NQ_GROUP(1, 128, 2, 8, 0, 1) NQ_GROUP(1, 128, 2, 8, 1, 2) NQ_GROUP(1, 128, 2, 8, 2, 4)
+    NQ_GROUP(1, 128, 3, 16, 0, 1) NQ_GROUP(1, 128, 3, 16, 1, 2) NQ_GROUP(1, 128, 3, 16, 2, 4)
+#undef NQ_GROUP
   }
 };
 }  // namespace

@@ -428,8 +428,10 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
                                        float* scales_out, int64_t ld_s, int64_t M, int64_t K,
                                        int32_t group, uint32_t flags, nq_stream_t stream) {
   const char* fn = "nq_per_token_group_quant_fp8";
-  nq_status st = check_flags(fn, flags, true, false, false);
+  nq_status st = check_flags(fn, flags, true, true, false);
   if (st != NQ_OK) return st;
+  if (flags & NQ_FLAG_VARIANT_MASK)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT applies to the norm calls only", fn);
   NQ_REQUIRE(M >= 0 && K >= 1, "%s: need M >= 0 and K >= 1", fn);
   if (group != 64 && group != 128) return fail(NQ_ERR_UNSUPPORTED, "%s: group %d not in {64, 128}", fn, group);
   NQ_REQUIRE(K % group == 0, "%s: K = %lld is not a multiple of group %d", fn, (long long)K, group);
@@ -447,13 +449,24 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   a.G = M * (K / group);
   a.flags = kernel_flags(flags, /*default_div=*/false);
   const bool vec = vec_bf16(x, ld_x) && aligned(q_out, 8) && ld_q % 8 == 0;
-  const int slot = nq::kGroupThreads / (group / 8);
-  // Four groups in flight per thread once there are enough groups to give
-  // every SM several CTAs that way; otherwise one, for more CTAs.
-  const int units = a.G >= int64_t(148) * slot * 4 * 2 ? 4 : 1;
+  // Team of 2^t lanes per group, 2^u groups per thread.  Many groups: teams
+  // of two lanes (each lane pays the group's scale once for 64 elements and
+  // a team still reads whole 32-byte sectors).  Few groups: 16 lanes per group
+  // for the shortest per-group latency.  NQ_FLAG_GROUP_SCHEDULE(t, u) forces it.
+  int lt = a.G >= int64_t(148) * 256 ? 1 : (group == 128 ? 4 : 3), lu = 0;
+  const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
+  if (ft || fk) {
+    if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
+    lt = int(ft);  // NQ_FLAG_GROUP_SCHEDULE stores t itself
+    lu = int(fk) - 1;
+    if (lt < 1 || lt > (group == 128 ? 4 : 3) || lu < 0 || lu > 2)
+      return fail(NQ_ERR_UNSUPPORTED, "%s: 2^%d lanes per group x 2^%d groups per thread is not built", fn, lt, lu);
+  }
+  const int tpg = 1 << lt, units = 1 << lu;
+  const int slot = nq::kGroupThreads / tpg;
   const int64_t grid = (a.G + int64_t(slot) * units - 1) / (int64_t(slot) * units);
   if (grid > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: too many groups", fn);
-  const void* k = nq::group_kernels()[group == 128 ? 1 : 0][units == 4 ? 1 : 0][vec ? 1 : 0];
+  const void* k = nq::group_kernels()[group == 128 ? 1 : 0][lt - 1][lu][vec ? 1 : 0];
   void* args[] = {&a};
   return launch(fn, k, unsigned(grid), nq::kGroupThreads, 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }

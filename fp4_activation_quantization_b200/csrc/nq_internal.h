@@ -83,8 +83,8 @@ const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();
 const RowKernels& row_kernels_rms_nvfp4();
 
-// Group kernel: [group == 128][units per thread: 0 -> 1, 1 -> 4][vec]
-using GroupTable = const void* [2][2][2];
+// Group kernel: [group == 128][log2(lanes per group) - 1][log2(groups per thread)][vec]
+using GroupTable = const void* [2][4][3][2];
 const GroupTable& group_kernels();
 constexpr int kGroupThreads = 256;
 

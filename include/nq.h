@@ -102,6 +102,9 @@ typedef enum nq_status {
  * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
+/* Group quantization's schedule (same bit field): 2^t lanes per group, 2^k
+ * groups per thread; see nq_per_token_group_quant_fp8. */
+#define NQ_FLAG_GROUP_SCHEDULE(t, k) ((((uint32_t)(t)) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 /* Force a kernel variant (tests and tuning; same bits either way): n = 1 keeps
  * the row in float32 registers; n = 2 keeps only the raw bf16 row and unpacks
  * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row.
@@ -182,7 +185,9 @@ nq_status nq_layernorm_quant_fp8(const void* x, int64_t ld_x, const float* gamma
  *   s = RN(absmax / 448), or with NQ_FLAG_UE8M0 the smallest power of two
  *   >= s (a zero group gives 2^-127).  group in {64, 128}; K % group == 0.
  * Default quantization: NQ_FLAG_SCALE_RECIP; a zero fp32 scale stores the
- * signed zeros of x.
+ * signed zeros of x.  NQ_FLAG_GROUP_SCHEDULE(t, k) forces the mapping (tests
+ * and tuning; same bits): 2^t lanes per group (t = 1..4 for group 128, 1..3
+ * for group 64) and 2^k groups per thread (k = 0..2).
  */
 nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out, int64_t ld_q,
                                        float* scales_out, int64_t ld_s, int64_t M, int64_t K,

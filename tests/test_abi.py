@@ -91,7 +91,9 @@ def test_validation_without_gpu(nq):
     assert L.nq_per_token_group_quant_fp8(FAKE, 200, FAKE, 200, FAKE, 2, 4, 200, 128, 0, None) == INV
     assert L.nq_per_token_group_quant_fp8(FAKE, 96, FAKE, 96, FAKE, 3, 4, 96, 32, 0, None) == UNS
     assert L.nq_per_token_group_quant_fp8(FAKE, 256, FAKE, 256, FAKE, 2, 4, 256, 128,
-                                          nq.flag_schedule(5, 0), None) == INV
+                                          nq.flag_group_schedule(5, 0), None) == UNS
+    assert L.nq_per_token_group_quant_fp8(FAKE, 256, FAKE, 256, FAKE, 2, 4, 256, 128,
+                                          nq.flag_variant(2), None) == INV
     assert L.nq_per_token_group_quant_fp8(None, 256, None, 256, None, 2, 0, 256, 128, 0, None) == nq.NQ_OK
     # LayerNorm rejects the bf16 double-rounding flag only when there is no norm: it has one, so fine;
     # it rejects UE8M0

@@ -305,6 +305,21 @@ def test_group_variants_and_strides(nq, group, flags_name):
         assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32)), off
 
 
+@pytest.mark.parametrize("group", [64, 128])
+def test_group_every_team_size(nq, group):
+    """Every built (lanes per group, groups per thread) mapping gives the oracle's bits."""
+    M, K = 333, 2048
+    w = S.make_group_inputs(M, K, seed=group + 11)
+    x = dev_bf16(w["x"])
+    for flags, of in ((0, 0), (nq.FLAG_UE8M0, oracle.UE8M0), (nq.FLAG_SCALE_DIV, oracle.DIV)):
+        eq, es = oracle.per_token_group_quant_fp8(w["x"], group, of)
+        for lt in range(1, (5 if group == 128 else 4)):
+            for lu in range(0, 3):
+                q, s = nq.nq_per_token_group_quant_fp8(x, group, flags=flags | nq.flag_group_schedule(lt, lu))
+                assert np.array_equal(host_u8(q), eq), (flags, lt, lu)
+                assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32)), (flags, lt, lu)
+
+
 def test_group_cvt_over_all_bf16_values(nq):
     """Groups whose absmax is 448 have scale 1, so their codes are the hardware
     e4m3 conversion of every finite bf16 value in [-448, 448]: compare with the oracle."""
