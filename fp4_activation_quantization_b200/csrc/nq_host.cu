@@ -450,10 +450,11 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   a.flags = kernel_flags(flags, /*default_div=*/false);
   const bool vec = vec_bf16(x, ld_x) && aligned(q_out, 8) && ld_q % 8 == 0;
   // Team of 2^t lanes per group, 2^u groups per thread.  Many groups: teams
-  // of two lanes (each lane pays the group's scale once for 64 elements and
-  // a team still reads whole 32-byte sectors).  Few groups: 16 lanes per group
-  // for the shortest per-group latency.  NQ_FLAG_GROUP_SCHEDULE(t, u) forces it.
-  int lt = a.G >= int64_t(148) * 256 ? 1 : (group == 128 ? 4 : 3), lu = 0;
+  // of four lanes, one group per thread (measured best on B200: each lane pays
+  // the group's scale once per 32 elements, a team reads 64 contiguous bytes,
+  // 56 registers).  Few groups: a lane per chunk for the shortest latency.
+  // NQ_FLAG_GROUP_SCHEDULE(t, u) forces it.
+  int lt = a.G >= int64_t(148) * 64 ? 2 : (group == 128 ? 4 : 3), lu = 0;
   const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
   if (ft || fk) {
     if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
