@@ -73,6 +73,9 @@ def _load():
                     ([P, I64, P, P, F, P, I64, I64, I64, F, U32], ctypes.c_int),
                 "oracle_per_token_group_quant_fp8":
                     ([P, I64, P, I64, P, I64, I64, I64, ctypes.c_int32, U32], ctypes.c_int),
+                "oracle_rmsnorm_quant_fp8_group":
+                    ([P, I64, P, P, I64, P, P, I64, P, I64, P, I64, I64, I64, ctypes.c_int32, F, U32],
+                     ctypes.c_int),
                 "oracle_rmsnorm_quant_nvfp4":
                     ([P, I64, P, P, I64, P, F, P, I64, P, I64, P, I64, I64, I64, F, U32],
                      ctypes.c_int),
@@ -251,6 +254,29 @@ def per_token_group_quant_fp8(x, group=128, flags=0):
                                                   group, flags)
     assert rc == 0
     return q, s
+
+
+def rmsnorm_quant_fp8_group(x, gamma, residual=None, group=128, eps=1e-6, flags=0, d=None,
+                            want_norm=False):
+    """RMSNorm (optional residual) + per-token-group e4m3 of y.
+
+    Returns ``(q uint8 [M, d], scales float32 [M, d/group], residual_out or
+    None, norm_out or None)``.
+    """
+    x = _c(x, np.uint16)
+    M = x.shape[0]
+    d = x.shape[1] if d is None else d
+    res = None if residual is None else _c(residual, np.uint16)
+    g = _c(gamma, np.uint16)
+    q = np.empty((M, d), np.uint8)
+    s = np.empty((M, d // group), np.float32)
+    ro = None if res is None else np.empty((M, d), np.uint16)
+    no = np.empty((M, d), np.uint16) if want_norm else None
+    rc = _load().oracle_rmsnorm_quant_fp8_group(
+        _p(x), _ld(x), _p(res), _p(ro), d, _p(g), _p(q), d, _p(s), d // group, _p(no), d, M, d, group,
+        eps, flags)
+    assert rc == 0
+    return q, s, ro, no
 
 
 def rmsnorm_quant_nvfp4(x, gamma, global_scale, residual=None, eps=1e-6, flags=0, d=None,

@@ -383,6 +383,43 @@ int oracle_per_token_group_quant_fp8(const uint16_t* x, int64_t ld_x, uint8_t* q
   return 0;
 }
 
+// RMSNorm (optional residual) + per-token-group e4m3 ([P4] Details: the fused
+// RMSNorm + group-quant path multiplies by the group scale's reciprocal, the
+// same numerics as the standalone group quantizer): y as in the other RMSNorm
+// calls, then per group of `group` consecutive y values s = RN(absmax / 448)
+// (UE8M0: next power of two), q = e4m3(RN(y * RN(1 / s))) (OR_DIV: RN(y / s));
+// a zero fp32 group scale stores the signed zeros of y.
+int oracle_rmsnorm_quant_fp8_group(const uint16_t* x, int64_t ld_x, const uint16_t* res_in,
+                                   uint16_t* res_out, int64_t ld_res, const uint16_t* gamma,
+                                   uint8_t* q, int64_t ld_q, float* scales, int64_t ld_s,
+                                   uint16_t* norm_out, int64_t ld_norm, int64_t M, int64_t d,
+                                   int32_t group, float eps, uint32_t flags) {
+  if (group <= 0 || d % group) return 1;
+  const bool div = use_div(flags, false);
+  const bool ue8m0 = (flags & OR_UE8M0) != 0;
+  std::vector<float> r, y;
+  for (int64_t m = 0; m < M; ++m) {
+    rms_row(x + m * ld_x, res_in ? res_in + m * ld_res : nullptr,
+            res_out ? res_out + m * ld_res : nullptr, gamma, d, eps, flags, r, y);
+    if (norm_out)
+      for (int64_t i = 0; i < d; ++i) norm_out[m * ld_norm + i] = f32_to_bf16(y[size_t(i)]);
+    for (int64_t g = 0; g < d / group; ++g) {
+      const float* ys = y.data() + g * group;
+      float amax = 0.0f;
+      for (int32_t i = 0; i < group; ++i) amax = std::fmax(amax, std::fabs(ys[i]));
+      float s = amax / kE4M3Max;
+      if (ue8m0) s = ue8m0_ceil(s);
+      scales[m * ld_s + g] = s;
+      const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
+      for (int32_t i = 0; i < group; ++i) {
+        float t = (s == 0.0f) ? ys[i] : (div ? ys[i] / s : ys[i] * inv);
+        q[m * ld_q + g * group + i] = e4m3_encode(t);
+      }
+    }
+  }
+  return 0;
+}
+
 // RMSNorm (optional residual) + NVFP4 ([P3] Description and commit notes):
 // per block of 16 consecutive elements, sf = e4m3(RN(RN(amax / 6) / g)),
 // element multiplier m = RN(1 / RN(dec(sf) * g)) (0 when that product is 0),

@@ -299,3 +299,56 @@ def test_static_zero_scale_is_ieee():
     q, _, _ = oracle.rmsnorm_quant_fp8_static(x, bf([1.0, 1.0, 0.0, 1.0]), 0.0, eps=1e-6)
     assert q[0, 0] == 0x7E and q[0, 1] == 0xFE and q[0, 3] == 0x7E
     assert q[0, 2] & 0x7F == 0x7F
+
+
+# ------------------------------------------- fused RMSNorm + group FP8 ----
+def test_golden_rms_group():
+    c = json.load(open(os.path.join(GOLDEN, "rows.json")))["rms_group"][0]
+    d = c["d"]
+    gamma = np.zeros(d, np.float32)
+    gamma[: len(c["gamma_head"])] = c["gamma_head"]
+    gamma[128] = c["gamma_at_128"]
+    x = bf(np.ones((1, d)))
+    for flags in (0, oracle.RECIP, oracle.DIV):
+        q, s, _, _ = oracle.rmsnorm_quant_fp8_group(x, bf(gamma), eps=c["eps"], flags=flags)
+        assert s[0, 0] == np.float32(c["scales"][0])
+        assert s[0, 1] == np.float32(c["gamma_at_128"]) / np.float32(448)
+        assert list(q[0, :4]) == c["codes_head"], c["why"]
+        assert q[0, 128] == c["code_at_128"]
+        assert not q[0, 4:128].any() and not q[0, 129:].any()
+
+
+@pytest.mark.parametrize("flags", [0, oracle.UE8M0, oracle.DIV])
+@pytest.mark.parametrize("residual", [False, True])
+def test_rms_group_composes_pinned_pieces(flags, residual):
+    """The fused result equals the pinned pieces composed in numpy: y from the
+    RMSNorm pin, per-group s = RN(absmax / 448) (or its UE8M0 ceil), the pinned
+    e4m3 encoder of RN(y * RN(1 / s)) (or RN(y / s))."""
+    M, d, G = 24, 1024, 128
+    w = S.make_rms_inputs(M, d, seed=3, residual=residual, x_outlier_channels=True)
+    q, s, ro, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"], w.get("residual"), flags=flags)
+    y = oracle.rms_y(w["x"], w["gamma"], w.get("residual"))
+    yg = y.reshape(M, d // G, G)
+    es = (np.abs(yg).max(axis=2) / np.float32(448)).astype(np.float32)
+    if flags & oracle.UE8M0:
+        es = oracle.ue8m0_ceil(es)
+    assert np.array_equal(s, es)
+    if flags & oracle.DIV:
+        t = (yg / es[..., None]).astype(np.float32)
+    else:
+        inv = np.where(es == 0, np.float32(0), np.float32(1) / es).astype(np.float32)
+        t = (yg * inv[..., None]).astype(np.float32)
+    assert np.array_equal(q, oracle.e4m3_encode(t).reshape(M, d))
+    if residual:
+        _, _, er, _ = oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"])
+        assert np.array_equal(ro, er)
+
+
+def test_rms_group_fused_vs_unfused():
+    """Quantizing fp32 y vs bf16-rounded y: a few percent of codes move by one ulp."""
+    w = S.make_rms_inputs(128, 4096, seed=4)
+    qf, sf_, _, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"], w["residual"])
+    qu, su, _, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"], w["residual"], flags=oracle.NORM_BF16_ROUND)
+    frac = (qf != qu).mean()
+    assert 0.01 <= frac <= 0.05
+    assert np.abs(e4m3_rank(qf) - e4m3_rank(qu)).max() <= 1
