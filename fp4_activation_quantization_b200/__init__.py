@@ -12,7 +12,8 @@ use, and that use raises ImportError when it has not been built
 Functions carry the C names:
 ``nq_fused_add_rmsnorm_quant_fp8``, ``nq_rmsnorm_quant_fp8_static``,
 ``nq_layernorm_quant_fp8``, ``nq_per_token_group_quant_fp8``,
-``nq_rmsnorm_quant_nvfp4``; plus ``nq_query_schedule``.
+``nq_rmsnorm_quant_nvfp4``, ``nq_rmsnorm_quant_fp8_group``; plus
+``nq_query_schedule``.
 """
 from __future__ import annotations
 
@@ -27,7 +28,8 @@ __all__ = [
     "flag_schedule", "flag_group_schedule", "flag_variant", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
-    "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4",
+    "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4", "OP_RMS_GROUP_FP8",
+    "nq_rmsnorm_quant_fp8_group",
 ]
 
 NQ_OK, NQ_ERR_INVALID_ARGUMENT, NQ_ERR_UNSUPPORTED, NQ_ERR_CUDA = 0, 1, 2, 3
@@ -37,7 +39,7 @@ FLAG_SCALE_DIV = 1 << 1
 FLAG_SCALE_RECIP = 1 << 2
 FLAG_UE8M0 = 1 << 3
 FLAG_NORM_BF16_ROUND = 1 << 4
-OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4 = 0, 1, 2, 3
+OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4, OP_RMS_GROUP_FP8 = 0, 1, 2, 3, 4
 
 
 def flag_schedule(log2_threads: int, log2_chunks: int) -> int:
@@ -81,9 +83,10 @@ def _load() -> ctypes.CDLL:
     L.nq_rmsnorm_quant_fp8_static.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, I64, I64, F, U32, P]
     L.nq_layernorm_quant_fp8.argtypes = [P, I64, P, P, P, P, I64, I64, I64, F, U32, P]
     L.nq_per_token_group_quant_fp8.argtypes = [P, I64, P, I64, P, I64, I64, I64, I32, U32, P]
+    L.nq_rmsnorm_quant_fp8_group.argtypes = [P, I64, P, P, I64, P, P, I64, P, I64, P, I64, I64, I64, I32, F, U32, P]
     L.nq_rmsnorm_quant_nvfp4.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, P, I64, I64, I64, F, U32, P]
     for name in ("nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
-                 "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4"):
+                 "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_rmsnorm_quant_fp8_group"):
         getattr(L, name).restype = st
     return L
 
@@ -279,6 +282,42 @@ def nq_per_token_group_quant_fp8(x, group: int = 128, *, q_out=None, scales_out=
         _check(_get_lib().nq_per_token_group_quant_fp8(_ptr(x), ld_x, _ptr(q_out), ld_q, _ptr(scales_out), ld_s, M, K,
                                                 group, flags, _stream(stream)), "nq_per_token_group_quant_fp8")
     return q_out, scales_out
+
+
+def nq_rmsnorm_quant_fp8_group(x, gamma, eps: float = 1e-6, *, group: int = 128, residual=None,
+                               residual_out=None, q_out=None, scales_out=None, norm_out=None,
+                               want_norm: bool = False, flags: int = 0, stream=None):
+    """RMSNorm (optional residual-add) + per-token-group e4m3 of y.
+
+    Returns ``(q float8_e4m3fn [M, d], scales float32 [M, d/group], residual_out
+    or None, norm_out or None)``.
+    """
+    M, d, ld_x = _rows(x, "x", torch.bfloat16)
+    _need(group > 0 and d % group == 0, f"d = {d} must be a multiple of group = {group}")
+    _vec(gamma, "gamma", torch.bfloat16, d)
+    ld_r = d
+    if residual is not None:
+        _, _, ld_r = _rows(residual, "residual", torch.bfloat16, d)
+        _need(residual.shape[0] == M, "residual must have M rows")
+        residual_out = _out(residual_out, (M, d), torch.bfloat16, x, "residual_out")
+        _need(_rows(residual_out, "residual_out", torch.bfloat16, d)[2] == ld_r,
+              "residual_out must have the row stride of residual")
+    else:
+        _need(residual_out is None, "residual_out needs residual")
+    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    scales_out = _out(scales_out, (M, d // group), torch.float32, x, "scales_out")
+    _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, d // group)
+    if want_norm and norm_out is None:
+        norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
+    _same_device(x, gamma, residual, residual_out, q_out, scales_out, norm_out)
+    with torch.cuda.device(x.device):
+        _check(_get_lib().nq_rmsnorm_quant_fp8_group(
+            _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(q_out), ld_q,
+            _ptr(scales_out), ld_s, _ptr(norm_out), ld_n, M, d, group, eps, flags, _stream(stream)),
+            "nq_rmsnorm_quant_fp8_group")
+    return q_out, scales_out, residual_out, norm_out
 
 
 def nq_rmsnorm_quant_nvfp4(x, gamma, global_scale, eps: float = 1e-6, *, residual=None, residual_out=None,

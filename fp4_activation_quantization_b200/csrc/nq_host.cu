@@ -147,6 +147,7 @@ const nq::RowKernels& table_of(int op) {
     case nq::kOpRmsDynFp8: return nq::row_kernels_rms_dyn();
     case nq::kOpRmsStaticFp8: return nq::row_kernels_rms_static();
     case nq::kOpLnStaticFp8: return nq::row_kernels_ln_static();
+    case nq::kOpRmsGroupFp8: return nq::row_kernels_rms_group();
     default: return nq::row_kernels_rms_nvfp4();
   }
 }
@@ -422,6 +423,48 @@ nq_status nq_rmsnorm_quant_nvfp4(const void* x, int64_t ld_x, const void* residu
   const bool vec = vec_bf16(x, ld_x) && vec_bf16(residual_in, ld_res) && vec_bf16(residual_out, ld_res) &&
                    aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) && aligned(q_out, 4) && ld_q % 4 == 0;
   return run_rows(fn, nq::kOpRmsNvfp4, a, vec, flags, stream);
+}
+
+nq_status nq_rmsnorm_quant_fp8_group(const void* x, int64_t ld_x, const void* residual_in,
+                                     void* residual_out, int64_t ld_res, const void* gamma, void* q_out,
+                                     int64_t ld_q, float* scales_out, int64_t ld_s, void* norm_out,
+                                     int64_t ld_norm, int64_t M, int64_t d, int32_t group, float eps,
+                                     uint32_t flags, nq_stream_t stream) {
+  const char* fn = "nq_rmsnorm_quant_fp8_group";
+  nq_status st = check_common(fn, M, d, eps);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, true, true, true)) != NQ_OK) return st;
+  if (group != 64 && group != 128) return fail(NQ_ERR_UNSUPPORTED, "%s: group %d not in {64, 128}", fn, group);
+  NQ_REQUIRE(d % group == 0, "%s: d = %lld is not a multiple of group %d", fn, (long long)d, group);
+  NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
+             "%s: residual_in and residual_out must both be given or both be NULL", fn);
+  NQ_REQUIRE(ld_x >= d && ld_q >= d && ld_s >= d / group && (!residual_in || ld_res >= d) &&
+                 (!norm_out || ld_norm >= d),
+             "%s: row strides too small", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && gamma && q_out && scales_out, "%s: x, gamma, q_out and scales_out are required", fn);
+  RowArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.res_in = static_cast<const uint16_t*>(residual_in);
+  a.res_out = static_cast<uint16_t*>(residual_out);
+  a.ld_res = ld_res;
+  a.gamma = gamma;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.scale_out = scales_out;
+  a.ld_scale = ld_s;
+  a.group = group;
+  a.norm_out = static_cast<uint16_t*>(norm_out);
+  a.ld_norm = ld_norm;
+  a.M = M;
+  a.d = int32_t(d);
+  a.eps = eps;
+  a.flags = kernel_flags(flags, /*default_div=*/false);
+  const bool vec = d % 8 == 0 && vec_bf16(x, ld_x) && vec_bf16(residual_in, ld_res) &&
+                   vec_bf16(residual_out, ld_res) && aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) &&
+                   aligned(q_out, 8) && ld_q % 8 == 0;
+  return run_rows(fn, nq::kOpRmsGroupFp8, a, vec, flags, stream);
 }
 
 nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out, int64_t ld_q,

@@ -12,7 +12,8 @@ enum RowOp : int {
   kOpRmsStaticFp8 = 1,  // RMSNorm (+residual) + static-scale e4m3
   kOpLnStaticFp8 = 2,   // LayerNorm + static-scale e4m3
   kOpRmsNvfp4 = 3,      // RMSNorm (+residual) + NVFP4
-  kNumRowOps = 4
+  kOpRmsGroupFp8 = 4,   // RMSNorm (+residual) + per-token-group e4m3
+  kNumRowOps = 5
 };
 
 // Kernel-side flag bits (the public NQ_FLAG_* values, repeated for the
@@ -32,7 +33,9 @@ struct RowArgs {
   const float* scale;  // device scalar: static scale or NVFP4 global scale
   uint8_t* q;          // e4m3 [M, ld_q] or packed e2m1 [M, ld_q]
   int64_t ld_q;
-  float* scale_out;  // float [M] (dynamic per-token)
+  float* scale_out;  // float [M] (dynamic per-token) or [M, ld_scale] (group scales)
+  int64_t ld_scale;
+  int32_t group;     // 64 or 128 (group op)
   uint8_t* sf;       // e4m3 block scales [M, ld_sf] (NVFP4)
   int64_t ld_sf;
   uint16_t* norm_out;  // bf16 [M, ld_norm] or null
@@ -82,6 +85,7 @@ const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();
 const RowKernels& row_kernels_rms_nvfp4();
+const RowKernels& row_kernels_rms_group();
 
 // Group kernel: [group == 128][log2(lanes per group) - 1][log2(groups per thread)][vec]
 using GroupTable = const void* [2][4][3][2];

@@ -106,6 +106,49 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
   }
 }
 
+// Per-token-group e4m3 of a row's y (chunk c of the row in v[k] for c = tid +
+// k*T): a group of G elements is G/8 consecutive chunks, held by G/8
+// consecutive threads of the group (T >= 32 and a multiple of G/8), so its
+// absmax is an xor-butterfly over those lanes; then s = RN(absmax / 448)
+// (UE8M0: next power of two), one reciprocal, q = e4m3(RN(y * RN(1 / s))).
+template <int T, int K, bool VEC, bool FULL>
+__device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
+                                                const float2 (&v)[K][4]) {
+  const int d = a.d;
+  const int C = FULL ? T * K : (d + 7) >> 3;
+  const int cpg = a.group >> 3;  // chunks per group
+  const bool div = (a.flags & kFlagDiv) != 0;
+  const bool ue8m0 = (a.flags & kFlagUe8m0) != 0;
+  uint8_t* qrow = a.q + row * a.ld_q;
+  float* srow = a.scale_out + row * a.ld_scale;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
+    for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+    float s = __fdiv_rn(m, kE4M3Max);
+    if (ue8m0) s = ue8m0_ceil(s);
+    const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+    float2 t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      t[i] = (div && s != 0.0f) ? make_float2(__fdiv_rn(v[k][i].x, s), __fdiv_rn(v[k][i].y, s))
+                                : mul2(v[k][i], f2(inv));
+    const uint2 codes = pack_pairs_e4m3(t);
+    if (FULL || (live && c < C)) {
+      if constexpr (VEC) {
+        *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qrow[8 * c + j] = uint8_t((j < 4 ? codes.x : codes.y) >> (8 * (j & 3)));
+      }
+      if ((c & (cpg - 1)) == 0) srow[c / cpg] = s;
+    }
+  }
+}
+
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.
@@ -295,6 +338,8 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
         if ((c & 1) == 0) sfrow[c >> 1] = uint8_t(sfc);
       }
     }
+  } else if constexpr (OP == kOpRmsGroupFp8) {
+    quantize_groups<T, K, VEC, FULL>(a, row, live, tid, v);
   } else {
     float s_div, s_inv;
     bool passthrough = false;
@@ -410,7 +455,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
 
   griddep_wait();
-  const float scale_in = __ldg(a.scale);
+  const float scale_in = (OP == kOpRmsGroupFp8) ? 1.0f : __ldg(a.scale);
   const float inv_static = __frcp_rn(scale_in);
 
   auto load = [&](int64_t row, uint4 (&xr)[K]) {
@@ -512,6 +557,24 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
         if (ok) {
           *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
           if ((c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
+        }
+      } else if constexpr (OP == kOpRmsGroupFp8) {
+        // the group's chunks are consecutive lanes (see quantize_groups)
+        const int cpg = a.group >> 3;
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+        for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+        float sg = __fdiv_rn(m, kE4M3Max);
+        if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
+        const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
+        float2 t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          t[i] = (div && sg != 0.0f) ? make_float2(__fdiv_rn(v[i].x, sg), __fdiv_rn(v[i].y, sg)) : mul2(v[i], f2(ig));
+        if (ok) {
+          *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_e4m3(t);
+          if ((c & (cpg - 1)) == 0) a.scale_out[row * a.ld_scale + c / cpg] = sg;
         }
       } else {
         float2 t[4];

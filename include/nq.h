@@ -6,7 +6,8 @@
  * residual, normalizes (RMSNorm or LayerNorm) in float32 registers and
  * quantizes the float32 result once, to e4m3 (FP8) or to NVFP4 (packed e2m1 +
  * e4m3 block scales).  A fifth call quantizes raw bf16 activations per group
- * of 128 (or 64) elements.
+ * of 128 (or 64) elements, and a sixth fuses RMSNorm with that group
+ * quantization.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -123,8 +124,8 @@ const char* nq_last_error(void);
 /*
  * Schedule the planner picks for a norm call (op: 0 = fused add+RMSNorm+
  * dynamic FP8, 1 = RMSNorm static FP8, 2 = LayerNorm static FP8, 3 = RMSNorm
- * NVFP4) at (M, d, flags): threads per row, 16-byte chunks per thread and rows
- * per CTA.  Pure host function; launches nothing.
+ * NVFP4, 4 = RMSNorm group FP8) at (M, d, flags): threads per row, 16-byte
+ * chunks per thread and rows per CTA.  Pure host function; launches nothing.
  */
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
                             int* chunks_per_thread, int* rows_per_cta);
@@ -192,6 +193,24 @@ nq_status nq_layernorm_quant_fp8(const void* x, int64_t ld_x, const float* gamma
 nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out, int64_t ld_q,
                                        float* scales_out, int64_t ld_s, int64_t M, int64_t K,
                                        int32_t group, uint32_t flags, nq_stream_t stream);
+
+/*
+ * RMSNorm (residual-add optional) + per-token-group e4m3 of y, for block-FP8
+ * GEMMs ("per_token_group_quant_8bit: multiply by reciprocal instead of
+ * dividing per element": Details, the fused RMSNorm + group-quant path).
+ *   x bf16 [M, ld_x]; residual_in / residual_out both NULL or both given;
+ *   gamma bf16 [d]; q_out e4m3 [M, ld_q]; scales_out float32 [M, ld_s],
+ *   d / group per row: s = RN(absmax(y over the group) / 448), or with
+ *   NQ_FLAG_UE8M0 the smallest power of two >= s; norm_out bf16 or NULL.
+ *   group in {64, 128}; d % group == 0.
+ * Default quantization: NQ_FLAG_SCALE_RECIP (y * RN(1 / s)), as the standalone
+ * group call; a zero fp32 scale stores the signed zeros of y.
+ */
+nq_status nq_rmsnorm_quant_fp8_group(const void* x, int64_t ld_x, const void* residual_in,
+                                     void* residual_out, int64_t ld_res, const void* gamma, void* q_out,
+                                     int64_t ld_q, float* scales_out, int64_t ld_s, void* norm_out,
+                                     int64_t ld_norm, int64_t M, int64_t d, int32_t group, float eps,
+                                     uint32_t flags, nq_stream_t stream);
 
 /*
  * RMSNorm (residual-add optional) + NVFP4 ("RMSNorm nvfp4 quant fusion for

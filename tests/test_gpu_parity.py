@@ -440,3 +440,53 @@ def test_variants_without_residual_bit_exact(nq, d, M, ld):
             assert np.array_equal(host_u8(q), e_ln), (var, sched)
             q, sf, _, _ = nq.nq_rmsnorm_quant_nvfp4(x, g, gs, 1e-6, flags=f)
             assert np.array_equal(host_u8(q), e_fp4[0]) and np.array_equal(host_u8(sf), e_fp4[1]), (var, sched)
+
+
+# ------------------------------------- fused RMSNorm + per-token-group FP8 ----
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("residual", [False, True])
+@pytest.mark.parametrize("d,M", [(128, 37), (512, 64), (2048, 9), (4096, 300), (7168, 20), (8192, 5)])
+def test_rms_group_bit_exact(nq, d, M, residual, group):
+    w = S.make_rms_inputs(M, d, seed=d + M, residual=residual, x_outlier_channels=True)
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    res = dev_bf16(w["residual"]) if residual else None
+    for flags, of in ((0, 0), (nq.FLAG_UE8M0, oracle.UE8M0), (nq.FLAG_SCALE_DIV, oracle.DIV)):
+        eq, es, er, en = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"], w.get("residual"), group=group,
+                                                        flags=of, want_norm=True)
+        gq = Guarded(M, d, torch.float8_e4m3fn)
+        gs = Guarded(M, d // group, torch.float32)
+        q, s, ro, no = nq.nq_rmsnorm_quant_fp8_group(x, g, 1e-6, group=group, residual=res, q_out=gq.view,
+                                                     scales_out=gs.view, want_norm=True, flags=flags)
+        torch.cuda.synchronize()
+        assert gq.guards_intact() and gs.guards_intact()
+        assert np.array_equal(host_u8(q), eq), flags
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32)), flags
+        assert np.array_equal(host_u16(no), en)
+        if residual:
+            assert np.array_equal(host_u16(ro), er)
+
+
+@pytest.mark.parametrize("d", [1024, 4096, 8192])
+def test_rms_group_every_schedule_and_variant(nq, d):
+    M = 17
+    w = S.make_rms_inputs(M, d, seed=d + 3, residual=False)
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    eq, es, _, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"])
+    scheds = all_schedules(d)
+    flags = [nq.flag_schedule(*s_) for s_ in scheds] + [nq.flag_variant(v) for v in (1, 2, 3)]
+    if (d + 7) // 8 <= 512:
+        flags.append(nq.flag_variant(2) | nq.flag_schedule(5, 4))
+    for f in flags:
+        q, s, _, _ = nq.nq_rmsnorm_quant_fp8_group(x, g, 1e-6, flags=f)
+        assert np.array_equal(host_u8(q), eq), hex(f)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32)), hex(f)
+
+
+def test_rms_group_misaligned_slice(nq):
+    M, d = 19, 1024
+    w = S.make_rms_inputs(M, d, seed=8, residual=True, ld_x=d + 8)
+    x = dev_bf16(w["x"])[:, 1:1 + d]
+    q, s, ro, _ = nq.nq_rmsnorm_quant_fp8_group(x, dev_bf16(w["gamma"]), 1e-6, residual=dev_bf16(w["residual"]))
+    eq, es, er, _ = oracle.rmsnorm_quant_fp8_group(w["x"][:, 1:1 + d], w["gamma"], w["residual"])
+    assert np.array_equal(host_u8(q), eq) and np.array_equal(host_u16(ro), er)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32))
