@@ -111,31 +111,59 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 // consecutive threads of the group (T >= 32 and a multiple of G/8), so its
 // absmax is an xor-butterfly over those lanes; then s = RN(absmax / 448)
 // (UE8M0: next power of two), one reciprocal, q = e4m3(RN(y * RN(1 / s))).
+// K <= 8, so a warp's K slots hold at most 32 groups (one per lane).
 template <int T, int K, bool VEC, bool FULL>
 __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
                                                 const float2 (&v)[K][4]) {
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
-  const int cpg = a.group >> 3;  // chunks per group
+  const int cpg = a.group >> 3;  // chunks per group: 8 or 16
+  const int gpw = 32 / cpg;      // groups per warp per chunk slot
+  const int lane = tid & 31;
   const bool div = (a.flags & kFlagDiv) != 0;
   const bool ue8m0 = (a.flags & kFlagUe8m0) != 0;
   uint8_t* qrow = a.q + row * a.ld_q;
   float* srow = a.scale_out + row * a.ld_scale;
+  // 1. group absmax of every chunk slot (xor-butterfly over the group's lanes)
+  float am[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
     for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    float s = __fdiv_rn(m, kE4M3Max);
-    if (ue8m0) s = ue8m0_ceil(s);
-    const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+    am[k] = m;
+  }
+  // 2. the warp holds K * gpw <= 32 groups: lane j computes the scale of group
+  //    (slot j / gpw, part j % gpw) once, instead of every lane computing the
+  //    scale of each of its K groups (a correctly rounded division and
+  //    reciprocal per group would otherwise dominate the instruction count).
+  float mine = 0.0f;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const float t = __shfl_sync(kFull, am[k], (lane % gpw) * cpg);
+    if (lane / gpw == k) mine = t;
+  }
+  float s = __fdiv_rn(mine, kE4M3Max);
+  if (ue8m0) s = ue8m0_ceil(s);
+  const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
+  {
+    const int kj = lane / gpw, part = lane % gpw;
+    const int c0 = (tid & ~31) + part * cpg + kj * T;  // first chunk of lane j's group
+    if (kj < K && (FULL || (live && c0 < C))) srow[c0 / cpg] = s;
+  }
+  // 3. each lane takes back the reciprocal (and scale) of its own groups
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const int src = k * gpw + lane / cpg;
+    const float ik = __shfl_sync(kFull, inv, src);
+    const float sk = div ? __shfl_sync(kFull, s, src) : 0.0f;
     float2 t[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      t[i] = (div && s != 0.0f) ? make_float2(__fdiv_rn(v[k][i].x, s), __fdiv_rn(v[k][i].y, s))
-                                : mul2(v[k][i], f2(inv));
+      t[i] = (div && sk != 0.0f) ? make_float2(__fdiv_rn(v[k][i].x, sk), __fdiv_rn(v[k][i].y, sk))
+                                 : mul2(v[k][i], f2(ik));
     const uint2 codes = pack_pairs_e4m3(t);
     if (FULL || (live && c < C)) {
       if constexpr (VEC) {
@@ -144,7 +172,6 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 #pragma unroll
         for (int j = 0; j < 8; ++j) qrow[8 * c + j] = uint8_t((j < 4 ? codes.x : codes.y) >> (8 * (j & 3)));
       }
-      if ((c & (cpg - 1)) == 0) srow[c / cpg] = s;
     }
   }
 }
