@@ -30,6 +30,7 @@ RECIP = 2
 UE8M0 = 4
 NORM_BF16_ROUND = 8
 SUM_PLAIN = 16
+E5M2 = 32
 
 E4M3_MAX = 448.0
 E2M1_MAX = 6.0
@@ -59,6 +60,8 @@ def _load():
                 "oracle_bf16_from_f32": ([P, P, I64], None),
                 "oracle_e4m3_encode": ([P, P, I64], None),
                 "oracle_e4m3_decode": ([P, P, I64], None),
+                "oracle_e5m2_encode": ([P, P, I64], None),
+                "oracle_e5m2_decode": ([P, P, I64], None),
                 "oracle_e2m1_encode": ([P, P, I64], None),
                 "oracle_e2m1_decode": ([P, P, I64], None),
                 "oracle_ue8m0_ceil": ([P, P, I64], None),
@@ -126,6 +129,20 @@ def e4m3_decode(c) -> np.ndarray:
     c = _c(c, np.uint8)
     out = np.empty(c.shape, np.float32)
     _load().oracle_e4m3_decode(_p(c), _p(out), c.size)
+    return out
+
+
+def e5m2_encode(v) -> np.ndarray:
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, np.uint8)
+    _load().oracle_e5m2_encode(_p(v), _p(out), v.size)
+    return out
+
+
+def e5m2_decode(c) -> np.ndarray:
+    c = _c(c, np.uint8)
+    out = np.empty(c.shape, np.float32)
+    _load().oracle_e5m2_decode(_p(c), _p(out), c.size)
     return out
 
 

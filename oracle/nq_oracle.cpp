@@ -40,8 +40,9 @@
 //  * canonical sum order (see canonical_sum) so that a parallel reduction with
 //    packed two-lane arithmetic can reproduce it exactly; OR_SUM_PLAIN
 //    switches to float64 sequential sums;
-//  * e4m3 / e2m1 encoders round to nearest, ties to even, and saturate to the
-//    largest finite magnitude (448 / 6);
+//  * e4m3 / e5m2 / e2m1 encoders round to nearest, ties to even, and saturate
+//    to the largest finite magnitude (448 / 57344 / 6); with e5m2 output the
+//    dynamic and group scales divide absmax by 57344;
 //  * NVFP4 global scale g is a dequantization multiplier (x ~ q * sf * g),
 //    block scale sf = e4m3(RN(RN(amax / 6) / g)), element multiplier
 //    m = RN(1 / RN(dec(sf) * g));
@@ -60,6 +61,7 @@ constexpr uint32_t OR_RECIP = 2u;           // quantize as RN(y * RN(1 / s))
 constexpr uint32_t OR_UE8M0 = 4u;           // power-of-two group scales
 constexpr uint32_t OR_NORM_BF16_ROUND = 8u; // round y to bf16 before quantizing
 constexpr uint32_t OR_SUM_PLAIN = 16u;      // float64 sequential sums
+constexpr uint32_t OR_E5M2 = 32u;           // FP8 outputs in e5m2 instead of e4m3
 
 constexpr float kE4M3Max = 448.0f;  // largest finite e4m3 magnitude (1.75 * 2^8)
 constexpr float kE2M1Max = 6.0f;    // largest e2m1 magnitude (1.5 * 2^2)
@@ -107,6 +109,42 @@ float e4m3_decode(uint8_t c) {
   if (ex == 0) return s * std::ldexp(float(m), -9);
   return s * std::ldexp(float(8 + m), ex - 10);
 }
+
+// ---- e5m2 (OCP FP8 E5M2): bias 15, 2 mantissa bits, largest finite 57344,
+// smallest subnormal 2^-16; infinities and NaNs exist but a saturating
+// conversion never produces an infinity.  [P2] Description: the output dtype
+// may be e5m2.  Round to nearest even, saturate. ----
+constexpr float kE5M2Max = 57344.0f;  // 1.75 * 2^15
+
+uint8_t e5m2_encode(float v) {
+  const uint8_t sign = (f2u(v) >> 31) ? 0x80 : 0x00;
+  if (std::isnan(v)) return uint8_t(sign | 0x7F);
+  float a = std::fabs(v);
+  if (a >= kE5M2Max) return uint8_t(sign | 0x7B);  // satfinite (inf included)
+  int e;
+  std::frexp(a, &e);
+  int E = e - 1;
+  if (a == 0.0f || E < -14) E = -14;  // subnormal range: quantum 2^-16
+  float n = std::nearbyint(std::ldexp(a, 2 - E));  // quantum 2^(E-2); ties to even
+  if (E == -14 && n < 4.0f) return uint8_t(sign | uint8_t(n));
+  if (n == 8.0f) { n = 4.0f; E += 1; }
+  return uint8_t(sign | uint8_t(((E + 15) << 2) | (int(n) - 4)));
+}
+
+float e5m2_decode(uint8_t c) {
+  const float s = (c & 0x80) ? -1.0f : 1.0f;
+  const int ex = (c >> 2) & 0x1F, m = c & 3;
+  if (ex == 31) return m ? std::nanf("") : s * INFINITY;
+  if (ex == 0) return s * std::ldexp(float(m), -16);
+  return s * std::ldexp(float(4 + m), ex - 17);
+}
+
+// The FP8 output format of a call: e4m3 by default, e5m2 with OR_E5M2.
+struct Fp8Out {
+  bool e5m2;
+  float max() const { return e5m2 ? kE5M2Max : kE4M3Max; }
+  uint8_t encode(float v) const { return e5m2 ? e5m2_encode(v) : e4m3_encode(v); }
+};
 
 // ---- e2m1 (FP4): bias 1, 1 mantissa bit; magnitudes {0,.5,1,1.5,2,3,4,6}.
 // [P3] Description: packed E2M1 elements. Round to nearest even, saturate. ----
@@ -251,6 +289,12 @@ void oracle_e4m3_encode(const float* in, uint8_t* out, int64_t n) {
 void oracle_e4m3_decode(const uint8_t* in, float* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = e4m3_decode(in[i]);
 }
+void oracle_e5m2_encode(const float* in, uint8_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e5m2_encode(in[i]);
+}
+void oracle_e5m2_decode(const uint8_t* in, float* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e5m2_decode(in[i]);
+}
 void oracle_e2m1_encode(const float* in, uint8_t* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = e2m1_encode(in[i]);
 }
@@ -296,6 +340,7 @@ int oracle_fused_add_rmsnorm_quant_fp8(const uint16_t* x, int64_t ld_x, const ui
                                        uint16_t* norm_out, int64_t ld_norm, int64_t M, int64_t d,
                                        float eps, uint32_t flags) {
   const bool div = use_div(flags, true);
+  const Fp8Out fmt{(flags & OR_E5M2) != 0};
   std::vector<float> r, y;
   for (int64_t m = 0; m < M; ++m) {
     rms_row(x + m * ld_x, res_in ? res_in + m * ld_res : nullptr,
@@ -304,12 +349,12 @@ int oracle_fused_add_rmsnorm_quant_fp8(const uint16_t* x, int64_t ld_x, const ui
       for (int64_t i = 0; i < d; ++i) norm_out[m * ld_norm + i] = f32_to_bf16(y[size_t(i)]);
     float amax = 0.0f;
     for (int64_t i = 0; i < d; ++i) amax = std::fmax(amax, std::fabs(y[size_t(i)]));
-    const float s = amax / kE4M3Max;
+    const float s = amax / fmt.max();
     scale_out[m] = s;
     const float inv = 1.0f / s;
     for (int64_t i = 0; i < d; ++i) {
       float t = (s == 0.0f) ? y[size_t(i)] : (div ? y[size_t(i)] / s : y[size_t(i)] * inv);
-      q[m * ld_q + i] = e4m3_encode(t);
+      q[m * ld_q + i] = fmt.encode(t);
     }
   }
   return 0;
@@ -325,6 +370,7 @@ int oracle_rmsnorm_quant_fp8_static(const uint16_t* x, int64_t ld_x, const uint1
                                     int64_t ld_norm, int64_t M, int64_t d, float eps,
                                     uint32_t flags) {
   const bool div = use_div(flags, false);
+  const Fp8Out fmt{(flags & OR_E5M2) != 0};
   const float inv = 1.0f / scale;
   std::vector<float> r, y;
   for (int64_t m = 0; m < M; ++m) {
@@ -333,7 +379,7 @@ int oracle_rmsnorm_quant_fp8_static(const uint16_t* x, int64_t ld_x, const uint1
     if (norm_out)
       for (int64_t i = 0; i < d; ++i) norm_out[m * ld_norm + i] = f32_to_bf16(y[size_t(i)]);
     for (int64_t i = 0; i < d; ++i)
-      q[m * ld_q + i] = e4m3_encode(div ? y[size_t(i)] / scale : y[size_t(i)] * inv);
+      q[m * ld_q + i] = fmt.encode(div ? y[size_t(i)] / scale : y[size_t(i)] * inv);
   }
   return 0;
 }
@@ -344,12 +390,13 @@ int oracle_layernorm_quant_fp8(const uint16_t* x, int64_t ld_x, const float* gam
                                const float* beta, float scale, uint8_t* q, int64_t ld_q,
                                int64_t M, int64_t d, float eps, uint32_t flags) {
   const bool div = use_div(flags, false);
+  const Fp8Out fmt{(flags & OR_E5M2) != 0};
   const float inv = 1.0f / scale;
   std::vector<float> c, y;
   for (int64_t m = 0; m < M; ++m) {
     ln_row(x + m * ld_x, gamma, beta, d, eps, flags, c, y);
     for (int64_t i = 0; i < d; ++i)
-      q[m * ld_q + i] = e4m3_encode(div ? y[size_t(i)] / scale : y[size_t(i)] * inv);
+      q[m * ld_q + i] = fmt.encode(div ? y[size_t(i)] / scale : y[size_t(i)] * inv);
   }
   return 0;
 }
@@ -364,19 +411,20 @@ int oracle_per_token_group_quant_fp8(const uint16_t* x, int64_t ld_x, uint8_t* q
   if (group <= 0 || K % group) return 1;
   const bool div = use_div(flags, false);
   const bool ue8m0 = (flags & OR_UE8M0) != 0;
+  const Fp8Out fmt{(flags & OR_E5M2) != 0};
   for (int64_t m = 0; m < M; ++m) {
     for (int64_t g = 0; g < K / group; ++g) {
       const uint16_t* xs = x + m * ld_x + g * group;
       float amax = 0.0f;
       for (int32_t i = 0; i < group; ++i) amax = std::fmax(amax, std::fabs(bf16_to_f32(xs[i])));
-      float s = amax / kE4M3Max;
+      float s = amax / fmt.max();
       if (ue8m0) s = ue8m0_ceil(s);
       scales[m * ld_s + g] = s;
       const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
       for (int32_t i = 0; i < group; ++i) {
         float v = bf16_to_f32(xs[i]);
         float t = (s == 0.0f) ? v : (div ? v / s : v * inv);
-        q[m * ld_q + g * group + i] = e4m3_encode(t);
+        q[m * ld_q + g * group + i] = fmt.encode(t);
       }
     }
   }
@@ -397,6 +445,7 @@ int oracle_rmsnorm_quant_fp8_group(const uint16_t* x, int64_t ld_x, const uint16
   if (group <= 0 || d % group) return 1;
   const bool div = use_div(flags, false);
   const bool ue8m0 = (flags & OR_UE8M0) != 0;
+  const Fp8Out fmt{(flags & OR_E5M2) != 0};
   std::vector<float> r, y;
   for (int64_t m = 0; m < M; ++m) {
     rms_row(x + m * ld_x, res_in ? res_in + m * ld_res : nullptr,
@@ -407,13 +456,13 @@ int oracle_rmsnorm_quant_fp8_group(const uint16_t* x, int64_t ld_x, const uint16
       const float* ys = y.data() + g * group;
       float amax = 0.0f;
       for (int32_t i = 0; i < group; ++i) amax = std::fmax(amax, std::fabs(ys[i]));
-      float s = amax / kE4M3Max;
+      float s = amax / fmt.max();
       if (ue8m0) s = ue8m0_ceil(s);
       scales[m * ld_s + g] = s;
       const float inv = (s == 0.0f) ? 0.0f : 1.0f / s;
       for (int32_t i = 0; i < group; ++i) {
         float t = (s == 0.0f) ? ys[i] : (div ? ys[i] / s : ys[i] * inv);
-        q[m * ld_q + g * group + i] = e4m3_encode(t);
+        q[m * ld_q + g * group + i] = fmt.encode(t);
       }
     }
   }

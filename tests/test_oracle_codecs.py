@@ -6,6 +6,9 @@
   e4m3 values, over every bf16 bit pattern and a million random float32
   values, and against torch's float -> float8_e4m3fn cast inside the finite
   range;
+* e5m2 decode of all 256 codes and encode of every bf16 pattern, random
+  float32 values and tie midpoints, against the bit fields, a brute-force
+  nearest-even search and torch's float8_e5m2;
 * e2m1 decode/encode against the bit-field definition and a brute-force
   search; page-independent tie cases from tests/golden;
 * UE8M0 against a brute-force smallest power of two;
@@ -167,3 +170,44 @@ def test_bf16_rounding_matches_torch():
     got = oracle.bf16_from_f32(v)
     exp = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(got, exp)
+
+
+def _e5m2_from_fields(code: int) -> float:
+    s = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 2) & 0x1F, code & 3
+    if e == 31:
+        return math.nan if m else s * math.inf
+    if e == 0:
+        return s * m * 2.0 ** -16
+    return s * (1 + m / 4) * 2.0 ** (e - 15)
+
+
+E5M2_MAGS = np.array([_e5m2_from_fields(c) for c in range(0x7C)], np.float64)  # 0x00..0x7B finite
+
+
+def test_e5m2_decode_matches_bitfields_and_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    dec = oracle.e5m2_decode(codes).astype(np.float64)
+    ref = np.array([_e5m2_from_fields(int(c)) for c in codes])
+    tdec = torch.from_numpy(codes).view(torch.float8_e5m2).to(torch.float64).numpy()
+    for a in (ref, tdec):
+        nan = np.isnan(a)
+        assert np.array_equal(np.isnan(dec), nan)
+        assert np.array_equal(dec[~nan], a[~nan])
+    assert dec[0x7B] == 57344.0 and dec[0x01] == 2.0 ** -16 and dec[0x7C] == np.inf
+
+
+def test_e5m2_encode_brute_force_and_torch():
+    bits = np.arange(65536, dtype=np.uint32)
+    v = (bits << 16).view(np.float32)
+    v = v[~np.isnan(v)]
+    rng = np.random.default_rng(9)
+    mag = np.exp2(rng.uniform(-20, 18, 300_000)).astype(np.float32)
+    mids = ((E5M2_MAGS[1:] + E5M2_MAGS[:-1]) / 2).astype(np.float32)
+    v = np.concatenate([v, mag, -mag, mids, -mids])
+    got = oracle.e5m2_encode(v)
+    exp = np.concatenate([_brute_nearest_even(c, E5M2_MAGS, 0x80, 0x7B) for c in np.array_split(v, 40)])
+    assert np.array_equal(got, exp)
+    inside = np.abs(v) <= 57344.0
+    t = torch.from_numpy(v[inside]).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(got[inside], t)

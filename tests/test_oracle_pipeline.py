@@ -352,3 +352,26 @@ def test_rms_group_fused_vs_unfused():
     frac = (qf != qu).mean()
     assert 0.01 <= frac <= 0.05
     assert np.abs(e4m3_rank(qf) - e4m3_rank(qu)).max() <= 1
+
+
+def test_e5m2_outputs_compose_pinned_pieces():
+    """With e5m2 output the dynamic scale is absmax / 57344 and the codes are the
+    pinned e5m2 encoder of RN(y / s); static and group paths likewise."""
+    w = S.make_rms_inputs(16, 1024, seed=21)
+    q, s, _, _ = oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"], flags=oracle.E5M2)
+    y = oracle.rms_y(w["x"], w["gamma"], w["residual"])
+    es = (np.abs(y).max(axis=1) / np.float32(57344)).astype(np.float32)
+    assert np.array_equal(s, es)
+    assert np.array_equal(q, oracle.e5m2_encode((y / es[:, None]).astype(np.float32)))
+    top = q[np.arange(16), np.argmax(np.abs(y), axis=1)]
+    assert np.all((top & 0x7F) == 0x7B)
+    qs, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, flags=oracle.E5M2)
+    y0 = oracle.rms_y(w["x"], w["gamma"])
+    assert np.array_equal(qs, oracle.e5m2_encode((y0 * (np.float32(1) / np.float32(0.05))).astype(np.float32)))
+    gw = S.make_group_inputs(8, 512, seed=2)
+    qg, sg = oracle.per_token_group_quant_fp8(gw["x"], 128, oracle.E5M2)
+    xf = oracle.bf16_to_f32(gw["x"]).reshape(8, 4, 128)
+    esg = (np.abs(xf).max(axis=2) / np.float32(57344)).astype(np.float32)
+    assert np.array_equal(sg, esg)
+    inv = (np.float32(1) / esg).astype(np.float32)
+    assert np.array_equal(qg, oracle.e5m2_encode((xf * inv[..., None]).astype(np.float32)).reshape(8, 512))
