@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
-    "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND",
+    "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND", "FLAG_E5M2",
     "flag_schedule", "flag_group_schedule", "flag_variant", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
@@ -39,6 +39,7 @@ FLAG_SCALE_DIV = 1 << 1
 FLAG_SCALE_RECIP = 1 << 2
 FLAG_UE8M0 = 1 << 3
 FLAG_NORM_BF16_ROUND = 1 << 4
+FLAG_E5M2 = 1 << 5
 OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4, OP_RMS_GROUP_FP8 = 0, 1, 2, 3, 4
 
 
@@ -178,6 +179,14 @@ def _out(t, shape, dtype, like: torch.Tensor, name: str):
     return t
 
 
+def _fp8_format(flags: int, q_out):
+    """(flags, dtype) of an FP8 call's codes: a float8_e5m2 ``q_out`` selects
+    e5m2 (FLAG_E5M2); otherwise the flag picks the dtype of a new ``q_out``."""
+    if q_out is not None and isinstance(q_out, torch.Tensor) and q_out.dtype == torch.float8_e5m2:
+        flags |= FLAG_E5M2
+    return flags, (torch.float8_e5m2 if flags & FLAG_E5M2 else torch.float8_e4m3fn)
+
+
 # ------------------------------------------------------------ the calls ----
 def nq_query_schedule(op: int, M: int, d: int, flags: int = 0):
     """(threads per row, 16-byte chunks per thread, rows per CTA) the planner picks."""
@@ -195,7 +204,9 @@ def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, res
     ``x`` bf16 [M, d] (may be a column slice), ``residual`` bf16 [M, d],
     ``gamma`` bf16 [d].  ``residual_out`` defaults to a new tensor; pass
     ``residual_out=residual`` for the in-place update.  Returns
-    ``(q float8_e4m3fn [M, d], scale float32 [M], residual_out, norm_out or None)``.
+    ``(q float8_e4m3fn [M, d], scale float32 [M], residual_out, norm_out or None)``;
+    with ``flags |= FLAG_E5M2`` or a float8_e5m2 ``q_out`` the codes are e5m2
+    and s = absmax / 57344 (this holds for every FP8 call).
     """
     M, d, ld_x = _rows(x, "x", torch.bfloat16)
     _, _, ld_r = _rows(residual, "residual", torch.bfloat16, d)
@@ -204,8 +215,9 @@ def nq_fused_add_rmsnorm_quant_fp8(x, residual, gamma, eps: float = 1e-6, *, res
     residual_out = _out(residual_out, (M, d), torch.bfloat16, x, "residual_out")
     _, _, ld_ro = _rows(residual_out, "residual_out", torch.bfloat16, d)
     _need(ld_ro == ld_r, "residual_out must have the row stride of residual")
-    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
-    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    flags, f8 = _fp8_format(flags, q_out)
+    q_out = _out(q_out, (M, d), f8, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", f8, d)
     scale_out = _out(scale_out, (M,), torch.float32, x, "scale_out")
     _vec(scale_out, "scale_out", torch.float32, M)
     if want_norm and norm_out is None:
@@ -239,8 +251,9 @@ def nq_rmsnorm_quant_fp8_static(x, gamma, scale, eps: float = 1e-6, *, residual=
               "residual_out must have the row stride of residual")
     else:
         _need(residual_out is None, "residual_out needs residual")
-    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
-    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    flags, f8 = _fp8_format(flags, q_out)
+    q_out = _out(q_out, (M, d), f8, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", f8, d)
     if want_norm and norm_out is None:
         norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
     ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
@@ -259,8 +272,9 @@ def nq_layernorm_quant_fp8(x, gamma, beta, scale, eps: float = 1e-5, *, q_out=No
     _vec(gamma, "gamma", torch.float32, d)
     _vec(beta, "beta", torch.float32, d)
     _scalar(scale, "scale")
-    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
-    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    flags, f8 = _fp8_format(flags, q_out)
+    q_out = _out(q_out, (M, d), f8, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", f8, d)
     _same_device(x, gamma, beta, scale, q_out)
     with torch.cuda.device(x.device):
         _check(_get_lib().nq_layernorm_quant_fp8(_ptr(x), ld_x, _ptr(gamma), _ptr(beta), _ptr(scale), _ptr(q_out),
@@ -273,8 +287,9 @@ def nq_per_token_group_quant_fp8(x, group: int = 128, *, q_out=None, scales_out=
     """Per-token-group e4m3. Returns ``(q float8_e4m3fn [M, K], scales float32 [M, K/group])``."""
     M, K, ld_x = _rows(x, "x", torch.bfloat16)
     _need(group > 0 and K % group == 0, f"K = {K} must be a multiple of group = {group}")
-    q_out = _out(q_out, (M, K), torch.float8_e4m3fn, x, "q_out")
-    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, K)
+    flags, f8 = _fp8_format(flags, q_out)
+    q_out = _out(q_out, (M, K), f8, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", f8, K)
     scales_out = _out(scales_out, (M, K // group), torch.float32, x, "scales_out")
     _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, K // group)
     _same_device(x, q_out, scales_out)
@@ -304,8 +319,9 @@ def nq_rmsnorm_quant_fp8_group(x, gamma, eps: float = 1e-6, *, group: int = 128,
               "residual_out must have the row stride of residual")
     else:
         _need(residual_out is None, "residual_out needs residual")
-    q_out = _out(q_out, (M, d), torch.float8_e4m3fn, x, "q_out")
-    _, _, ld_q = _rows(q_out, "q_out", torch.float8_e4m3fn, d)
+    flags, f8 = _fp8_format(flags, q_out)
+    q_out = _out(q_out, (M, d), f8, x, "q_out")
+    _, _, ld_q = _rows(q_out, "q_out", f8, d)
     scales_out = _out(scales_out, (M, d // group), torch.float32, x, "scales_out")
     _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, d // group)
     if want_norm and norm_out is None:

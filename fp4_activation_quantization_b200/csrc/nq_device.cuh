@@ -1,7 +1,7 @@
 // nq_device.cuh — device helpers shared by the sm_100a kernels of libnq.
 //
 // Format conversions use the hardware's packed converters
-// (cvt.rn.satfinite.e4m3x2.f32, cvt.rn.satfinite.e2m1x2.f32, cvt.rn.bf16x2.f32):
+// (cvt.rn.satfinite.{e4m3x2,e5m2x2,e2m1x2}.f32, cvt.rn.bf16x2.f32):
 // round to nearest even, saturate to the largest finite value.  Every other
 // float operation is written with an explicit IEEE intrinsic (__fadd_rn,
 // __fmul_rn, __fmaf_rn, __fdiv_rn, __frcp_rn, __fsqrt_rn) so that contraction
@@ -17,6 +17,7 @@ namespace nq {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kE4M3Max = 448.0f;
+constexpr float kE5M2Max = 57344.0f;
 constexpr float kE2M1Max = 6.0f;
 
 // ---------------------------------------------------------------- PDL -----
@@ -67,6 +68,27 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
   return out;
 }
 __device__ __forceinline__ uint32_t f32_to_e4m3(float a) { return pack_e4m3x4(a, 0.f, 0.f, 0.f) & 0xFFu; }
+
+// ---------------------------------------------------------------- e5m2 ----
+__device__ __forceinline__ uint32_t pack_e5m2x4(float a0, float a1, float a2, float a3) {
+  uint32_t out;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e5m2x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e5m2x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(out)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return out;
+}
+
+// The FP8 output format as a compile-time choice (E5: e5m2, else e4m3).
+template <bool E5>
+__device__ __forceinline__ uint32_t pack_fp8x4(float a0, float a1, float a2, float a3) {
+  if constexpr (E5) return pack_e5m2x4(a0, a1, a2, a3);
+  else return pack_e4m3x4(a0, a1, a2, a3);
+}
+template <bool E5>
+constexpr float fp8_max() { return E5 ? kE5M2Max : kE4M3Max; }
 
 // e4m3 code (never the NaN code here) -> float, exact.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {

@@ -1,10 +1,11 @@
-// nq_group.cu — per-token-group e4m3 quantization of raw bf16 activations
+// nq_group.cu — per-token-group FP8 quantization of raw bf16 activations
 // (vLLM PR #61343 "per_token_group_quant_8bit: multiply by reciprocal instead
 // of dividing per element": Overview and Details).
 //
-// Per group of GROUP consecutive elements of a row: s = RN(absmax / 448)
-// (UE8M0: the smallest power of two >= s), one correctly rounded reciprocal
-// per group, q = e4m3(RN(x * RN(1 / s))) (NQ_FLAG_SCALE_DIV: RN(x / s)).
+// Per group of GROUP consecutive elements of a row: s = RN(absmax / max)
+// (max = 448 for e4m3, 57344 for e5m2 (E5); UE8M0: the smallest power of two
+// >= s), one correctly rounded reciprocal per group,
+// q = fp8(RN(x * RN(1 / s))) (NQ_FLAG_SCALE_DIV: RN(x / s)).
 //
 // Mapping: the activations are a flat list of G = M * K / GROUP groups.  A
 // group (GROUP / 8 chunks of 16 bytes) is owned by a team of TPG lanes; lane j
@@ -20,7 +21,7 @@
 
 namespace nq {
 
-template <int GROUP, int TPG, int U, bool VEC>
+template <int GROUP, int TPG, int U, bool VEC, bool E5>
 __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a) {
   constexpr int CPG = GROUP / 8;             // chunks per group
   constexpr int CPL = CPG / TPG;             // chunks per lane
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
     }
 #pragma unroll
     for (int o = TPG / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    float s = __fdiv_rn(m, kE4M3Max);
+    float s = __fdiv_rn(m, fp8_max<E5>());
     if (ue8m0) s = ue8m0_ceil(s);
     const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
     const float2 inv2 = make_float2(inv, inv);
@@ -95,8 +96,8 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
           t[2 * e + 1] = q2.y;
         }
       }
-      const uint32_t lo = pack_e4m3x4(t[0], t[1], t[2], t[3]);
-      const uint32_t hi = pack_e4m3x4(t[4], t[5], t[6], t[7]);
+      const uint32_t lo = pack_fp8x4<E5>(t[0], t[1], t[2], t[3]);
+      const uint32_t hi = pack_fp8x4<E5>(t[4], t[5], t[6], t[7]);
       if (ok[u]) {
         if constexpr (VEC) {
           *reinterpret_cast<uint2*>(dst + 8 * c) = make_uint2(lo, hi);
@@ -114,13 +115,16 @@ namespace {
 struct GroupTableHolder {
   GroupTable t;
   GroupTableHolder() {
-    for (auto& x : t)
-      for (auto& y : x)
-        for (auto& z : y)
-          for (auto& w : z) w = nullptr;
-#define NQ_GROUP(GI, G, TI, TPG, UI, U)                                                  \
-  t[GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false>); \
-  t[GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true>);
+    for (auto& f : t)
+      for (auto& x : f)
+        for (auto& y : x)
+          for (auto& z : y)
+            for (auto& w : z) w = nullptr;
+#define NQ_GROUP(GI, G, TI, TPG, UI, U)                                                        \
+  t[0][GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false, false>); \
+  t[0][GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true, false>);  \
+  t[1][GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false, true>);  \
+  t[1][GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true, true>);
     // group 64 (8 chunks): teams of 2, 4, 8 lanes; group 128 (16 chunks): 2, 4, 8, 16
     NQ_GROUP(0, 64, 0, 2, 0, 1) NQ_GROUP(0, 64, 0, 2, 1, 2) NQ_GROUP(0, 64, 0, 2, 2, 4)
     NQ_GROUP(0, 64, 1, 4, 0, 1) NQ_GROUP(0, 64, 1, 4, 1, 2) NQ_GROUP(0, 64, 1, 4, 2, 4)

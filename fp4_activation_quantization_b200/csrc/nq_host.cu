@@ -34,8 +34,8 @@ nq_status fail(nq_status st, const char* fmt, ...) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
-                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_SCHEDULE_MASK |
-                                 NQ_FLAG_VARIANT_MASK;
+                                 NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_E5M2 |
+                                 NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
                       bool allow_bf16_round) {
@@ -59,6 +59,7 @@ uint32_t kernel_flags(uint32_t flags, bool default_div) {
   if (div) k |= nq::kFlagDiv;
   if (flags & NQ_FLAG_UE8M0) k |= nq::kFlagUe8m0;
   if (flags & NQ_FLAG_NORM_BF16_ROUND) k |= nq::kFlagNormBf16;
+  if (flags & NQ_FLAG_E5M2) k |= nq::kFlagE5m2;
   return k;
 }
 
@@ -142,12 +143,14 @@ nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
     if (!(cond)) return fail(NQ_ERR_INVALID_ARGUMENT, __VA_ARGS__); \
   } while (0)
 
-const nq::RowKernels& table_of(int op) {
+// Kernel table of an operation and FP8 output format (e5m2 never reaches
+// NVFP4: its entry point rejects the flag).
+const nq::RowKernels& table_of(int op, bool e5m2) {
   switch (op) {
-    case nq::kOpRmsDynFp8: return nq::row_kernels_rms_dyn();
-    case nq::kOpRmsStaticFp8: return nq::row_kernels_rms_static();
-    case nq::kOpLnStaticFp8: return nq::row_kernels_ln_static();
-    case nq::kOpRmsGroupFp8: return nq::row_kernels_rms_group();
+    case nq::kOpRmsDynFp8: return e5m2 ? nq::row_kernels_rms_dyn_e5m2() : nq::row_kernels_rms_dyn();
+    case nq::kOpRmsStaticFp8: return e5m2 ? nq::row_kernels_rms_static_e5m2() : nq::row_kernels_rms_static();
+    case nq::kOpLnStaticFp8: return e5m2 ? nq::row_kernels_ln_static_e5m2() : nq::row_kernels_ln_static();
+    case nq::kOpRmsGroupFp8: return e5m2 ? nq::row_kernels_rms_group_e5m2() : nq::row_kernels_rms_group();
     default: return nq::row_kernels_rms_nvfp4();
   }
 }
@@ -219,8 +222,9 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
   }
   const void* k = nullptr;
+  const nq::RowKernels& table = table_of(op, (flags & NQ_FLAG_E5M2) != 0);
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
-    const auto& raw = table_of(op).raw[s.log_t - nq::kMinLogT][s.log_k];
+    const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1] != nullptr) {
       const int64_t slots = resident_ctas(raw[1], threads);
       // Persistent pays once each resident CTA walks two or more rows.
@@ -233,7 +237,7 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     if (k == nullptr) k = raw[0];
   }
   if (k == nullptr) {
-    const auto& tab = table_of(op).direct[s.log_t - nq::kMinLogT][s.log_k];
+    const auto& tab = table.direct[s.log_t - nq::kMinLogT][s.log_k];
     k = tab[vec ? 1 : 0];
     // The predicate-free variant for rows that exactly fill the schedule, when
     // it does not need more registers (occupancy decides this kernel's speed).
@@ -393,6 +397,8 @@ nq_status nq_rmsnorm_quant_nvfp4(const void* x, int64_t ld_x, const void* residu
   nq_status st = check_common(fn, M, d, eps);
   if (st != NQ_OK) return st;
   if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
+  if (flags & NQ_FLAG_E5M2)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_E5M2 applies to the FP8 calls only", fn);
   NQ_REQUIRE(d % 16 == 0, "%s: d = %lld is not a multiple of 16", fn, (long long)d);
   NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
              "%s: residual_in and residual_out must both be given or both be NULL", fn);
@@ -510,7 +516,7 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   const int slot = nq::kGroupThreads / tpg;
   const int64_t grid = (a.G + int64_t(slot) * units - 1) / (int64_t(slot) * units);
   if (grid > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: too many groups", fn);
-  const void* k = nq::group_kernels()[group == 128 ? 1 : 0][lt - 1][lu][vec ? 1 : 0];
+  const void* k = nq::group_kernels()[(flags & NQ_FLAG_E5M2) ? 1 : 0][group == 128 ? 1 : 0][lt - 1][lu][vec ? 1 : 0];
   void* args[] = {&a};
   return launch(fn, k, unsigned(grid), nq::kGroupThreads, 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }

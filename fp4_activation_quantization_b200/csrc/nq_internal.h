@@ -21,6 +21,7 @@ enum RowOp : int {
 constexpr uint32_t kFlagDiv = 1u << 1;
 constexpr uint32_t kFlagUe8m0 = 1u << 3;
 constexpr uint32_t kFlagNormBf16 = 1u << 4;
+constexpr uint32_t kFlagE5m2 = 1u << 5;  // FP8 outputs in e5m2
 
 struct RowArgs {
   const uint16_t* x;  // bf16 [M, ld_x]
@@ -86,9 +87,13 @@ const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();
 const RowKernels& row_kernels_rms_nvfp4();
 const RowKernels& row_kernels_rms_group();
+const RowKernels& row_kernels_rms_dyn_e5m2();
+const RowKernels& row_kernels_rms_static_e5m2();
+const RowKernels& row_kernels_ln_static_e5m2();
+const RowKernels& row_kernels_rms_group_e5m2();
 
-// Group kernel: [group == 128][log2(lanes per group) - 1][log2(groups per thread)][vec]
-using GroupTable = const void* [2][4][3][2];
+// Group kernel: [e5m2][group == 128][log2(lanes per group) - 1][log2(groups per thread)][vec]
+using GroupTable = const void* [2][2][4][3][2];
 const GroupTable& group_kernels();
 constexpr int kGroupThreads = 256;
 

@@ -18,7 +18,8 @@
 //      optional bf16 norm_out;
 //   a5 scale: dynamic s = RN(max|y| / 448), static RN(1 / scale[0]), or the
 //      NVFP4 per-16 block scale e4m3(RN(RN(amax / 6) / g));
-//   a6 quantize, pack (cvt.rn.satfinite e4m3x2 / e2m1x2) and store.
+//   a6 quantize, pack (cvt.rn.satfinite e4m3x2 / e5m2x2 / e2m1x2) and store.
+//   With e5m2 output the largest code is 57344 instead of 448.
 //
 // The kernel is bound by instruction issue as much as by HBM, so every
 // per-element float operation is a packed two-lane one (add / mul / fma
@@ -48,8 +49,9 @@ __device__ __forceinline__ uint4 pack_pairs_bf16(const float2 (&v)[4]) {
   return make_uint4(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y), pack_bf16x2(v[2].x, v[2].y),
                     pack_bf16x2(v[3].x, v[3].y));
 }
-__device__ __forceinline__ uint2 pack_pairs_e4m3(const float2 (&t)[4]) {
-  return make_uint2(pack_e4m3x4(t[0].x, t[0].y, t[1].x, t[1].y), pack_e4m3x4(t[2].x, t[2].y, t[3].x, t[3].y));
+template <bool E5>
+__device__ __forceinline__ uint2 pack_pairs_fp8(const float2 (&t)[4]) {
+  return make_uint2(pack_fp8x4<E5>(t[0].x, t[0].y, t[1].x, t[1].y), pack_fp8x4<E5>(t[2].x, t[2].y, t[3].x, t[3].y));
 }
 
 // Chunk partial of the canonical order: even / odd accumulators from +0,
@@ -106,13 +108,14 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
   }
 }
 
-// Per-token-group e4m3 of a row's y (chunk c of the row in v[k] for c = tid +
+// Per-token-group FP8 of a row's y (chunk c of the row in v[k] for c = tid +
 // k*T): a group of G elements is G/8 consecutive chunks, held by G/8
 // consecutive threads of the group (T >= 32 and a multiple of G/8), so its
-// absmax is an xor-butterfly over those lanes; then s = RN(absmax / 448)
-// (UE8M0: next power of two), one reciprocal, q = e4m3(RN(y * RN(1 / s))).
-// K <= 8, so a warp's K slots hold at most 32 groups (one per lane).
-template <int T, int K, bool VEC, bool FULL>
+// absmax is an xor-butterfly over those lanes; then s = RN(absmax / max)
+// (max 448, or 57344 for e5m2; UE8M0: next power of two), one reciprocal,
+// q = fp8(RN(y * RN(1 / s))).  K <= 8, so a warp's K slots hold at most 32
+// groups (one per lane).
+template <bool E5, int T, int K, bool VEC, bool FULL>
 __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
                                                 const float2 (&v)[K][4]) {
   const int d = a.d;
@@ -144,7 +147,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
     const float t = __shfl_sync(kFull, am[k], (lane % gpw) * cpg);
     if (lane / gpw == k) mine = t;
   }
-  float s = __fdiv_rn(mine, kE4M3Max);
+  float s = __fdiv_rn(mine, fp8_max<E5>());
   if (ue8m0) s = ue8m0_ceil(s);
   const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
   {
@@ -164,7 +167,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
     for (int i = 0; i < 4; ++i)
       t[i] = (div && sk != 0.0f) ? make_float2(__fdiv_rn(v[k][i].x, sk), __fdiv_rn(v[k][i].y, sk))
                                  : mul2(v[k][i], f2(ik));
-    const uint2 codes = pack_pairs_e4m3(t);
+    const uint2 codes = pack_pairs_fp8<E5>(t);
     if (FULL || (live && c < C)) {
       if constexpr (VEC) {
         *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
@@ -179,7 +182,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.
-template <int OP, int T, int K, bool VEC, bool FULL>
+template <int OP, int T, int K, bool VEC, bool FULL, bool E5>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
                                             float* s_sum1, uint32_t* s_max) {
@@ -366,7 +369,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       }
     }
   } else if constexpr (OP == kOpRmsGroupFp8) {
-    quantize_groups<T, K, VEC, FULL>(a, row, live, tid, v);
+    quantize_groups<E5, T, K, VEC, FULL>(a, row, live, tid, v);
   } else {
     float s_div, s_inv;
     bool passthrough = false;
@@ -377,7 +380,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
         for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
       const float amax = row_max_nonneg<T>(m, s_max, tid);
-      const float s = __fdiv_rn(amax, kE4M3Max);
+      const float s = __fdiv_rn(amax, fp8_max<E5>());
       if (live && tid == 0) a.scale_out[row] = s;
       s_div = s;
       s_inv = __frcp_rn(s);
@@ -402,7 +405,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
         for (int i = 0; i < 4; ++i) t[i] = mul2(v[k][i], inv2);
       }
-      const uint2 codes = pack_pairs_e4m3(t);
+      const uint2 codes = pack_pairs_fp8<E5>(t);
       if (FULL || (live && c < C)) {
         if constexpr (VEC) {
           *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
@@ -422,7 +425,9 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 // registers halve occupancy), and so did shared-memory cp.async staging.
 // MODE 0: any alignment (scalar loads); 1: 16-byte rows; 2: 16-byte rows that
 // exactly fill the schedule (d == 8 * T * K, T > 32): no predicates at all.
-template <int OP, int T, int K, int MODE>
+// E5: FP8 outputs in e5m2 (a separate instantiation, so the e4m3 kernels
+// carry no branch on the format).
+template <int OP, int T, int K, int MODE, bool E5>
 __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
   constexpr bool VEC = MODE >= 1;
   constexpr bool FULL = MODE == 2;
@@ -444,7 +449,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   uint4 xr[K], rr[K];
   load_raw<T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
-  process_row<OP, T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+  process_row<OP, T, K, VEC, FULL, E5>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
@@ -465,7 +470,7 @@ constexpr int raw_min_blocks() {
   return blocks < 1 ? 1 : blocks;
 }
 
-template <int OP, int T, int K, bool PERSIST>
+template <int OP, int T, int K, bool PERSIST, bool E5>
 __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
     row_kernel_raw(const RowArgs a) {
   static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
@@ -592,7 +597,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
 #pragma unroll
         for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
         for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        float sg = __fdiv_rn(m, kE4M3Max);
+        float sg = __fdiv_rn(m, fp8_max<E5>());
         if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
         const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
         float2 t[4];
@@ -600,7 +605,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
         for (int i = 0; i < 4; ++i)
           t[i] = (div && sg != 0.0f) ? make_float2(__fdiv_rn(v[i].x, sg), __fdiv_rn(v[i].y, sg)) : mul2(v[i], f2(ig));
         if (ok) {
-          *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_e4m3(t);
+          *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
           if ((c & (cpg - 1)) == 0) a.scale_out[row * a.ld_scale + c / cpg] = sg;
         }
       } else {
@@ -608,7 +613,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
-        if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_e4m3(t);
+        if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
       }
     }
   };
@@ -641,9 +646,11 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   }
 }
 
-// Kernel table of one operation: every built (threads, chunks, vec) schedule.
-template <int OP>
+// Kernel table of one operation and FP8 output format: every built (threads,
+// chunks, vec) schedule.
+template <int OP, bool E5>
 struct RowTable {
+  static_assert(!(E5 && OP == kOpRmsNvfp4), "NVFP4 has no e5m2 form");
   RowKernels k;
   RowTable() {
     for (auto& x : k.direct)
@@ -654,13 +661,13 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
   if constexpr (OP != kOpRmsDynFp8) {                                                                          \
-    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false>); \
-    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true>);  \
+    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, E5>); \
+    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, E5>);  \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
-  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0>); \
-  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1>); \
-  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2>); \
+  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, E5>); \
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1, E5>); \
+  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2, E5>); \
   NQ_RAW(LT, LK)
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)

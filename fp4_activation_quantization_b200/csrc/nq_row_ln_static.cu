@@ -1,11 +1,11 @@
-// nq_row_ln_static.cu — instantiates the row kernel for LayerNorm + static-scale e4m3
-// (every built schedule, vector and scalar paths).  One file per operation so
-// that the kernels compile in parallel.
+// nq_row_ln_static.cu — instantiates the row kernel for LayerNorm + static-scale
+// e4m3 (every built schedule and variant).  One file per operation and FP8
+// format so that the kernels compile in parallel.
 #include "nq_row_kernel.cuh"
 
 namespace nq {
 const RowKernels& row_kernels_ln_static() {
-  static const RowTable<kOpLnStaticFp8> table;
+  static const RowTable<kOpLnStaticFp8, false> table;
   return table.k;
 }
 }  // namespace nq

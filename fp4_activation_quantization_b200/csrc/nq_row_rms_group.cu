@@ -1,11 +1,11 @@
-// nq_row_rms_group.cu — instantiates the row kernel for RMSNorm (+residual)
-// + per-token-group e4m3 (every built schedule and variant).  One file per
-// operation so that the kernels compile in parallel.
+// nq_row_rms_group.cu — instantiates the row kernel for RMSNorm (+residual) + per-token-group
+// e4m3 (every built schedule and variant).  One file per operation and FP8
+// format so that the kernels compile in parallel.
 #include "nq_row_kernel.cuh"
 
 namespace nq {
 const RowKernels& row_kernels_rms_group() {
-  static const RowTable<kOpRmsGroupFp8> table;
+  static const RowTable<kOpRmsGroupFp8, false> table;
   return table.k;
 }
 }  // namespace nq

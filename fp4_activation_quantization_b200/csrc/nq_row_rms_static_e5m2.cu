@@ -1,0 +1,11 @@
+// nq_row_rms_static_e5m2.cu — instantiates the row kernel for RMSNorm (+residual) + static-scale
+// e5m2 (every built schedule and variant).  One file per operation and FP8
+// format so that the kernels compile in parallel.
+#include "nq_row_kernel.cuh"
+
+namespace nq {
+const RowKernels& row_kernels_rms_static_e5m2() {
+  static const RowTable<kOpRmsStaticFp8, true> table;
+  return table.k;
+}
+}  // namespace nq

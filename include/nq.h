@@ -35,12 +35,13 @@
  * Numerics (identical on every schedule, reproduced exactly by the oracle):
  *   r = RN(x + residual) in float32; the bf16 residual_out is RN_bf16(r);
  *   row sums use a fixed chunked pairwise order (8 consecutive elements per
- *   chunk summed left to right from +0, then a pairwise tree over chunk index,
+ *   chunk; its even- and odd-position elements summed in order from +0 in two
+ *   accumulators, then RN(even + odd); then a pairwise tree over chunk index,
  *   highest index bit first);
  *   rstd = RN(1 / RN(sqrt(RN(mean + eps)))) with mean = RN(sum / d);
  *   RMSNorm y = RN(RN(r * rstd) * gamma); LayerNorm y = fma(RN((r - mu) * rstd),
- *   gamma, beta); e4m3 / e2m1 conversion rounds to nearest even and saturates
- *   to +-448 / +-6.
+ *   gamma, beta); e4m3 / e5m2 / e2m1 conversion rounds to nearest even and
+ *   saturates to +-448 / +-57344 / +-6.
  *
  * Sources (web pages, by title and section):
  *  - "Fusing RMSNorm and FP8 Quantization Under torch.compile" (netraruntime
@@ -98,6 +99,12 @@ typedef enum nq_status {
 /* Round y to bf16 before quantizing: reproduces the two-kernel (norm -> bf16
  * -> quant) numerics for A/B comparisons.  Not for production use. */
 #define NQ_FLAG_NORM_BF16_ROUND (1u << 4)
+/* FP8 outputs in e5m2 (5 exponent bits, 2 mantissa bits, largest finite
+ * 57344) instead of e4m3: the dynamic and group scales become
+ * RN(absmax / 57344) and the codes saturate to +-57344.  FP8 calls only
+ * (FlashInfer PR #3962 Description: the output tensor's FP8 type picks the
+ * format). */
+#define NQ_FLAG_E5M2 (1u << 5)
 /* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
  * thread (k = 0..3, t + k <= 11), with 2^(t+k) * 8 >= d.  Every schedule gives
  * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
