@@ -62,6 +62,9 @@ def _load():
                 "oracle_e4m3_decode": ([P, P, I64], None),
                 "oracle_e5m2_encode": ([P, P, I64], None),
                 "oracle_e5m2_decode": ([P, P, I64], None),
+                "oracle_sf_swizzled_size": ([I64, I64], I64),
+                "oracle_sf_swizzle": ([P, I64, I64, I64, P], None),
+                "oracle_group_scales_layout": ([P, I64, I64, ctypes.c_int, ctypes.c_int, I64, P], ctypes.c_int),
                 "oracle_e2m1_encode": ([P, P, I64], None),
                 "oracle_e2m1_decode": ([P, P, I64], None),
                 "oracle_ue8m0_ceil": ([P, P, I64], None),
@@ -324,3 +327,33 @@ def nvfp4_global_scale(x, gamma, residual=None, eps=1e-6, d=None) -> float:
     y = rms_y(x, gamma, residual, eps, d)
     amax = float(np.max(np.abs(y))) if y.size else 0.0
     return float(np.float32(amax / (E2M1_MAX * E4M3_MAX))) if amax > 0 else 1.0
+
+
+def sf_swizzle(sf) -> np.ndarray:
+    """Row-major block scales [rows, n] (uint8) -> the swizzled 128 x 4-tile
+    layout of block-scaled GEMMs, zero padded (flat uint8 array)."""
+    sf = _c(sf, np.uint8)
+    rows, n = sf.shape
+    out = np.empty(int(_load().oracle_sf_swizzled_size(rows, n)), np.uint8)
+    _load().oracle_sf_swizzle(_p(sf), n, rows, n, _p(out))
+    return out
+
+
+def group_scales_layout(s, col_major=False, packed=False, ld=None) -> np.ndarray:
+    """Row-major group scales [M, G] float32 -> the requested layout.
+
+    fp32: [M, G] (row-major) or [G, ld] (col_major, ld >= M).  packed (UE8M0
+    scales): uint32 words of four exponent bytes, [M, ld] with ld >= ceil(G/4)
+    or [ceil(G/4), ld] with ld >= M when col_major.
+    """
+    s = _c(s, np.float32)
+    M, G = s.shape
+    W = (G + 3) // 4
+    if ld is None:
+        ld = M if col_major else (W if packed else G)
+    shape = ((W if packed else G), ld) if col_major else (M, ld)
+    out = np.zeros(shape, np.uint32 if packed else np.float32)
+    rc = _load().oracle_group_scales_layout(_p(s), M, G, int(col_major), int(packed), ld, _p(out))
+    if rc != 0:
+        raise ValueError("packed UE8M0 layout needs power-of-two scales in [2^-127, 2^127]")
+    return out

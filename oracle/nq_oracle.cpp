@@ -505,4 +505,63 @@ int oracle_rmsnorm_quant_nvfp4(const uint16_t* x, int64_t ld_x, const uint16_t* 
   return 0;
 }
 
+// ---- GEMM-ready scale layouts ([P3] Description and commit notes: the
+// production NVFP4 quantizer writes its block scales in the swizzled layout
+// that block-scaled GEMMs read, with padding left uninitialized) ----
+//
+// Swizzled layout (the 128 x 4 scale-factor tile of block-scaled tensor-core
+// MMA in NVIDIA's public PTX ISA and cuBLAS documentation): the scale matrix
+// [rows, n] is cut into tiles of 128 rows x 4 columns, each stored whole as
+// 512 bytes; tiles are ordered by row tile, and within a row tile by column
+// tile.  Inside a tile, row r (0..127) and column c (0..3) sit at byte
+// 16 * (r % 32) + 4 * (r / 32) + c.  Rows pad to a multiple of 128 and columns
+// to a multiple of 4; padding bytes are zero here (a defined value).
+int64_t oracle_sf_swizzled_size(int64_t rows, int64_t n) {
+  return ((rows + 127) / 128 * 128) * ((n + 3) / 4 * 4);
+}
+
+void oracle_sf_swizzle(const uint8_t* sf, int64_t ld_sf, int64_t rows, int64_t n, uint8_t* out) {
+  const int64_t col_tiles = (n + 3) / 4;
+  std::memset(out, 0, size_t(oracle_sf_swizzled_size(rows, n)));
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t c = 0; c < n; ++c) {
+      const int64_t tile = (r / 128) * col_tiles + c / 4;
+      const int64_t rr = r % 128, cc = c % 4;
+      out[tile * 512 + 16 * (rr % 32) + 4 * (rr / 32) + cc] = sf[r * ld_sf + c];
+    }
+}
+
+// Group-scale layouts for per-token-group FP8 GEMMs.  s is the row-major
+// [M, G] float32 result.  col_major: element (m, g) at g * ld + m (M-major, as
+// a GEMM reading one k-block's scales for many tokens wants).  packed (UE8M0
+// scales only): the exponent byte e + 127 of s = 2^e, four consecutive groups
+// of a row per 32-bit word (group 4j + b in byte b, bytes past G zero); word
+// (m, j) at m * ld + j, or at j * ld + m when col_major.  Returns 0, or -1 if
+// packed and a scale is not a power of two in [2^-127, 2^127].
+int oracle_group_scales_layout(const float* s, int64_t M, int64_t G, int col_major, int packed, int64_t ld,
+                               void* out) {
+  if (!packed) {
+    float* o = static_cast<float*>(out);
+    for (int64_t m = 0; m < M; ++m)
+      for (int64_t g = 0; g < G; ++g) o[col_major ? g * ld + m : m * ld + g] = s[m * G + g];
+    return 0;
+  }
+  uint32_t* o = static_cast<uint32_t*>(out);
+  const int64_t W = (G + 3) / 4;
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t j = 0; j < W; ++j) {
+      uint32_t word = 0;
+      for (int64_t b = 0; b < 4 && 4 * j + b < G; ++b) {
+        const float v = s[m * G + 4 * j + b];
+        int e2 = 0;
+        const float f = std::frexp(v, &e2);  // v = f * 2^e2, f in [0.5, 1)
+        const int e = e2 - 1;
+        if (!(f == 0.5f) || e < -127 || e > 127) return -1;
+        word |= uint32_t(e + 127) << (8 * b);
+      }
+      o[col_major ? j * ld + m : m * ld + j] = word;
+    }
+  return 0;
+}
+
 }  // extern "C"
