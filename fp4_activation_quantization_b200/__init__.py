@@ -25,6 +25,7 @@ import torch
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
     "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND", "FLAG_E5M2",
+    "FLAG_SF_SWIZZLED", "sf_swizzled_size",
     "flag_schedule", "flag_group_schedule", "flag_variant", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
@@ -40,6 +41,7 @@ FLAG_SCALE_RECIP = 1 << 2
 FLAG_UE8M0 = 1 << 3
 FLAG_NORM_BF16_ROUND = 1 << 4
 FLAG_E5M2 = 1 << 5
+FLAG_SF_SWIZZLED = 1 << 6
 OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4, OP_RMS_GROUP_FP8 = 0, 1, 2, 3, 4
 
 
@@ -336,13 +338,20 @@ def nq_rmsnorm_quant_fp8_group(x, gamma, eps: float = 1e-6, *, group: int = 128,
     return q_out, scales_out, residual_out, norm_out
 
 
+def sf_swizzled_size(M: int, d: int) -> int:
+    """Bytes of the swizzled block-scale buffer of an [M, d] NVFP4 output."""
+    return ((M + 127) // 128 * 128) * ((d // 16 + 3) // 4 * 4)
+
+
 def nq_rmsnorm_quant_nvfp4(x, gamma, global_scale, eps: float = 1e-6, *, residual=None, residual_out=None,
                            q_out=None, sf_out=None, norm_out=None, want_norm: bool = False, flags: int = 0,
                            stream=None):
     """RMSNorm (optional residual-add) + NVFP4.
 
     Returns ``(q uint8 [M, d/2] packed e2m1, sf float8_e4m3fn [M, d/16],
-    residual_out or None, norm_out or None)``.
+    residual_out or None, norm_out or None)``.  With ``flags |=
+    FLAG_SF_SWIZZLED`` sf is the flat float8_e4m3fn buffer of
+    ``sf_swizzled_size(M, d)`` bytes in the swizzled 128 x 4-tile layout.
     """
     M, d, ld_x = _rows(x, "x", torch.bfloat16)
     _need(d % 16 == 0, f"d = {d} must be a multiple of 16")
@@ -359,8 +368,13 @@ def nq_rmsnorm_quant_nvfp4(x, gamma, global_scale, eps: float = 1e-6, *, residua
         _need(residual_out is None, "residual_out needs residual")
     q_out = _out(q_out, (M, d // 2), torch.uint8, x, "q_out")
     _, _, ld_q = _rows(q_out, "q_out", torch.uint8, d // 2)
-    sf_out = _out(sf_out, (M, d // 16), torch.float8_e4m3fn, x, "sf_out")
-    _, _, ld_sf = _rows(sf_out, "sf_out", torch.float8_e4m3fn, d // 16)
+    if flags & FLAG_SF_SWIZZLED:
+        sf_out = _out(sf_out, (sf_swizzled_size(M, d),), torch.float8_e4m3fn, x, "sf_out")
+        _need(sf_out.is_cuda and sf_out.is_contiguous(), "sf_out must be a contiguous CUDA tensor")
+        ld_sf = 0
+    else:
+        sf_out = _out(sf_out, (M, d // 16), torch.float8_e4m3fn, x, "sf_out")
+        _, _, ld_sf = _rows(sf_out, "sf_out", torch.float8_e4m3fn, d // 16)
     if want_norm and norm_out is None:
         norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
     ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d

@@ -35,11 +35,15 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
                                  NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_E5M2 |
-                                 NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK;
+                                 NQ_FLAG_SF_SWIZZLED | NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
-                      bool allow_bf16_round) {
+                      bool allow_bf16_round, bool nvfp4 = false) {
   if (flags & ~kKnownFlags) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: unknown flag bits 0x%x", fn, flags & ~kKnownFlags);
+  if ((flags & NQ_FLAG_E5M2) && nvfp4)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_E5M2 applies to the FP8 calls only", fn);
+  if ((flags & NQ_FLAG_SF_SWIZZLED) && !nvfp4)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SF_SWIZZLED applies to the NVFP4 call only", fn);
   if ((flags & NQ_FLAG_SCALE_DIV) && (flags & NQ_FLAG_SCALE_RECIP))
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
   if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
@@ -143,15 +147,15 @@ nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
     if (!(cond)) return fail(NQ_ERR_INVALID_ARGUMENT, __VA_ARGS__); \
   } while (0)
 
-// Kernel table of an operation and FP8 output format (e5m2 never reaches
-// NVFP4: its entry point rejects the flag).
-const nq::RowKernels& table_of(int op, bool e5m2) {
+// Kernel table of an operation and output form (alt: e5m2 codes for the FP8
+// operations, swizzled block scales for NVFP4).
+const nq::RowKernels& table_of(int op, bool alt) {
   switch (op) {
-    case nq::kOpRmsDynFp8: return e5m2 ? nq::row_kernels_rms_dyn_e5m2() : nq::row_kernels_rms_dyn();
-    case nq::kOpRmsStaticFp8: return e5m2 ? nq::row_kernels_rms_static_e5m2() : nq::row_kernels_rms_static();
-    case nq::kOpLnStaticFp8: return e5m2 ? nq::row_kernels_ln_static_e5m2() : nq::row_kernels_ln_static();
-    case nq::kOpRmsGroupFp8: return e5m2 ? nq::row_kernels_rms_group_e5m2() : nq::row_kernels_rms_group();
-    default: return nq::row_kernels_rms_nvfp4();
+    case nq::kOpRmsDynFp8: return alt ? nq::row_kernels_rms_dyn_e5m2() : nq::row_kernels_rms_dyn();
+    case nq::kOpRmsStaticFp8: return alt ? nq::row_kernels_rms_static_e5m2() : nq::row_kernels_rms_static();
+    case nq::kOpLnStaticFp8: return alt ? nq::row_kernels_ln_static_e5m2() : nq::row_kernels_ln_static();
+    case nq::kOpRmsGroupFp8: return alt ? nq::row_kernels_rms_group_e5m2() : nq::row_kernels_rms_group();
+    default: return alt ? nq::row_kernels_rms_nvfp4_swizzled() : nq::row_kernels_rms_nvfp4();
   }
 }
 
@@ -222,7 +226,7 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
   }
   const void* k = nullptr;
-  const nq::RowKernels& table = table_of(op, (flags & NQ_FLAG_E5M2) != 0);
+  const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0);
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
     const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1] != nullptr) {
@@ -396,18 +400,18 @@ nq_status nq_rmsnorm_quant_nvfp4(const void* x, int64_t ld_x, const void* residu
   const char* fn = "nq_rmsnorm_quant_nvfp4";
   nq_status st = check_common(fn, M, d, eps);
   if (st != NQ_OK) return st;
-  if ((st = check_flags(fn, flags, false, true, true)) != NQ_OK) return st;
-  if (flags & NQ_FLAG_E5M2)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_E5M2 applies to the FP8 calls only", fn);
+  if ((st = check_flags(fn, flags, false, true, true, /*nvfp4=*/true)) != NQ_OK) return st;
   NQ_REQUIRE(d % 16 == 0, "%s: d = %lld is not a multiple of 16", fn, (long long)d);
   NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
              "%s: residual_in and residual_out must both be given or both be NULL", fn);
-  NQ_REQUIRE(ld_x >= d && ld_q >= d / 2 && ld_sf >= d / 16 && (!residual_in || ld_res >= d) &&
+  const bool swizzled = (flags & NQ_FLAG_SF_SWIZZLED) != 0;  // ld_sf unused
+  NQ_REQUIRE(ld_x >= d && ld_q >= d / 2 && (swizzled || ld_sf >= d / 16) && (!residual_in || ld_res >= d) &&
                  (!norm_out || ld_norm >= d),
              "%s: row strides too small (ld_x >= d, ld_q >= d/2, ld_sf >= d/16)", fn);
   if (M == 0) return NQ_OK;
   NQ_REQUIRE(x && gamma && global_scale && q_out && sf_out,
              "%s: x, gamma, global_scale, q_out and sf_out are required", fn);
+  NQ_REQUIRE(!swizzled || aligned(sf_out, 4), "%s: swizzled sf_out must be 4-byte aligned", fn);
   RowArgs a{};
   a.x = static_cast<const uint16_t*>(x);
   a.ld_x = ld_x;

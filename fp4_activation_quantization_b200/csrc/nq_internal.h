@@ -91,6 +91,7 @@ const RowKernels& row_kernels_rms_dyn_e5m2();
 const RowKernels& row_kernels_rms_static_e5m2();
 const RowKernels& row_kernels_ln_static_e5m2();
 const RowKernels& row_kernels_rms_group_e5m2();
+const RowKernels& row_kernels_rms_nvfp4_swizzled();
 
 // Group kernel: [e5m2][group == 128][log2(lanes per group) - 1][log2(groups per thread)][vec]
 using GroupTable = const void* [2][2][4][3][2];

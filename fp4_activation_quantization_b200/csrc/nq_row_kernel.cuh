@@ -54,6 +54,29 @@ __device__ __forceinline__ uint2 pack_pairs_fp8(const float2 (&t)[4]) {
   return make_uint2(pack_fp8x4<E5>(t[0].x, t[0].y, t[1].x, t[1].y), pack_fp8x4<E5>(t[2].x, t[2].y, t[3].x, t[3].y));
 }
 
+// Swizzled block-scale layout of block-scaled tensor-core GEMMs (NVIDIA PTX
+// ISA / cuBLAS: 128-row x 4-column tiles of 512 bytes, row tiles outer; inside
+// a tile row r, column c at 16 (r % 32) + 4 (r / 32) + c): byte offset of the
+// 4-column word (row r, column tile jw) when a row has n_ct column tiles.
+__device__ __forceinline__ int64_t sf_swizzled_word(int64_t r, int jw, int n_ct) {
+  return ((r >> 7) * n_ct + jw) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+}
+// The four block scales of chunks c .. c + 7 (held by lanes l .. l + 7, l % 8
+// == 0; block b = chunks 2b, 2b + 1) as one little-endian word in lane l.
+__device__ __forceinline__ uint32_t sf_word4(uint32_t sfc) {
+  return sfc | (__shfl_down_sync(kFull, sfc, 2) << 8) | (__shfl_down_sync(kFull, sfc, 4) << 16) |
+         (__shfl_down_sync(kFull, sfc, 6) << 24);
+}
+// Zero padding of the swizzled layout for rows M .. roundup(M, 128): real row
+// `row` clears rows M + row, M + row + M, ... (every padding row once).
+template <int T>
+__device__ __forceinline__ void sf_zero_padding_rows(const RowArgs& a, int64_t row, int tid) {
+  const int64_t m_pad = (a.M + 127) & ~int64_t(127);
+  const int n_ct = (a.d / 16 + 3) / 4;
+  for (int64_t p = a.M + row; p < m_pad; p += a.M)
+    for (int j = tid; j < n_ct; j += T) *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(p, j, n_ct)) = 0u;
+}
+
 // Chunk partial of the canonical order: even / odd accumulators from +0,
 // then RN(even + odd).
 template <bool SQUARES>
@@ -182,10 +205,12 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.
-template <int OP, int T, int K, bool VEC, bool FULL, bool E5>
+template <int OP, int T, int K, bool VEC, bool FULL, bool ALT>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
                                             float* s_sum1, uint32_t* s_max) {
+  constexpr bool E5 = ALT && OP != kOpRmsNvfp4;   // e5m2 codes
+  constexpr bool SWZ = ALT && OP == kOpRmsNvfp4;  // swizzled block scales
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
   const bool live = FULL || live_in;
@@ -358,6 +383,11 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
         }
       }
       const uint32_t packed = pack_e2m1x8(t);
+      if constexpr (SWZ) {
+        const uint32_t word = sf_word4(sfc);  // padding columns come from zero chunks
+        if (ok && (c & 7) == 0)
+          *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(row, c >> 3, (C + 7) >> 3)) = word;
+      }
       if (ok) {
         if constexpr (VEC) {
           *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
@@ -365,8 +395,11 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
           for (int j = 0; j < 4; ++j) qrow[4 * c + j] = uint8_t(packed >> (8 * j));
         }
-        if ((c & 1) == 0) sfrow[c >> 1] = uint8_t(sfc);
+        if (!SWZ && (c & 1) == 0) sfrow[c >> 1] = uint8_t(sfc);
       }
+    }
+    if constexpr (SWZ) {
+      if (live) sf_zero_padding_rows<T>(a, row, tid);
     }
   } else if constexpr (OP == kOpRmsGroupFp8) {
     quantize_groups<E5, T, K, VEC, FULL>(a, row, live, tid, v);
@@ -425,9 +458,10 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 // registers halve occupancy), and so did shared-memory cp.async staging.
 // MODE 0: any alignment (scalar loads); 1: 16-byte rows; 2: 16-byte rows that
 // exactly fill the schedule (d == 8 * T * K, T > 32): no predicates at all.
-// E5: FP8 outputs in e5m2 (a separate instantiation, so the e4m3 kernels
-// carry no branch on the format).
-template <int OP, int T, int K, int MODE, bool E5>
+// ALT: the alternate output form, a separate instantiation so that the
+// default kernels carry no branch on it: e5m2 codes for the FP8 operations,
+// the swizzled block-scale layout for NVFP4.
+template <int OP, int T, int K, int MODE, bool ALT>
 __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
   constexpr bool VEC = MODE >= 1;
   constexpr bool FULL = MODE == 2;
@@ -449,7 +483,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   uint4 xr[K], rr[K];
   load_raw<T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
-  process_row<OP, T, K, VEC, FULL, E5>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+  process_row<OP, T, K, VEC, FULL, ALT>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
@@ -470,9 +504,11 @@ constexpr int raw_min_blocks() {
   return blocks < 1 ? 1 : blocks;
 }
 
-template <int OP, int T, int K, bool PERSIST, bool E5>
+template <int OP, int T, int K, bool PERSIST, bool ALT>
 __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
     row_kernel_raw(const RowArgs a) {
+  constexpr bool E5 = ALT && OP != kOpRmsNvfp4;   // e5m2 codes
+  constexpr bool SWZ = ALT && OP == kOpRmsNvfp4;  // swizzled block scales
   static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
   constexpr int W = T / 32;
@@ -586,9 +622,14 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
           }
         }
         const uint32_t packed = pack_e2m1x8(t);
+        if constexpr (SWZ) {
+          const uint32_t word = sf_word4(sfc);
+          if (ok && (c & 7) == 0)
+            *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(row, c >> 3, (C + 7) >> 3)) = word;
+        }
         if (ok) {
           *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
-          if ((c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
+          if (!SWZ && (c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
         }
       } else if constexpr (OP == kOpRmsGroupFp8) {
         // the group's chunks are consecutive lanes (see quantize_groups)
@@ -615,6 +656,9 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
           t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
         if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
       }
+    }
+    if constexpr (SWZ) {
+      if (live) sf_zero_padding_rows<T>(a, row, tid);
     }
   };
 
@@ -646,11 +690,10 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   }
 }
 
-// Kernel table of one operation and FP8 output format: every built (threads,
-// chunks, vec) schedule.
-template <int OP, bool E5>
+// Kernel table of one operation and output form (ALT: e5m2 codes, or the
+// swizzled NVFP4 block scales): every built (threads, chunks, vec) schedule.
+template <int OP, bool ALT>
 struct RowTable {
-  static_assert(!(E5 && OP == kOpRmsNvfp4), "NVFP4 has no e5m2 form");
   RowKernels k;
   RowTable() {
     for (auto& x : k.direct)
@@ -661,13 +704,13 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
   if constexpr (OP != kOpRmsDynFp8) {                                                                          \
-    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, E5>); \
-    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, E5>);  \
+    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, ALT>); \
+    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, ALT>);  \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
-  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, E5>); \
-  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1, E5>); \
-  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2, E5>); \
+  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, ALT>); \
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1, ALT>); \
+  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2, ALT>); \
   NQ_RAW(LT, LK)
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)

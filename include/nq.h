@@ -105,6 +105,16 @@ typedef enum nq_status {
  * (FlashInfer PR #3962 Description: the output tensor's FP8 type picks the
  * format). */
 #define NQ_FLAG_E5M2 (1u << 5)
+/* NVFP4 only: write the block scales in the swizzled layout that block-scaled
+ * tensor-core GEMMs read (TensorRT-LLM PR #14848 commit notes: the production
+ * quantizer's default).  The [M, d/16] scale matrix is cut into tiles of 128
+ * rows x 4 columns, 512 bytes each, stored row tile by row tile and, within a
+ * row tile, column tile by column tile; inside a tile, row r and column c are
+ * byte 16 * (r % 32) + 4 * (r / 32) + c (NVIDIA PTX ISA / cuBLAS block-scaling
+ * layout).  sf_out must hold roundup(M, 128) * roundup(d / 16, 4) bytes and be
+ * 4-byte aligned; ld_sf is ignored.  Padding rows and columns are written as
+ * zero. */
+#define NQ_FLAG_SF_SWIZZLED (1u << 6)
 /* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
  * thread (k = 0..3, t + k <= 11), with 2^(t+k) * 8 >= d.  Every schedule gives
  * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
@@ -228,7 +238,8 @@ nq_status nq_rmsnorm_quant_fp8_group(const void* x, int64_t ld_x, const void* re
  *     block_scale * g), read at kernel execution, positive and finite;
  *   q_out uint8 [M, ld_q] packed e2m1, element 2i in the low nibble of byte i
  *     (d / 2 bytes per row);
- *   sf_out uint8 [M, ld_sf] e4m3 block scales, one per 16 elements, row-major:
+ *   sf_out uint8 [M, ld_sf] e4m3 block scales, one per 16 elements, row-major
+ *     (NQ_FLAG_SF_SWIZZLED: the swizzled 128 x 4-tile layout instead):
  *     sf = e4m3(RN(RN(absmax / 6) / g)); element multiplier RN(1 / RN(sf * g));
  *   norm_out bf16 [M, ld_norm] or NULL.
  *   d % 16 == 0.

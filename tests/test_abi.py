@@ -46,7 +46,8 @@ def test_flag_values_match_header(nq):
     assert "#define NQ_MAX_D 16384" in text and nq.NQ_MAX_D == 16384
     for name, val in [("NQ_FLAG_PDL", nq.FLAG_PDL), ("NQ_FLAG_SCALE_DIV", nq.FLAG_SCALE_DIV),
                       ("NQ_FLAG_SCALE_RECIP", nq.FLAG_SCALE_RECIP), ("NQ_FLAG_UE8M0", nq.FLAG_UE8M0),
-                      ("NQ_FLAG_NORM_BF16_ROUND", nq.FLAG_NORM_BF16_ROUND), ("NQ_FLAG_E5M2", nq.FLAG_E5M2)]:
+                      ("NQ_FLAG_NORM_BF16_ROUND", nq.FLAG_NORM_BF16_ROUND), ("NQ_FLAG_E5M2", nq.FLAG_E5M2),
+                      ("NQ_FLAG_SF_SWIZZLED", nq.FLAG_SF_SWIZZLED)]:
         m = re.search(rf"#define {name} \(1u << (\d+)\)", text)
         assert m and (1 << int(m.group(1))) == val, name
 
@@ -90,6 +91,12 @@ def test_validation_without_gpu(nq):
     assert L.nq_rmsnorm_quant_nvfp4(FAKE, 32, None, None, 32, FAKE, FAKE, FAKE, 16, FAKE, 2, None, 32, 4, 32,
                                     1e-6, nq.FLAG_E5M2, None) == INV
     assert b"E5M2" in L.nq_last_error()
+    # swizzled block scales: NVFP4 only; the buffer must be 4-byte aligned; ld_sf is not checked
+    assert call_fused(nq, flags=nq.FLAG_SF_SWIZZLED) == INV
+    assert L.nq_rmsnorm_quant_nvfp4(FAKE, 32, None, None, 32, FAKE, FAKE, FAKE, 16, FAKE + 2, 0, None, 32, 4, 32,
+                                    1e-6, nq.FLAG_SF_SWIZZLED, None) == INV
+    assert b"4-byte" in L.nq_last_error()
+    assert nq.sf_swizzled_size(1, 16) == 128 * 4 and nq.sf_swizzled_size(129, 7168) == 256 * 448
     # group: K % group, group size, schedule flag not allowed
     assert L.nq_per_token_group_quant_fp8(FAKE, 200, FAKE, 200, FAKE, 2, 4, 200, 128, 0, None) == INV
     assert L.nq_per_token_group_quant_fp8(FAKE, 96, FAKE, 96, FAKE, 3, 4, 96, 32, 0, None) == UNS
