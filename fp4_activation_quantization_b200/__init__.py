@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "NQ_OK", "NQ_ERR_INVALID_ARGUMENT", "NQ_ERR_UNSUPPORTED", "NQ_ERR_CUDA", "NQ_MAX_D",
     "FLAG_PDL", "FLAG_SCALE_DIV", "FLAG_SCALE_RECIP", "FLAG_UE8M0", "FLAG_NORM_BF16_ROUND", "FLAG_E5M2",
-    "FLAG_SF_SWIZZLED", "sf_swizzled_size",
+    "FLAG_SF_SWIZZLED", "sf_swizzled_size", "FLAG_SCALES_COL_MAJOR", "FLAG_SCALES_PACKED_UE8M0",
     "flag_schedule", "flag_group_schedule", "flag_variant", "NQError", "lib", "library_path", "version",
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
@@ -42,6 +42,8 @@ FLAG_UE8M0 = 1 << 3
 FLAG_NORM_BF16_ROUND = 1 << 4
 FLAG_E5M2 = 1 << 5
 FLAG_SF_SWIZZLED = 1 << 6
+FLAG_SCALES_COL_MAJOR = 1 << 7
+FLAG_SCALES_PACKED_UE8M0 = 1 << 8
 OP_RMS_DYN_FP8, OP_RMS_STATIC_FP8, OP_LN_STATIC_FP8, OP_RMS_NVFP4, OP_RMS_GROUP_FP8 = 0, 1, 2, 3, 4
 
 
@@ -189,6 +191,30 @@ def _fp8_format(flags: int, q_out):
     return flags, (torch.float8_e5m2 if flags & FLAG_E5M2 else torch.float8_e4m3fn)
 
 
+def _group_scales(scales_out, M: int, G: int, flags: int, like: torch.Tensor):
+    """Group-scale output for the layout the flags select; returns (tensor, ld).
+
+    Row-major: float32 [M, G].  FLAG_SCALES_COL_MAJOR: a [M, G] view with
+    strides (1, ld) of a [G, ld] buffer.  FLAG_SCALES_PACKED_UE8M0: int32
+    words, [M, ceil(G/4)] (row-major) or its column-major view likewise.
+    """
+    packed = bool(flags & FLAG_SCALES_PACKED_UE8M0)
+    col = bool(flags & FLAG_SCALES_COL_MAJOR)
+    n = (G + 3) // 4 if packed else G
+    dtype = torch.int32 if packed else torch.float32
+    if scales_out is None:
+        buf = torch.empty((n, M) if col else (M, n), dtype=dtype, device=like.device)
+        return (buf.t() if col else buf), (M if col else n)
+    _need(isinstance(scales_out, torch.Tensor) and scales_out.is_cuda, "scales_out must be a CUDA tensor")
+    _need(scales_out.dtype == dtype and tuple(scales_out.shape) == (M, n),
+          f"scales_out must be {dtype} {(M, n)} for this layout")
+    if col:
+        _need(scales_out.stride(0) == 1 or M <= 1, "column-major scales_out needs stride(0) == 1")
+        return scales_out, (scales_out.stride(1) if n > 1 else max(scales_out.stride(1), M))
+    _need(scales_out.stride(1) == 1 or n <= 1, "scales_out must have a contiguous last dimension")
+    return scales_out, (scales_out.stride(0) if M > 1 else max(scales_out.stride(0), n))
+
+
 # ------------------------------------------------------------ the calls ----
 def nq_query_schedule(op: int, M: int, d: int, flags: int = 0):
     """(threads per row, 16-byte chunks per thread, rows per CTA) the planner picks."""
@@ -286,14 +312,14 @@ def nq_layernorm_quant_fp8(x, gamma, beta, scale, eps: float = 1e-5, *, q_out=No
 
 def nq_per_token_group_quant_fp8(x, group: int = 128, *, q_out=None, scales_out=None, flags: int = 0,
                                  stream=None):
-    """Per-token-group e4m3. Returns ``(q float8_e4m3fn [M, K], scales float32 [M, K/group])``."""
+    """Per-token-group e4m3. Returns ``(q float8_e4m3fn [M, K], scales float32 [M, K/group])``;
+    the scales follow the layout FLAG_SCALES_COL_MAJOR / FLAG_SCALES_PACKED_UE8M0 select."""
     M, K, ld_x = _rows(x, "x", torch.bfloat16)
     _need(group > 0 and K % group == 0, f"K = {K} must be a multiple of group = {group}")
     flags, f8 = _fp8_format(flags, q_out)
     q_out = _out(q_out, (M, K), f8, x, "q_out")
     _, _, ld_q = _rows(q_out, "q_out", f8, K)
-    scales_out = _out(scales_out, (M, K // group), torch.float32, x, "scales_out")
-    _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, K // group)
+    scales_out, ld_s = _group_scales(scales_out, M, K // group, flags, x)
     _same_device(x, q_out, scales_out)
     with torch.cuda.device(x.device):
         _check(_get_lib().nq_per_token_group_quant_fp8(_ptr(x), ld_x, _ptr(q_out), ld_q, _ptr(scales_out), ld_s, M, K,
@@ -324,8 +350,7 @@ def nq_rmsnorm_quant_fp8_group(x, gamma, eps: float = 1e-6, *, group: int = 128,
     flags, f8 = _fp8_format(flags, q_out)
     q_out = _out(q_out, (M, d), f8, x, "q_out")
     _, _, ld_q = _rows(q_out, "q_out", f8, d)
-    scales_out = _out(scales_out, (M, d // group), torch.float32, x, "scales_out")
-    _, _, ld_s = _rows(scales_out, "scales_out", torch.float32, d // group)
+    scales_out, ld_s = _group_scales(scales_out, M, d // group, flags, x)
     if want_norm and norm_out is None:
         norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
     ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d

@@ -69,6 +69,25 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
 }
 __device__ __forceinline__ uint32_t f32_to_e4m3(float a) { return pack_e4m3x4(a, 0.f, 0.f, 0.f) & 0xFFu; }
 
+// ------------------------------------------------------ group scales -----
+// Store the scale s of group g (of n_groups) of a row.  Float layout: element
+// row * rs + g * cs (row-major: rs = ld, cs = 1; column-major: rs = 1, cs =
+// ld).  Packed UE8M0 (s a power of two in [2^-127, 2^127]): its biased exponent
+// byte (the float's exponent field, 0 for the subnormal 2^-127) goes to byte
+// g % 4 of the 32-bit word at byte offset row * rs + (g / 4) * cs; the group
+// that ends a row also zeroes the word's unused bytes.
+__device__ __forceinline__ void store_group_scale(float* base, int64_t rs, int64_t cs, bool packed, int64_t row,
+                                                  int64_t g, int64_t n_groups, float s) {
+  if (!packed) {
+    base[row * rs + g * cs] = s;
+    return;
+  }
+  uint8_t* w = reinterpret_cast<uint8_t*>(base) + row * rs + (g >> 2) * cs;
+  w[g & 3] = uint8_t(__float_as_uint(s) >> 23);
+  if (g == n_groups - 1)
+    for (int j = int(g & 3) + 1; j < 4; ++j) w[j] = 0;
+}
+
 // ---------------------------------------------------------------- e5m2 ----
 __device__ __forceinline__ uint32_t pack_e5m2x4(float a0, float a1, float a2, float a3) {
   uint32_t out;

@@ -21,7 +21,7 @@
 
 namespace nq {
 
-template <int GROUP, int TPG, int U, bool VEC, bool E5>
+template <int GROUP, int TPG, int U, bool VEC, bool E5, bool LAYOUT>
 __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a) {
   constexpr int CPG = GROUP / 8;             // chunks per group
   constexpr int CPL = CPG / TPG;             // chunks per lane
@@ -107,7 +107,13 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
         }
       }
     }
-    if (ok[u] && lane_g == 0) a.s[row[u] * a.ld_s + cg[u]] = s;
+    if (ok[u] && lane_g == 0) {
+      if constexpr (LAYOUT)  // column-major or packed UE8M0
+        store_group_scale(a.s, a.ld_s, a.cs_s, (a.flags & kFlagScalesPacked) != 0, row[u], cg[u], a.groups_per_row,
+                          s);
+      else
+        a.s[row[u] * a.ld_s + cg[u]] = s;
+    }
   }
 }
 
@@ -116,15 +122,17 @@ struct GroupTableHolder {
   GroupTable t;
   GroupTableHolder() {
     for (auto& f : t)
-      for (auto& x : f)
-        for (auto& y : x)
-          for (auto& z : y)
-            for (auto& w : z) w = nullptr;
-#define NQ_GROUP(GI, G, TI, TPG, UI, U)                                                        \
-  t[0][GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false, false>); \
-  t[0][GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true, false>);  \
-  t[1][GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false, true>);  \
-  t[1][GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true, true>);
+      for (auto& l : f)
+        for (auto& x : l)
+          for (auto& y : x)
+            for (auto& z : y)
+              for (auto& w : z) w = nullptr;
+#define NQ_GROUP_FL(F, L, GI, G, TI, TPG, UI, U)                                                 \
+  t[F][L][GI][TI][UI][0] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, false, F, L>); \
+  t[F][L][GI][TI][UI][1] = reinterpret_cast<const void*>(&group_kernel<G, TPG, U, true, F, L>);
+#define NQ_GROUP(GI, G, TI, TPG, UI, U)                                                          \
+  NQ_GROUP_FL(false, false, GI, G, TI, TPG, UI, U) NQ_GROUP_FL(true, false, GI, G, TI, TPG, UI, U) \
+  NQ_GROUP_FL(false, true, GI, G, TI, TPG, UI, U) NQ_GROUP_FL(true, true, GI, G, TI, TPG, UI, U)
     // group 64 (8 chunks): teams of 2, 4, 8 lanes; group 128 (16 chunks): 2, 4, 8, 16
     NQ_GROUP(0, 64, 0, 2, 0, 1) NQ_GROUP(0, 64, 0, 2, 1, 2) NQ_GROUP(0, 64, 0, 2, 2, 4)
     NQ_GROUP(0, 64, 1, 4, 0, 1) NQ_GROUP(0, 64, 1, 4, 1, 2) NQ_GROUP(0, 64, 1, 4, 2, 4)
@@ -134,6 +142,7 @@ struct GroupTableHolder {
     NQ_GROUP(1, 128, 2, 8, 0, 1) NQ_GROUP(1, 128, 2, 8, 1, 2) NQ_GROUP(1, 128, 2, 8, 2, 4)
     NQ_GROUP(1, 128, 3, 16, 0, 1) NQ_GROUP(1, 128, 3, 16, 1, 2) NQ_GROUP(1, 128, 3, 16, 2, 4)
 #undef NQ_GROUP
+#undef NQ_GROUP_FL
   }
 };
 }  // namespace

@@ -35,7 +35,8 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 constexpr uint32_t kKnownFlags = NQ_FLAG_PDL | NQ_FLAG_SCALE_DIV | NQ_FLAG_SCALE_RECIP |
                                  NQ_FLAG_UE8M0 | NQ_FLAG_NORM_BF16_ROUND | NQ_FLAG_E5M2 |
-                                 NQ_FLAG_SF_SWIZZLED | NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK;
+                                 NQ_FLAG_SF_SWIZZLED | NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0 |
+                                 NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK;
 
 nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool allow_schedule,
                       bool allow_bf16_round, bool nvfp4 = false) {
@@ -46,8 +47,9 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SF_SWIZZLED applies to the NVFP4 call only", fn);
   if ((flags & NQ_FLAG_SCALE_DIV) && (flags & NQ_FLAG_SCALE_RECIP))
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCALE_DIV and NQ_FLAG_SCALE_RECIP are exclusive", fn);
-  if ((flags & NQ_FLAG_UE8M0) && !allow_ue8m0)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_UE8M0 applies to group quantization only", fn);
+  if ((flags & (NQ_FLAG_UE8M0 | NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) && !allow_ue8m0)
+    return fail(NQ_ERR_INVALID_ARGUMENT,
+                "%s: NQ_FLAG_UE8M0 / NQ_FLAG_SCALES_* apply to group quantization only", fn);
   if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK)) && !allow_schedule)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_VARIANT apply to the norm calls only", fn);
   if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 3)
@@ -64,12 +66,29 @@ uint32_t kernel_flags(uint32_t flags, bool default_div) {
   if (flags & NQ_FLAG_UE8M0) k |= nq::kFlagUe8m0;
   if (flags & NQ_FLAG_NORM_BF16_ROUND) k |= nq::kFlagNormBf16;
   if (flags & NQ_FLAG_E5M2) k |= nq::kFlagE5m2;
+  if (flags & NQ_FLAG_SCALES_PACKED_UE8M0) k |= nq::kFlagUe8m0 | nq::kFlagScalesPacked;
   return k;
 }
 
 struct Schedule {
   int log_t, log_k;
 };
+
+// Group-scale layout of the two group calls: checks ld_s and returns the
+// kernel's row / group strides (elements of float, or bytes when packed).
+nq_status group_scale_strides(const char* fn, uint32_t flags, int64_t M, int64_t groups, int64_t ld_s,
+                              int64_t* rs, int64_t* cs) {
+  const bool col = (flags & NQ_FLAG_SCALES_COL_MAJOR) != 0;
+  const bool packed = (flags & NQ_FLAG_SCALES_PACKED_UE8M0) != 0;
+  const int64_t need = col ? M : (packed ? (groups + 3) / 4 : groups);
+  if (ld_s < need)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: ld_s = %lld < %lld for this scale layout", fn, (long long)ld_s,
+                (long long)need);
+  const int64_t unit = packed ? 4 : 1;
+  *rs = col ? unit : unit * ld_s;
+  *cs = col ? unit * ld_s : unit;
+  return NQ_OK;
+}
 
 // Row -> thread mapping.  C = ceil(d / 8) chunks of 16 bytes, P = the next
 // power of two.  Rows of <= 1024 elements: one warp per row (eight rows per
@@ -148,13 +167,16 @@ nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
   } while (0)
 
 // Kernel table of an operation and output form (alt: e5m2 codes for the FP8
-// operations, swizzled block scales for NVFP4).
-const nq::RowKernels& table_of(int op, bool alt) {
+// operations, swizzled block scales for NVFP4; layout: column-major or packed
+// group scales).
+const nq::RowKernels& table_of(int op, bool alt, bool layout) {
   switch (op) {
     case nq::kOpRmsDynFp8: return alt ? nq::row_kernels_rms_dyn_e5m2() : nq::row_kernels_rms_dyn();
     case nq::kOpRmsStaticFp8: return alt ? nq::row_kernels_rms_static_e5m2() : nq::row_kernels_rms_static();
     case nq::kOpLnStaticFp8: return alt ? nq::row_kernels_ln_static_e5m2() : nq::row_kernels_ln_static();
-    case nq::kOpRmsGroupFp8: return alt ? nq::row_kernels_rms_group_e5m2() : nq::row_kernels_rms_group();
+    case nq::kOpRmsGroupFp8:
+      if (layout) return alt ? nq::row_kernels_rms_group_e5m2_layout() : nq::row_kernels_rms_group_layout();
+      return alt ? nq::row_kernels_rms_group_e5m2() : nq::row_kernels_rms_group();
     default: return alt ? nq::row_kernels_rms_nvfp4_swizzled() : nq::row_kernels_rms_nvfp4();
   }
 }
@@ -226,7 +248,8 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
   }
   const void* k = nullptr;
-  const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0);
+  const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0,
+                                        (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0);
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
     const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1] != nullptr) {
@@ -448,9 +471,10 @@ nq_status nq_rmsnorm_quant_fp8_group(const void* x, int64_t ld_x, const void* re
   NQ_REQUIRE(d % group == 0, "%s: d = %lld is not a multiple of group %d", fn, (long long)d, group);
   NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
              "%s: residual_in and residual_out must both be given or both be NULL", fn);
-  NQ_REQUIRE(ld_x >= d && ld_q >= d && ld_s >= d / group && (!residual_in || ld_res >= d) &&
-                 (!norm_out || ld_norm >= d),
+  NQ_REQUIRE(ld_x >= d && ld_q >= d && (!residual_in || ld_res >= d) && (!norm_out || ld_norm >= d),
              "%s: row strides too small", fn);
+  int64_t s_rs = 0, s_cs = 0;
+  if ((st = group_scale_strides(fn, flags, M, d / group, ld_s, &s_rs, &s_cs)) != NQ_OK) return st;
   if (M == 0) return NQ_OK;
   NQ_REQUIRE(x && gamma && q_out && scales_out, "%s: x, gamma, q_out and scales_out are required", fn);
   RowArgs a{};
@@ -463,7 +487,8 @@ nq_status nq_rmsnorm_quant_fp8_group(const void* x, int64_t ld_x, const void* re
   a.q = static_cast<uint8_t*>(q_out);
   a.ld_q = ld_q;
   a.scale_out = scales_out;
-  a.ld_scale = ld_s;
+  a.ld_scale = s_rs;
+  a.cs_scale = s_cs;
   a.group = group;
   a.norm_out = static_cast<uint16_t*>(norm_out);
   a.ld_norm = ld_norm;
@@ -488,7 +513,9 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   NQ_REQUIRE(M >= 0 && K >= 1, "%s: need M >= 0 and K >= 1", fn);
   if (group != 64 && group != 128) return fail(NQ_ERR_UNSUPPORTED, "%s: group %d not in {64, 128}", fn, group);
   NQ_REQUIRE(K % group == 0, "%s: K = %lld is not a multiple of group %d", fn, (long long)K, group);
-  NQ_REQUIRE(ld_x >= K && ld_q >= K && ld_s >= K / group, "%s: row strides too small", fn);
+  NQ_REQUIRE(ld_x >= K && ld_q >= K, "%s: row strides too small", fn);
+  int64_t s_rs = 0, s_cs = 0;
+  if ((st = group_scale_strides(fn, flags, M, K / group, ld_s, &s_rs, &s_cs)) != NQ_OK) return st;
   if (M == 0) return NQ_OK;
   NQ_REQUIRE(x && q_out && scales_out, "%s: x, q_out and scales_out are required", fn);
   GroupArgs a{};
@@ -497,7 +524,8 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   a.q = static_cast<uint8_t*>(q_out);
   a.ld_q = ld_q;
   a.s = scales_out;
-  a.ld_s = ld_s;
+  a.ld_s = s_rs;
+  a.cs_s = s_cs;
   a.groups_per_row = K / group;
   a.G = M * (K / group);
   a.flags = kernel_flags(flags, /*default_div=*/false);
@@ -520,7 +548,9 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   const int slot = nq::kGroupThreads / tpg;
   const int64_t grid = (a.G + int64_t(slot) * units - 1) / (int64_t(slot) * units);
   if (grid > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: too many groups", fn);
-  const void* k = nq::group_kernels()[(flags & NQ_FLAG_E5M2) ? 1 : 0][group == 128 ? 1 : 0][lt - 1][lu][vec ? 1 : 0];
+  const bool layout = (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0;
+  const void* k =
+      nq::group_kernels()[(flags & NQ_FLAG_E5M2) ? 1 : 0][layout ? 1 : 0][group == 128 ? 1 : 0][lt - 1][lu][vec ? 1 : 0];
   void* args[] = {&a};
   return launch(fn, k, unsigned(grid), nq::kGroupThreads, 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }

@@ -21,7 +21,12 @@ enum RowOp : int {
 constexpr uint32_t kFlagDiv = 1u << 1;
 constexpr uint32_t kFlagUe8m0 = 1u << 3;
 constexpr uint32_t kFlagNormBf16 = 1u << 4;
-constexpr uint32_t kFlagE5m2 = 1u << 5;  // FP8 outputs in e5m2
+constexpr uint32_t kFlagE5m2 = 1u << 5;           // FP8 outputs in e5m2
+constexpr uint32_t kFlagScalesPacked = 1u << 8;   // group scales as packed UE8M0 exponent bytes
+
+// Output-form bits of the kernel instantiations (template parameter OUT).
+constexpr int kOutAlt = 1;          // e5m2 codes (FP8 ops) / swizzled block scales (NVFP4)
+constexpr int kOutScaleLayout = 2;  // group ops: column-major or packed-UE8M0 group scales
 
 struct RowArgs {
   const uint16_t* x;  // bf16 [M, ld_x]
@@ -34,8 +39,9 @@ struct RowArgs {
   const float* scale;  // device scalar: static scale or NVFP4 global scale
   uint8_t* q;          // e4m3 [M, ld_q] or packed e2m1 [M, ld_q]
   int64_t ld_q;
-  float* scale_out;  // float [M] (dynamic per-token) or [M, ld_scale] (group scales)
-  int64_t ld_scale;
+  float* scale_out;  // float [M] (dynamic per-token) or the group scales
+  int64_t ld_scale;  // group scale (row, g) at row * ld_scale + g * cs_scale (elements; bytes
+  int64_t cs_scale;  // and g / 4 in place of g when packed, see store_group_scale)
   int32_t group;     // 64 or 128 (group op)
   uint8_t* sf;       // e4m3 block scales [M, ld_sf] (NVFP4)
   int64_t ld_sf;
@@ -52,8 +58,9 @@ struct GroupArgs {
   int64_t ld_x;
   uint8_t* q;  // e4m3 [M, ld_q]
   int64_t ld_q;
-  float* s;  // float [M, ld_s]
+  float* s;      // group scales: (row, g) at row * ld_s + g * cs_s (see store_group_scale)
   int64_t ld_s;
+  int64_t cs_s;
   int64_t groups_per_row;
   int64_t G;  // M * groups_per_row
   uint32_t flags;
@@ -92,9 +99,12 @@ const RowKernels& row_kernels_rms_static_e5m2();
 const RowKernels& row_kernels_ln_static_e5m2();
 const RowKernels& row_kernels_rms_group_e5m2();
 const RowKernels& row_kernels_rms_nvfp4_swizzled();
+const RowKernels& row_kernels_rms_group_layout();
+const RowKernels& row_kernels_rms_group_e5m2_layout();
 
-// Group kernel: [e5m2][group == 128][log2(lanes per group) - 1][log2(groups per thread)][vec]
-using GroupTable = const void* [2][2][4][3][2];
+// Group kernel: [e5m2][strided / packed scales][group == 128][log2(lanes per group) - 1]
+// [log2(groups per thread)][vec]
+using GroupTable = const void* [2][2][2][4][3][2];
 const GroupTable& group_kernels();
 constexpr int kGroupThreads = 256;
 

@@ -138,7 +138,7 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 // (max 448, or 57344 for e5m2; UE8M0: next power of two), one reciprocal,
 // q = fp8(RN(y * RN(1 / s))).  K <= 8, so a warp's K slots hold at most 32
 // groups (one per lane).
-template <bool E5, int T, int K, bool VEC, bool FULL>
+template <bool E5, bool LAYOUT, int T, int K, bool VEC, bool FULL>
 __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
                                                 const float2 (&v)[K][4]) {
   const int d = a.d;
@@ -176,7 +176,13 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
   {
     const int kj = lane / gpw, part = lane % gpw;
     const int c0 = (tid & ~31) + part * cpg + kj * T;  // first chunk of lane j's group
-    if (kj < K && (FULL || (live && c0 < C))) srow[c0 / cpg] = s;
+    if (kj < K && (FULL || (live && c0 < C))) {
+      if constexpr (LAYOUT)
+        store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
+                          c0 / cpg, d / a.group, s);
+      else
+        srow[c0 / cpg] = s;
+    }
   }
   // 3. each lane takes back the reciprocal (and scale) of its own groups
 #pragma unroll
@@ -205,12 +211,13 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.
-template <int OP, int T, int K, bool VEC, bool FULL, bool ALT>
+template <int OP, int T, int K, bool VEC, bool FULL, int OUT>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
                                             float* s_sum1, uint32_t* s_max) {
-  constexpr bool E5 = ALT && OP != kOpRmsNvfp4;   // e5m2 codes
-  constexpr bool SWZ = ALT && OP == kOpRmsNvfp4;  // swizzled block scales
+  constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
+  constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
+  constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
   const bool live = FULL || live_in;
@@ -402,7 +409,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       if (live) sf_zero_padding_rows<T>(a, row, tid);
     }
   } else if constexpr (OP == kOpRmsGroupFp8) {
-    quantize_groups<E5, T, K, VEC, FULL>(a, row, live, tid, v);
+    quantize_groups<E5, LAYOUT, T, K, VEC, FULL>(a, row, live, tid, v);
   } else {
     float s_div, s_inv;
     bool passthrough = false;
@@ -458,10 +465,11 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 // registers halve occupancy), and so did shared-memory cp.async staging.
 // MODE 0: any alignment (scalar loads); 1: 16-byte rows; 2: 16-byte rows that
 // exactly fill the schedule (d == 8 * T * K, T > 32): no predicates at all.
-// ALT: the alternate output form, a separate instantiation so that the
-// default kernels carry no branch on it: e5m2 codes for the FP8 operations,
-// the swizzled block-scale layout for NVFP4.
-template <int OP, int T, int K, int MODE, bool ALT>
+// OUT: output-form bits, each a separate instantiation so that the default
+// kernels carry no branch on them.  kOutAlt: e5m2 codes for the FP8
+// operations, the swizzled block-scale layout for NVFP4; kOutScaleLayout
+// (group operation): strided or packed-UE8M0 group scales.
+template <int OP, int T, int K, int MODE, int OUT>
 __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
   constexpr bool VEC = MODE >= 1;
   constexpr bool FULL = MODE == 2;
@@ -483,7 +491,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   uint4 xr[K], rr[K];
   load_raw<T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
-  process_row<OP, T, K, VEC, FULL, ALT>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+  process_row<OP, T, K, VEC, FULL, OUT>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
@@ -504,11 +512,12 @@ constexpr int raw_min_blocks() {
   return blocks < 1 ? 1 : blocks;
 }
 
-template <int OP, int T, int K, bool PERSIST, bool ALT>
+template <int OP, int T, int K, bool PERSIST, int OUT>
 __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
     row_kernel_raw(const RowArgs a) {
-  constexpr bool E5 = ALT && OP != kOpRmsNvfp4;   // e5m2 codes
-  constexpr bool SWZ = ALT && OP == kOpRmsNvfp4;  // swizzled block scales
+  constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
+  constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
+  constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
   static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
   constexpr int W = T / 32;
@@ -647,7 +656,13 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
           t[i] = (div && sg != 0.0f) ? make_float2(__fdiv_rn(v[i].x, sg), __fdiv_rn(v[i].y, sg)) : mul2(v[i], f2(ig));
         if (ok) {
           *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
-          if ((c & (cpg - 1)) == 0) a.scale_out[row * a.ld_scale + c / cpg] = sg;
+          if ((c & (cpg - 1)) == 0) {
+            if constexpr (LAYOUT)
+              store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
+                                c / cpg, d / a.group, sg);
+            else
+              a.scale_out[row * a.ld_scale + c / cpg] = sg;
+          }
         }
       } else {
         float2 t[4];
@@ -690,9 +705,9 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   }
 }
 
-// Kernel table of one operation and output form (ALT: e5m2 codes, or the
-// swizzled NVFP4 block scales): every built (threads, chunks, vec) schedule.
-template <int OP, bool ALT>
+// Kernel table of one operation and output form (OUT bits): every built
+// (threads, chunks, vec) schedule.
+template <int OP, int OUT>
 struct RowTable {
   RowKernels k;
   RowTable() {
@@ -704,13 +719,13 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
   if constexpr (OP != kOpRmsDynFp8) {                                                                          \
-    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, ALT>); \
-    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, ALT>);  \
+    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT>); \
+    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT>);  \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
-  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, ALT>); \
-  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1, ALT>); \
-  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2, ALT>); \
+  k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, OUT>); \
+  k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1, OUT>); \
+  if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2, OUT>); \
   NQ_RAW(LT, LK)
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)

@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_ln_static() {
-  static const RowTable<kOpLnStaticFp8, false> table;
+  static const RowTable<kOpLnStaticFp8, 0> table;
   return table.k;
 }
 }  // namespace nq

@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_ln_static_e5m2() {
-  static const RowTable<kOpLnStaticFp8, true> table;
+  static const RowTable<kOpLnStaticFp8, kOutAlt> table;
   return table.k;
 }
 }  // namespace nq

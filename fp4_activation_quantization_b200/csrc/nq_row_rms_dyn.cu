@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_rms_dyn() {
-  static const RowTable<kOpRmsDynFp8, false> table;
+  static const RowTable<kOpRmsDynFp8, 0> table;
   return table.k;
 }
 }  // namespace nq

@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_rms_group() {
-  static const RowTable<kOpRmsGroupFp8, false> table;
+  static const RowTable<kOpRmsGroupFp8, 0> table;
   return table.k;
 }
 }  // namespace nq

@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_rms_group_e5m2() {
-  static const RowTable<kOpRmsGroupFp8, true> table;
+  static const RowTable<kOpRmsGroupFp8, kOutAlt> table;
   return table.k;
 }
 }  // namespace nq

@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_rms_nvfp4() {
-  static const RowTable<kOpRmsNvfp4, false> table;
+  static const RowTable<kOpRmsNvfp4, 0> table;
   return table.k;
 }
 }  // namespace nq

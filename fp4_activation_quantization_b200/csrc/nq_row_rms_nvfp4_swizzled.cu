@@ -6,7 +6,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_rms_nvfp4_swizzled() {
-  static const RowTable<kOpRmsNvfp4, true> table;
+  static const RowTable<kOpRmsNvfp4, kOutAlt> table;
   return table.k;
 }
 }  // namespace nq

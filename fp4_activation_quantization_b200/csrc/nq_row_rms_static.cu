@@ -5,7 +5,7 @@
 
 namespace nq {
 const RowKernels& row_kernels_rms_static() {
-  static const RowTable<kOpRmsStaticFp8, false> table;
+  static const RowTable<kOpRmsStaticFp8, 0> table;
   return table.k;
 }
 }  // namespace nq

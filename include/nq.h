@@ -115,6 +115,19 @@ typedef enum nq_status {
  * 4-byte aligned; ld_sf is ignored.  Padding rows and columns are written as
  * zero. */
 #define NQ_FLAG_SF_SWIZZLED (1u << 6)
+/* Group calls only: GEMM-ready group-scale layouts (for per-token-group FP8
+ * GEMMs that read one k-block's scales for many tokens at once).
+ * NQ_FLAG_SCALES_COL_MAJOR: float scale (m, g) at scales_out[g * ld_s + m],
+ *   ld_s >= M (M-major).
+ * NQ_FLAG_SCALES_PACKED_UE8M0 (implies NQ_FLAG_UE8M0): scales_out holds
+ *   32-bit words, each the biased exponent bytes (e + 127 of the scale 2^e) of
+ *   four consecutive groups of a row, group 4j + b in byte b (little-endian);
+ *   bytes past the row's last group are zero.  Word (m, j) at
+ *   ((uint32_t*)scales_out)[m * ld_s + j] with ld_s >= ceil(G / 4), or with
+ *   NQ_FLAG_SCALES_COL_MAJOR at [j * ld_s + m] with ld_s >= M.
+ * ld_s counts floats, or 32-bit words when packed. */
+#define NQ_FLAG_SCALES_COL_MAJOR (1u << 7)
+#define NQ_FLAG_SCALES_PACKED_UE8M0 (1u << 8)
 /* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
  * thread (k = 0..3, t + k <= 11), with 2^(t+k) * 8 >= d.  Every schedule gives
  * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
@@ -199,9 +212,11 @@ nq_status nq_layernorm_quant_fp8(const void* x, int64_t ld_x, const float* gamma
  * Per-token-group e4m3 of raw bf16 activations ("per_token_group_quant_8bit:
  * multiply by reciprocal instead of dividing per element": Overview, Details).
  *   x bf16 [M, ld_x] (first K columns); q_out e4m3 [M, ld_q];
- *   scales_out float32 [M, ld_s] row-major, K / group scales per row:
- *   s = RN(absmax / 448), or with NQ_FLAG_UE8M0 the smallest power of two
- *   >= s (a zero group gives 2^-127).  group in {64, 128}; K % group == 0.
+ *   scales_out float32 [M, ld_s] row-major, K / group scales per row
+ *   (NQ_FLAG_SCALES_COL_MAJOR / NQ_FLAG_SCALES_PACKED_UE8M0: the GEMM-ready
+ *   layouts above): s = RN(absmax / 448) (57344 with NQ_FLAG_E5M2), or with
+ *   NQ_FLAG_UE8M0 the smallest power of two >= s (a zero group gives 2^-127).
+ *   group in {64, 128}; K % group == 0.
  * Default quantization: NQ_FLAG_SCALE_RECIP; a zero fp32 scale stores the
  * signed zeros of x.  NQ_FLAG_GROUP_SCHEDULE(t, k) forces the mapping (tests
  * and tuning; same bits): 2^t lanes per group (t = 1..4 for group 128, 1..3
@@ -217,8 +232,9 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
  * dividing per element": Details, the fused RMSNorm + group-quant path).
  *   x bf16 [M, ld_x]; residual_in / residual_out both NULL or both given;
  *   gamma bf16 [d]; q_out e4m3 [M, ld_q]; scales_out float32 [M, ld_s],
- *   d / group per row: s = RN(absmax(y over the group) / 448), or with
- *   NQ_FLAG_UE8M0 the smallest power of two >= s; norm_out bf16 or NULL.
+ *   d / group per row, or a layout of NQ_FLAG_SCALES_*: s = RN(absmax(y over
+ *   the group) / 448), or with NQ_FLAG_UE8M0 the smallest power of two >= s;
+ *   norm_out bf16 or NULL.
  *   group in {64, 128}; d % group == 0.
  * Default quantization: NQ_FLAG_SCALE_RECIP (y * RN(1 / s)), as the standalone
  * group call; a zero fp32 scale stores the signed zeros of y.

@@ -47,7 +47,9 @@ def test_flag_values_match_header(nq):
     for name, val in [("NQ_FLAG_PDL", nq.FLAG_PDL), ("NQ_FLAG_SCALE_DIV", nq.FLAG_SCALE_DIV),
                       ("NQ_FLAG_SCALE_RECIP", nq.FLAG_SCALE_RECIP), ("NQ_FLAG_UE8M0", nq.FLAG_UE8M0),
                       ("NQ_FLAG_NORM_BF16_ROUND", nq.FLAG_NORM_BF16_ROUND), ("NQ_FLAG_E5M2", nq.FLAG_E5M2),
-                      ("NQ_FLAG_SF_SWIZZLED", nq.FLAG_SF_SWIZZLED)]:
+                      ("NQ_FLAG_SF_SWIZZLED", nq.FLAG_SF_SWIZZLED),
+                      ("NQ_FLAG_SCALES_COL_MAJOR", nq.FLAG_SCALES_COL_MAJOR),
+                      ("NQ_FLAG_SCALES_PACKED_UE8M0", nq.FLAG_SCALES_PACKED_UE8M0)]:
         m = re.search(rf"#define {name} \(1u << (\d+)\)", text)
         assert m and (1 << int(m.group(1))) == val, name
 
@@ -97,6 +99,17 @@ def test_validation_without_gpu(nq):
                                     1e-6, nq.FLAG_SF_SWIZZLED, None) == INV
     assert b"4-byte" in L.nq_last_error()
     assert nq.sf_swizzled_size(1, 16) == 128 * 4 and nq.sf_swizzled_size(129, 7168) == 256 * 448
+    # group-scale layouts: group calls only; ld_s checked per layout (M = 4, K = 640 -> 5 groups, 2 words)
+    assert call_fused(nq, flags=nq.FLAG_SCALES_COL_MAJOR) == INV
+    col, packed = nq.FLAG_SCALES_COL_MAJOR, nq.FLAG_SCALES_PACKED_UE8M0
+    for flags, ld_ok, ld_bad in ((0, 5, 4), (col, 4, 3), (packed, 2, 1), (col | packed, 4, 3)):
+        assert L.nq_per_token_group_quant_fp8(FAKE, 640, FAKE, 640, FAKE, ld_bad, 4, 640, 128, flags,
+                                              None) == INV, flags
+        assert b"ld_s" in L.nq_last_error()
+        assert L.nq_per_token_group_quant_fp8(None, 640, None, 640, None, ld_ok, 0, 640, 128, flags,
+                                              None) == nq.NQ_OK, flags
+        assert L.nq_rmsnorm_quant_fp8_group(FAKE, 640, None, None, 640, FAKE, FAKE, 640, FAKE, ld_bad, None, 640,
+                                            4, 640, 128, 1e-6, flags, None) == INV, flags
     # group: K % group, group size, schedule flag not allowed
     assert L.nq_per_token_group_quant_fp8(FAKE, 200, FAKE, 200, FAKE, 2, 4, 200, 128, 0, None) == INV
     assert L.nq_per_token_group_quant_fp8(FAKE, 96, FAKE, 96, FAKE, 3, 4, 96, 32, 0, None) == UNS
