@@ -60,6 +60,11 @@ def group_bytes(M, K, g=128):
     return M * (3 * K + 4 * (K // g))      # x read, e4m3 + fp32 scales write
 
 
+def rms_group_bytes(M, d, residual, g=128):
+    # x (+ residual read and write) bf16, e4m3 write, fp32 group scales; bf16 gamma
+    return M * ((6 * d if residual else 2 * d) + d + 4 * (d // g)) + 2 * d
+
+
 def nvfp4_bytes(M, d, residual):
     per = (6 * d if residual else 2 * d) + d // 2 + d // 16
     return M * per + 2 * d + 4
@@ -475,6 +480,23 @@ def run_sweep(nq):
             rows.append({"op": f"per_token_group_quant_fp8[{tag}]", "M": M, "K": K, "us": round(us, 3),
                          "GBps": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4)})
             del xs, qs, sc
+    for d in (4096, 7168):
+        g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
+        for M in (1, 256, 8192, 32768):
+            for residual in (False, True):
+                nb = rms_group_bytes(M, d, residual)
+                S = sets_for(nb)
+                xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)]
+                rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)] if residual else None
+                qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S)]
+                sc = [torch.empty(M, d // 128, dtype=torch.float32, device="cuda") for _ in range(S)]
+                us = _time_graph(lambda i: nq.nq_rmsnorm_quant_fp8_group(
+                    xs[i], g, 1e-6, residual=rs[i] if residual else None,
+                    residual_out=rs[i] if residual else None, q_out=qs[i], scales_out=sc[i]), S)
+                rows.append({"op": "rmsnorm_quant_fp8_group" + ("+res" if residual else ""), "M": M, "d": d,
+                             "us": round(us, 3), "GBps": round(nb / us / 1e3, 1),
+                             "frac": round(nb / us / 1e3 / peak, 4)})
+                del xs, rs, qs, sc
     gs = torch.tensor([0.004], dtype=torch.float32, device="cuda")
     for d, ld in ((7168, 7168), (1536, 2112), (512, 512)):
         g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
@@ -575,7 +597,8 @@ def run_case(args):
     bf = torch.bfloat16
     g = torch.Generator(device="cuda").manual_seed(0)
     x = torch.randn(M, d, device="cuda", generator=g).to(bf)
-    res = torch.randn(M, d, device="cuda", generator=g).to(bf) if op in ("fused_add_rmsnorm_quant_fp8", "nvfp4_res") else None
+    res = (torch.randn(M, d, device="cuda", generator=g).to(bf)
+           if op in ("fused_add_rmsnorm_quant_fp8", "nvfp4_res", "rmsnorm_quant_fp8_group_res") else None)
     gam = (1 + 0.1 * torch.randn(d, device="cuda", generator=g)).to(bf)
     gl = 1 + 0.1 * torch.randn(d, device="cuda", generator=g)
     bl = 0.02 * torch.randn(d, device="cuda", generator=g)
@@ -591,6 +614,8 @@ def run_case(args):
             nq.nq_rmsnorm_quant_nvfp4(x, gam, sc, 1e-6, residual=res, residual_out=res)
         elif op == "per_token_group_quant_fp8":
             nq.nq_per_token_group_quant_fp8(x, 128)
+        elif op in ("rmsnorm_quant_fp8_group", "rmsnorm_quant_fp8_group_res"):
+            nq.nq_rmsnorm_quant_fp8_group(x, gam, 1e-6, residual=res, residual_out=res)
     torch.cuda.synchronize()
     print("ok")
 
@@ -610,7 +635,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--case", choices=["rmsnorm_quant_fp8_static", "layernorm_quant_fp8",
                                        "fused_add_rmsnorm_quant_fp8", "nvfp4", "nvfp4_res",
-                                       "per_token_group_quant_fp8"],
+                                       "per_token_group_quant_fp8", "rmsnorm_quant_fp8_group",
+                                       "rmsnorm_quant_fp8_group_res"],
                     help="run one call --iters times on M x d and exit (for profiler captures)")
     ap.add_argument("--M", type=int, default=16384)
     ap.add_argument("--d", type=int, default=4096)

@@ -30,7 +30,7 @@ __all__ = [
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4", "OP_RMS_GROUP_FP8",
-    "nq_rmsnorm_quant_fp8_group",
+    "nq_rmsnorm_quant_fp8_group", "nq_check_device_errors",
 ]
 
 NQ_OK, NQ_ERR_INVALID_ARGUMENT, NQ_ERR_UNSUPPORTED, NQ_ERR_CUDA = 0, 1, 2, 3
@@ -58,7 +58,8 @@ def flag_group_schedule(log2_lanes: int, log2_groups: int) -> int:
 
 
 def flag_variant(n: int) -> int:
-    """NQ_FLAG_VARIANT(n): 1 register rows, 2 raw rows, 3 raw rows persistent (0 = automatic)."""
+    """NQ_FLAG_VARIANT(n): 1 register rows, 2 raw rows, 3 raw rows persistent, 4 rows staged in
+    shared memory by one bulk copy, 5 persistent ring of bulk copies (0 = automatic)."""
     return (n & 0x7) << 24
 
 
@@ -81,6 +82,7 @@ def _load() -> ctypes.CDLL:
     L.nq_version.argtypes, L.nq_version.restype = [], ctypes.c_int
     L.nq_status_string.argtypes, L.nq_status_string.restype = [st], ctypes.c_char_p
     L.nq_last_error.argtypes, L.nq_last_error.restype = [], ctypes.c_char_p
+    L.nq_check_device_errors.argtypes, L.nq_check_device_errors.restype = [], st
     L.nq_query_schedule.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     L.nq_query_schedule.restype = st
@@ -114,6 +116,12 @@ def __getattr__(name):  # module attribute `lib`, loaded on first access
 
 def version() -> int:
     return _get_lib().nq_version()
+
+
+def nq_check_device_errors() -> None:
+    """Raise NQError if a kernel's bounded wait for its own copy gave up since
+    the last check (synchronous; clears the device error word)."""
+    _check(_get_lib().nq_check_device_errors(), "nq_check_device_errors")
 
 
 class NQError(RuntimeError):

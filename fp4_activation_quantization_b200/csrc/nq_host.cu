@@ -14,6 +14,11 @@
 #include "nq.h"
 #include "nq_internal.h"
 
+// Device error word of this library: bit 0 is set by a kernel whose bounded
+// wait on its own bulk copy gave up (read and cleared by
+// nq_check_device_errors).  A symbol, not an allocation.
+__device__ uint32_t g_nq_device_error;
+
 namespace {
 
 using nq::RowArgs;
@@ -52,8 +57,8 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
                 "%s: NQ_FLAG_UE8M0 / NQ_FLAG_SCALES_* apply to group quantization only", fn);
   if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK)) && !allow_schedule)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_VARIANT apply to the norm calls only", fn);
-  if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 3)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT(n) takes n in 0..3", fn);
+  if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 5)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT(n) takes n in 0..5", fn);
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -92,12 +97,18 @@ nq_status group_scale_strides(const char* fn, uint32_t flags, int64_t M, int64_t
 
 // Row -> thread mapping.  C = ceil(d / 8) chunks of 16 bytes, P = the next
 // power of two.  Rows of <= 1024 elements: one warp per row (eight rows per
-// CTA), 2^max(0, log P - 5) chunks per thread.  Wider rows: one CTA per row
-// with four chunks per thread (64 bytes of the row per thread, 128 with a
-// residual, in flight at once).  Few rows (M < 148, fewer than one per SM):
-// spread the row over up to 1024 threads with one or two chunks each, which
-// shortens the per-row critical path.  Every mapping gives identical bits.
-nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedule* s, bool raw = false) {
+// CTA), 2^max(0, log P - 5) chunks per thread.  Wider rows: one CTA per row;
+// the chunks per thread follow rows per SM (measured on B200 for every
+// operation at d = 2816 ... 8192, M = 148 ... 65536):
+//   M < 148 (fewer rows than SMs): up to 1024 threads, one or two chunks each;
+//   M < 192 and P <= 512: one chunk per thread; M < 384: two;
+//   P <= 512 (d <= 4096): two for the residual-add dynamic path at any M
+//     (more rows in flight per SM beat the longer per-thread chain), and for
+//     static RMSNorm, LayerNorm and NVFP4 while M < 768;
+//   otherwise four (64 bytes of the row per thread, 128 with a residual, in
+//   flight at once).
+// Every mapping gives identical bits.
+nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags, Schedule* s, bool raw = false) {
   const int64_t C = (d + 7) / 8;
   int lp = 0;
   while ((int64_t(1) << lp) < C) ++lp;
@@ -120,11 +131,47 @@ nq_status plan_rows(const char* fn, int64_t M, int64_t d, uint32_t flags, Schedu
     s->log_t = lp < 10 ? lp : 10;
     s->log_k = lp - s->log_t;
   } else {
-    s->log_t = lp - 2 < 10 ? lp - 2 : 10;
-    s->log_k = lp - s->log_t;
+    int lk = 2;
+    if (M < 192 && lp <= 9) lk = 0;
+    else if (M < 384) lk = 1;
+    else if (lp <= 9 && (op == nq::kOpRmsDynFp8 ||
+                         (M < 768 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8 || op == nq::kOpRmsNvfp4))))
+      lk = 1;
+    int lt = lp - lk;
+    if (lt > 10) lt = 10;
+    s->log_t = lt;
+    s->log_k = lp - lt;
   }
   if (!nq::schedule_built(s->log_t, s->log_k))
     return fail(NQ_ERR_UNSUPPORTED, "%s: no built schedule for d = %lld", fn, (long long)d);
+  return NQ_OK;
+}
+
+// Ring kernels (NQ_FLAG_VARIANT(5)): 2^t >= 64 threads per row and 2^k <= 4
+// chunks per thread; automatically two chunks per thread where the row allows
+// (half the gamma / beta registers of four).
+nq_status plan_ring(const char* fn, int64_t d, uint32_t flags, Schedule* s) {
+  const int64_t C = (d + 7) / 8;
+  int lp = 0;
+  while ((int64_t(1) << lp) < C) ++lp;
+  const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
+  if (ft || fk) {
+    if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
+    const int lt = int(ft) + 4, lk = int(fk) - 1;
+    if (!nq::ring_schedule_built(lt, lk))
+      return fail(NQ_ERR_UNSUPPORTED, "%s: ring schedule of 2^%d threads x 2^%d chunks is not built", fn, lt, lk);
+    if ((int64_t(1) << (lt + lk)) < C)
+      return fail(NQ_ERR_INVALID_ARGUMENT, "%s: schedule covers %lld chunks, a row has %lld", fn,
+                  (long long)(int64_t(1) << (lt + lk)), (long long)C);
+    *s = {lt, lk};
+    return NQ_OK;
+  }
+  int lt = lp - 1;
+  lt = lt < 6 ? 6 : (lt > nq::kMaxLogT ? nq::kMaxLogT : lt);
+  const int lk = lp > lt ? lp - lt : 0;
+  if (!nq::ring_schedule_built(lt, lk))
+    return fail(NQ_ERR_UNSUPPORTED, "%s: no ring schedule for d = %lld", fn, (long long)d);
+  *s = {lt, lk};
   return NQ_OK;
 }
 
@@ -196,11 +243,50 @@ int kernel_regs(const void* k) {
   return regs;
 }
 
+// Device address of g_nq_device_error on the current device (cached per device).
+std::mutex g_err_mu;
+uint32_t* g_err_ptr[64] = {};
+uint32_t* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (g_err_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_nq_device_error) == cudaSuccess) g_err_ptr[dev] = static_cast<uint32_t*>(p);
+    else (void)cudaGetLastError();
+  }
+  return g_err_ptr[dev];
+}
+
+// Dynamic shared memory above the default 48 KB needs a per-kernel opt-in.
+std::mutex g_smem_mu;
+std::vector<std::pair<const void*, size_t>> g_smem;
+bool allow_smem(const void* k, size_t bytes) {
+  if (bytes <= 48 * 1024) return true;
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  for (const auto& p : g_smem)
+    if (p.first == k && p.second >= bytes) return true;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  g_smem.push_back({k, bytes});
+  return true;
+}
+
 // SM count and resident CTAs per SM of a kernel (host queries, cached).
+struct OccKey {
+  const void* k;
+  size_t smem;
+  int occ;
+};
 std::mutex g_occ_mu;
-std::vector<std::pair<const void*, int>> g_occ;
+std::vector<OccKey> g_occ;
 int g_sms = 0;
-int64_t resident_ctas(const void* k, int block) {
+int64_t resident_ctas(const void* k, int block, size_t smem = 0) {
   std::lock_guard<std::mutex> lk(g_occ_mu);
   if (g_sms == 0) {
     int dev = 0, n = 0;
@@ -211,13 +297,13 @@ int64_t resident_ctas(const void* k, int block) {
     g_sms = n;
   }
   for (const auto& p : g_occ)
-    if (p.first == k) return int64_t(g_sms) * p.second;
+    if (p.k == k && p.smem == smem) return int64_t(g_sms) * p.occ;
   int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, block, 0) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, block, smem) != cudaSuccess) {
     (void)cudaGetLastError();
     occ = 0;
   }
-  g_occ.push_back({k, occ});
+  g_occ.push_back({k, smem, occ});
   return int64_t(g_sms) * occ;
 }
 
@@ -226,14 +312,16 @@ int64_t resident_ctas(const void* k, int block) {
 // Kernel variants (same bits): register rows (row_kernel: the row as float32
 // in registers; any op, any alignment), raw rows (row_kernel_raw: ops without
 // a residual, 16-byte rows, one CTA per row, raw bf16 kept and unpacked per
-// pass), and raw rows persistent (one CTA per resident slot, next row
-// prefetched).  NQ_FLAG_VARIANT forces one where it applies.
+// pass), raw rows persistent (one CTA per resident slot, next row
+// prefetched), and staged rows (row_kernel_staged: the row copied to shared
+// memory by one bulk copy).  NQ_FLAG_VARIANT forces one where it applies.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   const bool has_res = a.res_in != nullptr;
   uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
-  const bool raw_forced = (variant == 2 || variant == 3) && vec && !has_res && op != nq::kOpRmsDynFp8;
+  const bool raw_forced = variant >= 2 && vec && !has_res && op != nq::kOpRmsDynFp8;
+  const bool ring = variant == 5 && raw_forced;
   Schedule s;
-  nq_status st = plan_rows(fn, a.M, a.d, flags, &s, raw_forced);
+  nq_status st = ring ? plan_ring(fn, a.d, flags, &s) : plan_rows(fn, op, a.M, a.d, flags, &s, raw_forced);
   if (st != NQ_OK) return st;
   const int threads = 1 << s.log_t;
   const int rows = nq::rows_per_cta(threads);
@@ -242,14 +330,36 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     // Automatic choice, from measurements on B200: static RMSNorm gains from
     // raw rows (fewer registers, more CTAs per SM) and, once every resident
     // CTA gets two or more rows, from the persistent prefetching form; NVFP4
-    // gains from raw rows on wide rows; LayerNorm (two reductions in a row)
-    // does not, and keeps float32 rows.
+    // gains from raw rows on wide rows; LayerNorm from raw rows once a row
+    // has 1024 elements or more (up to 1.37x at d = 7168: its float32 row
+    // would hold twice the registers).
     if (op == nq::kOpRmsStaticFp8) variant = 3;
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
+    else if (op == nq::kOpLnStaticFp8 && a.d >= 1024) variant = 2;
   }
   const void* k = nullptr;
+  size_t smem = 0;
   const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0,
                                         (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0);
+  if (ring) {
+    // Ring depth 4 while four rows take at most 64 KB, else 2; one CTA per
+    // resident slot (the occupancy query counts the ring's shared memory).
+    const int depth_idx = int64_t(a.d) * 2 * 4 <= 64 * 1024 ? 1 : 0;
+    k = table.ring[s.log_t - nq::kMinLogT][s.log_k][depth_idx];
+    smem = size_t(depth_idx ? 4 : 2) * size_t(a.d) * 2;
+    if (k == nullptr) return fail(NQ_ERR_UNSUPPORTED, "%s: ring kernel not built", fn);
+    if (!allow_smem(k, smem))
+      return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
+    const int64_t slots = resident_ctas(k, threads, smem);
+    if (slots <= 0) return fail(NQ_ERR_UNSUPPORTED, "%s: ring kernel does not fit on an SM", fn);
+    grid = grid < slots ? grid : slots;
+  }
+  if (vec && !has_res && op != nq::kOpRmsDynFp8 && variant == 4) {
+    k = table.staged[s.log_t - nq::kMinLogT][s.log_k];
+    smem = nq::staged_smem_bytes(threads, a.d);
+    if (k != nullptr && !allow_smem(k, smem))
+      return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
+  }
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
     const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1] != nullptr) {
@@ -273,8 +383,10 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
       if (r_full > 0 && r_vec > 0 && r_full <= r_vec) k = tab[2];
     }
   }
+  a.err = device_error_word();
+  if (a.err == nullptr) return fail(NQ_ERR_CUDA, "%s: no CUDA device", fn);
   void* args[] = {&a};
-  return launch(fn, k, unsigned(grid), unsigned(threads * rows), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
+  return launch(fn, k, unsigned(grid), unsigned(threads * rows), smem, args, (flags & NQ_FLAG_PDL) != 0, stream);
 }
 
 bool vec_bf16(const void* p, int64_t ld) { return p == nullptr || (aligned(p, 16) && ld % 8 == 0); }
@@ -297,6 +409,22 @@ const char* nq_status_string(nq_status status) {
 
 const char* nq_last_error(void) { return g_last_error.c_str(); }
 
+nq_status nq_check_device_errors(void) {
+  const char* fn = "nq_check_device_errors";
+  uint32_t* p = device_error_word();
+  if (p == nullptr) return fail(NQ_ERR_CUDA, "%s: no CUDA device", fn);
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, p, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    const cudaError_t e = cudaGetLastError();
+    return fail(NQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  }
+  if (word == 0) return NQ_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) (void)cudaGetLastError();
+  return fail(NQ_ERR_CUDA, "%s: a kernel's bounded wait for its bulk copy gave up (error word 0x%x); the "
+              "outputs of that launch are not meaningful", fn, word);
+}
+
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
                             int* chunks_per_thread, int* rows_per_cta) {
   const char* fn = "nq_query_schedule";
@@ -305,7 +433,7 @@ nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* t
   nq_status st = check_common(fn, M, d, 1.0f);
   if (st != NQ_OK) return st;
   Schedule s;
-  st = plan_rows(fn, M, d, flags, &s);
+  st = plan_rows(fn, op, M, d, flags, &s);
   if (st != NQ_OK) return st;
   *threads_per_row = 1 << s.log_t;
   *chunks_per_thread = 1 << s.log_k;

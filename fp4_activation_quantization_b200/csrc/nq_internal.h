@@ -51,6 +51,7 @@ struct RowArgs {
   int32_t d;
   float eps;
   uint32_t flags;  // kFlag* bits; kFlagDiv set means divide, clear means reciprocal
+  uint32_t* err;   // device error word: bit 0 set when a bounded wait gave up
 };
 
 struct GroupArgs {
@@ -85,10 +86,20 @@ inline bool raw_schedule_built(int log_t, int log_k) {
   return schedule_built(log_t, log_k) || (log_t == 5 && log_k == 4);
 }
 using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
+using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2];
+// Ring kernels: T >= 64 threads per row, K <= 4 chunks per thread; [.][.][ring depth 2 or 4]
+using RingTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK][2];
+inline bool ring_schedule_built(int log_t, int log_k) {
+  return log_t >= 6 && log_t <= kMaxLogT && log_k >= 0 && log_k <= 2 && log_t + log_k <= 11;
+}
 struct RowKernels {
   KernelTable direct;  // one row per thread group
   RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent]
+  StagedTable staged;  // rows without residual staged in shared memory by a bulk copy
+  RingTable ring;      // rows without residual through a ring of bulk copies, persistent
 };
+// Dynamic shared memory of a staged-row kernel: its rows of d bf16.
+inline size_t staged_smem_bytes(int threads, int64_t d) { return size_t(rows_per_cta(threads)) * size_t(d) * 2; }
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();

@@ -494,6 +494,192 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   process_row<OP, T, K, VEC, FULL, OUT>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
+// Per-chunk gamma (RMSNorm: bf16) or gamma and beta (LayerNorm: float32) of
+// chunk slot k = tid + k * T, zero past the row.  GammaLoads fetches them from
+// global memory (through L1) at each use; GammaRegs holds a thread's chunks in
+// registers for a CTA that processes many rows on the same columns.
+template <int T>
+struct GammaLoads {
+  const RowArgs& a;
+  int tid, C;
+  __device__ __forceinline__ void ln(int k, float4& g0, float4& g1, float4& e0, float4& e1) const {
+    const int c = tid + k * T;
+    g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
+    if (c < C) {
+      const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
+      g0 = __ldg(reinterpret_cast<const float4*>(gp));
+      g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
+      e0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
+      e1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
+    }
+  }
+  __device__ __forceinline__ uint4 rms(int k) const {
+    const int c = tid + k * T;
+    uint4 gu = make_uint4(0u, 0u, 0u, 0u);
+    if (c < C) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
+    return gu;
+  }
+};
+
+template <bool LN, int T, int K>
+struct GammaRegs {
+  float4 g0[LN ? K : 1], g1[LN ? K : 1], e0[LN ? K : 1], e1[LN ? K : 1];
+  uint4 gu[LN ? 1 : K];
+  __device__ __forceinline__ void load(const RowArgs& a, int tid, int C) {
+    const GammaLoads<T> from{a, tid, C};
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      if constexpr (LN) from.ln(k, g0[k], g1[k], e0[k], e1[k]);
+      else gu[k] = from.rms(k);
+    }
+  }
+  __device__ __forceinline__ void ln(int k, float4& a0, float4& a1, float4& b0, float4& b1) const {
+    a0 = g0[k], a1 = g1[k], b0 = e0[k], b1 = e1[k];
+  }
+  __device__ __forceinline__ uint4 rms(int k) const { return gu[k]; }
+};
+
+// a3..a6 of one row without residual whose raw bf16 chunks come from src(k)
+// (registers, or the row staged in shared memory) and whose gamma / beta come
+// from gam.  Rows past M (warp rows only) compute on zeros and store nothing.
+template <int OP, int T, int K, int OUT, typename Src, typename Gam, typename Hook>
+__device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, int tid, Src&& src, const Gam& gam,
+                                                float* b0, float* b1, float scale_in, float inv_static,
+                                                Hook&& after_first_sum) {
+  constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
+  constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
+  constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
+  const int d = a.d;
+  const int C = d >> 3;
+  const float fd = float(d);
+  const bool div = (a.flags & kFlagDiv) != 0;
+  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
+  const bool live = row < a.M;  // rows past M (warp rows only) compute on zeros and store nothing
+  float part[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    float2 v[4];
+    unpack_pairs(src(k), v);
+    part[k] = chunk_partial<OP != kOpLnStaticFp8>(v);
+  }
+  const float total = row_total<T, K>(part, b0, tid);
+  after_first_sum();  // every thread of the row group has read its chunks
+  float rstd, mean = 0.0f;
+  if constexpr (OP == kOpLnStaticFp8) {
+    mean = __fdiv_rn(total, fd);
+    const float2 nm = f2(-mean);
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      float2 v[4];
+      unpack_pairs(src(k), v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = (c < C) ? add2(v[i], nm) : f2(0.0f);
+      part[k] = chunk_partial<true>(v);
+    }
+    const float sq = row_total<T, K>(part, b1, tid);
+    rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
+  } else {
+    rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
+  }
+  const float2 rs2 = f2(rstd), nm = f2(-mean), inv2 = f2(inv_static);
+  uint8_t* qrow = a.q + row * a.ld_q;
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const bool ok = live && c < C;
+    float2 v[4];
+    unpack_pairs(src(k), v);
+    if constexpr (OP == kOpLnStaticFp8) {
+      float4 g0, g1, e0, e1;
+      gam.ln(k, g0, g1, e0, e1);
+      const float2 g[4] = {make_float2(g0.x, g0.y), make_float2(g0.z, g0.w), make_float2(g1.x, g1.y),
+                           make_float2(g1.z, g1.w)};
+      const float2 b[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w), make_float2(e1.x, e1.y),
+                           make_float2(e1.z, e1.w)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = fma2(mul2(add2(v[i], nm), rs2), g[i], b[i]);
+    } else {
+      float2 g[4];
+      unpack_pairs(gam.rms(k), g);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = mul2(mul2(v[i], rs2), g[i]);
+    }
+    if (bf16_round) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = make_float2(round_bf16(v[i].x), round_bf16(v[i].y));
+    }
+    if constexpr (OP != kOpLnStaticFp8) {
+      if (a.norm_out != nullptr && ok)
+        *reinterpret_cast<uint4*>(a.norm_out + row * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
+    }
+    if constexpr (OP == kOpRmsNvfp4) {
+      float m8 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));  // chunks c, c^1 form a block
+      const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), scale_in));
+      const float S = __fmul_rn(e4m3_to_f32(sfc), scale_in);
+      const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (div && S != 0.0f) {
+          t[2 * i] = __fdiv_rn(v[i].x, S);
+          t[2 * i + 1] = __fdiv_rn(v[i].y, S);
+        } else {
+          const float2 q = mul2(v[i], f2(mult));
+          t[2 * i] = q.x;
+          t[2 * i + 1] = q.y;
+        }
+      }
+      const uint32_t packed = pack_e2m1x8(t);
+      if constexpr (SWZ) {
+        const uint32_t word = sf_word4(sfc);
+        if (ok && (c & 7) == 0)
+          *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(row, c >> 3, (C + 7) >> 3)) = word;
+      }
+      if (ok) {
+        *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
+        if (!SWZ && (c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
+      }
+    } else if constexpr (OP == kOpRmsGroupFp8) {
+      // the group's chunks are consecutive lanes (see quantize_groups)
+      const int cpg = a.group >> 3;
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+      float sg = __fdiv_rn(m, fp8_max<E5>());
+      if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
+      const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
+      float2 t[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        t[i] = (div && sg != 0.0f) ? make_float2(__fdiv_rn(v[i].x, sg), __fdiv_rn(v[i].y, sg)) : mul2(v[i], f2(ig));
+      if (ok) {
+        *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
+        if ((c & (cpg - 1)) == 0) {
+          if constexpr (LAYOUT)
+            store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
+                              c / cpg, d / a.group, sg);
+          else
+            a.scale_out[row * a.ld_scale + c / cpg] = sg;
+        }
+      }
+    } else {
+      float2 t[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
+      if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
+    }
+  }
+  if constexpr (SWZ) {
+    if (live) sf_zero_padding_rows<T>(a, row, tid);
+  }
+}
+
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
 // residual), 16-byte rows, T > 32.  Only the raw bf16 chunks are kept (half
 // the registers of float32); each pass unpacks them again.  With PERSIST the
@@ -515,9 +701,6 @@ constexpr int raw_min_blocks() {
 template <int OP, int T, int K, bool PERSIST, int OUT>
 __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
     row_kernel_raw(const RowArgs a) {
-  constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
-  constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
-  constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
   static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
   constexpr int W = T / 32;
@@ -525,11 +708,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
   const int64_t group = int64_t(blockIdx.x) * R + int64_t(threadIdx.x / T);
   const int64_t n_groups = int64_t(gridDim.x) * R;
-  const int d = a.d;
-  const int C = d >> 3;
-  const float fd = float(d);
-  const bool div = (a.flags & kFlagDiv) != 0;
-  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
+  const int C = a.d >> 3;
 
   griddep_wait();
   const float scale_in = (OP == kOpRmsGroupFp8) ? 1.0f : __ldg(a.scale);
@@ -544,137 +723,8 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
     }
   };
   auto process = [&](int64_t row, const uint4 (&xr)[K], float* b0, float* b1) {
-    const bool live = row < a.M;  // rows past M (warp rows only) compute on zeros and store nothing
-    float part[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      float2 v[4];
-      unpack_pairs(xr[k], v);
-      part[k] = chunk_partial<OP != kOpLnStaticFp8>(v);
-    }
-    const float total = row_total<T, K>(part, b0, tid);
-    float rstd, mean = 0.0f;
-    if constexpr (OP == kOpLnStaticFp8) {
-      mean = __fdiv_rn(total, fd);
-      const float2 nm = f2(-mean);
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const int c = tid + k * T;
-        float2 v[4];
-        unpack_pairs(xr[k], v);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = (c < C) ? add2(v[i], nm) : f2(0.0f);
-        part[k] = chunk_partial<true>(v);
-      }
-      const float sq = row_total<T, K>(part, b1, tid);
-      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
-    } else {
-      rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
-    }
-    const float2 rs2 = f2(rstd), nm = f2(-mean), inv2 = f2(inv_static);
-    uint8_t* qrow = a.q + row * a.ld_q;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      const bool ok = live && c < C;
-      float2 v[4];
-      unpack_pairs(xr[k], v);
-      if constexpr (OP == kOpLnStaticFp8) {
-        float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
-        if (c < C) {
-          const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
-          g0 = __ldg(reinterpret_cast<const float4*>(gp));
-          g1 = __ldg(reinterpret_cast<const float4*>(gp + 4));
-          e0 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c));
-          e1 = __ldg(reinterpret_cast<const float4*>(a.beta + 8 * c + 4));
-        }
-        const float2 g[4] = {make_float2(g0.x, g0.y), make_float2(g0.z, g0.w), make_float2(g1.x, g1.y),
-                             make_float2(g1.z, g1.w)};
-        const float2 b[4] = {make_float2(e0.x, e0.y), make_float2(e0.z, e0.w), make_float2(e1.x, e1.y),
-                             make_float2(e1.z, e1.w)};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = fma2(mul2(add2(v[i], nm), rs2), g[i], b[i]);
-      } else {
-        uint4 gu = make_uint4(0u, 0u, 0u, 0u);
-        if (c < C) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
-        float2 g[4];
-        unpack_pairs(gu, g);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = mul2(mul2(v[i], rs2), g[i]);
-      }
-      if (bf16_round) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = make_float2(round_bf16(v[i].x), round_bf16(v[i].y));
-      }
-      if constexpr (OP != kOpLnStaticFp8) {
-        if (a.norm_out != nullptr && ok)
-          *reinterpret_cast<uint4*>(a.norm_out + row * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
-      }
-      if constexpr (OP == kOpRmsNvfp4) {
-        float m8 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
-        const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));  // chunks c, c^1 form a block
-        const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), scale_in));
-        const float S = __fmul_rn(e4m3_to_f32(sfc), scale_in);
-        const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
-        float t[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (div && S != 0.0f) {
-            t[2 * i] = __fdiv_rn(v[i].x, S);
-            t[2 * i + 1] = __fdiv_rn(v[i].y, S);
-          } else {
-            const float2 q = mul2(v[i], f2(mult));
-            t[2 * i] = q.x;
-            t[2 * i + 1] = q.y;
-          }
-        }
-        const uint32_t packed = pack_e2m1x8(t);
-        if constexpr (SWZ) {
-          const uint32_t word = sf_word4(sfc);
-          if (ok && (c & 7) == 0)
-            *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(row, c >> 3, (C + 7) >> 3)) = word;
-        }
-        if (ok) {
-          *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
-          if (!SWZ && (c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
-        }
-      } else if constexpr (OP == kOpRmsGroupFp8) {
-        // the group's chunks are consecutive lanes (see quantize_groups)
-        const int cpg = a.group >> 3;
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
-        for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        float sg = __fdiv_rn(m, fp8_max<E5>());
-        if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
-        const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
-        float2 t[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          t[i] = (div && sg != 0.0f) ? make_float2(__fdiv_rn(v[i].x, sg), __fdiv_rn(v[i].y, sg)) : mul2(v[i], f2(ig));
-        if (ok) {
-          *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
-          if ((c & (cpg - 1)) == 0) {
-            if constexpr (LAYOUT)
-              store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
-                                c / cpg, d / a.group, sg);
-            else
-              a.scale_out[row * a.ld_scale + c / cpg] = sg;
-          }
-        }
-      } else {
-        float2 t[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
-        if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
-      }
-    }
-    if constexpr (SWZ) {
-      if (live) sf_zero_padding_rows<T>(a, row, tid);
-    }
+    process_raw_row<OP, T, K, OUT>(a, row, tid, [&](int k) { return xr[k]; }, GammaLoads<T>{a, tid, C}, b0, b1,
+                                   scale_in, inv_static, [] {});
   };
 
   if constexpr (!PERSIST) {
@@ -705,6 +755,148 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   }
 }
 
+// Rows without a residual, staged in shared memory: one thread per row issues
+// a single bulk asynchronous copy of the whole row (the TMA engine) that
+// completes on an mbarrier, and every pass re-reads the row from shared memory.
+// The row costs no registers while it is in flight or being processed, so
+// many more rows fit on an SM than with register rows (whose occupancy the row
+// data limits); the launch bound asks for at most 40 registers per thread.
+template <int T>
+constexpr int staged_min_blocks() {
+  constexpr int threads = (T == 32) ? 256 : T;
+  constexpr int blocks = 65536 / (threads * 40);
+  return blocks < 1 ? 1 : (blocks > 16 ? 16 : blocks);
+}
+
+template <int OP, int T, int K, int OUT>
+__global__ void __launch_bounds__(T == 32 ? 256 : T, (staged_min_blocks<T>())) row_kernel_staged(const RowArgs a) {
+  static_assert(OP != kOpRmsDynFp8, "staged rows: no residual");
+  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
+  constexpr int W = T / 32;
+  extern __shared__ __align__(128) uint4 s_rows[];  // R rows of d / 8 chunks
+  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
+  __shared__ __align__(8) uint64_t s_bar[R];
+  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
+  const int rsel = (T == 32) ? int(threadIdx.x >> 5) : 0;
+  const int64_t row = int64_t(blockIdx.x) * R + rsel;
+  const int C = a.d >> 3;
+  const uint4* xs = s_rows + int64_t(rsel) * C;
+
+  if (int(threadIdx.x) < R) mbar_init(&s_bar[threadIdx.x], 1);
+  fence_mbar_init();
+  __syncthreads();
+  griddep_wait();
+  const bool live = row < a.M;
+  if (live && tid == 0) {
+    const uint32_t bytes = uint32_t(a.d) * 2u;
+    mbar_arrive_expect_tx(&s_bar[rsel], bytes);
+    bulk_g2s(s_rows + int64_t(rsel) * C, a.x + row * a.ld_x, bytes, &s_bar[rsel]);
+  }
+  griddep_launch_dependents();
+  if (!live) return;  // a whole warp of a warp-per-row CTA: it takes part in no later barrier
+  const float scale_in = (OP == kOpRmsGroupFp8) ? 1.0f : __ldg(a.scale);
+  const float inv_static = __frcp_rn(scale_in);
+  if (!mbar_wait_bounded(&s_bar[rsel], 0)) {
+    // The copy did not land in time: record it, give the copy one more bounded
+    // wait, and finish the row anyway so that every thread meets the same
+    // barriers (its outputs are then not meaningful).
+    atomicOr(a.err, 1u);
+    (void)mbar_wait_bounded(&s_bar[rsel], 0);
+  }
+  process_raw_row<OP, T, K, OUT>(
+      a, row, tid,
+      [&](int k) {
+        const int c = tid + k * T;
+        return c < C ? xs[c] : make_uint4(0u, 0u, 0u, 0u);
+      },
+      GammaLoads<T>{a, tid, C}, s_sum[0], s_sum[1], scale_in, inv_static, [] {});
+}
+
+// Persistent rows without a residual through a ring of S row buffers in
+// shared memory.  CTA b walks rows b, b + G, b + 2G, ... (G = grid size).
+// Thread 0 keeps S bulk copies in flight: each lands one whole row and
+// completes on that stage's mbarrier.  A row is copied once from shared
+// memory into registers (raw bf16); after the row's first reduction barrier,
+// no thread reads the stage any more, so thread 0 refills it with the row S
+// steps ahead.  Gamma (and beta) of the thread's fixed columns stay in
+// registers for the whole kernel, so per row the L1 carries only the row
+// itself and its outputs.  Waits are bounded as in row_kernel_staged.
+template <int OP, int T, int K>
+constexpr int ring_min_blocks() {
+  // registers: gamma / beta (RMSNorm 4, LayerNorm 16 per chunk), the raw row
+  // (4 per chunk), ~48 working
+  constexpr int regs = (OP == kOpLnStaticFp8 ? 16 : 4) * K + 4 * K + 48;
+  constexpr int blocks = 65536 / (T * regs);
+  return blocks < 1 ? 1 : blocks;
+}
+
+template <int OP, int T, int K, int S, int OUT>
+__global__ void __launch_bounds__(T, (ring_min_blocks<OP, T, K>())) row_kernel_ring(const RowArgs a) {
+  static_assert(OP != kOpRmsDynFp8, "ring rows: no residual");
+  static_assert(T >= 64, "ring rows: one row per CTA");
+  constexpr int W = T / 32;
+  extern __shared__ __align__(128) uint4 s_ring[];  // S stages of d / 8 chunks
+  __shared__ __align__(16) float s_sum[2][W * 32];
+  __shared__ __align__(8) uint64_t s_full[S];
+  const int tid = int(threadIdx.x);
+  const int C = a.d >> 3;
+  const int64_t G = gridDim.x;
+  const uint32_t bytes = uint32_t(a.d) * 2u;
+
+  if (tid < S) mbar_init(&s_full[tid], 1);
+  fence_mbar_init();
+  __syncthreads();
+  griddep_wait();
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) {
+      const int64_t r = int64_t(blockIdx.x) + int64_t(i) * G;
+      if (r < a.M) {
+        mbar_arrive_expect_tx(&s_full[i], bytes);
+        bulk_g2s(s_ring + int64_t(i) * C, a.x + r * a.ld_x, bytes, &s_full[i]);
+      }
+    }
+  }
+  GammaRegs<OP == kOpLnStaticFp8, T, K> gam;
+  gam.load(a, tid, C);
+  const float scale_in = (OP == kOpRmsGroupFp8) ? 1.0f : __ldg(a.scale);
+  const float inv_static = __frcp_rn(scale_in);
+  bool released = false;
+  int j = 0;
+  for (int64_t row = blockIdx.x; row < a.M; row += G, ++j) {
+    const int st = j % S;
+    const uint32_t parity = uint32_t(j / S) & 1u;
+    const int64_t refill = row + int64_t(S) * G;  // the row this stage takes next
+    if (!released && refill >= a.M) {
+      griddep_launch_dependents();  // every load of this CTA is issued
+      released = true;
+    }
+    if (!mbar_wait_bounded(&s_full[st], parity)) {
+      atomicOr(a.err, 1u);  // see row_kernel_staged
+      (void)mbar_wait_bounded(&s_full[st], parity);
+    }
+    const uint4* xs = s_ring + int64_t(st) * C;
+    uint4 xr[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      xr[k] = c < C ? xs[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // Reduction buffers: LayerNorm's two sums use both (each separated from
+    // its next use by the other sum's barrier); single sums alternate by row.
+    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
+    process_raw_row<OP, T, K, OUT>(
+        a, row, tid, [&](int k) { return xr[k]; }, gam, b0, s_sum[1], scale_in, inv_static, [&] {
+          if (tid == 0 && refill < a.M) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive_expect_tx(&s_full[st], bytes);
+            bulk_g2s(s_ring + int64_t(st) * C, a.x + refill * a.ld_x, bytes, &s_full[st]);
+          }
+        });
+  }
+  if (!released) griddep_launch_dependents();
+}
+
 // Kernel table of one operation and output form (OUT bits): every built
 // (threads, chunks, vec) schedule.
 template <int OP, int OUT>
@@ -717,10 +909,16 @@ struct RowTable {
     for (auto& x : k.raw)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
+    for (auto& x : k.staged)
+      for (auto& y : x) y = nullptr;
+    for (auto& x : k.ring)
+      for (auto& y : x)
+        for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
   if constexpr (OP != kOpRmsDynFp8) {                                                                          \
     k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT>); \
     k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT>);  \
+    k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK), OUT>);     \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, OUT>); \
@@ -734,6 +932,17 @@ struct RowTable {
     NQ_DIRECT(9, 0) NQ_DIRECT(9, 1) NQ_DIRECT(9, 2)
     NQ_DIRECT(10, 0) NQ_DIRECT(10, 1)
     NQ_RAW(5, 4)  // one warp per row, 16 chunks per lane (rows of up to 4096 elements)
+#define NQ_RING(LT, LK)                                                                                           \
+  if constexpr (OP != kOpRmsDynFp8) {                                                                             \
+    k.ring[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_ring<OP, (1 << LT), (1 << LK), 2, OUT>); \
+    k.ring[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_ring<OP, (1 << LT), (1 << LK), 4, OUT>); \
+  }
+    NQ_RING(6, 0) NQ_RING(6, 1) NQ_RING(6, 2)
+    NQ_RING(7, 0) NQ_RING(7, 1) NQ_RING(7, 2)
+    NQ_RING(8, 0) NQ_RING(8, 1) NQ_RING(8, 2)
+    NQ_RING(9, 0) NQ_RING(9, 1) NQ_RING(9, 2)
+    NQ_RING(10, 0) NQ_RING(10, 1)
+#undef NQ_RING
 #undef NQ_DIRECT
 #undef NQ_RAW
   }

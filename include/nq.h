@@ -138,16 +138,26 @@ typedef enum nq_status {
 #define NQ_FLAG_GROUP_SCHEDULE(t, k) ((((uint32_t)(t)) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 /* Force a kernel variant (tests and tuning; same bits either way): n = 1 keeps
  * the row in float32 registers; n = 2 keeps only the raw bf16 row and unpacks
- * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row.
- * n = 2, 3 apply to 16-byte-aligned rows without a residual and are ignored
- * otherwise; with them NQ_FLAG_SCHEDULE also accepts t = 5, k = 4 (one warp
- * per row, 16 chunks per lane, rows of up to 4096 elements).  0 = automatic. */
+ * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row;
+ * n = 4 stages the row in shared memory with one bulk asynchronous copy and
+ * re-reads it there on every pass; n = 5 runs persistent CTAs that keep a ring
+ * of bulk copies of upcoming rows in flight and hold gamma (and beta) in
+ * registers (t >= 6, k <= 2 with NQ_FLAG_SCHEDULE).  n = 2..5 apply to
+ * 16-byte-aligned rows without a residual and are ignored otherwise; with
+ * n = 2..4, NQ_FLAG_SCHEDULE also accepts t = 5, k = 4 (one warp per row, 16
+ * chunks per lane, rows of up to 4096 elements).  0 = automatic. */
 #define NQ_FLAG_VARIANT(n) ((((uint32_t)(n)) & 0x7u) << 24)
 #define NQ_FLAG_VARIANT_MASK (0x7u << 24)
 /* Library version (major * 10000 + minor * 100 + patch). */
 int nq_version(void);
 /* Static text of a status code. */
 const char* nq_status_string(nq_status status);
+/* Synchronous: read and clear this library's device error word on the current
+ * device.  NQ_OK if no kernel recorded an error since the last check;
+ * NQ_ERR_CUDA (message in nq_last_error) if a kernel's bounded wait for its
+ * own bulk copy into shared memory gave up (about one second), in which case
+ * that launch's outputs are not meaningful.  Kernels never trap or hang. */
+nq_status nq_check_device_errors(void);
 /* Message of the last failing call on this thread ("" if none). */
 const char* nq_last_error(void);
 

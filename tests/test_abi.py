@@ -124,20 +124,26 @@ def test_validation_without_gpu(nq):
                                     None) == INV
 
 
-@pytest.mark.parametrize("M,d,exp", [
-    (64, 2816, (512, 1, 1)),      # fewer rows than SMs: one chunk per thread
-    (4096, 2816, (128, 4, 1)),    # rows > 1024 elements: one CTA per row, 4 chunks per thread
-    (4096, 4096, (128, 4, 1)),
-    (65536, 8192, (256, 4, 1)),
-    (8192, 7168, (256, 4, 1)),
-    (8192, 512, (32, 2, 8)),      # narrow rows: one warp per row, 8 rows per CTA
-    (8192, 1536, (64, 4, 1)),
-    (1, 8192, (1024, 1, 1)),      # a single row spreads over 1024 threads
-    (16, 16384, (1024, 2, 1)),
-    (1, 100, (32, 1, 8)),
+@pytest.mark.parametrize("op,M,d,exp", [
+    (0, 64, 2816, (512, 1, 1)),      # fewer rows than SMs: one chunk per thread
+    (0, 4096, 2816, (256, 2, 1)),    # residual-add dynamic, d <= 4096: two chunks per thread at any M
+    (0, 4096, 4096, (256, 2, 1)),
+    (0, 65536, 8192, (256, 4, 1)),   # wider rows: four chunks per thread
+    (0, 8192, 7168, (256, 4, 1)),
+    (0, 8192, 512, (32, 2, 8)),      # narrow rows: one warp per row, 8 rows per CTA
+    (0, 8192, 1536, (128, 2, 1)),
+    (0, 1, 8192, (1024, 1, 1)),      # a single row spreads over 1024 threads
+    (0, 16, 16384, (1024, 2, 1)),
+    (0, 1, 100, (32, 1, 8)),
+    (1, 4096, 4096, (128, 4, 1)),    # static RMSNorm: four chunks once there are many rows per SM
+    (1, 600, 4096, (256, 2, 1)),     # ... two below 768 rows
+    (1, 160, 4096, (512, 1, 1)),     # ... one below 192 rows
+    (1, 300, 7168, (512, 2, 1)),     # two below 384 rows
+    (2, 512, 4096, (256, 2, 1)),
+    (4, 600, 4096, (128, 4, 1)),     # fused group: four chunks from 384 rows
 ])
-def test_planner(nq, M, d, exp):
-    assert nq.nq_query_schedule(0, M, d) == exp
+def test_planner(nq, op, M, d, exp):
+    assert nq.nq_query_schedule(op, M, d) == exp
 
 
 def test_planner_forced_schedules(nq):
