@@ -30,7 +30,7 @@ __all__ = [
     "nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4", "OP_RMS_GROUP_FP8",
-    "nq_rmsnorm_quant_fp8_group", "nq_check_device_errors",
+    "nq_rmsnorm_quant_fp8_group", "nq_check_device_errors", "nq_selftest_division",
 ]
 
 NQ_OK, NQ_ERR_INVALID_ARGUMENT, NQ_ERR_UNSUPPORTED, NQ_ERR_CUDA = 0, 1, 2, 3
@@ -83,6 +83,8 @@ def _load() -> ctypes.CDLL:
     L.nq_status_string.argtypes, L.nq_status_string.restype = [st], ctypes.c_char_p
     L.nq_last_error.argtypes, L.nq_last_error.restype = [], ctypes.c_char_p
     L.nq_check_device_errors.argtypes, L.nq_check_device_errors.restype = [], st
+    L.nq_selftest_division.argtypes = [U32, ctypes.c_uint64, P, I32, P, P]
+    L.nq_selftest_division.restype = st
     L.nq_query_schedule.argtypes = [ctypes.c_int, I64, I64, U32, ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     L.nq_query_schedule.restype = st
@@ -116,6 +118,18 @@ def __getattr__(name):  # module attribute `lib`, loaded on first access
 
 def version() -> int:
     return _get_lib().nq_version()
+
+
+def nq_selftest_division(divisors, a_bits_begin: int = 0, count: int = 1 << 32, stream=None) -> int:
+    """Mismatches of the dynamic path's bounded division against the correctly
+    rounded quotient, over a bit range of dividends and float32 CUDA `divisors`."""
+    _need(isinstance(divisors, torch.Tensor) and divisors.is_cuda and divisors.dtype == torch.float32
+          and divisors.dim() == 1 and divisors.is_contiguous(), "divisors must be a contiguous float32 CUDA vector")
+    out = torch.zeros(1, dtype=torch.int64, device=divisors.device)
+    with torch.cuda.device(divisors.device):
+        _check(_get_lib().nq_selftest_division(a_bits_begin, count, _ptr(divisors), divisors.numel(), _ptr(out),
+                                               _stream(stream)), "nq_selftest_division")
+    return int(out.item())
 
 
 def nq_check_device_errors() -> None:

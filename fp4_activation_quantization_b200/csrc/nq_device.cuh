@@ -117,6 +117,35 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
 }
 __device__ __forceinline__ uint32_t f32_to_e4m3(float a) { return pack_e4m3x4(a, 0.f, 0.f, 0.f) & 0xFFu; }
 
+// ------------------------------------------------ bounded division ------
+// RN(a / b) for one divisor b shared by many quotients, from r = RN(1 / b)
+// (correctly rounded).  q0 = RN(a r) is within 1.5 ulp of a / b; each step
+// t = q b - a (fma), q' = q + t (-r) (fma) is the FMA remainder correction of
+// Markstein (IBM J. Res. Dev. 34(1), 1990; Muller et al., "Handbook of
+// Floating-Point Arithmetic", FMA-based division).  The first step brings q
+// within one ulp, and the second then rounds correctly while the remainders
+// are normal.  Contract, for b in [2^-60, 2^100] and |a / b| <= 2^17 (the
+// callers guarantee both): the result is RN(a / b) bit for bit when
+// |a / b| >= 2^-24; smaller quotients keep the sign of a / b and stay below
+// 2^-20, so their e4m3 / e5m2 code is the same signed zero.  The remainder is
+// taken as q b - a (not a - q b) so that a zero quotient keeps the sign of a.
+// nq_selftest_division checks this over every float32 dividend.
+constexpr float kFastDivMinDivisor = 8.6736173798840355e-19f;  // 2^-60
+constexpr float kFastDivMaxDivisor = 1.2676506002282294e30f;   // 2^100
+__device__ __forceinline__ bool fast_div_ok(float b) { return b >= kFastDivMinDivisor && b <= kFastDivMaxDivisor; }
+__device__ __forceinline__ float div_rn_by(float a, float b, float nr) {
+  const float q0 = __fmul_rn(a, -nr);
+  const float q1 = __fmaf_rn(__fmaf_rn(q0, b, -a), nr, q0);
+  return __fmaf_rn(__fmaf_rn(q1, b, -a), nr, q1);
+}
+// Two lanes at once (packed fp32x2, each lane rounding as its scalar form).
+__device__ __forceinline__ float2 div2_rn_by(float2 a, float2 b2, float2 nr2) {
+  const float2 na = make_float2(-a.x, -a.y);
+  const float2 q0 = __fmul2_rn(a, make_float2(-nr2.x, -nr2.y));
+  const float2 q1 = __ffma2_rn(__ffma2_rn(q0, b2, na), nr2, q0);
+  return __ffma2_rn(__ffma2_rn(q1, b2, na), nr2, q1);
+}
+
 // ------------------------------------------------------ group scales -----
 // Store the scale s of group g (of n_groups) of a row.  Float layout: element
 // row * rs + g * cs (row-major: rs = ld, cs = 1; column-major: rs = 1, cs =

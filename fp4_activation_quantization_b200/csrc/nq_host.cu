@@ -12,12 +12,44 @@
 #include <vector>
 
 #include "nq.h"
+#include "nq_device.cuh"
 #include "nq_internal.h"
 
 // Device error word of this library: bit 0 is set by a kernel whose bounded
 // wait on its own bulk copy gave up (read and cleared by
 // nq_check_device_errors).  A symbol, not an allocation.
 __device__ uint32_t g_nq_device_error;
+
+// Exhaustive check of the bounded division (nq_selftest_division): for
+// a = the float with bits a_begin + i and each divisor b in its domain, count
+// quotients q of div_rn_by / div2_rn_by that break its contract against the
+// correctly rounded ref = __fdiv_rn(a, b): q == ref bit for bit when
+// |ref| >= 2^-24; below, q has the sign of ref and |q| < 2^-20, so both give
+// the same (signed zero) FP8 code.
+__device__ __forceinline__ unsigned selftest_bad(float q, float ref) {
+  if (fabsf(ref) >= 5.9604645e-08f) return __float_as_uint(q) != __float_as_uint(ref);  // 2^-24
+  return ((__float_as_uint(q) ^ __float_as_uint(ref)) >> 31) | (fabsf(q) >= 9.5367432e-07f);  // 2^-20
+}
+__global__ void __launch_bounds__(256) selftest_division_kernel(uint32_t a_begin, uint64_t count, const float* divs,
+                                                                int n_div, unsigned long long* mismatches) {
+  unsigned long long local = 0;
+  const uint64_t stride = uint64_t(gridDim.x) * blockDim.x;
+  for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+    const float a = __uint_as_float(uint32_t(a_begin + i));
+    const float a2 = __uint_as_float(uint32_t(a_begin + i) ^ 0x80000000u);  // the other sign, second lane
+    for (int j = 0; j < n_div; ++j) {
+      const float b = divs[j];
+      if (!nq::fast_div_ok(b) || !(fabsf(a) <= 131072.0f * b)) continue;  // outside the domain (NaN too)
+      const float nr = -__frcp_rn(b);
+      const float ref = __fdiv_rn(a, b), ref2 = __fdiv_rn(a2, b);
+      const float2 q2 = nq::div2_rn_by(make_float2(a, a2), make_float2(b, b), make_float2(nr, nr));
+      local += selftest_bad(nq::div_rn_by(a, b, nr), ref);
+      local += selftest_bad(q2.x, ref) + selftest_bad(q2.y, ref2);
+    }
+  }
+  for (int o = 16; o >= 1; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+  if ((threadIdx.x & 31) == 0 && local) atomicAdd(mismatches, local);
+}
 
 namespace {
 
@@ -408,6 +440,29 @@ const char* nq_status_string(nq_status status) {
 }
 
 const char* nq_last_error(void) { return g_last_error.c_str(); }
+
+nq_status nq_selftest_division(uint32_t a_bits_begin, uint64_t count, const float* divisors, int32_t n_divisors,
+                               unsigned long long* mismatches, nq_stream_t stream) {
+  const char* fn = "nq_selftest_division";
+  NQ_REQUIRE(count <= (uint64_t(1) << 32) && uint64_t(a_bits_begin) + count <= (uint64_t(1) << 32),
+             "%s: the bit range must stay within 32 bits", fn);
+  NQ_REQUIRE(n_divisors >= 0 && (n_divisors == 0 || divisors != nullptr) && mismatches != nullptr,
+             "%s: divisors and mismatches are required", fn);
+  if (count == 0 || n_divisors == 0) return NQ_OK;
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      (void)cudaGetLastError();
+      sms = 148;
+    }
+  }
+  const uint64_t blocks = (count + 255) / 256;
+  const unsigned grid = unsigned(blocks < uint64_t(sms) * 16 ? blocks : uint64_t(sms) * 16);
+  void* args[] = {&a_bits_begin, &count, &divisors, &n_divisors, &mismatches};
+  return launch(fn, reinterpret_cast<const void*>(&selftest_division_kernel), grid, 256, 0, args, false,
+                static_cast<cudaStream_t>(stream));
+}
 
 nq_status nq_check_device_errors(void) {
   const char* fn = "nq_check_device_errors";

@@ -431,6 +431,11 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     }
     uint8_t* qrow = a.q + row * a.ld_q;
     const float2 inv2 = f2(s_inv);
+    // Dynamic scale with division: |y / s| <= 448 (57344), so the bounded
+    // division from RN(1 / s) is exact (nq_device.cuh); tiny scales keep the
+    // library division.
+    const bool fast = (OP == kOpRmsDynFp8) && div && fast_div_ok(s_div);
+    const float2 s2 = f2(s_div), nr2 = f2(-s_inv);
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
@@ -438,6 +443,9 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       if (passthrough) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) t[i] = v[k][i];
+      } else if (fast) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = div2_rn_by(v[k][i], s2, nr2);
       } else if (div) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) t[i] = make_float2(__fdiv_rn(v[k][i].x, s_div), __fdiv_rn(v[k][i].y, s_div));

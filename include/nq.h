@@ -158,6 +158,19 @@ const char* nq_status_string(nq_status status);
  * own bulk copy into shared memory gave up (about one second), in which case
  * that launch's outputs are not meaningful.  Kernels never trap or hang. */
 nq_status nq_check_device_errors(void);
+/* Diagnostic (tests): checks, on the device, the bounded division the dynamic
+ * FP8 path uses for RN(y / s) (a correctly rounded reciprocal r = RN(1 / s),
+ * then two FMA remainder corrections; Markstein 1990).  For every a whose
+ * bits are a_bits_begin .. a_bits_begin + count - 1 (and -a), and every
+ * divisor b of divisors[n_divisors] (device memory) in the domain the kernels
+ * use it on (b in [2^-60, 2^100], |a / b| <= 2^17), compares the scalar and the
+ * packed forms with the correctly rounded quotient and adds to *mismatches (a
+ * device unsigned long long) the quotients that break the contract: equal bit
+ * for bit when |a / b| >= 2^-24, else the same sign and magnitude < 2^-20 (so
+ * the same signed-zero FP8 code).
+ * Asynchronous on stream. */
+nq_status nq_selftest_division(uint32_t a_bits_begin, uint64_t count, const float* divisors, int32_t n_divisors,
+                               unsigned long long* mismatches, nq_stream_t stream);
 /* Message of the last failing call on this thread ("" if none). */
 const char* nq_last_error(void);
 
