@@ -16,6 +16,12 @@
 namespace nq {
 
 constexpr unsigned kFull = 0xffffffffu;
+
+// A compile-time bool passed to generic lambdas (decltype(tag)::value).
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
 constexpr float kE4M3Max = 448.0f;
 constexpr float kE5M2Max = 57344.0f;
 constexpr float kE2M1Max = 6.0f;

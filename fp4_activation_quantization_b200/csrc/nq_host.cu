@@ -364,10 +364,12 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     // CTA gets two or more rows, from the persistent prefetching form; NVFP4
     // gains from raw rows on wide rows; LayerNorm from raw rows once a row
     // has 1024 elements or more (up to 1.37x at d = 7168: its float32 row
-    // would hold twice the registers).
+    // would hold twice the registers); the fused group quantization from raw
+    // rows at every width (1.13x - 1.26x).
     if (op == nq::kOpRmsStaticFp8) variant = 3;
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
     else if (op == nq::kOpLnStaticFp8 && a.d >= 1024) variant = 2;
+    else if (op == nq::kOpRmsGroupFp8) variant = 2;
   }
   const void* k = nullptr;
   size_t smem = 0;

@@ -140,13 +140,12 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 // groups (one per lane).
 template <bool E5, bool LAYOUT, int T, int K, bool VEC, bool FULL>
 __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
-                                                const float2 (&v)[K][4]) {
+                                                const float2 (&v)[K][4], bool div) {
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
   const int cpg = a.group >> 3;  // chunks per group: 8 or 16
   const int gpw = 32 / cpg;      // groups per warp per chunk slot
   const int lane = tid & 31;
-  const bool div = (a.flags & kFlagDiv) != 0;
   const bool ue8m0 = (a.flags & kFlagUe8m0) != 0;
   uint8_t* qrow = a.q + row * a.ld_q;
   float* srow = a.scale_out + row * a.ld_scale;
@@ -221,7 +220,8 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
   const bool live = FULL || live_in;
-  const bool div = (a.flags & kFlagDiv) != 0;
+  const bool div_flag = (a.flags & kFlagDiv) != 0;
+  const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
   // ---- a2: r = x + residual, residual_out; a3: chunk partials
   float2 v[K][4];
   float part[K];
@@ -278,9 +278,16 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
   }
 
+  // ---- a4..a6.  The plain form (the call's default quantization, no bf16
+  // rounding, no norm output) is a separate copy with those flags folded
+  // away, so its per-chunk code carries no branch on them (K >= 4, below).
+  auto finish = [&](auto plain_tag) {
+  constexpr bool PLAIN = decltype(plain_tag)::value;
+  const bool div = PLAIN ? (OP == kOpRmsDynFp8) : div_flag;
+  const bool bf16_round = PLAIN ? false : bf16_flag;
+  uint16_t* const norm_out = PLAIN ? nullptr : a.norm_out;
   // ---- a4: normalize (y overwrites v); gamma / beta fetched now, through L1
   const float2 rs2 = f2(rstd);
-  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
@@ -337,8 +344,8 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     }
   }
   if constexpr (OP != kOpLnStaticFp8) {
-    if (a.norm_out != nullptr) {
-      uint16_t* nrow = a.norm_out + row * a.ld_norm;
+    if (norm_out != nullptr) {
+      uint16_t* nrow = norm_out + row * a.ld_norm;
 #pragma unroll
       for (int k = 0; k < K; ++k) {
         const int c = tid + k * T;
@@ -409,7 +416,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       if (live) sf_zero_padding_rows<T>(a, row, tid);
     }
   } else if constexpr (OP == kOpRmsGroupFp8) {
-    quantize_groups<E5, LAYOUT, T, K, VEC, FULL>(a, row, live, tid, v);
+    quantize_groups<E5, LAYOUT, T, K, VEC, FULL>(a, row, live, tid, v, div);
   } else {
     float s_div, s_inv;
     bool passthrough = false;
@@ -430,29 +437,8 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       s_inv = __frcp_rn(s_div);
     }
     uint8_t* qrow = a.q + row * a.ld_q;
-    const float2 inv2 = f2(s_inv);
-    // Dynamic scale with division: |y / s| <= 448 (57344), so the bounded
-    // division from RN(1 / s) is exact (nq_device.cuh); tiny scales keep the
-    // library division.
-    const bool fast = (OP == kOpRmsDynFp8) && div && fast_div_ok(s_div);
-    const float2 s2 = f2(s_div), nr2 = f2(-s_inv);
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
+    auto store_codes = [&](int k, const float2 (&t)[4]) {
       const int c = tid + k * T;
-      float2 t[4];
-      if (passthrough) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = v[k][i];
-      } else if (fast) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = div2_rn_by(v[k][i], s2, nr2);
-      } else if (div) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = make_float2(__fdiv_rn(v[k][i].x, s_div), __fdiv_rn(v[k][i].y, s_div));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) t[i] = mul2(v[k][i], inv2);
-      }
       const uint2 codes = pack_pairs_fp8<E5>(t);
       if (FULL || (live && c < C)) {
         if constexpr (VEC) {
@@ -463,8 +449,47 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
             if (8 * c + j < d) qrow[8 * c + j] = uint8_t((j < 4 ? codes.x : codes.y) >> (8 * (j & 3)));
         }
       }
+    };
+    // Dynamic scale with division: |y / s| <= 448 (57344), so the bounded
+    // division from RN(1 / s) is exact (nq_device.cuh); tiny scales keep the
+    // library division.  Each form is its own loop.
+    const bool fast = (OP == kOpRmsDynFp8) && div && fast_div_ok(s_div);
+    if (passthrough) {
+#pragma unroll
+      for (int k = 0; k < K; ++k) store_codes(k, v[k]);
+    } else if (fast) {
+      const float2 s2 = f2(s_div), nr2 = f2(-s_inv);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        float2 t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = div2_rn_by(v[k][i], s2, nr2);
+        store_codes(k, t);
+      }
+    } else if (div) {
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        float2 t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = make_float2(__fdiv_rn(v[k][i].x, s_div), __fdiv_rn(v[k][i].y, s_div));
+        store_codes(k, t);
+      }
+    } else {
+      const float2 inv2 = f2(s_inv);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        float2 t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) t[i] = mul2(v[k][i], inv2);
+        store_codes(k, t);
+      }
     }
   }
+  };
+  // Measured on B200: the second copy pays with four chunks per thread
+  // (4-7 %), but costs an SM slot with two or fewer (38 -> 43 registers).
+  if (K >= 4 && !bf16_flag && a.norm_out == nullptr && div_flag == (OP == kOpRmsDynFp8)) finish(BoolTag<true>{});
+  else finish(BoolTag<false>{});
 }
 
 // One row per thread group: loads straight to registers.  Many small CTAs per
@@ -560,8 +585,8 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   const int d = a.d;
   const int C = d >> 3;
   const float fd = float(d);
-  const bool div = (a.flags & kFlagDiv) != 0;
-  const bool bf16_round = (a.flags & kFlagNormBf16) != 0;
+  const bool div_flag = (a.flags & kFlagDiv) != 0;
+  const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
   const bool live = row < a.M;  // rows past M (warp rows only) compute on zeros and store nothing
   float part[K];
 #pragma unroll
@@ -592,6 +617,15 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   }
   const float2 rs2 = f2(rstd), nm = f2(-mean), inv2 = f2(inv_static);
   uint8_t* qrow = a.q + row * a.ld_q;
+  // Pass 3.  The plain form (reciprocal quantization, no bf16 rounding, no
+  // norm output: the default of every call) is a separate copy of the loop
+  // with those flags folded away, so the per-chunk code carries no branch on
+  // them and no library-division call site.
+  auto pass3 = [&](auto plain_tag) {
+  constexpr bool PLAIN = decltype(plain_tag)::value;
+  const bool div = PLAIN ? false : div_flag;
+  const bool bf16_round = PLAIN ? false : bf16_flag;
+  uint16_t* const norm_out = PLAIN ? nullptr : a.norm_out;
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
@@ -618,8 +652,8 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
       for (int i = 0; i < 4; ++i) v[i] = make_float2(round_bf16(v[i].x), round_bf16(v[i].y));
     }
     if constexpr (OP != kOpLnStaticFp8) {
-      if (a.norm_out != nullptr && ok)
-        *reinterpret_cast<uint4*>(a.norm_out + row * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
+      if (norm_out != nullptr && ok)
+        *reinterpret_cast<uint4*>(norm_out + row * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
     }
     if constexpr (OP == kOpRmsNvfp4) {
       float m8 = 0.0f;
@@ -683,6 +717,9 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
       if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
     }
   }
+  };
+  if (!div_flag && !bf16_flag && a.norm_out == nullptr) pass3(BoolTag<true>{});
+  else pass3(BoolTag<false>{});
   if constexpr (SWZ) {
     if (live) sf_zero_padding_rows<T>(a, row, tid);
   }
