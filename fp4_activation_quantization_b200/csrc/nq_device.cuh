@@ -152,6 +152,17 @@ __device__ __forceinline__ float2 div2_rn_by(float2 a, float2 b2, float2 nr2) {
   return __ffma2_rn(__ffma2_rn(q1, b2, na), nr2, q1);
 }
 
+// s = RN(amax / max) for the FP8 format's largest value (448 or 57344):
+// the bounded division where its quotient lies in [2^-24, 2^17], else the
+// library division; always the correctly rounded quotient.
+template <bool E5>
+__device__ __forceinline__ float fp8_scale_of(float amax) {
+  constexpr float kMax = E5 ? 57344.0f : 448.0f;
+  constexpr float kNegRcp = -(1.0f / kMax);
+  constexpr float kLo = 5.9604645e-08f, kHi = 131072.0f;  // 2^-24, 2^17
+  return (amax >= kMax * kLo && amax <= kMax * kHi) ? div_rn_by(amax, kMax, kNegRcp) : __fdiv_rn(amax, kMax);
+}
+
 // ------------------------------------------------------ group scales -----
 // Store the scale s of group g (of n_groups) of a row.  Float layout: element
 // row * rs + g * cs (row-major: rs = ld, cs = 1; column-major: rs = 1, cs =

@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
     }
 #pragma unroll
     for (int o = TPG / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    float s = __fdiv_rn(m, fp8_max<E5>());
+    float s = fp8_scale_of<E5>(m);
     if (ue8m0) s = ue8m0_ceil(s);
     const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
     const float2 inv2 = make_float2(inv, inv);

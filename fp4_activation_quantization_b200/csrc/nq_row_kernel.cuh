@@ -77,6 +77,38 @@ __device__ __forceinline__ void sf_zero_padding_rows(const RowArgs& a, int64_t r
     for (int j = tid; j < n_ct; j += T) *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(p, j, n_ct)) = 0u;
 }
 
+// NVFP4 block scale of a 16-element block with absmax amax under the global
+// scale g: sf = e4m3(RN(RN(amax / 6) / g)), S = RN(dec(sf) * g) and the
+// element multiplier RN(1 / S) (0 when S == 0).  Both divisions use the
+// bounded division (nq_device.cuh) where its quotient lies in [2^-24, 2^17]
+// and its divisor in range (ngr = -RN(1 / g), g_fast = g in range), else the
+// library division, so the result is always the correctly rounded one.
+struct Nvfp4Scale {
+  uint32_t code;
+  float mult;
+};
+__device__ __forceinline__ Nvfp4Scale nvfp4_block_scale(float amax, float g, float ngr, bool g_fast) {
+  constexpr float kSix = 6.0f, kNegRcpSix = -(1.0f / 6.0f);
+  constexpr float kLo = 5.9604645e-08f, kHi = 131072.0f;  // 2^-24, 2^17
+  const float x = (amax >= kSix * kLo && amax <= kSix * kHi) ? div_rn_by(amax, kSix, kNegRcpSix)
+                                                             : __fdiv_rn(amax, kSix);
+  const float q = (g_fast && x >= g * kLo && x <= g * kHi) ? div_rn_by(x, g, ngr) : __fdiv_rn(x, g);
+  const uint32_t code = f32_to_e4m3(q);
+  const float S = __fmul_rn(e4m3_to_f32(code), g);
+  return {code, (S == 0.0f) ? 0.0f : __frcp_rn(S)};
+}
+// Block scales of two chunk slots whose blocks each span this lane and its
+// xor-1 partner: the even lane computes slot 0's, the odd lane slot 1's, and
+// they swap, so each scale is computed once per pair instead of twice.
+__device__ __forceinline__ void nvfp4_pair_scales(float amax0, float amax1, int tid, float g, float ngr, bool g_fast,
+                                                  Nvfp4Scale& s0, Nvfp4Scale& s1) {
+  const bool odd = (tid & 1) != 0;
+  const Nvfp4Scale m = nvfp4_block_scale(odd ? amax1 : amax0, g, ngr, g_fast);
+  const Nvfp4Scale o = {__shfl_xor_sync(kFull, m.code, 1), __shfl_xor_sync(kFull, m.mult, 1)};
+  s0 = odd ? o : m;
+  s1 = odd ? m : o;
+}
+
 // Chunk partial of the canonical order: even / odd accumulators from +0,
 // then RN(even + odd).
 template <bool SQUARES>
@@ -169,7 +201,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
     const float t = __shfl_sync(kFull, am[k], (lane % gpw) * cpg);
     if (lane / gpw == k) mine = t;
   }
-  float s = __fdiv_rn(mine, fp8_max<E5>());
+  float s = fp8_scale_of<E5>(mine);
   if (ue8m0) s = ue8m0_ceil(s);
   const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
   {
@@ -367,21 +399,22 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   // ---- a5 + a6: scale, quantize, pack, store
   if constexpr (OP == kOpRmsNvfp4) {
     const float g = __ldg(a.scale);
+    const float ngr = -__frcp_rn(g);
+    const bool g_fast = fast_div_ok(g);
     uint8_t* qrow = a.q + row * a.ld_q;
     uint8_t* sfrow = a.sf + row * a.ld_sf;
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      const bool ok = FULL || (live && c < C);
+    // A 16-element block is chunks (c, c^1), held by lanes (t, t^1).
+    auto block_amax = [&](int k) {
       float m8 = 0.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
-      // A 16-element block is chunks (c, c^1), held by lanes (t, t^1).
-      const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
-      const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), g));
-      const float S = __fmul_rn(e4m3_to_f32(sfc), g);
-      const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+      return fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
+    };
+    auto quant_store = [&](int k, const Nvfp4Scale& sc) {
+      const int c = tid + k * T;
+      const bool ok = FULL || (live && c < C);
       float t[8];
+      const float S = div ? __fmul_rn(e4m3_to_f32(sc.code), g) : 0.0f;
       if (div && S != 0.0f) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -391,14 +424,14 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float2 q = mul2(v[k][i], f2(mult));
+          const float2 q = mul2(v[k][i], f2(sc.mult));
           t[2 * i] = q.x;
           t[2 * i + 1] = q.y;
         }
       }
       const uint32_t packed = pack_e2m1x8(t);
       if constexpr (SWZ) {
-        const uint32_t word = sf_word4(sfc);  // padding columns come from zero chunks
+        const uint32_t word = sf_word4(sc.code);  // padding columns come from zero chunks
         if (ok && (c & 7) == 0)
           *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(row, c >> 3, (C + 7) >> 3)) = word;
       }
@@ -409,8 +442,19 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
           for (int j = 0; j < 4; ++j) qrow[4 * c + j] = uint8_t(packed >> (8 * j));
         }
-        if (!SWZ && (c & 1) == 0) sfrow[c >> 1] = uint8_t(sfc);
+        if (!SWZ && (c & 1) == 0) sfrow[c >> 1] = uint8_t(sc.code);
       }
+    };
+    if constexpr (K >= 2) {
+#pragma unroll
+      for (int k = 0; k < K; k += 2) {
+        Nvfp4Scale s0, s1;
+        nvfp4_pair_scales(block_amax(k), block_amax(k + 1), tid, g, ngr, g_fast, s0, s1);
+        quant_store(k, s0);
+        quant_store(k + 1, s1);
+      }
+    } else {
+      quant_store(0, nvfp4_block_scale(block_amax(0), g, ngr, g_fast));
     }
     if constexpr (SWZ) {
       if (live) sf_zero_padding_rows<T>(a, row, tid);
@@ -427,7 +471,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
         for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
       const float amax = row_max_nonneg<T>(m, s_max, tid);
-      const float s = __fdiv_rn(amax, fp8_max<E5>());
+      const float s = fp8_scale_of<E5>(amax);
       if (live && tid == 0) a.scale_out[row] = s;
       s_div = s;
       s_inv = __frcp_rn(s);
@@ -626,11 +670,10 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   const bool div = PLAIN ? false : div_flag;
   const bool bf16_round = PLAIN ? false : bf16_flag;
   uint16_t* const norm_out = PLAIN ? nullptr : a.norm_out;
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
+  // y of chunk slot k (and its bf16 norm output)
+  auto norm_chunk = [&](int k, float2 (&v)[4]) {
     const int c = tid + k * T;
     const bool ok = live && c < C;
-    float2 v[4];
     unpack_pairs(src(k), v);
     if constexpr (OP == kOpLnStaticFp8) {
       float4 g0, g1, e0, e1;
@@ -655,14 +698,20 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
       if (norm_out != nullptr && ok)
         *reinterpret_cast<uint4*>(norm_out + row * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
     }
-    if constexpr (OP == kOpRmsNvfp4) {
+  };
+  if constexpr (OP == kOpRmsNvfp4) {
+    const float ngr = -__frcp_rn(scale_in);
+    const bool g_fast = fast_div_ok(scale_in);
+    auto block_amax = [&](const float2 (&v)[4]) {  // chunks c, c^1 (lanes t, t^1) form a block
       float m8 = 0.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
-      const float amax = fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));  // chunks c, c^1 form a block
-      const uint32_t sfc = f32_to_e4m3(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), scale_in));
-      const float S = __fmul_rn(e4m3_to_f32(sfc), scale_in);
-      const float mult = (S == 0.0f) ? 0.0f : __frcp_rn(S);
+      return fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
+    };
+    auto quant_store = [&](int k, const float2 (&v)[4], const Nvfp4Scale& sc) {
+      const int c = tid + k * T;
+      const bool ok = live && c < C;
+      const float S = div ? __fmul_rn(e4m3_to_f32(sc.code), scale_in) : 0.0f;
       float t[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -670,29 +719,53 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
           t[2 * i] = __fdiv_rn(v[i].x, S);
           t[2 * i + 1] = __fdiv_rn(v[i].y, S);
         } else {
-          const float2 q = mul2(v[i], f2(mult));
+          const float2 q = mul2(v[i], f2(sc.mult));
           t[2 * i] = q.x;
           t[2 * i + 1] = q.y;
         }
       }
       const uint32_t packed = pack_e2m1x8(t);
       if constexpr (SWZ) {
-        const uint32_t word = sf_word4(sfc);
+        const uint32_t word = sf_word4(sc.code);
         if (ok && (c & 7) == 0)
           *reinterpret_cast<uint32_t*>(a.sf + sf_swizzled_word(row, c >> 3, (C + 7) >> 3)) = word;
       }
       if (ok) {
         *reinterpret_cast<uint32_t*>(qrow + 4 * c) = packed;
-        if (!SWZ && (c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sfc);
+        if (!SWZ && (c & 1) == 0) a.sf[row * a.ld_sf + (c >> 1)] = uint8_t(sc.code);
       }
-    } else if constexpr (OP == kOpRmsGroupFp8) {
+    };
+    if constexpr (K >= 2) {
+#pragma unroll
+      for (int k = 0; k < K; k += 2) {
+        float2 v0[4], v1[4];
+        norm_chunk(k, v0);
+        norm_chunk(k + 1, v1);
+        Nvfp4Scale s0, s1;
+        nvfp4_pair_scales(block_amax(v0), block_amax(v1), tid, scale_in, ngr, g_fast, s0, s1);
+        quant_store(k, v0, s0);
+        quant_store(k + 1, v1, s1);
+      }
+    } else {
+      float2 v[4];
+      norm_chunk(0, v);
+      quant_store(0, v, nvfp4_block_scale(block_amax(v), scale_in, ngr, g_fast));
+    }
+  } else {
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const bool ok = live && c < C;
+    float2 v[4];
+    norm_chunk(k, v);
+    if constexpr (OP == kOpRmsGroupFp8) {
       // the group's chunks are consecutive lanes (see quantize_groups)
       const int cpg = a.group >> 3;
       float m = 0.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
       for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-      float sg = __fdiv_rn(m, fp8_max<E5>());
+      float sg = fp8_scale_of<E5>(m);
       if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
       const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
       float2 t[4];
@@ -716,6 +789,7 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
         t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
       if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
     }
+  }
   }
   };
   if (!div_flag && !bf16_flag && a.norm_out == nullptr) pass3(BoolTag<true>{});
