@@ -89,8 +89,8 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
                 "%s: NQ_FLAG_UE8M0 / NQ_FLAG_SCALES_* apply to group quantization only", fn);
   if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK)) && !allow_schedule)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_VARIANT apply to the norm calls only", fn);
-  if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 5)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT(n) takes n in 0..5", fn);
+  if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 6)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT(n) takes n in 0..6", fn);
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -137,6 +137,7 @@ nq_status group_scale_strides(const char* fn, uint32_t flags, int64_t M, int64_t
 //   P <= 512 (d <= 4096): two for the residual-add dynamic path at any M
 //     (more rows in flight per SM beat the longer per-thread chain), and for
 //     static RMSNorm, LayerNorm and NVFP4 while M < 768;
+//   LayerNorm with P = 1024 and M >= 768: eight;
 //   otherwise four (64 bytes of the row per thread, 128 with a residual, in
 //   flight at once).
 // Every mapping gives identical bits.
@@ -169,6 +170,9 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
     else if (lp <= 9 && (op == nq::kOpRmsDynFp8 ||
                          (M < 768 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8 || op == nq::kOpRmsNvfp4))))
       lk = 1;
+    // LayerNorm takes two rows per CTA (run_rows); with P = 1024 it runs
+    // best at eight chunks per thread (8192 x 7168: 54.1 -> 49.9 us).
+    if (op == nq::kOpLnStaticFp8 && lp == 10 && M >= 768) lk = 3;
     int lt = lp - lk;
     if (lt > 10) lt = 10;
     s->log_t = lt;
@@ -365,9 +369,12 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     // gains from raw rows on wide rows; LayerNorm from raw rows once a row
     // has 1024 elements or more (up to 1.37x at d = 7168: its float32 row
     // would hold twice the registers); the fused group quantization from raw
-    // rows at every width (1.13x - 1.26x).
+    // rows at every width (1.13x - 1.26x).  LayerNorm rows wider than a warp
+    // take two rows per CTA (gamma / beta loaded once for both: 1.27x at
+    // 65536 x 4096).
     if (op == nq::kOpRmsStaticFp8) variant = 3;
     else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
+    else if (op == nq::kOpLnStaticFp8 && threads > 32) variant = 6;
     else if (op == nq::kOpLnStaticFp8 && a.d >= 1024) variant = 2;
     else if (op == nq::kOpRmsGroupFp8) variant = 2;
   }
@@ -387,6 +394,11 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     const int64_t slots = resident_ctas(k, threads, smem);
     if (slots <= 0) return fail(NQ_ERR_UNSUPPORTED, "%s: ring kernel does not fit on an SM", fn);
     grid = grid < slots ? grid : slots;
+  }
+  if (vec && !has_res && variant == 6 && threads > 32 &&
+      (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
+    k = table.raw2[s.log_t - nq::kMinLogT][s.log_k];
+    if (k != nullptr) grid = (a.M + 1) / 2;
   }
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && variant == 4) {
     k = table.staged[s.log_t - nq::kMinLogT][s.log_k];

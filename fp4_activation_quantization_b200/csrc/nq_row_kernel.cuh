@@ -799,6 +799,179 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   }
 }
 
+// Two rows per thread group on the same columns (static RMSNorm and
+// LayerNorm without residual): each thread loads its gamma (and beta) chunk
+// once for both rows, and both rows' sums share one barrier.  The per-row
+// arithmetic and its order are those of process_raw_row.
+template <int T, int K>
+__device__ __forceinline__ void row_totals2(float (&part)[2][K], float (&out)[2], float* red, int tid) {
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+#pragma unroll
+    for (int h = K / 2; h >= 1; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) part[r][i] = __fadd_rn(part[r][i], part[r][i + h]);
+    out[r] = part[r][0];
+  }
+  if constexpr (T > 32) {
+    constexpr int W = T / 32;
+    const int lane = tid & 31, w = tid >> 5;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) red[(r * W + w) * 32 + lane] = out[r];
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float p[W];
+#pragma unroll
+      for (int i = 0; i < W; ++i) p[i] = red[(r * W + i) * 32 + lane];
+#pragma unroll
+      for (int h = W / 2; h >= 1; h >>= 1)
+#pragma unroll
+        for (int i = 0; i < h; ++i) p[i] = __fadd_rn(p[i], p[i + h]);
+      out[r] = p[0];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) out[r] = __fadd_rn(out[r], __shfl_xor_sync(kFull, out[r], o));
+}
+
+template <int OP, int T, int K, int OUT>
+__device__ __forceinline__ void process_raw_rows2(const RowArgs& a, const int64_t (&row)[2], int tid,
+                                                  const uint4 (&xr)[2][K], float* b0, float* b1, float scale_in,
+                                                  float inv_static) {
+  static_assert(OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8, "two-row form: static RMSNorm / LayerNorm");
+  constexpr bool E5 = (OUT & kOutAlt) != 0;
+  constexpr bool LN = OP == kOpLnStaticFp8;
+  const int d = a.d;
+  const int C = d >> 3;
+  const float fd = float(d);
+  const bool div_flag = (a.flags & kFlagDiv) != 0;
+  const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
+  float part[2][K], total[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      float2 v[4];
+      unpack_pairs(xr[r][k], v);
+      part[r][k] = chunk_partial<!LN>(v);
+    }
+  row_totals2<T, K>(part, total, b0, tid);
+  float rstd[2], mean[2] = {0.0f, 0.0f};
+  if constexpr (LN) {
+    float sq[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      mean[r] = __fdiv_rn(total[r], fd);
+      const float2 nm = f2(-mean[r]);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        const int c = tid + k * T;
+        float2 v[4];
+        unpack_pairs(xr[r][k], v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = (c < C) ? add2(v[i], nm) : f2(0.0f);
+        part[r][k] = chunk_partial<true>(v);
+      }
+    }
+    row_totals2<T, K>(part, sq, b1, tid);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) rstd[r] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq[r], fd), a.eps)));
+  } else {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) rstd[r] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total[r], fd), a.eps)));
+  }
+  const GammaLoads<T> gam{a, tid, C};
+  auto pass3 = [&](auto plain_tag) {
+    constexpr bool PLAIN = decltype(plain_tag)::value;
+    const bool div = PLAIN ? false : div_flag;
+    const bool bf16_round = PLAIN ? false : bf16_flag;
+    uint16_t* const norm_out = PLAIN ? nullptr : a.norm_out;
+    const float2 inv2 = f2(inv_static);
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      float2 g[4], b[4];
+      if constexpr (LN) {
+        float4 g0, g1, e0, e1;
+        gam.ln(k, g0, g1, e0, e1);
+        g[0] = make_float2(g0.x, g0.y); g[1] = make_float2(g0.z, g0.w);
+        g[2] = make_float2(g1.x, g1.y); g[3] = make_float2(g1.z, g1.w);
+        b[0] = make_float2(e0.x, e0.y); b[1] = make_float2(e0.z, e0.w);
+        b[2] = make_float2(e1.x, e1.y); b[3] = make_float2(e1.z, e1.w);
+      } else {
+        unpack_pairs(gam.rms(k), g);
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const bool ok = row[r] < a.M && c < C;
+        float2 v[4];
+        unpack_pairs(xr[r][k], v);
+        const float2 rs2 = f2(rstd[r]);
+        if constexpr (LN) {
+          const float2 nm = f2(-mean[r]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = fma2(mul2(add2(v[i], nm), rs2), g[i], b[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = mul2(mul2(v[i], rs2), g[i]);
+        }
+        if (bf16_round) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = make_float2(round_bf16(v[i].x), round_bf16(v[i].y));
+        }
+        if constexpr (!LN) {
+          if (norm_out != nullptr && ok)
+            *reinterpret_cast<uint4*>(norm_out + row[r] * a.ld_norm + 8 * c) = pack_pairs_bf16(v);
+        }
+        float2 t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
+        if (ok) *reinterpret_cast<uint2*>(a.q + row[r] * a.ld_q + 8 * c) = pack_pairs_fp8<E5>(t);
+      }
+    }
+  };
+  if (!div_flag && !bf16_flag && a.norm_out == nullptr) pass3(BoolTag<true>{});
+  else pass3(BoolTag<false>{});
+}
+
+template <int T, int K>
+constexpr int raw2_min_blocks() {
+  constexpr int cap = 8 * K + 64;  // two raw rows (4 registers per chunk each) + working set
+  constexpr int blocks = 65536 / (T * (cap < 64 ? 64 : cap));
+  return blocks < 1 ? 1 : blocks;
+}
+
+// Two rows per CTA (T >= 64), raw bf16 chunks in registers, not persistent.
+template <int OP, int T, int K, int OUT>
+__global__ void __launch_bounds__(T, (raw2_min_blocks<T, K>())) row_kernel_raw2(const RowArgs a) {
+  static_assert(T >= 64, "two-row form: one CTA per row pair");
+  constexpr int W = T / 32;
+  __shared__ __align__(16) float s_sum[2][2 * W * 32];
+  const int tid = int(threadIdx.x);
+  const int C = a.d >> 3;
+  const int64_t row[2] = {int64_t(blockIdx.x) * 2, int64_t(blockIdx.x) * 2 + 1};
+  griddep_wait();
+  const float scale_in = __ldg(a.scale);
+  const float inv_static = __frcp_rn(scale_in);
+  uint4 xr[2][K];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const uint16_t* xrow = a.x + row[r] * a.ld_x;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      xr[r][k] = (row[r] < a.M && c < C) ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  griddep_launch_dependents();
+  process_raw_rows2<OP, T, K, OUT>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
+}
+
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
 // residual), 16-byte rows, T > 32.  Only the raw bf16 chunks are kept (half
 // the registers of float32); each pass unpacks them again.  With PERSIST the
@@ -1030,6 +1203,8 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
     for (auto& x : k.staged)
       for (auto& y : x) y = nullptr;
+    for (auto& x : k.raw2)
+      for (auto& y : x) y = nullptr;
     for (auto& x : k.ring)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
@@ -1038,6 +1213,10 @@ struct RowTable {
     k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT>); \
     k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT>);  \
     k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK), OUT>);     \
+  }                                                                                                            \
+  if constexpr (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8) {                                               \
+    if constexpr (LT > 5 && LK <= 3)                                                                           \
+      k.raw2[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_raw2<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT>); \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, OUT>); \

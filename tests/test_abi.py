@@ -141,6 +141,7 @@ def test_validation_without_gpu(nq):
     (1, 300, 7168, (512, 2, 1)),     # two below 384 rows
     (2, 512, 4096, (256, 2, 1)),
     (4, 600, 4096, (128, 4, 1)),     # fused group: four chunks from 384 rows
+    (2, 8192, 7168, (128, 8, 1)),    # LayerNorm, P = 1024: eight chunks per thread
 ])
 def test_planner(nq, op, M, d, exp):
     assert nq.nq_query_schedule(op, M, d) == exp

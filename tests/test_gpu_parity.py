@@ -568,3 +568,25 @@ def test_ring_rows_output_forms(nq):
     assert np.array_equal(s.cpu().numpy().view(np.uint32),
                           oracle.group_scales_layout(es, col_major=True, packed=True).T)
     nq.nq_check_device_errors()
+
+
+@pytest.mark.parametrize("d,M", [(512, 7), (1024, 1), (2816, 301), (4096, 4097), (7168, 64), (16384, 33)])
+def test_two_row_variant_every_schedule(nq, d, M):
+    """NQ_FLAG_VARIANT(6): two rows per CTA on the same columns (static RMSNorm and LayerNorm),
+    every schedule with at least 64 threads, odd and even M."""
+    w = S.make_rms_inputs(M, d, seed=d * 3 + M, residual=False, x_outlier_channels=True)
+    lw = S.make_ln_inputs(M, d, seed=d * 3 + M + 1)
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    e_st, _, e_no = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, want_norm=True)
+    e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
+    e_div, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, flags=oracle.DIV)
+    lx, lgam, lbet = dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"])
+    for sched in [None] + [s_ for s_ in all_schedules(d) if s_[0] > 5]:
+        f = nq.flag_variant(6) | (0 if sched is None else nq.flag_schedule(*sched))
+        q, _, no = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, want_norm=True, flags=f)
+        assert np.array_equal(host_u8(q), e_st) and np.array_equal(host_u16(no), e_no), ("rms", sched)
+        q, _, _ = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, flags=f | nq.FLAG_SCALE_DIV)
+        assert np.array_equal(host_u8(q), e_div), ("rms div", sched)
+        q = nq.nq_layernorm_quant_fp8(lx, lgam, lbet, sc, 1e-6, flags=f)
+        assert np.array_equal(host_u8(q), e_ln), ("ln", sched)
