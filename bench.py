@@ -11,7 +11,8 @@ device time.
 Timing: inputs are generated on the device (seeded), and a step uses one of S
 rotating input/output sets whose total (S x 96 MiB) is several times the
 126 MB L2, so no step finds its inputs in L2.  Calls are captured into CUDA
-graphs of S launches and replayed back to back; CUDA events on the launching
+graphs of S launches (with programmatic dependent launch; ``--no-pdl``
+without) and replayed back to back; CUDA events on the launching
 stream bracket the whole timed region (exactly K steps) and every graph, which
 gives each kernel's mean launch duration for the roofline.  Multi-GPU runs
 (torchrun, one process per GPU) give every rank the same per-GPU workload
@@ -19,7 +20,8 @@ gives each kernel's mean launch duration for the roofline.  Multi-GPU runs
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 instead, on a bounded sample per step.  ``--sweep`` adds a per-configuration
-table (fused add+RMSNorm+dynamic FP8 sweep, group FP8, NVFP4) under "sweep".
+table (fused add+RMSNorm+dynamic FP8 sweep, group FP8, fused RMSNorm + group
+FP8, NVFP4) under "sweep".
 """
 from __future__ import annotations
 
@@ -276,7 +278,10 @@ def run_gpu_arm(args):
     set_bytes = M * d * 2 * 2 + M * d * 2          # two bf16 inputs + two e4m3 outputs
     S = max(8, -(-4 * L2_BYTES // set_bytes))      # > 4x L2 in flight between reuses
     wl = Workload(nq, M, d, S, seed=1234 + rank)
-    flags = nq.FLAG_PDL if args.pdl else 0
+    # Programmatic dependent launch: each kernel waits (griddepcontrol.wait)
+    # for the previous one before its first read, so no work is skipped; its
+    # CTAs are resident earlier, as when these kernels follow a GEMM.
+    flags = 0 if args.no_pdl else nq.FLAG_PDL
     g_rms, g_ln = wl.capture(wl.rms, S, flags), wl.capture(wl.ln, S, flags)
     K, W = args.steps, max(3, args.warmup)
     q_full, r = divmod(K, S)
@@ -393,7 +398,7 @@ def run_gpu_arm(args):
         "config": {"workload": "RMSNorm->e4m3 static + LayerNorm->e4m3 static, M=4096 tokens, d=4096",
                    "M": M, "d": d, "scale": SCALE, "eps": EPS, "io": "bf16 in, e4m3 out, fp32 math",
                    "l2": f"inputs rotate over {S} sets ({S * set_bytes / 2**20:.0f} MiB, > L2 126 MB)",
-                   "graphs": f"CUDA graphs of {S} launches replayed back to back", "pdl": bool(args.pdl),
+                   "graphs": f"CUDA graphs of {S} launches replayed back to back", "pdl": not args.no_pdl,
                    "parallelism": f"replicas x{world} (rows shard, no collective)"},
         "per_call": {"nq_rmsnorm_quant_fp8_static": {"us": round(rms_us, 3),
                                                      "GBps": round(rms_static_bytes(M, d) / rms_us / 1e3, 1)},
@@ -626,7 +631,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=40)
     ap.add_argument("--impl", choices=["nq", "reference"], default="nq")
-    ap.add_argument("--pdl", action="store_true", help="launch with programmatic dependent launch")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch (default: with)")
     ap.add_argument("--sweep", action="store_true", help="add the per-configuration table")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
