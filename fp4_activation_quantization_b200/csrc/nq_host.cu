@@ -395,9 +395,8 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     if (slots <= 0) return fail(NQ_ERR_UNSUPPORTED, "%s: ring kernel does not fit on an SM", fn);
     grid = grid < slots ? grid : slots;
   }
-  if (vec && !has_res && variant == 6 && threads > 32 &&
-      (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
-    k = table.raw2[s.log_t - nq::kMinLogT][s.log_k];
+  if (vec && !has_res && variant == 6 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
+    k = table.rows2[s.log_t - nq::kMinLogT][s.log_k];
     if (k != nullptr) grid = (a.M + 1) / 2;
   }
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && variant == 4) {

@@ -97,7 +97,7 @@ struct RowKernels {
   RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent]
   StagedTable staged;  // rows without residual staged in shared memory by a bulk copy
   RingTable ring;      // rows without residual through a ring of bulk copies, persistent
-  StagedTable raw2;    // two rows per CTA on the same columns (static RMSNorm / LayerNorm)
+  StagedTable rows2;   // two rows per CTA on the same columns (static RMSNorm / LayerNorm)
 };
 // Dynamic shared memory of a staged-row kernel: its rows of d bf16.
 inline size_t staged_smem_bytes(int threads, int64_t d) { return size_t(rows_per_cta(threads)) * size_t(d) * 2; }

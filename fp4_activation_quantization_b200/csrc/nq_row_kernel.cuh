@@ -799,14 +799,14 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   }
 }
 
-// Two rows per thread group on the same columns (static RMSNorm and
+// NR rows per thread group on the same columns (static RMSNorm and
 // LayerNorm without residual): each thread loads its gamma (and beta) chunk
-// once for both rows, and both rows' sums share one barrier.  The per-row
+// once for all NR rows, and the rows' sums share one barrier.  The per-row
 // arithmetic and its order are those of process_raw_row.
-template <int T, int K>
-__device__ __forceinline__ void row_totals2(float (&part)[2][K], float (&out)[2], float* red, int tid) {
+template <int T, int K, int NR>
+__device__ __forceinline__ void row_totals_n(float (&part)[NR][K], float (&out)[NR], float* red, int tid) {
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
+  for (int r = 0; r < NR; ++r) {
 #pragma unroll
     for (int h = K / 2; h >= 1; h >>= 1)
 #pragma unroll
@@ -817,10 +817,10 @@ __device__ __forceinline__ void row_totals2(float (&part)[2][K], float (&out)[2]
     constexpr int W = T / 32;
     const int lane = tid & 31, w = tid >> 5;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) red[(r * W + w) * 32 + lane] = out[r];
+    for (int r = 0; r < NR; ++r) red[(r * W + w) * 32 + lane] = out[r];
     __syncthreads();
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < NR; ++r) {
       float p[W];
 #pragma unroll
       for (int i = 0; i < W; ++i) p[i] = red[(r * W + i) * 32 + lane];
@@ -834,13 +834,13 @@ __device__ __forceinline__ void row_totals2(float (&part)[2][K], float (&out)[2]
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1)
 #pragma unroll
-    for (int r = 0; r < 2; ++r) out[r] = __fadd_rn(out[r], __shfl_xor_sync(kFull, out[r], o));
+    for (int r = 0; r < NR; ++r) out[r] = __fadd_rn(out[r], __shfl_xor_sync(kFull, out[r], o));
 }
 
-template <int OP, int T, int K, int OUT>
-__device__ __forceinline__ void process_raw_rows2(const RowArgs& a, const int64_t (&row)[2], int tid,
-                                                  const uint4 (&xr)[2][K], float* b0, float* b1, float scale_in,
-                                                  float inv_static) {
+template <int OP, int T, int K, int OUT, int NR>
+__device__ __forceinline__ void process_raw_rows_n(const RowArgs& a, const int64_t (&row)[NR], int tid,
+                                                   const uint4 (&xr)[NR][K], float* b0, float* b1, float scale_in,
+                                                   float inv_static) {
   static_assert(OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8, "two-row form: static RMSNorm / LayerNorm");
   constexpr bool E5 = (OUT & kOutAlt) != 0;
   constexpr bool LN = OP == kOpLnStaticFp8;
@@ -849,21 +849,21 @@ __device__ __forceinline__ void process_raw_rows2(const RowArgs& a, const int64_
   const float fd = float(d);
   const bool div_flag = (a.flags & kFlagDiv) != 0;
   const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
-  float part[2][K], total[2];
+  float part[NR][K], total[NR];
 #pragma unroll
-  for (int r = 0; r < 2; ++r)
+  for (int r = 0; r < NR; ++r)
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       float2 v[4];
       unpack_pairs(xr[r][k], v);
       part[r][k] = chunk_partial<!LN>(v);
     }
-  row_totals2<T, K>(part, total, b0, tid);
-  float rstd[2], mean[2] = {0.0f, 0.0f};
+  row_totals_n<T, K, NR>(part, total, b0, tid);
+  float rstd[NR], mean[NR] = {};
   if constexpr (LN) {
-    float sq[2];
+    float sq[NR];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < NR; ++r) {
       mean[r] = __fdiv_rn(total[r], fd);
       const float2 nm = f2(-mean[r]);
 #pragma unroll
@@ -876,12 +876,12 @@ __device__ __forceinline__ void process_raw_rows2(const RowArgs& a, const int64_
         part[r][k] = chunk_partial<true>(v);
       }
     }
-    row_totals2<T, K>(part, sq, b1, tid);
+    row_totals_n<T, K, NR>(part, sq, b1, tid);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) rstd[r] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq[r], fd), a.eps)));
+    for (int r = 0; r < NR; ++r) rstd[r] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq[r], fd), a.eps)));
   } else {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) rstd[r] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total[r], fd), a.eps)));
+    for (int r = 0; r < NR; ++r) rstd[r] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total[r], fd), a.eps)));
   }
   const GammaLoads<T> gam{a, tid, C};
   auto pass3 = [&](auto plain_tag) {
@@ -905,7 +905,7 @@ __device__ __forceinline__ void process_raw_rows2(const RowArgs& a, const int64_
         unpack_pairs(gam.rms(k), g);
       }
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
+      for (int r = 0; r < NR; ++r) {
         const bool ok = row[r] < a.M && c < C;
         float2 v[4];
         unpack_pairs(xr[r][k], v);
@@ -938,28 +938,32 @@ __device__ __forceinline__ void process_raw_rows2(const RowArgs& a, const int64_
   else pass3(BoolTag<false>{});
 }
 
-template <int T, int K>
-constexpr int raw2_min_blocks() {
-  constexpr int cap = 8 * K + 64;  // two raw rows (4 registers per chunk each) + working set
+template <int T, int K, int NR>
+constexpr int rows_n_min_blocks() {
+  constexpr int cap = 4 * NR * K + 64;  // NR raw rows (4 registers per chunk each) + working set
   constexpr int blocks = 65536 / (T * (cap < 64 ? 64 : cap));
   return blocks < 1 ? 1 : blocks;
 }
 
-// Two rows per CTA (T >= 64), raw bf16 chunks in registers, not persistent.
-template <int OP, int T, int K, int OUT>
-__global__ void __launch_bounds__(T, (raw2_min_blocks<T, K>())) row_kernel_raw2(const RowArgs a) {
-  static_assert(T >= 64, "two-row form: one CTA per row pair");
+// NR rows per CTA (T >= 64), raw bf16 chunks in registers, not persistent.
+// Built for NR = 2; four rows per CTA measured slower on B200 (their raw
+// rows spill or halve the resident CTAs).
+template <int OP, int T, int K, int OUT, int NR>
+__global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel_rows_n(const RowArgs a) {
+  static_assert(T >= 64, "multi-row form: one CTA per group of NR rows");
   constexpr int W = T / 32;
-  __shared__ __align__(16) float s_sum[2][2 * W * 32];
+  __shared__ __align__(16) float s_sum[2][NR * W * 32];
   const int tid = int(threadIdx.x);
   const int C = a.d >> 3;
-  const int64_t row[2] = {int64_t(blockIdx.x) * 2, int64_t(blockIdx.x) * 2 + 1};
+  int64_t row[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) row[r] = int64_t(blockIdx.x) * NR + r;
   griddep_wait();
   const float scale_in = __ldg(a.scale);
   const float inv_static = __frcp_rn(scale_in);
-  uint4 xr[2][K];
+  uint4 xr[NR][K];
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
+  for (int r = 0; r < NR; ++r) {
     const uint16_t* xrow = a.x + row[r] * a.ld_x;
 #pragma unroll
     for (int k = 0; k < K; ++k) {
@@ -969,7 +973,7 @@ __global__ void __launch_bounds__(T, (raw2_min_blocks<T, K>())) row_kernel_raw2(
     }
   }
   griddep_launch_dependents();
-  process_raw_rows2<OP, T, K, OUT>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
+  process_raw_rows_n<OP, T, K, OUT, NR>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
 }
 
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
@@ -1203,7 +1207,7 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
     for (auto& x : k.staged)
       for (auto& y : x) y = nullptr;
-    for (auto& x : k.raw2)
+    for (auto& x : k.rows2)
       for (auto& y : x) y = nullptr;
     for (auto& x : k.ring)
       for (auto& y : x)
@@ -1216,7 +1220,7 @@ struct RowTable {
   }                                                                                                            \
   if constexpr (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8) {                                               \
     if constexpr (LT > 5 && LK <= 3)                                                                           \
-      k.raw2[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_raw2<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT>); \
+      k.rows2[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2>); \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, OUT>); \

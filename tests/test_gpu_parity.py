@@ -582,11 +582,11 @@ def test_two_row_variant_every_schedule(nq, d, M):
     e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
     e_div, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, flags=oracle.DIV)
     lx, lgam, lbet = dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"])
-    for sched in [None] + [s_ for s_ in all_schedules(d) if s_[0] > 5]:
-        f = nq.flag_variant(6) | (0 if sched is None else nq.flag_schedule(*sched))
+    for var, sched in [(v, s_) for v in (6,) for s_ in [None] + [s_ for s_ in all_schedules(d) if s_[0] > 5]]:
+        f = nq.flag_variant(var) | (0 if sched is None else nq.flag_schedule(*sched))
         q, _, no = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, want_norm=True, flags=f)
-        assert np.array_equal(host_u8(q), e_st) and np.array_equal(host_u16(no), e_no), ("rms", sched)
+        assert np.array_equal(host_u8(q), e_st) and np.array_equal(host_u16(no), e_no), ("rms", var, sched)
         q, _, _ = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, flags=f | nq.FLAG_SCALE_DIV)
-        assert np.array_equal(host_u8(q), e_div), ("rms div", sched)
+        assert np.array_equal(host_u8(q), e_div), ("rms div", var, sched)
         q = nq.nq_layernorm_quant_fp8(lx, lgam, lbet, sc, 1e-6, flags=f)
-        assert np.array_equal(host_u8(q), e_ln), ("ln", sched)
+        assert np.array_equal(host_u8(q), e_ln), ("ln", var, sched)
