@@ -123,6 +123,20 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
 }
 __device__ __forceinline__ uint32_t f32_to_e4m3(float a) { return pack_e4m3x4(a, 0.f, 0.f, 0.f) & 0xFFu; }
 
+// ------------------------------------------------------------ absmax -----
+// max(m, |v_0|, ..., |v_7|) with three-input max.f32 (sm_100), half the
+// instructions of a two-input chain; exact, and the same result.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float absmax8(const float2 (&v)[4], float m) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = fmax3(m, fabsf(v[i].x), fabsf(v[i].y));
+  return m;
+}
+
 // ------------------------------------------------ bounded division ------
 // RN(a / b) for one divisor b shared by many quotients, from r = RN(1 / b)
 // (correctly rounded).  q0 = RN(a r) is within 1.5 ulp of a / b; each step

@@ -66,10 +66,10 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
     float m = 0.0f;
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {
-      float v[8];
-      unpack_bf16x8(raw[u][j], v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+      const uint4 w = raw[u][j];
+      const float2 v[4] = {make_float2(bf16_lo(w.x), bf16_hi(w.x)), make_float2(bf16_lo(w.y), bf16_hi(w.y)),
+                           make_float2(bf16_lo(w.z), bf16_hi(w.z)), make_float2(bf16_lo(w.w), bf16_hi(w.w))};
+      m = absmax8(v, m);
     }
 #pragma unroll
     for (int o = TPG / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));

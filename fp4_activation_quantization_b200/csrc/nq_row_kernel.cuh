@@ -185,9 +185,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
   float am[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
+    float m = absmax8(v[k], 0.0f);
     for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
     am[k] = m;
   }
@@ -405,9 +403,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     uint8_t* sfrow = a.sf + row * a.ld_sf;
     // A 16-element block is chunks (c, c^1), held by lanes (t, t^1).
     auto block_amax = [&](int k) {
-      float m8 = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
+      const float m8 = absmax8(v[k], 0.0f);
       return fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
     };
     auto quant_store = [&](int k, const Nvfp4Scale& sc) {
@@ -468,8 +464,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < K; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[k][i].x), fabsf(v[k][i].y)));
+        m = absmax8(v[k], m);
       const float amax = row_max_nonneg<T>(m, s_max, tid);
       const float s = fp8_scale_of<E5>(amax);
       if (live && tid == 0) a.scale_out[row] = s;
@@ -703,9 +698,7 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
     const float ngr = -__frcp_rn(scale_in);
     const bool g_fast = fast_div_ok(scale_in);
     auto block_amax = [&](const float2 (&v)[4]) {  // chunks c, c^1 (lanes t, t^1) form a block
-      float m8 = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) m8 = fmaxf(m8, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      const float m8 = absmax8(v, 0.0f);
       return fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
     };
     auto quant_store = [&](int k, const float2 (&v)[4], const Nvfp4Scale& sc) {
@@ -761,9 +754,7 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
     if constexpr (OP == kOpRmsGroupFp8) {
       // the group's chunks are consecutive lanes (see quantize_groups)
       const int cpg = a.group >> 3;
-      float m = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+      float m = absmax8(v, 0.0f);
       for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
       float sg = fp8_scale_of<E5>(m);
       if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
