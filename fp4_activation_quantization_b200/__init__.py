@@ -31,6 +31,7 @@ __all__ = [
     "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_query_schedule",
     "OP_RMS_DYN_FP8", "OP_RMS_STATIC_FP8", "OP_LN_STATIC_FP8", "OP_RMS_NVFP4", "OP_RMS_GROUP_FP8",
     "nq_rmsnorm_quant_fp8_group", "nq_check_device_errors", "nq_selftest_division",
+    "nq_fused_add_rmsnorm_quant_fp8_moe",
 ]
 
 NQ_OK, NQ_ERR_INVALID_ARGUMENT, NQ_ERR_UNSUPPORTED, NQ_ERR_CUDA = 0, 1, 2, 3
@@ -94,8 +95,11 @@ def _load() -> ctypes.CDLL:
     L.nq_per_token_group_quant_fp8.argtypes = [P, I64, P, I64, P, I64, I64, I64, I32, U32, P]
     L.nq_rmsnorm_quant_fp8_group.argtypes = [P, I64, P, P, I64, P, P, I64, P, I64, P, I64, I64, I64, I32, F, U32, P]
     L.nq_rmsnorm_quant_nvfp4.argtypes = [P, I64, P, P, I64, P, P, P, I64, P, I64, P, I64, I64, I64, F, U32, P]
+    L.nq_fused_add_rmsnorm_quant_fp8_moe.argtypes = [P, I64, P, P, I64, P, P, I32, I64, P, I64, P, I64, P, I64,
+                                                     I64, I64, I32, F, U32, P]
     for name in ("nq_fused_add_rmsnorm_quant_fp8", "nq_rmsnorm_quant_fp8_static", "nq_layernorm_quant_fp8",
-                 "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_rmsnorm_quant_fp8_group"):
+                 "nq_per_token_group_quant_fp8", "nq_rmsnorm_quant_nvfp4", "nq_rmsnorm_quant_fp8_group",
+                 "nq_fused_add_rmsnorm_quant_fp8_moe"):
         getattr(L, name).restype = st
     return L
 
@@ -432,3 +436,49 @@ def nq_rmsnorm_quant_nvfp4(x, gamma, global_scale, eps: float = 1e-6, *, residua
             ld_q, _ptr(sf_out), ld_sf, _ptr(norm_out), ld_n, M, d, eps, flags, _stream(stream)),
             "nq_rmsnorm_quant_nvfp4")
     return q_out, sf_out, residual_out, norm_out
+
+
+def nq_fused_add_rmsnorm_quant_fp8_moe(x, gamma, dest, rows: int, eps: float = 1e-6, *, group: int = 0,
+                                       residual=None, residual_out=None, q_out=None, scales_out=None,
+                                       norm_out=None, want_norm: bool = False, flags: int = 0, stream=None):
+    """Residual-add (optional) + RMSNorm + e4m3 stored into a MoE layer's permuted input.
+
+    ``dest`` int32 [M, topk] (CUDA): the permuted row of each (token, slot), < 0
+    skips.  ``group`` 0 gives one dynamic scale per token, 64 / 128 per-token-
+    group scales.  Returns ``(q float8_e4m3fn [rows, d], scales float32 [rows]
+    or [rows, d/group], residual_out or None, norm_out or None)``.
+    """
+    M, d, ld_x = _rows(x, "x", torch.bfloat16)
+    _vec(gamma, "gamma", torch.bfloat16, d)
+    _need(isinstance(dest, torch.Tensor) and dest.is_cuda and dest.dtype == torch.int32 and dest.dim() == 2
+          and dest.shape[0] == M and dest.is_contiguous(), "dest must be a contiguous int32 CUDA tensor [M, topk]")
+    topk = dest.shape[1]
+    _need(group in (0, 64, 128) and (group == 0 or d % group == 0), f"group must be 0, 64 or 128 dividing d = {d}")
+    ld_r = d
+    if residual is not None:
+        _, _, ld_r = _rows(residual, "residual", torch.bfloat16, d)
+        _need(residual.shape[0] == M, "residual must have M rows")
+        residual_out = _out(residual_out, (M, d), torch.bfloat16, x, "residual_out")
+        _need(_rows(residual_out, "residual_out", torch.bfloat16, d)[2] == ld_r,
+              "residual_out must have the row stride of residual")
+    else:
+        _need(residual_out is None, "residual_out needs residual")
+    q_out = _out(q_out, (rows, d), torch.float8_e4m3fn, x, "q_out")
+    ld_q = q_out.stride(0) if rows > 1 else d
+    _need(q_out.stride(-1) == 1 or d <= 1, "q_out must have a contiguous last dimension")
+    if group == 0:
+        scales_out = _out(scales_out, (rows,), torch.float32, x, "scales_out")
+        ld_s = 1
+    else:
+        scales_out = _out(scales_out, (rows, d // group), torch.float32, x, "scales_out")
+        ld_s = scales_out.stride(0) if rows > 1 else d // group
+    if want_norm and norm_out is None:
+        norm_out = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    ld_n = _rows(norm_out, "norm_out", torch.bfloat16, d)[2] if norm_out is not None else d
+    _same_device(x, gamma, dest, residual, residual_out, q_out, scales_out, norm_out)
+    with torch.cuda.device(x.device):
+        _check(_get_lib().nq_fused_add_rmsnorm_quant_fp8_moe(
+            _ptr(x), ld_x, _ptr(residual), _ptr(residual_out), ld_r, _ptr(gamma), _ptr(dest), topk, rows,
+            _ptr(q_out), ld_q, _ptr(scales_out), ld_s, _ptr(norm_out), ld_n, M, d, group, eps, flags,
+            _stream(stream)), "nq_fused_add_rmsnorm_quant_fp8_moe")
+    return q_out, scales_out, residual_out, norm_out

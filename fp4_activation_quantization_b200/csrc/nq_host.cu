@@ -252,7 +252,8 @@ nq_status check_common(const char* fn, int64_t M, int64_t d, float eps) {
 // Kernel table of an operation and output form (alt: e5m2 codes for the FP8
 // operations, swizzled block scales for NVFP4; layout: column-major or packed
 // group scales).
-const nq::RowKernels& table_of(int op, bool alt, bool layout) {
+const nq::RowKernels& table_of(int op, bool alt, bool layout, bool scatter) {
+  if (scatter) return op == nq::kOpRmsDynFp8 ? nq::row_kernels_rms_dyn_scatter() : nq::row_kernels_rms_group_scatter();
   switch (op) {
     case nq::kOpRmsDynFp8: return alt ? nq::row_kernels_rms_dyn_e5m2() : nq::row_kernels_rms_dyn();
     case nq::kOpRmsStaticFp8: return alt ? nq::row_kernels_rms_static_e5m2() : nq::row_kernels_rms_static();
@@ -354,6 +355,7 @@ int64_t resident_ctas(const void* k, int block, size_t smem = 0) {
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   const bool has_res = a.res_in != nullptr;
   uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
+  if (a.dest != nullptr) variant = 1;  // MoE scatter: register rows only
   const bool raw_forced = variant >= 2 && vec && !has_res && op != nq::kOpRmsDynFp8;
   const bool ring = variant == 5 && raw_forced;
   Schedule s;
@@ -380,8 +382,10 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   }
   const void* k = nullptr;
   size_t smem = 0;
+  const bool scatter = a.dest != nullptr;
   const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0,
-                                        (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0);
+                                        (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0,
+                                        scatter);
   if (ring) {
     // Ring depth 4 while four rows take at most 64 KB, else 2; one CTA per
     // resident slot (the occupancy query counts the ring's shared memory).
@@ -489,8 +493,9 @@ nq_status nq_check_device_errors(void) {
   if (word == 0) return NQ_OK;
   const uint32_t zero = 0;
   if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) (void)cudaGetLastError();
-  return fail(NQ_ERR_CUDA, "%s: a kernel's bounded wait for its bulk copy gave up (error word 0x%x); the "
-              "outputs of that launch are not meaningful", fn, word);
+  return fail(NQ_ERR_CUDA, "%s: device error word 0x%x (bit 0: a bounded wait for a bulk copy gave up, that "
+              "launch's outputs are not meaningful; bit 1: a MoE destination row was out of range and skipped)",
+              fn, word);
 }
 
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
@@ -696,6 +701,59 @@ nq_status nq_rmsnorm_quant_fp8_group(const void* x, int64_t ld_x, const void* re
                    vec_bf16(residual_out, ld_res) && aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) &&
                    aligned(q_out, 8) && ld_q % 8 == 0;
   return run_rows(fn, nq::kOpRmsGroupFp8, a, vec, flags, stream);
+}
+
+nq_status nq_fused_add_rmsnorm_quant_fp8_moe(const void* x, int64_t ld_x, const void* residual_in,
+                                             void* residual_out, int64_t ld_res, const void* gamma,
+                                             const int32_t* dest, int32_t topk, int64_t rows, void* q_out,
+                                             int64_t ld_q, float* scales_out, int64_t ld_s, void* norm_out,
+                                             int64_t ld_norm, int64_t M, int64_t d, int32_t group, float eps,
+                                             uint32_t flags, nq_stream_t stream) {
+  const char* fn = "nq_fused_add_rmsnorm_quant_fp8_moe";
+  nq_status st = check_common(fn, M, d, eps);
+  if (st != NQ_OK) return st;
+  if ((st = check_flags(fn, flags, group != 0, true, true)) != NQ_OK) return st;
+  if (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0 | NQ_FLAG_VARIANT_MASK))
+    return fail(NQ_ERR_UNSUPPORTED, "%s: e4m3 codes, row-major scales and the automatic variant only", fn);
+  if (group != 0 && group != 64 && group != 128)
+    return fail(NQ_ERR_UNSUPPORTED, "%s: group %d not in {0 (per token), 64, 128}", fn, group);
+  NQ_REQUIRE(group == 0 || d % group == 0, "%s: d = %lld is not a multiple of group %d", fn, (long long)d, group);
+  NQ_REQUIRE(topk >= 1 && topk <= 64, "%s: topk = %d not in 1..64", fn, topk);
+  NQ_REQUIRE(rows >= 0 && rows <= int64_t(0x7fffffff), "%s: rows = %lld out of range", fn, (long long)rows);
+  NQ_REQUIRE((residual_in == nullptr) == (residual_out == nullptr),
+             "%s: residual_in and residual_out must both be given or both be NULL", fn);
+  NQ_REQUIRE(ld_x >= d && ld_q >= d && (group == 0 || ld_s >= d / group) && (!residual_in || ld_res >= d) &&
+                 (!norm_out || ld_norm >= d),
+             "%s: row strides too small", fn);
+  if (M == 0) return NQ_OK;
+  NQ_REQUIRE(x && gamma && dest && (rows == 0 || (q_out && scales_out)),
+             "%s: x, gamma, dest, q_out and scales_out are required", fn);
+  RowArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.ld_x = ld_x;
+  a.res_in = static_cast<const uint16_t*>(residual_in);
+  a.res_out = static_cast<uint16_t*>(residual_out);
+  a.ld_res = ld_res;
+  a.gamma = gamma;
+  a.q = static_cast<uint8_t*>(q_out);
+  a.ld_q = ld_q;
+  a.scale_out = scales_out;
+  a.ld_scale = group == 0 ? 1 : ld_s;
+  a.cs_scale = 1;
+  a.group = group;
+  a.norm_out = static_cast<uint16_t*>(norm_out);
+  a.ld_norm = ld_norm;
+  a.M = M;
+  a.d = int32_t(d);
+  a.eps = eps;
+  a.flags = kernel_flags(flags, /*default_div=*/group == 0);
+  a.dest = dest;
+  a.topk = topk;
+  a.dest_rows = rows;
+  const bool vec = d % 8 == 0 && vec_bf16(x, ld_x) && vec_bf16(residual_in, ld_res) &&
+                   vec_bf16(residual_out, ld_res) && aligned(gamma, 16) && vec_bf16(norm_out, ld_norm) &&
+                   aligned(q_out, 8) && ld_q % 8 == 0;
+  return run_rows(fn, group == 0 ? nq::kOpRmsDynFp8 : nq::kOpRmsGroupFp8, a, vec, flags, stream);
 }
 
 nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out, int64_t ld_q,

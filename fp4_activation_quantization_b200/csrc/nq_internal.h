@@ -27,6 +27,7 @@ constexpr uint32_t kFlagScalesPacked = 1u << 8;   // group scales as packed UE8M
 // Output-form bits of the kernel instantiations (template parameter OUT).
 constexpr int kOutAlt = 1;          // e5m2 codes (FP8 ops) / swizzled block scales (NVFP4)
 constexpr int kOutScaleLayout = 2;  // group ops: column-major or packed-UE8M0 group scales
+constexpr int kOutScatter = 4;      // dynamic / group FP8 rows stored to MoE destination rows
 
 struct RowArgs {
   const uint16_t* x;  // bf16 [M, ld_x]
@@ -51,7 +52,10 @@ struct RowArgs {
   int32_t d;
   float eps;
   uint32_t flags;  // kFlag* bits; kFlagDiv set means divide, clear means reciprocal
-  uint32_t* err;   // device error word: bit 0 set when a bounded wait gave up
+  uint32_t* err;   // device error word: bit 0 a bounded wait gave up, bit 1 a destination row out of range
+  const int32_t* dest;  // [M, topk] destination rows (kOutScatter); < 0 skips
+  int32_t topk;
+  int64_t dest_rows;    // rows of q / scales when scattering
 };
 
 struct GroupArgs {
@@ -113,6 +117,8 @@ const RowKernels& row_kernels_rms_group_e5m2();
 const RowKernels& row_kernels_rms_nvfp4_swizzled();
 const RowKernels& row_kernels_rms_group_layout();
 const RowKernels& row_kernels_rms_group_e5m2_layout();
+const RowKernels& row_kernels_rms_dyn_scatter();
+const RowKernels& row_kernels_rms_group_scatter();
 
 // Group kernel: [e5m2][strided / packed scales][group == 128][log2(lanes per group) - 1]
 // [log2(groups per thread)][vec]

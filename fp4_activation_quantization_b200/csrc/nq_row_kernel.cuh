@@ -109,6 +109,23 @@ __device__ __forceinline__ void nvfp4_pair_scales(float amax0, float amax1, int 
   s1 = odd ? m : o;
 }
 
+// MoE dispatch: calls f(r) for each destination row r of `row` (dest[row *
+// topk + j] >= 0); a destination at or past dest_rows is skipped and recorded
+// in bit 1 of the device error word.
+template <typename F>
+__device__ __forceinline__ void for_each_dest(const RowArgs& a, int64_t row, F&& f) {
+  const int32_t* dp = a.dest + row * a.topk;
+  for (int j = 0; j < a.topk; ++j) {
+    const int32_t r = __ldg(dp + j);
+    if (r < 0) continue;
+    if (r >= a.dest_rows) {
+      atomicOr(a.err, 2u);
+      continue;
+    }
+    f(int64_t(r));
+  }
+}
+
 // Chunk partial of the canonical order: even / odd accumulators from +0,
 // then RN(even + odd).
 template <bool SQUARES>
@@ -163,6 +180,32 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
   }
 }
 
+// The FP8 codes of a row's K chunk slots, stored to each of its destination
+// rows (MoE dispatch).
+template <int T, int K, bool VEC, bool FULL>
+__device__ __forceinline__ void scatter_codes(const RowArgs& a, int64_t row, bool live, int tid,
+                                              const uint2 (&codes)[K]) {
+  if (!live) return;
+  const int d = a.d;
+  const int C = FULL ? T * K : (d + 7) >> 3;
+  for_each_dest(a, row, [&](int64_t r) {
+    uint8_t* qrow = a.q + r * a.ld_q;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const int c = tid + k * T;
+      if (FULL || c < C) {
+        if constexpr (VEC) {
+          *reinterpret_cast<uint2*>(qrow + 8 * c) = codes[k];
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (8 * c + j < d) qrow[8 * c + j] = uint8_t((j < 4 ? codes[k].x : codes[k].y) >> (8 * (j & 3)));
+        }
+      }
+    }
+  });
+}
+
 // Per-token-group FP8 of a row's y (chunk c of the row in v[k] for c = tid +
 // k*T): a group of G elements is G/8 consecutive chunks, held by G/8
 // consecutive threads of the group (T >= 32 and a multiple of G/8), so its
@@ -170,7 +213,7 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 // (max 448, or 57344 for e5m2; UE8M0: next power of two), one reciprocal,
 // q = fp8(RN(y * RN(1 / s))).  K <= 8, so a warp's K slots hold at most 32
 // groups (one per lane).
-template <bool E5, bool LAYOUT, int T, int K, bool VEC, bool FULL>
+template <bool E5, bool LAYOUT, int T, int K, bool VEC, bool FULL, bool SCATTER = false>
 __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
                                                 const float2 (&v)[K][4], bool div) {
   const int d = a.d;
@@ -206,7 +249,9 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
     const int kj = lane / gpw, part = lane % gpw;
     const int c0 = (tid & ~31) + part * cpg + kj * T;  // first chunk of lane j's group
     if (kj < K && (FULL || (live && c0 < C))) {
-      if constexpr (LAYOUT)
+      if constexpr (SCATTER)
+        for_each_dest(a, row, [&](int64_t r) { a.scale_out[r * a.ld_scale + c0 / cpg] = s; });
+      else if constexpr (LAYOUT)
         store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
                           c0 / cpg, d / a.group, s);
       else
@@ -214,6 +259,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
     }
   }
   // 3. each lane takes back the reciprocal (and scale) of its own groups
+  uint2 kept[SCATTER ? K : 1];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
@@ -226,7 +272,9 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
       t[i] = (div && sk != 0.0f) ? make_float2(__fdiv_rn(v[k][i].x, sk), __fdiv_rn(v[k][i].y, sk))
                                  : mul2(v[k][i], f2(ik));
     const uint2 codes = pack_pairs_fp8<E5>(t);
-    if (FULL || (live && c < C)) {
+    if constexpr (SCATTER) {
+      kept[k] = codes;
+    } else if (FULL || (live && c < C)) {
       if constexpr (VEC) {
         *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
       } else {
@@ -235,6 +283,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
       }
     }
   }
+  if constexpr (SCATTER) scatter_codes<T, K, VEC, FULL>(a, row, live, tid, kept);
 }
 
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
@@ -247,6 +296,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
   constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
   constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
+  constexpr bool SCATTER = (OUT & kOutScatter) != 0;          // MoE destination rows
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
   const bool live = FULL || live_in;
@@ -456,7 +506,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       if (live) sf_zero_padding_rows<T>(a, row, tid);
     }
   } else if constexpr (OP == kOpRmsGroupFp8) {
-    quantize_groups<E5, LAYOUT, T, K, VEC, FULL>(a, row, live, tid, v, div);
+    quantize_groups<E5, LAYOUT, T, K, VEC, FULL, SCATTER>(a, row, live, tid, v, div);
   } else {
     float s_div, s_inv;
     bool passthrough = false;
@@ -467,7 +517,11 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
         m = absmax8(v[k], m);
       const float amax = row_max_nonneg<T>(m, s_max, tid);
       const float s = fp8_scale_of<E5>(amax);
-      if (live && tid == 0) a.scale_out[row] = s;
+      if constexpr (SCATTER) {
+        if (live && tid == 0) for_each_dest(a, row, [&](int64_t r) { a.scale_out[r] = s; });
+      } else {
+        if (live && tid == 0) a.scale_out[row] = s;
+      }
       s_div = s;
       s_inv = __frcp_rn(s);
       passthrough = (s == 0.0f);  // zero row: store the signed zeros of y
@@ -476,9 +530,14 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       s_inv = __frcp_rn(s_div);
     }
     uint8_t* qrow = a.q + row * a.ld_q;
+    uint2 kept[SCATTER ? K : 1];
     auto store_codes = [&](int k, const float2 (&t)[4]) {
       const int c = tid + k * T;
       const uint2 codes = pack_pairs_fp8<E5>(t);
+      if constexpr (SCATTER) {
+        kept[k] = codes;
+        return;
+      }
       if (FULL || (live && c < C)) {
         if constexpr (VEC) {
           *reinterpret_cast<uint2*>(qrow + 8 * c) = codes;
@@ -523,6 +582,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
         store_codes(k, t);
       }
     }
+    if constexpr (SCATTER) scatter_codes<T, K, VEC, FULL>(a, row, live, tid, kept);
   }
   };
   // Measured on B200: the second copy pays with four chunks per thread
@@ -1204,7 +1264,7 @@ struct RowTable {
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
-  if constexpr (OP != kOpRmsDynFp8) {                                                                          \
+  if constexpr (OP != kOpRmsDynFp8 && !(OUT & kOutScatter)) {                                                  \
     k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT>); \
     k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT>);  \
     k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK), OUT>);     \
@@ -1226,7 +1286,7 @@ struct RowTable {
     NQ_DIRECT(10, 0) NQ_DIRECT(10, 1)
     NQ_RAW(5, 4)  // one warp per row, 16 chunks per lane (rows of up to 4096 elements)
 #define NQ_RING(LT, LK)                                                                                           \
-  if constexpr (OP != kOpRmsDynFp8) {                                                                             \
+  if constexpr (OP != kOpRmsDynFp8 && !(OUT & kOutScatter)) {                                                     \
     k.ring[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_ring<OP, (1 << LT), (1 << LK), 2, OUT>); \
     k.ring[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_ring<OP, (1 << LT), (1 << LK), 4, OUT>); \
   }

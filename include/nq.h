@@ -157,8 +157,10 @@ const char* nq_status_string(nq_status status);
 /* Synchronous: read and clear this library's device error word on the current
  * device.  NQ_OK if no kernel recorded an error since the last check;
  * NQ_ERR_CUDA (message in nq_last_error) if a kernel's bounded wait for its
- * own bulk copy into shared memory gave up (about one second), in which case
- * that launch's outputs are not meaningful.  Kernels never trap or hang. */
+ * own bulk copy into shared memory gave up (about one second; bit 0), in which
+ * case that launch's outputs are not meaningful, or if a MoE destination row
+ * was out of range (bit 1; the store was skipped).  Kernels never trap or
+ * hang. */
 nq_status nq_check_device_errors(void);
 /* Diagnostic (tests): checks, on the device, the bounded division the dynamic
  * FP8 path uses for RN(y / s) (a correctly rounded reciprocal r = RN(1 / s),
@@ -232,6 +234,35 @@ nq_status nq_layernorm_quant_fp8(const void* x, int64_t ld_x, const float* gamma
                                  const float* beta, const float* scale, void* q_out, int64_t ld_q,
                                  int64_t M, int64_t d, float eps, uint32_t flags,
                                  nq_stream_t stream);
+
+/*
+ * Residual-add (optional) + RMSNorm + e4m3, stored straight into the permuted
+ * input of a mixture-of-experts layer ("Fusing RMSNorm and FP8 Quantization
+ * Under torch.compile", "What we'd tell anyone shipping this": the MoE expert
+ * path quantizes inside the fused-MoE kernel and needs its own analogous
+ * fusion).  Each token is normalized and quantized once, exactly as by
+ * nq_fused_add_rmsnorm_quant_fp8 (group == 0: dynamic per-token scale,
+ * division by default) or nq_rmsnorm_quant_fp8_group (group 64 or 128:
+ * per-token-group scales, reciprocal by default), and its codes and scales
+ * are written to each of its destination rows.
+ *   dest int32 [M, topk] device memory: the row of (token t, slot j) in the
+ *     experts' permuted input (e.g. expert-major, as the MoE alignment step
+ *     lays it out); < 0 skips the slot (a dropped token).  A destination
+ *     >= rows is skipped and sets bit 1 of the device error word
+ *     (nq_check_device_errors).  topk in 1..64.
+ *   q_out e4m3 [rows, ld_q]; scales_out float32 [rows] (group == 0) or
+ *     [rows, ld_s] row-major (group scales).  Rows no slot targets are not
+ *     written.  x, residual_in / residual_out, gamma, norm_out as in
+ *     nq_rmsnorm_quant_fp8_group (residual_out and norm_out in token order).
+ * e4m3 only, row-major scales, automatic schedule; NQ_FLAG_UE8M0 applies with
+ * group scales.
+ */
+nq_status nq_fused_add_rmsnorm_quant_fp8_moe(const void* x, int64_t ld_x, const void* residual_in,
+                                             void* residual_out, int64_t ld_res, const void* gamma,
+                                             const int32_t* dest, int32_t topk, int64_t rows, void* q_out,
+                                             int64_t ld_q, float* scales_out, int64_t ld_s, void* norm_out,
+                                             int64_t ld_norm, int64_t M, int64_t d, int32_t group, float eps,
+                                             uint32_t flags, nq_stream_t stream);
 
 /*
  * Per-token-group e4m3 of raw bf16 activations ("per_token_group_quant_8bit:

@@ -357,3 +357,19 @@ def group_scales_layout(s, col_major=False, packed=False, ld=None) -> np.ndarray
     if rc != 0:
         raise ValueError("packed UE8M0 layout needs power-of-two scales in [2^-127, 2^127]")
     return out
+
+
+def moe_scatter(q, scales, dest, rows):
+    """Rows of a per-token result in the experts' permuted order: row
+    dest[t, j] of the output is token t's row, for every slot j with
+    dest[t, j] >= 0 (the definition of the dispatch; rows nobody targets stay
+    zero).  q [M, n] -> [rows, n]; scales [M] or [M, G] likewise."""
+    q = np.asarray(q)
+    s = np.asarray(scales)
+    dest = np.asarray(dest)
+    qo = np.zeros((rows,) + q.shape[1:], q.dtype)
+    so = np.zeros((rows,) + s.shape[1:], s.dtype)
+    t, j = np.nonzero(dest >= 0)
+    qo[dest[t, j]] = q[t]
+    so[dest[t, j]] = s[t]
+    return qo, so

@@ -200,3 +200,32 @@ def make_group_inputs(M: int, K: int, seed: int = 0, outlier_p: float = 0.001,
     w["x"] = f64_to_bf16_bits(v).reshape(M, K)
     w.update(M=M, K=K, seed=seed)
     return w
+
+
+SID_ROUTE = 6
+
+
+def make_moe_routing(M: int, E: int, topk: int, seed: int = 0, drop_p: float = 0.0) -> Workload:
+    """Synthetic MoE routing: each token picks `topk` distinct experts (uniform,
+    seeded), and every (token, slot) gets the row it occupies in the experts'
+    permuted input: expert-major, and by (token, slot) within an expert.  With
+    drop_p > 0, that fraction of (token, slot) pairs is dropped (row -1), as a
+    capacity limit would.  This is routing data for the tests and the sweep, not
+    part of the method."""
+    keys = uniform01(seed, SID_ROUTE, M * E).reshape(M, E)
+    topk_ids = np.argsort(keys, axis=1, kind="stable")[:, :topk].astype(np.int32)
+    flat_e = topk_ids.reshape(-1).astype(np.int64)
+    keep = np.ones(M * topk, bool)
+    if drop_p > 0:
+        keep = uniform01(seed, SID_ROUTE + 1, M * topk) > drop_p
+    order = np.lexsort((np.arange(M * topk), flat_e))  # by expert, then (token, slot)
+    order = order[keep[order]]
+    dest = np.full(M * topk, -1, np.int64)
+    dest[order] = np.arange(order.size)
+    counts = np.bincount(flat_e[keep], minlength=E)
+    w = Workload()
+    w["topk_ids"] = topk_ids
+    w["dest"] = dest.reshape(M, topk).astype(np.int32)
+    w["expert_offsets"] = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    w.update(M=M, E=E, topk=topk, rows=int(order.size), seed=seed)
+    return w

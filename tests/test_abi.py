@@ -99,6 +99,14 @@ def test_validation_without_gpu(nq):
                                     1e-6, nq.FLAG_SF_SWIZZLED, None) == INV
     assert b"4-byte" in L.nq_last_error()
     assert nq.sf_swizzled_size(1, 16) == 128 * 4 and nq.sf_swizzled_size(129, 7168) == 256 * 448
+    # MoE dispatch: topk, group and the unsupported flags are checked on the host
+    def moe(topk=2, group=0, flags=0, rows=8, dest=FAKE):
+        return L.nq_fused_add_rmsnorm_quant_fp8_moe(FAKE, 256, FAKE, FAKE, 256, FAKE, dest, topk, rows, FAKE, 256,
+                                                    FAKE, 2, None, 256, 4, 256, group, 1e-6, flags, None)
+    assert moe(topk=0) == INV and moe(topk=65) == INV
+    assert moe(group=32) == UNS and moe(flags=nq.FLAG_E5M2) == UNS
+    assert moe(flags=nq.FLAG_UE8M0) == INV  # UE8M0 needs group scales
+    assert moe(dest=None) == INV and moe(rows=-1) == INV
     # group-scale layouts: group calls only; ld_s checked per layout (M = 4, K = 640 -> 5 groups, 2 words)
     assert call_fused(nq, flags=nq.FLAG_SCALES_COL_MAJOR) == INV
     col, packed = nq.FLAG_SCALES_COL_MAJOR, nq.FLAG_SCALES_PACKED_UE8M0
