@@ -67,6 +67,12 @@ def rms_group_bytes(M, d, residual, g=128):
     return M * ((6 * d if residual else 2 * d) + d + 4 * (d // g)) + 2 * d
 
 
+def moe_bytes(M, d, topk, group, residual=True):
+    # x (+ residual read and write) bf16, topk copies of the e4m3 row and its scales, dest; bf16 gamma
+    per_scale = 4 if group == 0 else 4 * (d // group)
+    return M * ((6 * d if residual else 2 * d) + topk * (d + per_scale + 4)) + 2 * d
+
+
 def nvfp4_bytes(M, d, residual):
     per = (6 * d if residual else 2 * d) + d // 2 + d // 16
     return M * per + 2 * d + 4
@@ -502,6 +508,28 @@ def run_sweep(nq):
                              "us": round(us, 3), "GBps": round(nb / us / 1e3, 1),
                              "frac": round(nb / us / 1e3 / peak, 4)})
                 del xs, rs, qs, sc
+    import synthetic as S
+    d, E, topk = 7168, 256, 8
+    g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
+    for M in (256, 4096, 32768):
+        route = S.make_moe_routing(M, E, topk, seed=M)
+        dest = torch.from_numpy(route["dest"]).cuda()
+        n_rows = route["rows"]
+        for group in (0, 128):
+            nb = moe_bytes(M, d, topk, group)
+            S_ = sets_for(nb)
+            xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S_)]
+            rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S_)]
+            qs = [torch.empty(n_rows, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S_)]
+            sc = [torch.empty((n_rows, d // 128) if group else (n_rows,), dtype=torch.float32, device="cuda")
+                  for _ in range(S_)]
+            us = _time_graph(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8_moe(
+                xs[i], g, dest, n_rows, 1e-6, group=group, residual=rs[i], residual_out=rs[i], q_out=qs[i],
+                scales_out=sc[i]), S_)
+            rows.append({"op": "fused_add_rmsnorm_quant_fp8_moe" + ("[group128]" if group else "[per-token]"),
+                         "M": M, "d": d, "experts": E, "topk": topk, "us": round(us, 3),
+                         "GBps": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4)})
+            del xs, rs, qs, sc
     gs = torch.tensor([0.004], dtype=torch.float32, device="cuda")
     for d, ld in ((7168, 7168), (1536, 2112), (512, 512)):
         g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
