@@ -368,14 +368,15 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     // Automatic choice, from measurements on B200: static RMSNorm gains from
     // raw rows (fewer registers, more CTAs per SM) and, once every resident
     // CTA gets two or more rows, from the persistent prefetching form; NVFP4
-    // gains from raw rows on wide rows; LayerNorm from raw rows once a row
+    // from raw rows once a row is wider than a warp (10-15 % at d = 1536 ...
+    // 3584); LayerNorm from raw rows once a row
     // has 1024 elements or more (up to 1.37x at d = 7168: its float32 row
     // would hold twice the registers); the fused group quantization from raw
     // rows at every width (1.13x - 1.26x).  LayerNorm rows wider than a warp
     // take two rows per CTA (gamma / beta loaded once for both: 1.27x at
     // 65536 x 4096).
     if (op == nq::kOpRmsStaticFp8) variant = 3;
-    else if (op == nq::kOpRmsNvfp4 && a.d >= 4096) variant = 2;
+    else if (op == nq::kOpRmsNvfp4 && threads > 32) variant = 2;
     else if (op == nq::kOpLnStaticFp8 && threads > 32) variant = 6;
     else if (op == nq::kOpLnStaticFp8 && a.d >= 1024) variant = 2;
     else if (op == nq::kOpRmsGroupFp8) variant = 2;
