@@ -121,7 +121,13 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
       : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
   return out;
 }
-__device__ __forceinline__ uint32_t f32_to_e4m3(float a) { return pack_e4m3x4(a, 0.f, 0.f, 0.f) & 0xFFu; }
+// One float -> its e4m3 code (one converter instruction; the pair's other
+// half is e4m3(+0) = 0x00).
+__device__ __forceinline__ uint32_t f32_to_e4m3(float a) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(h) : "f"(a), "f"(0.0f));
+  return h;
+}
 
 // ------------------------------------------------------------ absmax -----
 // max(m, |v_0|, ..., |v_7|) with three-input max.f32 (sm_100), half the
@@ -217,12 +223,19 @@ __device__ __forceinline__ uint32_t pack_fp8x4(float a0, float a1, float a2, flo
 template <bool E5>
 constexpr float fp8_max() { return E5 ? kE5M2Max : kE4M3Max; }
 
-// e4m3 code (never the NaN code here) -> float, exact.
+// e4m3 code (low byte of c) -> float, exact: the hardware converter widens
+// e4m3 to f16 (every e4m3 value, NaN included, is an f16 value), then f16 ->
+// f32.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
-  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
-  const float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))  // (1 + m/8) 2^(e-7)
-                      : __fmul_rn(float(m), 0.001953125f);                 // m 2^-9
-  return (c & 0x80u) ? -mag : mag;
+  float f;
+  asm("{\n\t.reg .b16 c8, lo, hi;\n\t.reg .b32 h2;\n\t"
+      "cvt.u16.u32 c8, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h2, c8;\n\t"
+      "mov.b32 {lo, hi}, h2;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t}"
+      : "=f"(f)
+      : "r"(c & 0xFFu));
+  return f;
 }
 
 // ---------------------------------------------------------------- e2m1 ----

@@ -79,20 +79,34 @@ __device__ __forceinline__ void sf_zero_padding_rows(const RowArgs& a, int64_t r
 
 // NVFP4 block scale of a 16-element block with absmax amax under the global
 // scale g: sf = e4m3(RN(RN(amax / 6) / g)), S = RN(dec(sf) * g) and the
-// element multiplier RN(1 / S) (0 when S == 0).  Both divisions use the
-// bounded division (nq_device.cuh) where its quotient lies in [2^-24, 2^17]
-// and its divisor in range (ngr = -RN(1 / g), g_fast = g in range), else the
-// library division, so the result is always the correctly rounded one.
+// element multiplier RN(1 / S) (0 when S == 0).  Both divisions take the
+// bounded division (nq_device.cuh); where a quotient is nonzero and outside
+// [2^-24, 2^17], or g is outside the divisor range (ngr = -RN(1 / g), g_fast
+// = g in range), the lane takes the library division instead, so the result
+// is always the correctly rounded one.  That case is tested once per warp,
+// so the library division is a branch that ordinary data never enter.  Every
+// lane of the warp must call this together.
 struct Nvfp4Scale {
   uint32_t code;
   float mult;
 };
+// The library-division form of the quotient, out of line: in the raw-row
+// kernels (64 registers) ptxas then keeps the common path free of spills.
+static __device__ __noinline__ float nvfp4_block_quotient_lib(float amax, float g) {
+  return __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
+}
+template <bool OUT_OF_LINE>
 __device__ __forceinline__ Nvfp4Scale nvfp4_block_scale(float amax, float g, float ngr, bool g_fast) {
   constexpr float kSix = 6.0f, kNegRcpSix = -(1.0f / 6.0f);
   constexpr float kLo = 5.9604645e-08f, kHi = 131072.0f;  // 2^-24, 2^17
-  const float x = (amax >= kSix * kLo && amax <= kSix * kHi) ? div_rn_by(amax, kSix, kNegRcpSix)
-                                                             : __fdiv_rn(amax, kSix);
-  const float q = (g_fast && x >= g * kLo && x <= g * kHi) ? div_rn_by(x, g, ngr) : __fdiv_rn(x, g);
+  float x = div_rn_by(amax, kSix, kNegRcpSix);
+  float q = div_rn_by(x, g, ngr);
+  // A zero quotient is exact (0 * r, then zero remainders) once ngr is finite.
+  const bool fast = (amax == 0.0f || (amax >= kSix * kLo && amax <= kSix * kHi)) &&
+                    (g_fast && (x == 0.0f || (x >= g * kLo && x <= g * kHi)));
+  if (!__all_sync(kFull, fast)) {
+    if (!fast) q = OUT_OF_LINE ? nvfp4_block_quotient_lib(amax, g) : __fdiv_rn(__fdiv_rn(amax, kSix), g);
+  }
   const uint32_t code = f32_to_e4m3(q);
   const float S = __fmul_rn(e4m3_to_f32(code), g);
   return {code, (S == 0.0f) ? 0.0f : __frcp_rn(S)};
@@ -100,10 +114,11 @@ __device__ __forceinline__ Nvfp4Scale nvfp4_block_scale(float amax, float g, flo
 // Block scales of two chunk slots whose blocks each span this lane and its
 // xor-1 partner: the even lane computes slot 0's, the odd lane slot 1's, and
 // they swap, so each scale is computed once per pair instead of twice.
+template <bool OUT_OF_LINE>
 __device__ __forceinline__ void nvfp4_pair_scales(float amax0, float amax1, int tid, float g, float ngr, bool g_fast,
                                                   Nvfp4Scale& s0, Nvfp4Scale& s1) {
   const bool odd = (tid & 1) != 0;
-  const Nvfp4Scale m = nvfp4_block_scale(odd ? amax1 : amax0, g, ngr, g_fast);
+  const Nvfp4Scale m = nvfp4_block_scale<OUT_OF_LINE>(odd ? amax1 : amax0, g, ngr, g_fast);
   const Nvfp4Scale o = {__shfl_xor_sync(kFull, m.code, 1), __shfl_xor_sync(kFull, m.mult, 1)};
   s0 = odd ? o : m;
   s1 = odd ? m : o;
@@ -335,7 +350,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   float rstd;
   if constexpr (OP == kOpLnStaticFp8) {
     // Centre on the row mean (RN(r - mean) == RN(r + (-mean))), then the
-    // biased variance; padding elements stay exactly zero.
+    // biased variance; padding elements of a partial chunk are zeroed.
     const float2 nm = f2(-__fdiv_rn(total, fd));
 #pragma unroll
     for (int k = 0; k < K; ++k) {
@@ -348,9 +363,10 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
           if (8 * c + 2 * i >= d) t.x = 0.0f;
           if (8 * c + 2 * i + 1 >= d) t.y = 0.0f;
         }
-        v[k][i] = ok ? t : f2(0.0f);
+        v[k][i] = t;
       }
-      part[k] = chunk_partial<true>(v[k]);
+      // a chunk slot past the row adds +0 (its values are never stored)
+      part[k] = ok ? chunk_partial<true>(v[k]) : 0.0f;
     }
     const float sq = row_total<T, K>(part, s_sum1, tid);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
@@ -495,12 +511,12 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
       for (int k = 0; k < K; k += 2) {
         Nvfp4Scale s0, s1;
-        nvfp4_pair_scales(block_amax(k), block_amax(k + 1), tid, g, ngr, g_fast, s0, s1);
+        nvfp4_pair_scales<false>(block_amax(k), block_amax(k + 1), tid, g, ngr, g_fast, s0, s1);
         quant_store(k, s0);
         quant_store(k + 1, s1);
       }
     } else {
-      quant_store(0, nvfp4_block_scale(block_amax(0), g, ngr, g_fast));
+      quant_store(0, nvfp4_block_scale<false>(block_amax(0), g, ngr, g_fast));
     }
     if constexpr (SWZ) {
       if (live) sf_zero_padding_rows<T>(a, row, tid);
@@ -706,8 +722,10 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
       float2 v[4];
       unpack_pairs(src(k), v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = (c < C) ? add2(v[i], nm) : f2(0.0f);
-      part[k] = chunk_partial<true>(v);
+      for (int i = 0; i < 4; ++i) v[i] = add2(v[i], nm);
+      // a chunk slot past the row adds +0 (as zero chunks would): one select
+      // per chunk instead of one per element
+      part[k] = (c < C) ? chunk_partial<true>(v) : 0.0f;
     }
     const float sq = row_total<T, K>(part, b1, tid);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
@@ -795,14 +813,14 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
         norm_chunk(k, v0);
         norm_chunk(k + 1, v1);
         Nvfp4Scale s0, s1;
-        nvfp4_pair_scales(block_amax(v0), block_amax(v1), tid, scale_in, ngr, g_fast, s0, s1);
+        nvfp4_pair_scales<true>(block_amax(v0), block_amax(v1), tid, scale_in, ngr, g_fast, s0, s1);
         quant_store(k, v0, s0);
         quant_store(k + 1, v1, s1);
       }
     } else {
       float2 v[4];
       norm_chunk(0, v);
-      quant_store(0, v, nvfp4_block_scale(block_amax(v), scale_in, ngr, g_fast));
+      quant_store(0, v, nvfp4_block_scale<true>(block_amax(v), scale_in, ngr, g_fast));
     }
   } else {
 #pragma unroll
@@ -923,8 +941,11 @@ __device__ __forceinline__ void process_raw_rows_n(const RowArgs& a, const int64
         float2 v[4];
         unpack_pairs(xr[r][k], v);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = (c < C) ? add2(v[i], nm) : f2(0.0f);
-        part[r][k] = chunk_partial<true>(v);
+        for (int i = 0; i < 4; ++i) v[i] = (K >= 8 && c >= C) ? f2(0.0f) : add2(v[i], nm);
+        // A chunk slot past the row adds +0, as a zero chunk would: one
+        // select per chunk.  (With eight chunks per thread the per-element
+        // form above is kept: ptxas spills less with it.)
+        part[r][k] = (K < 8 && c >= C) ? 0.0f : chunk_partial<true>(v);
       }
     }
     row_totals_n<T, K, NR>(part, sq, b1, tid);
