@@ -60,7 +60,8 @@ def flag_group_schedule(log2_lanes: int, log2_groups: int) -> int:
 
 def flag_variant(n: int) -> int:
     """NQ_FLAG_VARIANT(n): 1 register rows, 2 raw rows, 3 raw rows persistent, 4 rows staged in
-    shared memory by one bulk copy, 5 persistent ring of bulk copies (0 = automatic)."""
+    shared memory by one bulk copy, 5 persistent ring of bulk copies, 6 two rows per CTA, 7 two
+    rows per CTA with persistent CTAs prefetching by cp.async (0 = automatic)."""
     return (n & 0x7) << 24
 
 

@@ -89,8 +89,6 @@ nq_status check_flags(const char* fn, uint32_t flags, bool allow_ue8m0, bool all
                 "%s: NQ_FLAG_UE8M0 / NQ_FLAG_SCALES_* apply to group quantization only", fn);
   if ((flags & (NQ_FLAG_SCHEDULE_MASK | NQ_FLAG_VARIANT_MASK)) && !allow_schedule)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE / NQ_FLAG_VARIANT apply to the norm calls only", fn);
-  if (((flags & NQ_FLAG_VARIANT_MASK) >> 24) > 6)
-    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_VARIANT(n) takes n in 0..6", fn);
   if ((flags & NQ_FLAG_NORM_BF16_ROUND) && !allow_bf16_round)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_NORM_BF16_ROUND needs a norm", fn);
   return NQ_OK;
@@ -403,6 +401,18 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   if (vec && !has_res && variant == 6 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
     k = table.rows2[s.log_t - nq::kMinLogT][s.log_k];
     if (k != nullptr) grid = (a.M + 1) / 2;
+  }
+  if (vec && !has_res && variant == 7 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
+    k = table.rows2p[s.log_t - nq::kMinLogT][s.log_k];
+    if (k != nullptr) {
+      smem = nq::rows2p_smem_bytes(threads, 1 << s.log_k);
+      if (!allow_smem(k, smem))
+        return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
+      const int64_t slots = resident_ctas(k, threads, smem);
+      if (slots <= 0) return fail(NQ_ERR_UNSUPPORTED, "%s: two-row persistent kernel does not fit on an SM", fn);
+      const int64_t pairs = (a.M + 1) / 2;
+      grid = pairs < slots ? pairs : slots;
+    }
   }
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && variant == 4) {
     k = table.staged[s.log_t - nq::kMinLogT][s.log_k];

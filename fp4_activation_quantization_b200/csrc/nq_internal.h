@@ -102,9 +102,13 @@ struct RowKernels {
   StagedTable staged;  // rows without residual staged in shared memory by a bulk copy
   RingTable ring;      // rows without residual through a ring of bulk copies, persistent
   StagedTable rows2;   // two rows per CTA on the same columns (static RMSNorm / LayerNorm)
+  StagedTable rows2p;  // rows2 with persistent CTAs prefetching the next two rows by cp.async
 };
 // Dynamic shared memory of a staged-row kernel: its rows of d bf16.
 inline size_t staged_smem_bytes(int threads, int64_t d) { return size_t(rows_per_cta(threads)) * size_t(d) * 2; }
+// Dynamic shared memory of the persistent two-row kernel: two stages of two
+// rows of threads x chunks 16-byte slots.
+inline size_t rows2p_smem_bytes(int threads, int chunks) { return size_t(2) * 2u * size_t(chunks) * size_t(threads) * 16u; }
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();

@@ -1048,6 +1048,68 @@ __global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel
   process_raw_rows_n<OP, T, K, OUT, NR>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
 }
 
+// NR rows per CTA as row_kernel_rows_n, with persistent CTAs that keep the
+// next group of NR rows in flight: CTA b takes groups b, b + G, b + 2G, ...
+// (G = grid size).  Each thread copies its own chunks of the next group into
+// its own slots of a two-stage shared-memory buffer with cp.async while it
+// processes the current group, so the prefetch holds no registers (the
+// register-prefetching raw kernel gives a quarter of its registers to it).
+// Thread t's 16-byte slot for (stage, row r, chunk k) is ((stage * NR + r) *
+// K + k) * T + t: consecutive threads, consecutive slots, no bank conflicts.
+template <int OP, int T, int K, int OUT, int NR>
+__global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel_rows_n_async(const RowArgs a) {
+  static_assert(T >= 64, "multi-row form: one CTA per group of NR rows");
+  constexpr int W = T / 32;
+  __shared__ __align__(16) float s_sum[2][NR * W * 32];
+  extern __shared__ __align__(16) uint4 s_stage[];  // [2][NR][K][T]
+  const int tid = int(threadIdx.x);
+  const int C = a.d >> 3;
+  const int64_t G = gridDim.x;
+  const int64_t n_groups = (a.M + NR - 1) / NR;
+  griddep_wait();
+  const float scale_in = __ldg(a.scale);
+  const float inv_static = __frcp_rn(scale_in);
+  // Issue group p's copies into stage st and commit them (an empty group past
+  // the last one, so that one wait count serves every step).
+  auto issue = [&](int64_t p, int st) {
+    if (p < n_groups) {
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const int64_t row = p * NR + r;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const int c = tid + k * T;
+          const bool ok = row < a.M && c < C;
+          const uint16_t* src = ok ? a.x + row * a.ld_x + 8 * c : a.x;
+          cp_async16(&s_stage[((st * NR + r) * K + k) * T + tid], src, ok);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  int64_t p = blockIdx.x;
+  issue(p, 0);
+  for (int j = 0; p < n_groups; ++j, p += G) {
+    const int64_t next = p + G;
+    issue(next, (j + 1) & 1);
+    if (next >= n_groups) griddep_launch_dependents();  // every load of this CTA is issued
+    cp_async_wait<1>();                                  // group p has landed
+    uint4 xr[NR][K];
+    int64_t row[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      row[r] = p * NR + r;
+#pragma unroll
+      for (int k = 0; k < K; ++k) xr[r][k] = s_stage[(((j & 1) * NR + r) * K + k) * T + tid];
+    }
+    // LayerNorm's two sums use both buffers (each separated from its next
+    // use by the other sum's barrier); a single sum alternates by step.
+    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
+    process_raw_rows_n<OP, T, K, OUT, NR>(a, row, tid, xr, b0, s_sum[1], scale_in, inv_static);
+  }
+  if (blockIdx.x >= n_groups) griddep_launch_dependents();
+}
+
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
 // residual), 16-byte rows, T > 32.  Only the raw bf16 chunks are kept (half
 // the registers of float32); each pass unpacks them again.  With PERSIST the
@@ -1281,6 +1343,8 @@ struct RowTable {
       for (auto& y : x) y = nullptr;
     for (auto& x : k.rows2)
       for (auto& y : x) y = nullptr;
+    for (auto& x : k.rows2p)
+      for (auto& y : x) y = nullptr;
     for (auto& x : k.ring)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
@@ -1291,8 +1355,10 @@ struct RowTable {
     k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK), OUT>);     \
   }                                                                                                            \
   if constexpr (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8) {                                               \
-    if constexpr (LT > 5 && LK <= 3)                                                                           \
+    if constexpr (LT > 5 && LK <= 3) {                                                                         \
       k.rows2[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2>); \
+      k.rows2p[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_rows_n_async<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2>); \
+    }                                                                                                          \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, OUT>); \

@@ -144,7 +144,9 @@ typedef enum nq_status {
  * of bulk copies of upcoming rows in flight and hold gamma (and beta) in
  * registers (t >= 6, k <= 2 with NQ_FLAG_SCHEDULE); n = 6 (static RMSNorm
  * and LayerNorm, t >= 6) gives each CTA two rows on the same columns, so each
- * thread loads its gamma / beta once for both.  n = 2..6 apply to
+ * thread loads its gamma / beta once for both; n = 7 is n = 6 with persistent
+ * CTAs, each thread copying its chunks of the CTA's next two rows into shared
+ * memory (cp.async) while it processes the current two.  n = 2..7 apply to
  * 16-byte-aligned rows without a residual and are ignored otherwise; with
  * n = 2..4, NQ_FLAG_SCHEDULE also accepts t = 5, k = 4 (one warp per row, 16
  * chunks per lane, rows of up to 4096 elements).  0 = automatic. */

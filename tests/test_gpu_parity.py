@@ -573,7 +573,8 @@ def test_ring_rows_output_forms(nq):
 @pytest.mark.parametrize("d,M", [(512, 7), (1024, 1), (2816, 301), (4096, 4097), (7168, 64), (16384, 33)])
 def test_two_row_variant_every_schedule(nq, d, M):
     """NQ_FLAG_VARIANT(6): two rows per CTA on the same columns (static RMSNorm and LayerNorm),
-    every schedule with at least 64 threads, odd and even M."""
+    and NQ_FLAG_VARIANT(7), the same with persistent CTAs prefetching their next two rows by
+    cp.async; every schedule with at least 64 threads, odd and even M."""
     w = S.make_rms_inputs(M, d, seed=d * 3 + M, residual=False, x_outlier_channels=True)
     lw = S.make_ln_inputs(M, d, seed=d * 3 + M + 1)
     x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
@@ -582,7 +583,7 @@ def test_two_row_variant_every_schedule(nq, d, M):
     e_ln = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-6)
     e_div, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, flags=oracle.DIV)
     lx, lgam, lbet = dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"])
-    for var, sched in [(v, s_) for v in (6,) for s_ in [None] + [s_ for s_ in all_schedules(d) if s_[0] > 5]]:
+    for var, sched in [(v, s_) for v in (6, 7) for s_ in [None] + [s_ for s_ in all_schedules(d) if s_[0] > 5]]:
         f = nq.flag_variant(var) | (0 if sched is None else nq.flag_schedule(*sched))
         q, _, no = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, want_norm=True, flags=f)
         assert np.array_equal(host_u8(q), e_st) and np.array_equal(host_u16(no), e_no), ("rms", var, sched)
