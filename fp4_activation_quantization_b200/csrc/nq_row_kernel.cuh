@@ -233,8 +233,9 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
                                                 const float2 (&v)[K][4], bool div) {
   const int d = a.d;
   const int C = FULL ? T * K : (d + 7) >> 3;
-  const int cpg = a.group >> 3;  // chunks per group: 8 or 16
-  const int gpw = 32 / cpg;      // groups per warp per chunk slot
+  const int lcpg = (a.group == 128) ? 4 : 3;  // log2(chunks per group): groups are 64 or 128
+  const int cpg = 1 << lcpg;                   // chunks per group: 8 or 16
+  const int gpw = 32 >> lcpg;                  // groups per warp per chunk slot
   const int lane = tid & 31;
   const bool ue8m0 = (a.flags & kFlagUe8m0) != 0;
   uint8_t* qrow = a.q + row * a.ld_q;
@@ -254,23 +255,23 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
   float mine = 0.0f;
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const float t = __shfl_sync(kFull, am[k], (lane % gpw) * cpg);
-    if (lane / gpw == k) mine = t;
+    const float t = __shfl_sync(kFull, am[k], (lane & (gpw - 1)) << lcpg);
+    if ((lane >> (5 - lcpg)) == k) mine = t;
   }
   float s = fp8_scale_of<E5>(mine);
   if (ue8m0) s = ue8m0_ceil(s);
   const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
   {
-    const int kj = lane / gpw, part = lane % gpw;
-    const int c0 = (tid & ~31) + part * cpg + kj * T;  // first chunk of lane j's group
+    const int kj = lane >> (5 - lcpg), part = lane & (gpw - 1);
+    const int c0 = (tid & ~31) + (part << lcpg) + kj * T;  // first chunk of lane j's group
     if (kj < K && (FULL || (live && c0 < C))) {
       if constexpr (SCATTER)
-        for_each_dest(a, row, [&](int64_t r) { a.scale_out[r * a.ld_scale + c0 / cpg] = s; });
+        for_each_dest(a, row, [&](int64_t r) { a.scale_out[r * a.ld_scale + (c0 >> lcpg)] = s; });
       else if constexpr (LAYOUT)
         store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
-                          c0 / cpg, d / a.group, s);
+                          c0 >> lcpg, d >> (lcpg + 3), s);
       else
-        srow[c0 / cpg] = s;
+        srow[c0 >> lcpg] = s;
     }
   }
   // 3. each lane takes back the reciprocal (and scale) of its own groups
@@ -278,7 +279,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
-    const int src = k * gpw + lane / cpg;
+    const int src = k * gpw + (lane >> lcpg);
     const float ik = __shfl_sync(kFull, inv, src);
     const float sk = div ? __shfl_sync(kFull, s, src) : 0.0f;
     float2 t[4];
@@ -822,21 +823,31 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
       norm_chunk(0, v);
       quant_store(0, v, nvfp4_block_scale<true>(block_amax(v), scale_in, ngr, g_fast));
     }
-  } else {
-#pragma unroll
-  for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
-    const bool ok = live && c < C;
-    float2 v[4];
-    norm_chunk(k, v);
-    if constexpr (OP == kOpRmsGroupFp8) {
-      // the group's chunks are consecutive lanes (see quantize_groups)
-      const int cpg = a.group >> 3;
+  } else if constexpr (OP == kOpRmsGroupFp8) {
+    // The group's chunks are consecutive lanes (see quantize_groups).  Chunk
+    // slots go in pairs: the warp holds 2 * gpw groups of a pair, and lane j
+    // < 2 * gpw computes the scale of group (slot j / gpw, part j % gpw) once
+    // (a correctly rounded division and reciprocal); every lane then takes
+    // its own two groups' scale and reciprocal by shuffles.  Group sizes are
+    // 64 or 128, so every index below is a shift or a mask.
+    const int lcpg = (a.group == 128) ? 4 : 3;  // log2(chunks per group)
+    const int cpg = 1 << lcpg, gpw = 32 >> lcpg;
+    const int lane = tid & 31;
+    const bool ue8m0 = (a.flags & kFlagUe8m0) != 0;
+    const bool packed = (a.flags & kFlagScalesPacked) != 0;
+    const int64_t n_groups = d >> (lcpg + 3);
+    auto group_max = [&](const float2 (&v)[4]) {
       float m = absmax8(v, 0.0f);
       for (int o = cpg >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-      float sg = fp8_scale_of<E5>(m);
-      if (a.flags & kFlagUe8m0) sg = ue8m0_ceil(sg);
-      const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
+      return m;
+    };
+    auto scale_of = [&](float m) {
+      const float sg = fp8_scale_of<E5>(m);
+      return ue8m0 ? ue8m0_ceil(sg) : sg;
+    };
+    auto quant_store = [&](int k, const float2 (&v)[4], float sg, float ig) {
+      const int c = tid + k * T;
+      const bool ok = live && c < C;
       float2 t[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -845,19 +856,45 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
         *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
         if ((c & (cpg - 1)) == 0) {
           if constexpr (LAYOUT)
-            store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, (a.flags & kFlagScalesPacked) != 0, row,
-                              c / cpg, d / a.group, sg);
+            store_group_scale(a.scale_out, a.ld_scale, a.cs_scale, packed, row, c >> lcpg, n_groups, sg);
           else
-            a.scale_out[row * a.ld_scale + c / cpg] = sg;
+            a.scale_out[row * a.ld_scale + (c >> lcpg)] = sg;
         }
       }
-    } else {
-      float2 t[4];
+    };
+    if constexpr (K >= 2) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
-      if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
+      for (int k = 0; k < K; k += 2) {
+        float2 v0[4], v1[4];
+        norm_chunk(k, v0);
+        norm_chunk(k + 1, v1);
+        const float m0 = group_max(v0), m1 = group_max(v1);
+        const int first = (lane & (gpw - 1)) << lcpg;  // first lane of group part j % gpw
+        const float t0 = __shfl_sync(kFull, m0, first), t1 = __shfl_sync(kFull, m1, first);
+        const float sg = scale_of(lane < gpw ? t0 : t1);  // lanes >= 2 gpw: unused
+        const float ig = (sg == 0.0f) ? 0.0f : __frcp_rn(sg);
+        const int own = lane >> lcpg;  // this lane's group part
+        quant_store(k, v0, __shfl_sync(kFull, sg, own), __shfl_sync(kFull, ig, own));
+        quant_store(k + 1, v1, __shfl_sync(kFull, sg, gpw + own), __shfl_sync(kFull, ig, gpw + own));
+      }
+    } else {
+      float2 v[4];
+      norm_chunk(0, v);
+      const float sg = scale_of(group_max(v));
+      quant_store(0, v, sg, (sg == 0.0f) ? 0.0f : __frcp_rn(sg));
     }
+  } else {
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int c = tid + k * T;
+    const bool ok = live && c < C;
+    float2 v[4];
+    norm_chunk(k, v);
+    float2 t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      t[i] = div ? make_float2(__fdiv_rn(v[i].x, scale_in), __fdiv_rn(v[i].y, scale_in)) : mul2(v[i], inv2);
+    if (ok) *reinterpret_cast<uint2*>(qrow + 8 * c) = pack_pairs_fp8<E5>(t);
   }
   }
   };
