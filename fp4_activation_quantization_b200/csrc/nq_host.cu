@@ -421,17 +421,20 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
       return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
   }
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
+    // The narrow copy tests for chunk slots past the row; a row that fills
+    // the schedule (d == 8 * threads * chunks) takes the copy without tests.
+    const int narrow = a.d == (8 * int64_t(threads)) << s.log_k ? 0 : 1;
     const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
-    if (variant == 3 && raw[1] != nullptr) {
-      const int64_t slots = resident_ctas(raw[1], threads);
+    if (variant == 3 && raw[1][narrow] != nullptr) {
+      const int64_t slots = resident_ctas(raw[1][narrow], threads);
       // Persistent pays once each resident CTA walks two or more rows.
       const bool forced = ((flags & NQ_FLAG_VARIANT_MASK) >> 24) == 3;
       if (slots > 0 && (forced || grid >= 2 * slots)) {
-        k = raw[1];
+        k = raw[1][narrow];
         grid = grid < slots ? grid : slots;
       }
     }
-    if (k == nullptr) k = raw[0];
+    if (k == nullptr) k = raw[0][narrow];
   }
   if (k == nullptr) {
     const auto& tab = table.direct[s.log_t - nq::kMinLogT][s.log_k];

@@ -89,7 +89,7 @@ using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][3];
 inline bool raw_schedule_built(int log_t, int log_k) {
   return schedule_built(log_t, log_k) || (log_t == 5 && log_k == 4);
 }
-using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
+using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2][2];
 using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2];
 // Ring kernels: T >= 64 threads per row, K <= 4 chunks per thread; [.][.][ring depth 2 or 4]
 using RingTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK][2];
@@ -98,7 +98,7 @@ inline bool ring_schedule_built(int log_t, int log_k) {
 }
 struct RowKernels {
   KernelTable direct;  // one row per thread group
-  RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent]
+  RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent][row narrower than T * K * 8]
   StagedTable staged;  // rows without residual staged in shared memory by a bulk copy
   RingTable ring;      // rows without residual through a ring of bulk copies, persistent
   StagedTable rows2;   // two rows per CTA on the same columns (static RMSNorm / LayerNorm)

@@ -691,7 +691,7 @@ struct GammaRegs {
 // a3..a6 of one row without residual whose raw bf16 chunks come from src(k)
 // (registers, or the row staged in shared memory) and whose gamma / beta come
 // from gam.  Rows past M (warp rows only) compute on zeros and store nothing.
-template <int OP, int T, int K, int OUT, typename Src, typename Gam, typename Hook>
+template <int OP, int T, int K, int OUT, bool NARROW, typename Src, typename Gam, typename Hook>
 __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, int tid, Src&& src, const Gam& gam,
                                                 float* b0, float* b1, float scale_in, float inv_static,
                                                 Hook&& after_first_sum) {
@@ -704,12 +704,25 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   const bool div_flag = (a.flags & kFlagDiv) != 0;
   const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
   const bool live = row < a.M;  // rows past M (warp rows only) compute on zeros and store nothing
+  // NARROW: the row may be narrower than the schedule (C < T * K, d not a
+  // power of two), so chunk slot k of this thread's warp may lie wholly past
+  // it; such a slot is skipped (its partial sums are +0, as zero chunks would
+  // give).  The test is warp-uniform.  The lower half of the slots is never
+  // dead for a schedule the planner picks (T * K is the smallest power of two
+  // >= C), so only the upper half is tested; a dead lower slot of a forced,
+  // wider schedule is computed on zeros.  Rows that fill the schedule take
+  // the NARROW = false copy, free of these tests (they cost 2-4 % there).
+  const int wbase = tid & ~31;
+  auto slot_live = [&](int k) { return !NARROW || k < K / 2 || wbase + k * T < C; };
   float part[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    float2 v[4];
-    unpack_pairs(src(k), v);
-    part[k] = chunk_partial<OP != kOpLnStaticFp8>(v);
+    part[k] = 0.0f;
+    if (slot_live(k)) {
+      float2 v[4];
+      unpack_pairs(src(k), v);
+      part[k] = chunk_partial<OP != kOpLnStaticFp8>(v);
+    }
   }
   const float total = row_total<T, K>(part, b0, tid);
   after_first_sum();  // every thread of the row group has read its chunks
@@ -720,13 +733,16 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       const int c = tid + k * T;
-      float2 v[4];
-      unpack_pairs(src(k), v);
+      part[k] = 0.0f;
+      if (slot_live(k)) {
+        float2 v[4];
+        unpack_pairs(src(k), v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = add2(v[i], nm);
-      // a chunk slot past the row adds +0 (as zero chunks would): one select
-      // per chunk instead of one per element
-      part[k] = (c < C) ? chunk_partial<true>(v) : 0.0f;
+        for (int i = 0; i < 4; ++i) v[i] = add2(v[i], nm);
+        // a chunk past the row adds +0 (as a zero chunk would): one select
+        // per chunk instead of one per element
+        part[k] = (c < C) ? chunk_partial<true>(v) : 0.0f;
+      }
     }
     const float sq = row_total<T, K>(part, b1, tid);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
@@ -811,6 +827,14 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
     if constexpr (K >= 2) {
 #pragma unroll
       for (int k = 0; k < K; k += 2) {
+        if (!slot_live(k + 1)) {  // slot k alone (its own block scales), or nothing
+          if (slot_live(k)) {
+            float2 v[4];
+            norm_chunk(k, v);
+            quant_store(k, v, nvfp4_block_scale<true>(block_amax(v), scale_in, ngr, g_fast), true);
+          }
+          continue;
+        }
         float2 v0[4], v1[4];
         norm_chunk(k, v0);
         norm_chunk(k + 1, v1);
@@ -875,6 +899,15 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
     if constexpr (K >= 2) {
 #pragma unroll
       for (int k = 0; k < K; k += 2) {
+        if (!slot_live(k + 1)) {  // slot k alone (every lane its group's scale), or nothing
+          if (slot_live(k)) {
+            float2 v[4];
+            norm_chunk(k, v);
+            const float sg = scale_of(group_max(v));
+            quant_store(k, v, sg, (sg == 0.0f) ? 0.0f : __frcp_rn(sg));
+          }
+          continue;
+        }
         float2 v0[4], v1[4];
         norm_chunk(k, v0);
         norm_chunk(k + 1, v1);
@@ -896,6 +929,7 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
   } else {
 #pragma unroll
   for (int k = 0; k < K; ++k) {
+    if (!slot_live(k)) continue;
     const int c = tid + k * T;
     const bool ok = live && c < C;
     float2 v[4];
@@ -1175,7 +1209,7 @@ constexpr int raw_min_blocks() {
   return blocks < 1 ? 1 : blocks;
 }
 
-template <int OP, int T, int K, bool PERSIST, int OUT>
+template <int OP, int T, int K, bool PERSIST, int OUT, bool NARROW>
 __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
     row_kernel_raw(const RowArgs a) {
   static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
@@ -1200,7 +1234,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
     }
   };
   auto process = [&](int64_t row, const uint4 (&xr)[K], float* b0, float* b1) {
-    process_raw_row<OP, T, K, OUT>(a, row, tid, [&](int k) { return xr[k]; }, GammaLoads<T>{a, tid, C}, b0, b1,
+    process_raw_row<OP, T, K, OUT, NARROW>(a, row, tid, [&](int k) { return xr[k]; }, GammaLoads<T>{a, tid, C}, b0, b1,
                                    scale_in, inv_static, [] {});
   };
 
@@ -1280,7 +1314,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (staged_min_blocks<T>())) r
     atomicOr(a.err, 1u);
     (void)mbar_wait_bounded(&s_bar[rsel], 0);
   }
-  process_raw_row<OP, T, K, OUT>(
+  process_raw_row<OP, T, K, OUT, true>(
       a, row, tid,
       [&](int k) {
         const int c = tid + k * T;
@@ -1362,7 +1396,7 @@ __global__ void __launch_bounds__(T, (ring_min_blocks<OP, T, K>())) row_kernel_r
     // Reduction buffers: LayerNorm's two sums use both (each separated from
     // its next use by the other sum's barrier); single sums alternate by row.
     float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
-    process_raw_row<OP, T, K, OUT>(
+    process_raw_row<OP, T, K, OUT, true>(
         a, row, tid, [&](int k) { return xr[k]; }, gam, b0, s_sum[1], scale_in, inv_static, [&] {
           if (tid == 0 && refill < a.M) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1385,7 +1419,8 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
     for (auto& x : k.raw)
       for (auto& y : x)
-        for (auto& z : y) z = nullptr;
+        for (auto& z : y)
+          for (auto& w : z) w = nullptr;
     for (auto& x : k.staged)
       for (auto& y : x) y = nullptr;
     for (auto& x : k.rows2)
@@ -1397,8 +1432,10 @@ struct RowTable {
         for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
   if constexpr (OP != kOpRmsDynFp8 && !(OUT & kOutScatter)) {                                                  \
-    k.raw[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT>); \
-    k.raw[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT>);  \
+    k.raw[LT - kMinLogT][LK][0][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT, false>); \
+    k.raw[LT - kMinLogT][LK][1][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT, false>);  \
+    k.raw[LT - kMinLogT][LK][0][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT, true>);  \
+    k.raw[LT - kMinLogT][LK][1][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT, true>);   \
     k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK), OUT>);     \
   }                                                                                                            \
   if constexpr (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8) {                                               \
