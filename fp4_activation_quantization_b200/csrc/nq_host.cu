@@ -426,11 +426,17 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     const int narrow = a.d == (8 * int64_t(threads)) << s.log_k ? 0 : 1;
     const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1][narrow] != nullptr) {
-      const int64_t slots = resident_ctas(raw[1][narrow], threads);
+      // Persistent CTAs of the RMSNorm-type operations hold gamma as fp32 in
+      // shared memory.
+      const size_t gsmem = nq::raw_gamma_smem_bytes(op, a.d);
+      if (!allow_smem(raw[1][narrow], gsmem))
+        return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, gsmem);
+      const int64_t slots = resident_ctas(raw[1][narrow], threads * rows, gsmem);
       // Persistent pays once each resident CTA walks two or more rows.
       const bool forced = ((flags & NQ_FLAG_VARIANT_MASK) >> 24) == 3;
       if (slots > 0 && (forced || grid >= 2 * slots)) {
         k = raw[1][narrow];
+        smem = gsmem;
         grid = grid < slots ? grid : slots;
       }
     }

@@ -106,6 +106,9 @@ struct RowKernels {
 };
 // Dynamic shared memory of a staged-row kernel: its rows of d bf16.
 inline size_t staged_smem_bytes(int threads, int64_t d) { return size_t(rows_per_cta(threads)) * size_t(d) * 2; }
+// Dynamic shared memory of a persistent raw-row kernel: gamma as fp32 for the
+// RMSNorm-type operations (LayerNorm reads gamma / beta through L1).
+inline size_t raw_gamma_smem_bytes(int op, int64_t d) { return op == kOpLnStaticFp8 ? 0 : size_t(d) * 4u; }
 // Dynamic shared memory of the persistent two-row kernel: two stages of two
 // rows of threads x chunks 16-byte slots.
 inline size_t rows2p_smem_bytes(int threads, int chunks) { return size_t(2) * 2u * size_t(chunks) * size_t(threads) * 16u; }

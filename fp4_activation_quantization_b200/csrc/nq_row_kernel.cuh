@@ -668,6 +668,25 @@ struct GammaLoads {
     if (c < C) gu = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c));
     return gu;
   }
+  __device__ __forceinline__ void rms2(int k, float2 (&g)[4]) const { unpack_pairs(rms(k), g); }
+};
+
+// RMSNorm gamma (bf16) widened to fp32 once per persistent CTA and kept in
+// shared memory: per chunk two conflict-free 16-byte loads replace a load and
+// eight integer unpack instructions on every row.  Chunk c's first four
+// values are lo[c], the last four hi[c].
+template <int T, int K>
+struct GammaSmem {
+  const float4* lo;
+  const float4* hi;
+  int tid, C;
+  __device__ __forceinline__ void rms2(int k, float2 (&g)[4]) const {
+    const int c = tid + k * T;
+    float4 l = make_float4(0.f, 0.f, 0.f, 0.f), h = l;
+    if (c < C) l = lo[c], h = hi[c];
+    g[0] = make_float2(l.x, l.y), g[1] = make_float2(l.z, l.w), g[2] = make_float2(h.x, h.y),
+    g[3] = make_float2(h.z, h.w);
+  }
 };
 
 template <bool LN, int T, int K>
@@ -686,6 +705,7 @@ struct GammaRegs {
     a0 = g0[k], a1 = g1[k], b0 = e0[k], b1 = e1[k];
   }
   __device__ __forceinline__ uint4 rms(int k) const { return gu[k]; }
+  __device__ __forceinline__ void rms2(int k, float2 (&g)[4]) const { unpack_pairs(gu[k], g); }
 };
 
 // a3..a6 of one row without residual whose raw bf16 chunks come from src(k)
@@ -776,7 +796,7 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
       for (int i = 0; i < 4; ++i) v[i] = fma2(mul2(add2(v[i], nm), rs2), g[i], b[i]);
     } else {
       float2 g[4];
-      unpack_pairs(gam.rms(k), g);
+      gam.rms2(k, g);
 #pragma unroll
       for (int i = 0; i < 4; ++i) v[i] = mul2(mul2(v[i], rs2), g[i]);
     }
@@ -1233,9 +1253,30 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
       xr[k] = (row < a.M && c < C) ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
     }
   };
+  // Persistent CTAs of the RMSNorm-type operations keep gamma as fp32 in
+  // (dynamic) shared memory, widened once by the whole CTA (raw_gamma_smem_bytes)
+  // while the first row's load is in flight.
+  constexpr bool GSMEM = PERSIST && OP != kOpLnStaticFp8;
+  extern __shared__ __align__(16) float4 s_gamma[];  // [2][C]: GSMEM only
+  auto stage_gamma = [&] {
+    if constexpr (GSMEM) {
+      for (int c = int(threadIdx.x); c < C; c += int(blockDim.x)) {
+        float2 g[4];
+        unpack_pairs(__ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c)), g);
+        s_gamma[c] = make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
+        s_gamma[C + c] = make_float4(g[2].x, g[2].y, g[3].x, g[3].y);
+      }
+      __syncthreads();
+    }
+  };
   auto process = [&](int64_t row, const uint4 (&xr)[K], float* b0, float* b1) {
-    process_raw_row<OP, T, K, OUT, NARROW>(a, row, tid, [&](int k) { return xr[k]; }, GammaLoads<T>{a, tid, C}, b0, b1,
-                                   scale_in, inv_static, [] {});
+    if constexpr (GSMEM)
+      process_raw_row<OP, T, K, OUT, NARROW>(a, row, tid, [&](int k) { return xr[k]; },
+                                             GammaSmem<T, K>{s_gamma, s_gamma + C, tid, C}, b0, b1, scale_in,
+                                             inv_static, [] {});
+    else
+      process_raw_row<OP, T, K, OUT, NARROW>(a, row, tid, [&](int k) { return xr[k]; }, GammaLoads<T>{a, tid, C}, b0,
+                                             b1, scale_in, inv_static, [] {});
   };
 
   if constexpr (!PERSIST) {
@@ -1250,6 +1291,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
     uint4 xa[K], xb[K];
     int64_t row = group;
     load(row, xa);
+    stage_gamma();
     for (int parity = 0; row < a.M; parity ^= 1) {
       const int64_t next = row + n_groups;
       if (next >= a.M) griddep_launch_dependents();  // nothing left to load
