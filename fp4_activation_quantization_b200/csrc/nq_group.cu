@@ -42,7 +42,9 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const GroupArgs a)
   for (int u = 0; u < U; ++u) {
     const int64_t g = base + int64_t(u) * SLOT + slot;
     ok[u] = g < a.G;
-    row[u] = ok[u] ? g / a.groups_per_row : 0;
+    row[u] = !ok[u] ? 0
+             : a.row_magic ? int64_t((uint64_t(uint32_t(g)) * a.row_magic) >> a.row_shift)
+                           : g / a.groups_per_row;
     cg[u] = ok[u] ? g - row[u] * a.groups_per_row : 0;
     const uint16_t* src = a.x + row[u] * a.ld_x + cg[u] * GROUP;
 #pragma unroll

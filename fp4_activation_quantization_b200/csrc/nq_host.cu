@@ -802,6 +802,12 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   a.cs_s = s_cs;
   a.groups_per_row = K / group;
   a.G = M * (K / group);
+  if (a.G < (int64_t(1) << 31)) {
+    int l = 0;
+    while ((int64_t(1) << l) < a.groups_per_row) ++l;
+    a.row_shift = 32 + l;
+    a.row_magic = ((uint64_t(1) << a.row_shift) + uint64_t(a.groups_per_row) - 1) / uint64_t(a.groups_per_row);
+  }
   a.flags = kernel_flags(flags, /*default_div=*/false);
   const bool vec = vec_bf16(x, ld_x) && aligned(q_out, 8) && ld_q % 8 == 0;
   // Team of 2^t lanes per group, 2^u groups per thread.  Many groups: teams

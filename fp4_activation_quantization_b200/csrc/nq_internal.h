@@ -68,6 +68,14 @@ struct GroupArgs {
   int64_t cs_s;
   int64_t groups_per_row;
   int64_t G;  // M * groups_per_row
+  // Row of flat group g (g / groups_per_row) without a 64-bit division: for G
+  // < 2^31, (g * row_magic) >> row_shift with row_shift = 32 + ceil(log2
+  // groups_per_row) and row_magic = ceil(2^row_shift / groups_per_row) < 2^33
+  // is exact (the error g * (row_magic - 2^row_shift / gpr) / 2^row_shift stays
+  // below 1 / (2 gpr), Granlund and Montgomery, PLDI 1994).  row_magic = 0:
+  // divide.
+  uint64_t row_magic;
+  int32_t row_shift;
   uint32_t flags;
 };
 
