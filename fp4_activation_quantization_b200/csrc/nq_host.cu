@@ -165,9 +165,12 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
     int lk = 2;
     if (M < 192 && lp <= 9) lk = 0;
     else if (M < 384) lk = 1;
-    else if (lp <= 9 && (op == nq::kOpRmsDynFp8 ||
+    else if (lp <= 9 && ((op == nq::kOpRmsDynFp8 && !(lp == 9 && C < (int64_t(1) << lp))) ||
                          (M < 768 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8 || op == nq::kOpRmsNvfp4))))
       lk = 1;
+    // (The dynamic path keeps four chunks for rows of 257 ... 511 chunks, d =
+    // 2056 ... 4088: their upper slots are skipped whole per warp, 65536 x
+    // 2816: 225 -> 197 us.)
     // LayerNorm takes two rows per CTA (run_rows); with P = 1024 it runs
     // best at eight chunks per thread (8192 x 7168: 54.1 -> 49.9 us).
     if (op == nq::kOpLnStaticFp8 && lp == 10 && M >= 768) lk = 3;
@@ -445,6 +448,14 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   if (k == nullptr) {
     const auto& tab = table.direct[s.log_t - nq::kMinLogT][s.log_k];
     k = tab[vec ? 1 : 0];
+    // 16-byte rows narrower than the schedule skip the chunk slots wholly
+    // past the row (mode 3), when that needs no more registers (measured on
+    // B200: with fewer registers 3-15 % faster at d = 1536 ... 7168; with
+    // more, at two chunks per thread, 4 % slower).
+    if (vec && a.d < (8 * int64_t(threads)) << s.log_k && tab[3] != nullptr) {
+      const int r_narrow = kernel_regs(tab[3]), r_vec = kernel_regs(tab[1]);
+      if (r_narrow > 0 && r_vec > 0 && r_narrow <= r_vec) k = tab[3];
+    }
     // The predicate-free variant for rows that exactly fill the schedule, when
     // it does not need more registers (occupancy decides this kernel's speed).
     if (vec && threads > 32 && a.d == (8 * int64_t(threads)) << s.log_k && tab[2] != nullptr) {

@@ -90,8 +90,9 @@ inline bool schedule_built(int log_t, int log_k) {
 
 // Host-side kernel tables (pointer to the __global__ stub), one per
 // translation unit: [log_t - 5][log_k][mode], mode 0 = any alignment,
-// 1 = 16-byte rows, 2 = 16-byte rows with d == 8 * threads * chunks (t > 5).
-using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][3];
+// 1 = 16-byte rows, 2 = 16-byte rows with d == 8 * threads * chunks (t > 5),
+// 3 = 16-byte rows with d < 8 * threads * chunks (k > 0).
+using KernelTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 1][4];
 // Raw-row schedules: those of the direct kernel, plus one warp per row with 16
 // chunks per lane (t = 5, k = 4).
 inline bool raw_schedule_built(int log_t, int log_k) {

@@ -305,7 +305,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.
-template <int OP, int T, int K, bool VEC, bool FULL, int OUT>
+template <int OP, int T, int K, bool VEC, bool FULL, int OUT, bool NARROW = false>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
                                             float* s_sum1, uint32_t* s_max) {
@@ -318,12 +318,25 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   const bool live = FULL || live_in;
   const bool div_flag = (a.flags & kFlagDiv) != 0;
   const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
+  // NARROW (16-byte rows narrower than the schedule): a chunk slot that lies
+  // wholly past the row for this warp is skipped in every per-chunk step
+  // except the NVFP4 and group quantization (which run on its zeros); its
+  // sums are +0, as zero chunks give.  Only the upper half of the slots can
+  // be dead for a planned schedule (see process_raw_row).
+  const int wbase = tid & ~31;
+  auto slot_live = [&](int k) { return !NARROW || k < K / 2 || wbase + k * T < C; };
   // ---- a2: r = x + residual, residual_out; a3: chunk partials
   float2 v[K][4];
   float part[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     const int c = tid + k * T;
+    if (!slot_live(k)) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = f2(0.0f);
+      part[k] = 0.0f;
+      continue;
+    }
     unpack_pairs(xr[k], v[k]);
     if (has_res) {
       float2 t[4];
@@ -355,6 +368,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     const float2 nm = f2(-__fdiv_rn(total, fd));
 #pragma unroll
     for (int k = 0; k < K; ++k) {
+      if (!slot_live(k)) continue;  // part[k] is +0 already
       const int c = tid + k * T;
       const bool ok = FULL || (live && c < C);
 #pragma unroll
@@ -387,6 +401,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   const float2 rs2 = f2(rstd);
 #pragma unroll
   for (int k = 0; k < K; ++k) {
+    if (!slot_live(k)) continue;  // y stays 0
     const int c = tid + k * T;
     const bool gok = FULL || c < C;
     if constexpr (OP == kOpLnStaticFp8) {
@@ -531,7 +546,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       float m = 0.0f;
 #pragma unroll
       for (int k = 0; k < K; ++k)
-        m = absmax8(v[k], m);
+        if (slot_live(k)) m = absmax8(v[k], m);
       const float amax = row_max_nonneg<T>(m, s_max, tid);
       const float s = fp8_scale_of<E5>(amax);
       if constexpr (SCATTER) {
@@ -571,11 +586,13 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     const bool fast = (OP == kOpRmsDynFp8) && div && fast_div_ok(s_div);
     if (passthrough) {
 #pragma unroll
-      for (int k = 0; k < K; ++k) store_codes(k, v[k]);
+      for (int k = 0; k < K; ++k)
+        if (slot_live(k)) store_codes(k, v[k]);
     } else if (fast) {
       const float2 s2 = f2(s_div), nr2 = f2(-s_inv);
 #pragma unroll
       for (int k = 0; k < K; ++k) {
+        if (!slot_live(k)) continue;
         float2 t[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) t[i] = div2_rn_by(v[k][i], s2, nr2);
@@ -584,6 +601,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     } else if (div) {
 #pragma unroll
       for (int k = 0; k < K; ++k) {
+        if (!slot_live(k)) continue;
         float2 t[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) t[i] = make_float2(__fdiv_rn(v[k][i].x, s_div), __fdiv_rn(v[k][i].y, s_div));
@@ -593,6 +611,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       const float2 inv2 = f2(s_inv);
 #pragma unroll
       for (int k = 0; k < K; ++k) {
+        if (!slot_live(k)) continue;
         float2 t[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) t[i] = mul2(v[k][i], inv2);
@@ -613,7 +632,9 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 // next row into a second register set measured slower on B200 (the doubled
 // registers halve occupancy), and so did shared-memory cp.async staging.
 // MODE 0: any alignment (scalar loads); 1: 16-byte rows; 2: 16-byte rows that
-// exactly fill the schedule (d == 8 * T * K, T > 32): no predicates at all.
+// exactly fill the schedule (d == 8 * T * K, T > 32): no predicates at all;
+// 3: 16-byte rows narrower than the schedule (d < 8 * T * K): chunk slots
+// wholly past the row are skipped per warp.
 // OUT: output-form bits, each a separate instantiation so that the default
 // kernels carry no branch on them.  kOutAlt: e5m2 codes for the FP8
 // operations, the swizzled block-scale layout for NVFP4; kOutScaleLayout
@@ -622,6 +643,7 @@ template <int OP, int T, int K, int MODE, int OUT>
 __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a) {
   constexpr bool VEC = MODE >= 1;
   constexpr bool FULL = MODE == 2;
+  constexpr bool NARROW = MODE == 3;
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA
   constexpr int W = T / 32;             // warps per row
   static_assert(K == 1 || K == 2 || K == 4 || K == 8, "chunks per thread");
@@ -640,7 +662,7 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   uint4 xr[K], rr[K];
   load_raw<T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
-  process_row<OP, T, K, VEC, FULL, OUT>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+  process_row<OP, T, K, VEC, FULL, OUT, NARROW>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
 }
 
 // Per-chunk gamma (RMSNorm: bf16) or gamma and beta (LayerNorm: float32) of
@@ -1490,6 +1512,7 @@ struct RowTable {
   k.direct[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 0, OUT>); \
   k.direct[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 1, OUT>); \
   if (LT > 5) k.direct[LT - kMinLogT][LK][2] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 2, OUT>); \
+  if constexpr (LK > 0) k.direct[LT - kMinLogT][LK][3] = reinterpret_cast<const void*>(&row_kernel<OP, (1 << LT), (1 << LK), 3, OUT>); \
   NQ_RAW(LT, LK)
     NQ_DIRECT(5, 0) NQ_DIRECT(5, 1) NQ_DIRECT(5, 2) NQ_DIRECT(5, 3)
     NQ_DIRECT(6, 0) NQ_DIRECT(6, 1) NQ_DIRECT(6, 2) NQ_DIRECT(6, 3)

@@ -134,8 +134,9 @@ def test_validation_without_gpu(nq):
 
 @pytest.mark.parametrize("op,M,d,exp", [
     (0, 64, 2816, (512, 1, 1)),      # fewer rows than SMs: one chunk per thread
-    (0, 4096, 2816, (256, 2, 1)),    # residual-add dynamic, d <= 4096: two chunks per thread at any M
-    (0, 4096, 4096, (256, 2, 1)),
+    (0, 4096, 4096, (256, 2, 1)),    # residual-add dynamic, d <= 4096: two chunks per thread at any M ...
+    (0, 4096, 2816, (128, 4, 1)),    # ... except rows narrower than the 512-chunk schedule: four
+    (0, 4096, 2048, (128, 2, 1)),
     (0, 65536, 8192, (256, 4, 1)),   # wider rows: four chunks per thread
     (0, 8192, 7168, (256, 4, 1)),
     (0, 8192, 512, (32, 2, 8)),      # narrow rows: one warp per row, 8 rows per CTA
