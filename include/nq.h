@@ -184,7 +184,8 @@ const char* nq_last_error(void);
  * Schedule the planner picks for a norm call (op: 0 = fused add+RMSNorm+
  * dynamic FP8, 1 = RMSNorm static FP8, 2 = LayerNorm static FP8, 3 = RMSNorm
  * NVFP4, 4 = RMSNorm group FP8) at (M, d, flags): threads per row, 16-byte
- * chunks per thread and rows per CTA.  Pure host function; launches nothing.
+ * chunks per thread and rows per CTA; for op 3, the call without a residual.
+ * Pure host function; launches nothing.
  */
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,
                             int* chunks_per_thread, int* rows_per_cta);

@@ -591,3 +591,35 @@ def test_two_row_variant_every_schedule(nq, d, M):
         assert np.array_equal(host_u8(q), e_div), ("rms div", var, sched)
         q = nq.nq_layernorm_quant_fp8(lx, lgam, lbet, sc, 1e-6, flags=f)
         assert np.array_equal(host_u8(q), e_ln), ("ln", var, sched)
+
+
+# -------------------------------------- rows narrower than the schedule ----
+@pytest.mark.parametrize("residual", [False, True])
+def test_narrow_rows_partial_warps_every_schedule(nq, residual):
+    """Rows narrower than their power-of-two schedule, with a chunk count that is not a multiple
+    of 32, so that one warp of a chunk slot is partly inside the row and the warps after it are
+    wholly past it (the slots the register-row and raw-row kernels skip).  NVFP4 (d = 2832),
+    group 64 (d = 2880) and group 128 (d = 2944), every schedule, bit-exact with the oracle."""
+    M = 37
+    for d, kind, group in ((2832, "nvfp4", 0), (2880, "group", 64), (2944, "group", 128)):
+        assert ((d // 8) % 32) != 0
+        w = S.make_rms_inputs(M, d, seed=d + residual, residual=residual, x_outlier_channels=True)
+        x, gam = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+        res = dev_bf16(w["residual"]) if residual else None
+        if kind == "nvfp4":
+            g = oracle.nvfp4_global_scale(w["x"], w["gamma"], w.get("residual"), d=d)
+            eq, esf, er, _ = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], g, residual=w.get("residual"), d=d)
+            gs = torch.tensor([g], dtype=torch.float32, device="cuda")
+        else:
+            eq, es, er, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"], w.get("residual"), group=group)
+        for sched in [None, *all_schedules(d)]:
+            f = 0 if sched is None else nq.flag_schedule(*sched)
+            if kind == "nvfp4":
+                q, sf, ro, _ = nq.nq_rmsnorm_quant_nvfp4(x, gam, gs, 1e-6, residual=res, flags=f)
+                assert np.array_equal(host_u8(sf), esf), (d, sched, "block scales")
+            else:
+                q, s, ro, _ = nq.nq_rmsnorm_quant_fp8_group(x, gam, 1e-6, group=group, residual=res, flags=f)
+                assert np.array_equal(s.cpu().numpy().view(np.uint32), es.view(np.uint32)), (d, sched, "scales")
+            assert np.array_equal(host_u8(q), eq), (d, sched, "codes")
+            if residual:
+                assert np.array_equal(host_u16(ro), er), (d, sched, "residual_out")
