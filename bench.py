@@ -79,8 +79,12 @@ def nvfp4_bytes(M, d, residual):
 
 
 def kernel_source_hash() -> str:
+    """Hash of the device-code sources (every csrc file except the host-side
+    launcher nq_host.cu): a profile's counters stay valid while it matches."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "fp4_activation_quantization_b200", "csrc", "*"))):
+        if os.path.basename(p) == "nq_host.cu":
+            continue
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())

@@ -308,8 +308,11 @@ uint32_t* device_error_word() {
 // Dynamic shared memory above the default 48 KB needs a per-kernel opt-in.
 std::mutex g_smem_mu;
 std::vector<std::pair<const void*, size_t>> g_smem;
+// Opt kernel k in to `bytes` of dynamic shared memory.  Set whenever a kernel
+// takes any: the 48 KB default covers static and dynamic memory together, so
+// 48 KB of dynamic memory on top of a kernel's static buffers needs it too.
 bool allow_smem(const void* k, size_t bytes) {
-  if (bytes <= 48 * 1024) return true;
+  if (bytes == 0) return true;
   std::lock_guard<std::mutex> lk(g_smem_mu);
   for (const auto& p : g_smem)
     if (p.first == k && p.second >= bytes) return true;

@@ -623,3 +623,23 @@ def test_narrow_rows_partial_warps_every_schedule(nq, residual):
             assert np.array_equal(host_u8(q), eq), (d, sched, "codes")
             if residual:
                 assert np.array_equal(host_u16(ro), er), (d, sched, "residual_out")
+
+
+@pytest.mark.parametrize("d", [11264, 12288, 16384])
+def test_static_persistent_wide_rows(nq, d):
+    """Persistent raw rows keep gamma as fp32 in dynamic shared memory (4 d bytes: 44, 48 and
+    64 KB here, on top of the kernel's static buffers).  Static RMSNorm and NVFP4, automatic and
+    forced persistent variant, bit-exact with the oracle."""
+    M = 700
+    w = S.make_rms_inputs(M, d, seed=d, residual=False)
+    x, gam = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    eq, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05)
+    g = oracle.nvfp4_global_scale(w["x"], w["gamma"], d=d)
+    e4, esf, _, _ = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], g, d=d)
+    gs = torch.tensor([g], dtype=torch.float32, device="cuda")
+    for f in (0, nq.flag_variant(3)):
+        q, _, _ = nq.nq_rmsnorm_quant_fp8_static(x, gam, sc, 1e-6, flags=f)
+        assert np.array_equal(host_u8(q), eq), f
+        q4, sf, _, _ = nq.nq_rmsnorm_quant_nvfp4(x, gam, gs, 1e-6, flags=f)
+        assert np.array_equal(host_u8(q4), e4) and np.array_equal(host_u8(sf), esf), f
