@@ -175,11 +175,11 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
     // LayerNorm takes two rows per CTA (run_rows); with P = 1024 it runs
     // best at eight chunks per thread (8192 x 7168: 54.1 -> 49.9 us).
     if (op == nq::kOpLnStaticFp8 && lp == 10 && M >= 768) lk = 3;
-    // NVFP4 without residual (raw rows) on rows narrower than a schedule of
-    // 512 or more chunks: eight chunks per thread, so that the dead upper
-    // slots fall on whole slots of every warp (8192 x 7168: 45.3 -> 42.4 us,
-    // 65536 x 2816: 142.5 -> 130.2 us).
-    if (op == nq::kOpRmsNvfp4 && !has_res && lp >= 9 && lp <= 10 && C < (int64_t(1) << lp) && M >= 768) lk = 3;
+    // NVFP4 without residual (raw rows): eight chunks per thread for P = 1024
+    // (8192 x 8192: 87.8 -> 85.4 us; 8192 x 7168: 45.3 -> 42.4 us, its dead
+    // upper slots then whole slots of every warp) and for rows narrower than
+    // P = 512 (65536 x 2816: 142.5 -> 130.2 us); at d = 4096 four stay faster.
+    if (op == nq::kOpRmsNvfp4 && !has_res && M >= 768 && (lp == 10 || (lp == 9 && C < (int64_t(1) << lp)))) lk = 3;
     int lt = lp - lk;
     if (lt > 10) lt = 10;
     s->log_t = lt;

@@ -151,9 +151,10 @@ def test_validation_without_gpu(nq):
     (2, 512, 4096, (256, 2, 1)),
     (4, 600, 4096, (128, 4, 1)),     # fused group: four chunks from 384 rows
     (2, 8192, 7168, (128, 8, 1)),    # LayerNorm, P = 1024: eight chunks per thread
-    (3, 8192, 7168, (128, 8, 1)),    # NVFP4 without residual, rows narrower than P >= 512: eight
+    (3, 8192, 7168, (128, 8, 1)),    # NVFP4 without residual, rows narrower than P = 512: eight
     (3, 8192, 2816, (64, 8, 1)),
-    (3, 8192, 8192, (256, 4, 1)),    # ... but four on rows that fill it
+    (3, 8192, 8192, (128, 8, 1)),    # ... and at P = 1024 whatever the width
+    (3, 8192, 4096, (128, 4, 1)),    # ... but four on rows that fill P = 512
     (3, 8192, 1536, (64, 4, 1)),
 ])
 def test_planner(nq, op, M, d, exp):
