@@ -411,7 +411,8 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     grid = grid < slots ? grid : slots;
   }
   if (vec && !has_res && variant == 6 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
-    k = table.rows2[s.log_t - nq::kMinLogT][s.log_k];
+    // The narrow copy skips chunk slots wholly past rows narrower than the schedule.
+    k = table.rows2[s.log_t - nq::kMinLogT][s.log_k][a.d < (8 * int64_t(threads)) << s.log_k ? 1 : 0];
     if (k != nullptr) grid = (a.M + 1) / 2;
   }
   if (vec && !has_res && variant == 7 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {

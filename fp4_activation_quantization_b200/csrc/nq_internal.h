@@ -100,6 +100,7 @@ inline bool raw_schedule_built(int log_t, int log_k) {
 }
 using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2][2];
 using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2];
+using Rows2Table = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
 // Ring kernels: T >= 64 threads per row, K <= 4 chunks per thread; [.][.][ring depth 2 or 4]
 using RingTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK][2];
 inline bool ring_schedule_built(int log_t, int log_k) {
@@ -110,7 +111,7 @@ struct RowKernels {
   RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent][row narrower than T * K * 8]
   StagedTable staged;  // rows without residual staged in shared memory by a bulk copy
   RingTable ring;      // rows without residual through a ring of bulk copies, persistent
-  StagedTable rows2;   // two rows per CTA on the same columns (static RMSNorm / LayerNorm)
+  Rows2Table rows2;    // two rows per CTA on the same columns (static RMSNorm / LayerNorm): [.][.][narrow row]
   StagedTable rows2p;  // rows2 with persistent CTAs prefetching the next two rows by cp.async
 };
 // Dynamic shared memory of a staged-row kernel: its rows of d bf16.

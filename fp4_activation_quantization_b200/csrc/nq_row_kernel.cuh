@@ -1029,7 +1029,7 @@ __device__ __forceinline__ void row_totals_n(float (&part)[NR][K], float (&out)[
     for (int r = 0; r < NR; ++r) out[r] = __fadd_rn(out[r], __shfl_xor_sync(kFull, out[r], o));
 }
 
-template <int OP, int T, int K, int OUT, int NR>
+template <int OP, int T, int K, int OUT, int NR, bool NARROW = false>
 __device__ __forceinline__ void process_raw_rows_n(const RowArgs& a, const int64_t (&row)[NR], int tid,
                                                    const uint4 (&xr)[NR][K], float* b0, float* b1, float scale_in,
                                                    float inv_static) {
@@ -1041,11 +1041,21 @@ __device__ __forceinline__ void process_raw_rows_n(const RowArgs& a, const int64
   const float fd = float(d);
   const bool div_flag = (a.flags & kFlagDiv) != 0;
   const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
+  // NARROW: chunk slots wholly past the row for this warp are skipped (see
+  // process_raw_row).
+  const int wbase = tid & ~31;
+  auto slot_live = [&](int k) { return k < K / 2 || wbase + k * T < C; };
   float part[NR][K], total[NR];
 #pragma unroll
   for (int r = 0; r < NR; ++r)
 #pragma unroll
     for (int k = 0; k < K; ++k) {
+      if constexpr (NARROW) {
+        if (!slot_live(k)) {
+          part[r][k] = 0.0f;
+          continue;
+        }
+      }
       float2 v[4];
       unpack_pairs(xr[r][k], v);
       part[r][k] = chunk_partial<!LN>(v);
@@ -1061,6 +1071,12 @@ __device__ __forceinline__ void process_raw_rows_n(const RowArgs& a, const int64
 #pragma unroll
       for (int k = 0; k < K; ++k) {
         const int c = tid + k * T;
+        if constexpr (NARROW) {
+          if (!slot_live(k)) {
+            part[r][k] = 0.0f;
+            continue;
+          }
+        }
         float2 v[4];
         unpack_pairs(xr[r][k], v);
 #pragma unroll
@@ -1087,6 +1103,9 @@ __device__ __forceinline__ void process_raw_rows_n(const RowArgs& a, const int64
     const float2 inv2 = f2(inv_static);
 #pragma unroll
     for (int k = 0; k < K; ++k) {
+      if constexpr (NARROW) {
+        if (!slot_live(k)) continue;
+      }
       const int c = tid + k * T;
       float2 g[4], b[4];
       if constexpr (LN) {
@@ -1143,7 +1162,7 @@ constexpr int rows_n_min_blocks() {
 // NR rows per CTA (T >= 64), raw bf16 chunks in registers, not persistent.
 // Built for NR = 2; four rows per CTA measured slower on B200 (their raw
 // rows spill or halve the resident CTAs).
-template <int OP, int T, int K, int OUT, int NR>
+template <int OP, int T, int K, int OUT, int NR, bool NARROW>
 __global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel_rows_n(const RowArgs a) {
   static_assert(T >= 64, "multi-row form: one CTA per group of NR rows");
   constexpr int W = T / 32;
@@ -1168,7 +1187,7 @@ __global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel
     }
   }
   griddep_launch_dependents();
-  process_raw_rows_n<OP, T, K, OUT, NR>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
+  process_raw_rows_n<OP, T, K, OUT, NR, NARROW>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
 }
 
 // NR rows per CTA as row_kernel_rows_n, with persistent CTAs that keep the
@@ -1488,7 +1507,8 @@ struct RowTable {
     for (auto& x : k.staged)
       for (auto& y : x) y = nullptr;
     for (auto& x : k.rows2)
-      for (auto& y : x) y = nullptr;
+      for (auto& y : x)
+        for (auto& z : y) z = nullptr;
     for (auto& x : k.rows2p)
       for (auto& y : x) y = nullptr;
     for (auto& x : k.ring)
@@ -1504,7 +1524,8 @@ struct RowTable {
   }                                                                                                            \
   if constexpr (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8) {                                               \
     if constexpr (LT > 5 && LK <= 3) {                                                                         \
-      k.rows2[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2>); \
+      k.rows2[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2, false>); \
+      k.rows2[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2, true>); \
       k.rows2p[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_rows_n_async<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2>); \
     }                                                                                                          \
   }
