@@ -176,7 +176,7 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
     // best at eight chunks per thread (8192 x 7168: 54.1 -> 49.9 us).
     if (op == nq::kOpLnStaticFp8 && lp == 10 && M >= 768) lk = 3;
     // NVFP4 without residual (raw rows): eight chunks per thread for P = 1024
-    // (8192 x 8192: 87.8 -> 85.4 us; 8192 x 7168: 45.3 -> 42.4 us, its dead
+    // (16384 x 8192: 87.8 -> 85.4 us; 8192 x 7168: 45.3 -> 42.4 us, its dead
     // upper slots then whole slots of every warp) and for rows narrower than
     // P = 512 (65536 x 2816: 142.5 -> 130.2 us); at d = 4096 four stay faster.
     if (op == nq::kOpRmsNvfp4 && !has_res && M >= 768 && (lp == 10 || (lp == 9 && C < (int64_t(1) << lp)))) lk = 3;
