@@ -160,7 +160,11 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
     s->log_t = 5;
     s->log_k = lp > 5 ? lp - 5 : 0;
   } else if (M < 148) {
-    s->log_t = lp < 10 ? lp : 10;
+    // Fewer rows than SMs: latency first.  Up to 512 threads with one chunk
+    // each; rows of 4097 ... 8192 elements take 512 threads with two chunks,
+    // not 1024 with one (1 x 8192 dynamic: 3.20 -> 2.56 us, 64 x 7168:
+    // 3.50 -> 2.64 us; 8-13 % for the NVFP4 and group forms).
+    s->log_t = lp < 10 ? lp : (lp == 10 ? 9 : 10);
     s->log_k = lp - s->log_t;
   } else {
     int lk = 2;

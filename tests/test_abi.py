@@ -141,7 +141,8 @@ def test_validation_without_gpu(nq):
     (0, 8192, 7168, (256, 4, 1)),
     (0, 8192, 512, (32, 2, 8)),      # narrow rows: one warp per row, 8 rows per CTA
     (0, 8192, 1536, (128, 2, 1)),
-    (0, 1, 8192, (1024, 1, 1)),      # a single row spreads over 1024 threads
+    (0, 1, 8192, (512, 2, 1)),       # a single row: 512 threads with two chunks each ...
+    (0, 100, 4096, (512, 1, 1)),     # ... or one
     (0, 16, 16384, (1024, 2, 1)),
     (0, 1, 100, (32, 1, 8)),
     (1, 4096, 4096, (128, 4, 1)),    # static RMSNorm: four chunks once there are many rows per SM
