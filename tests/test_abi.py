@@ -170,3 +170,25 @@ def test_planner_forced_schedules(nq):
     with pytest.raises(nq.NQError):
         nq.nq_query_schedule(0, 100, 64, nq.flag_schedule(10, 2))    # not built (t + k > 11)
     assert nq.nq_query_schedule(0, 100, 8192, nq.flag_schedule(7, 3)) == (128, 8, 1)
+
+
+def test_planner_properties(nq):
+    """Over a grid of operations, row counts and widths, the automatic schedule covers the row
+    with the fewest chunk slots a power-of-two schedule allows (or one warp with one chunk),
+    stays within the built schedules, and puts eight rows in a CTA exactly when a warp owns a
+    row."""
+    Ms = [1, 16, 100, 147, 148, 191, 192, 383, 384, 767, 768, 4096, 65536]
+    ds = [8, 64, 512, 1000, 1024, 1536, 2048, 2816, 4096, 4104, 7168, 8192, 12288, 16384]
+    for op in range(5):
+        for M in Ms:
+            for d in ds:
+                if op == 3 and d % 16:
+                    continue
+                T, K, R = nq.nq_query_schedule(op, M, d)
+                C = (d + 7) // 8
+                P = 1 << max(0, (C - 1).bit_length())
+                assert T & (T - 1) == 0 and 32 <= T <= 1024, (op, M, d, T)
+                assert K in (1, 2, 4, 8), (op, M, d, K)
+                assert T * K >= C, (op, M, d, T, K)
+                assert T * K == max(P, 32), (op, M, d, T, K)
+                assert R == (8 if T == 32 else 1), (op, M, d, T, R)
