@@ -375,3 +375,40 @@ def test_e5m2_outputs_compose_pinned_pieces():
     assert np.array_equal(sg, esg)
     inv = (np.float32(1) / esg).astype(np.float32)
     assert np.array_equal(qg, oracle.e5m2_encode((xf * inv[..., None]).astype(np.float32)).reshape(8, 512))
+
+
+# --------------------------------------------------- MoE dispatch scatter ----
+def test_moe_scatter_golden_dispatch():
+    """The oracle's MoE dispatch against a dispatch worked by hand
+    (tests/golden/moe_dispatch.json: 3 tokens, top-2, one dropped slot, one
+    row nobody targets).  A transposed destination index, a gather in place
+    of the scatter, or a dropped slot (-1) wrapping to the last row each fail
+    it."""
+    c = json.load(open(os.path.join(GOLDEN, "moe_dispatch.json")))
+    dest = np.array(c["dest"], np.int32)
+    q = np.array(c["q"], np.uint8)
+    for key, exp_key, dtype in (("scale", "expected_scale", np.float32),
+                                ("group_scales", "expected_group_scales", np.float32)):
+        qo, so = oracle.moe_scatter(q, np.array(c[key], dtype), dest, c["rows"])
+        assert qo.dtype == np.uint8 and qo.shape == (c["rows"], q.shape[1])
+        assert np.array_equal(qo, np.array(c["expected_q"], np.uint8))
+        assert np.array_equal(so, np.array(c[exp_key], dtype))
+
+
+def test_moe_scatter_counts_against_routing():
+    """Every row the router assigns receives exactly one token's row: rows that
+    several slots name cannot occur (the routing is a permutation of the kept
+    slots), and each kept slot's row equals its token's row."""
+    r = S.make_moe_routing(50, 16, 4, seed=5, drop_p=0.1)
+    dest = r["dest"]
+    kept = dest[dest >= 0]
+    assert len(np.unique(kept)) == len(kept) and kept.max() < r["rows"]
+    q = np.arange(50 * 8, dtype=np.uint8).reshape(50, 8) % 251
+    s = np.arange(50, dtype=np.float32) + 1
+    qo, so = oracle.moe_scatter(q, s, dest, r["rows"])
+    for t in range(50):
+        for j in range(4):
+            if dest[t, j] >= 0:
+                assert np.array_equal(qo[dest[t, j]], q[t]) and so[dest[t, j]] == s[t]
+    untouched = np.setdiff1d(np.arange(r["rows"]), kept)
+    assert not qo[untouched].any() and not so[untouched].any()
