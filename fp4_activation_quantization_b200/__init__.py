@@ -59,9 +59,8 @@ def flag_group_schedule(log2_lanes: int, log2_groups: int) -> int:
 
 
 def flag_variant(n: int) -> int:
-    """NQ_FLAG_VARIANT(n): 1 register rows, 2 raw rows, 3 raw rows persistent, 4 rows staged in
-    shared memory by one bulk copy, 5 persistent ring of bulk copies, 6 two rows per CTA, 7 two
-    rows per CTA with persistent CTAs prefetching by cp.async (0 = automatic)."""
+    """NQ_FLAG_VARIANT(n): 1 register rows, 2 raw rows, 3 raw rows persistent, 6 two rows per CTA
+    (0 = automatic; 4, 5 and 7 are not built)."""
     return (n & 0x7) << 24
 
 
@@ -138,8 +137,9 @@ def nq_selftest_division(divisors, a_bits_begin: int = 0, count: int = 1 << 32, 
 
 
 def nq_check_device_errors() -> None:
-    """Raise NQError if a kernel's bounded wait for its own copy gave up since
-    the last check (synchronous; clears the device error word)."""
+    """Raise NQError if a kernel recorded an error since the last check (a MoE
+    destination row out of range).  Synchronous: waits for every stream of the
+    current device, then reads and clears the device error word atomically."""
     _check(_get_lib().nq_check_device_errors(), "nq_check_device_errors")
 
 

@@ -15,10 +15,16 @@
 #include "nq_device.cuh"
 #include "nq_internal.h"
 
-// Device error word of this library: bit 0 is set by a kernel whose bounded
-// wait on its own bulk copy gave up (read and cleared by
-// nq_check_device_errors).  A symbol, not an allocation.
+// Device error word of this library: bit 1 is set by a MoE dispatch whose
+// destination row was out of range (read and cleared by
+// nq_check_device_errors).  A symbol, not an allocation; one per device.
 __device__ uint32_t g_nq_device_error;
+// Where take_error_word leaves the word it cleared, for the host to read.
+__device__ uint32_t g_nq_device_error_taken;
+
+// Read and clear the error word in one atomic step, so that a bit a kernel
+// sets between the read and the clear cannot be lost.
+__global__ void take_error_word_kernel() { g_nq_device_error_taken = atomicExch(&g_nq_device_error, 0u); }
 
 // Exhaustive check of the bounded division (nq_selftest_division): for
 // a = the float with bits a_begin + i and each divisor b in its domain, count
@@ -194,34 +200,6 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
   return NQ_OK;
 }
 
-// Ring kernels (NQ_FLAG_VARIANT(5)): 2^t >= 64 threads per row and 2^k <= 4
-// chunks per thread; automatically two chunks per thread where the row allows
-// (half the gamma / beta registers of four).
-nq_status plan_ring(const char* fn, int64_t d, uint32_t flags, Schedule* s) {
-  const int64_t C = (d + 7) / 8;
-  int lp = 0;
-  while ((int64_t(1) << lp) < C) ++lp;
-  const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
-  if (ft || fk) {
-    if (!ft || !fk) return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE needs both fields", fn);
-    const int lt = int(ft) + 4, lk = int(fk) - 1;
-    if (!nq::ring_schedule_built(lt, lk))
-      return fail(NQ_ERR_UNSUPPORTED, "%s: ring schedule of 2^%d threads x 2^%d chunks is not built", fn, lt, lk);
-    if ((int64_t(1) << (lt + lk)) < C)
-      return fail(NQ_ERR_INVALID_ARGUMENT, "%s: schedule covers %lld chunks, a row has %lld", fn,
-                  (long long)(int64_t(1) << (lt + lk)), (long long)C);
-    *s = {lt, lk};
-    return NQ_OK;
-  }
-  int lt = lp - 1;
-  lt = lt < 6 ? 6 : (lt > nq::kMaxLogT ? nq::kMaxLogT : lt);
-  const int lk = lp > lt ? lp - lt : 0;
-  if (!nq::ring_schedule_built(lt, lk))
-    return fail(NQ_ERR_UNSUPPORTED, "%s: no ring schedule for d = %lld", fn, (long long)d);
-  *s = {lt, lk};
-  return NQ_OK;
-}
-
 nq_status launch(const char* fn, const void* kernel, unsigned grid, unsigned block, size_t smem,
                  void** args, bool pdl, cudaStream_t stream) {
   if (kernel == nullptr) return fail(NQ_ERR_UNSUPPORTED, "%s: kernel variant not built", fn);
@@ -276,104 +254,139 @@ const nq::RowKernels& table_of(int op, bool alt, bool layout, bool scatter) {
   }
 }
 
-// Registers per thread of a kernel (host query, cached per kernel).
+// The current CUDA device (-1 when there is none or it is out of the caches'
+// range).  Kernel attributes, the shared-memory opt-in and occupancy are per
+// device, so the caches below are keyed by (device, kernel).
+constexpr int kMaxDevices = 64;
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return -1;
+  }
+  return dev;
+}
+
+// Registers per thread of a kernel (host query, cached per device and kernel).
+struct RegsKey {
+  int dev;
+  const void* k;
+  int regs;
+};
 std::mutex g_regs_mu;
-std::vector<std::pair<const void*, int>> g_regs;
+std::vector<RegsKey> g_regs;
 int kernel_regs(const void* k) {
+  const int dev = current_device();
+  if (dev < 0) return -1;
   std::lock_guard<std::mutex> lk(g_regs_mu);
   for (const auto& p : g_regs)
-    if (p.first == k) return p.second;
+    if (p.dev == dev && p.k == k) return p.regs;
   cudaFuncAttributes attr;
   int regs = -1;
   if (cudaFuncGetAttributes(&attr, k) == cudaSuccess) regs = attr.numRegs;
   else (void)cudaGetLastError();
-  g_regs.push_back({k, regs});
+  g_regs.push_back({dev, k, regs});
   return regs;
 }
 
-// Device address of g_nq_device_error on the current device (cached per device).
+// Device address of a __device__ symbol on the current device (cached per
+// device: each device holds its own copy of the symbol).
 std::mutex g_err_mu;
-uint32_t* g_err_ptr[64] = {};
-uint32_t* device_error_word() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    (void)cudaGetLastError();
-    return nullptr;
-  }
+uint32_t* g_err_ptr[kMaxDevices] = {};
+uint32_t* g_taken_ptr[kMaxDevices] = {};
+uint32_t* symbol_on_device(uint32_t** cache, const void* symbol) {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
   std::lock_guard<std::mutex> lk(g_err_mu);
-  if (g_err_ptr[dev] == nullptr) {
+  if (cache[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_nq_device_error) == cudaSuccess) g_err_ptr[dev] = static_cast<uint32_t*>(p);
+    if (cudaGetSymbolAddress(&p, symbol) == cudaSuccess) cache[dev] = static_cast<uint32_t*>(p);
     else (void)cudaGetLastError();
   }
-  return g_err_ptr[dev];
+  return cache[dev];
 }
+uint32_t* device_error_word() { return symbol_on_device(g_err_ptr, &g_nq_device_error); }
 
-// Dynamic shared memory above the default 48 KB needs a per-kernel opt-in.
+// Dynamic shared memory above the default 48 KB needs an opt-in per device
+// and kernel.
+struct SmemKey {
+  int dev;
+  const void* k;
+  size_t bytes;
+};
 std::mutex g_smem_mu;
-std::vector<std::pair<const void*, size_t>> g_smem;
-// Opt kernel k in to `bytes` of dynamic shared memory.  Set whenever a kernel
-// takes any: the 48 KB default covers static and dynamic memory together, so
-// 48 KB of dynamic memory on top of a kernel's static buffers needs it too.
+std::vector<SmemKey> g_smem;
+// Opt kernel k in to `bytes` of dynamic shared memory on the current device.
+// Set whenever a kernel takes any: the 48 KB default covers static and
+// dynamic memory together, so 48 KB of dynamic memory on top of a kernel's
+// static buffers needs it too.
 bool allow_smem(const void* k, size_t bytes) {
   if (bytes == 0) return true;
+  const int dev = current_device();
+  if (dev < 0) return false;
   std::lock_guard<std::mutex> lk(g_smem_mu);
   for (const auto& p : g_smem)
-    if (p.first == k && p.second >= bytes) return true;
+    if (p.dev == dev && p.k == k && p.bytes >= bytes) return true;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) != cudaSuccess) {
     (void)cudaGetLastError();
     return false;
   }
-  g_smem.push_back({k, bytes});
+  g_smem.push_back({dev, k, bytes});
   return true;
 }
 
-// SM count and resident CTAs per SM of a kernel (host queries, cached).
+// SM count of each device and resident CTAs per SM of a kernel (host queries,
+// cached per device).
 struct OccKey {
+  int dev;
   const void* k;
+  int block;
   size_t smem;
   int occ;
 };
 std::mutex g_occ_mu;
 std::vector<OccKey> g_occ;
-int g_sms = 0;
+int g_sms[kMaxDevices] = {};
 int64_t resident_ctas(const void* k, int block, size_t smem = 0) {
+  const int dev = current_device();
+  if (dev < 0) return 0;
   std::lock_guard<std::mutex> lk(g_occ_mu);
-  if (g_sms == 0) {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
       (void)cudaGetLastError();
       return 0;
     }
-    g_sms = n;
+    g_sms[dev] = n;
   }
   for (const auto& p : g_occ)
-    if (p.k == k && p.smem == smem) return int64_t(g_sms) * p.occ;
+    if (p.dev == dev && p.k == k && p.block == block && p.smem == smem) return int64_t(g_sms[dev]) * p.occ;
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, block, smem) != cudaSuccess) {
     (void)cudaGetLastError();
     occ = 0;
   }
-  g_occ.push_back({k, smem, occ});
-  return int64_t(g_sms) * occ;
+  g_occ.push_back({dev, k, block, smem, occ});
+  return int64_t(g_sms[dev]) * occ;
 }
 
-// Shared tail of the four norm calls.
+// Shared tail of the norm calls.
 //
 // Kernel variants (same bits): register rows (row_kernel: the row as float32
 // in registers; any op, any alignment), raw rows (row_kernel_raw: ops without
-// a residual, 16-byte rows, one CTA per row, raw bf16 kept and unpacked per
-// pass), raw rows persistent (one CTA per resident slot, next row
-// prefetched), and staged rows (row_kernel_staged: the row copied to shared
-// memory by one bulk copy).  NQ_FLAG_VARIANT forces one where it applies.
+// a residual, 16-byte rows, raw bf16 kept and unpacked per pass), raw rows
+// persistent (one CTA per resident slot, next row prefetched), and two rows
+// per CTA (row_kernel_rows_n: static RMSNorm / LayerNorm).  NQ_FLAG_VARIANT
+// forces one where it applies.
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   const bool has_res = a.res_in != nullptr;
   uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
+  if (variant == 4 || variant == 5 || variant == 7)
+    return fail(NQ_ERR_UNSUPPORTED, "%s: NQ_FLAG_VARIANT(%u) is not built (variants 1, 2, 3 and 6 are)", fn, variant);
   if (a.dest != nullptr) variant = 1;  // MoE scatter: register rows only
   const bool raw_forced = variant >= 2 && vec && !has_res && op != nq::kOpRmsDynFp8;
-  const bool ring = variant == 5 && raw_forced;
   Schedule s;
-  nq_status st = ring ? plan_ring(fn, a.d, flags, &s) : plan_rows(fn, op, a.M, a.d, flags, &s, raw_forced, has_res);
+  nq_status st = plan_rows(fn, op, a.M, a.d, flags, &s, raw_forced, has_res);
   if (st != NQ_OK) return st;
   const int threads = 1 << s.log_t;
   const int rows = nq::rows_per_cta(threads);
@@ -401,41 +414,10 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
   const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0,
                                         (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0,
                                         scatter);
-  if (ring) {
-    // Ring depth 4 while four rows take at most 64 KB, else 2; one CTA per
-    // resident slot (the occupancy query counts the ring's shared memory).
-    const int depth_idx = int64_t(a.d) * 2 * 4 <= 64 * 1024 ? 1 : 0;
-    k = table.ring[s.log_t - nq::kMinLogT][s.log_k][depth_idx];
-    smem = size_t(depth_idx ? 4 : 2) * size_t(a.d) * 2;
-    if (k == nullptr) return fail(NQ_ERR_UNSUPPORTED, "%s: ring kernel not built", fn);
-    if (!allow_smem(k, smem))
-      return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
-    const int64_t slots = resident_ctas(k, threads, smem);
-    if (slots <= 0) return fail(NQ_ERR_UNSUPPORTED, "%s: ring kernel does not fit on an SM", fn);
-    grid = grid < slots ? grid : slots;
-  }
   if (vec && !has_res && variant == 6 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
     // The narrow copy skips chunk slots wholly past rows narrower than the schedule.
     k = table.rows2[s.log_t - nq::kMinLogT][s.log_k][a.d < (8 * int64_t(threads)) << s.log_k ? 1 : 0];
     if (k != nullptr) grid = (a.M + 1) / 2;
-  }
-  if (vec && !has_res && variant == 7 && threads > 32 && (op == nq::kOpRmsStaticFp8 || op == nq::kOpLnStaticFp8)) {
-    k = table.rows2p[s.log_t - nq::kMinLogT][s.log_k];
-    if (k != nullptr) {
-      smem = nq::rows2p_smem_bytes(threads, 1 << s.log_k);
-      if (!allow_smem(k, smem))
-        return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
-      const int64_t slots = resident_ctas(k, threads, smem);
-      if (slots <= 0) return fail(NQ_ERR_UNSUPPORTED, "%s: two-row persistent kernel does not fit on an SM", fn);
-      const int64_t pairs = (a.M + 1) / 2;
-      grid = pairs < slots ? pairs : slots;
-    }
-  }
-  if (vec && !has_res && op != nq::kOpRmsDynFp8 && variant == 4) {
-    k = table.staged[s.log_t - nq::kMinLogT][s.log_k];
-    smem = nq::staged_smem_bytes(threads, a.d);
-    if (k != nullptr && !allow_smem(k, smem))
-      return fail(NQ_ERR_UNSUPPORTED, "%s: %zu bytes of shared memory per CTA not available", fn, smem);
   }
   if (vec && !has_res && op != nq::kOpRmsDynFp8 && (variant == 2 || variant == 3)) {
     // The narrow copy tests for chunk slots past the row; a row that fills
@@ -528,19 +510,25 @@ nq_status nq_selftest_division(uint32_t a_bits_begin, uint64_t count, const floa
 
 nq_status nq_check_device_errors(void) {
   const char* fn = "nq_check_device_errors";
-  uint32_t* p = device_error_word();
-  if (p == nullptr) return fail(NQ_ERR_CUDA, "%s: no CUDA device", fn);
+  uint32_t* taken = symbol_on_device(g_taken_ptr, &g_nq_device_error_taken);
+  if (device_error_word() == nullptr || taken == nullptr) return fail(NQ_ERR_CUDA, "%s: no CUDA device", fn);
+  // Every kernel on every stream of this device first (torch's side streams
+  // do not synchronize with the legacy stream), then one thread swaps the word
+  // for zero, then the legacy-stream copy reads what it took.
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) {
+    take_error_word_kernel<<<1, 1, 0, 0>>>();
+    e = cudaGetLastError();
+  }
   uint32_t word = 0;
-  if (cudaMemcpy(&word, p, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
-    const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaMemcpy(&word, taken, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
     return fail(NQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
   }
   if (word == 0) return NQ_OK;
-  const uint32_t zero = 0;
-  if (cudaMemcpy(p, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) (void)cudaGetLastError();
-  return fail(NQ_ERR_CUDA, "%s: device error word 0x%x (bit 0: a bounded wait for a bulk copy gave up, that "
-              "launch's outputs are not meaningful; bit 1: a MoE destination row was out of range and skipped)",
-              fn, word);
+  return fail(NQ_ERR_CUDA, "%s: device error word 0x%x (bit 1: a MoE destination row was out of range; its "
+              "store was skipped)", fn, word);
 }
 
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,

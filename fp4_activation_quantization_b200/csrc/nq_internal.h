@@ -52,7 +52,7 @@ struct RowArgs {
   int32_t d;
   float eps;
   uint32_t flags;  // kFlag* bits; kFlagDiv set means divide, clear means reciprocal
-  uint32_t* err;   // device error word: bit 0 a bounded wait gave up, bit 1 a destination row out of range
+  uint32_t* err;   // device error word: bit 1 a destination row out of range
   const int32_t* dest;  // [M, topk] destination rows (kOutScatter); < 0 skips
   int32_t topk;
   int64_t dest_rows;    // rows of q / scales when scattering
@@ -99,29 +99,15 @@ inline bool raw_schedule_built(int log_t, int log_k) {
   return schedule_built(log_t, log_k) || (log_t == 5 && log_k == 4);
 }
 using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2][2];
-using StagedTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2];
 using Rows2Table = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
-// Ring kernels: T >= 64 threads per row, K <= 4 chunks per thread; [.][.][ring depth 2 or 4]
-using RingTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK][2];
-inline bool ring_schedule_built(int log_t, int log_k) {
-  return log_t >= 6 && log_t <= kMaxLogT && log_k >= 0 && log_k <= 2 && log_t + log_k <= 11;
-}
 struct RowKernels {
   KernelTable direct;  // one row per thread group
   RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent][row narrower than T * K * 8]
-  StagedTable staged;  // rows without residual staged in shared memory by a bulk copy
-  RingTable ring;      // rows without residual through a ring of bulk copies, persistent
   Rows2Table rows2;    // two rows per CTA on the same columns (static RMSNorm / LayerNorm): [.][.][narrow row]
-  StagedTable rows2p;  // rows2 with persistent CTAs prefetching the next two rows by cp.async
 };
-// Dynamic shared memory of a staged-row kernel: its rows of d bf16.
-inline size_t staged_smem_bytes(int threads, int64_t d) { return size_t(rows_per_cta(threads)) * size_t(d) * 2; }
 // Dynamic shared memory of a persistent raw-row kernel: gamma as fp32 for the
 // RMSNorm-type operations (LayerNorm reads gamma / beta through L1).
 inline size_t raw_gamma_smem_bytes(int op, int64_t d) { return op == kOpLnStaticFp8 ? 0 : size_t(d) * 4u; }
-// Dynamic shared memory of the persistent two-row kernel: two stages of two
-// rows of threads x chunks 16-byte slots.
-inline size_t rows2p_smem_bytes(int threads, int chunks) { return size_t(2) * 2u * size_t(chunks) * size_t(threads) * 16u; }
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();

@@ -666,9 +666,8 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
 }
 
 // Per-chunk gamma (RMSNorm: bf16) or gamma and beta (LayerNorm: float32) of
-// chunk slot k = tid + k * T, zero past the row.  GammaLoads fetches them from
-// global memory (through L1) at each use; GammaRegs holds a thread's chunks in
-// registers for a CTA that processes many rows on the same columns.
+// chunk slot k = tid + k * T, zero past the row, fetched from global memory
+// (through L1) at each use.
 template <int T>
 struct GammaLoads {
   const RowArgs& a;
@@ -711,32 +710,11 @@ struct GammaSmem {
   }
 };
 
-template <bool LN, int T, int K>
-struct GammaRegs {
-  float4 g0[LN ? K : 1], g1[LN ? K : 1], e0[LN ? K : 1], e1[LN ? K : 1];
-  uint4 gu[LN ? 1 : K];
-  __device__ __forceinline__ void load(const RowArgs& a, int tid, int C) {
-    const GammaLoads<T> from{a, tid, C};
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      if constexpr (LN) from.ln(k, g0[k], g1[k], e0[k], e1[k]);
-      else gu[k] = from.rms(k);
-    }
-  }
-  __device__ __forceinline__ void ln(int k, float4& a0, float4& a1, float4& b0, float4& b1) const {
-    a0 = g0[k], a1 = g1[k], b0 = e0[k], b1 = e1[k];
-  }
-  __device__ __forceinline__ uint4 rms(int k) const { return gu[k]; }
-  __device__ __forceinline__ void rms2(int k, float2 (&g)[4]) const { unpack_pairs(gu[k], g); }
-};
-
 // a3..a6 of one row without residual whose raw bf16 chunks come from src(k)
-// (registers, or the row staged in shared memory) and whose gamma / beta come
-// from gam.  Rows past M (warp rows only) compute on zeros and store nothing.
-template <int OP, int T, int K, int OUT, bool NARROW, typename Src, typename Gam, typename Hook>
+// (registers) and whose gamma / beta come from gam.  Rows past M (warp rows only) compute on zeros and store nothing.
+template <int OP, int T, int K, int OUT, bool NARROW, typename Src, typename Gam>
 __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, int tid, Src&& src, const Gam& gam,
-                                                float* b0, float* b1, float scale_in, float inv_static,
-                                                Hook&& after_first_sum) {
+                                                float* b0, float* b1, float scale_in, float inv_static) {
   constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
   constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
   constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
@@ -767,7 +745,6 @@ __device__ __forceinline__ void process_raw_row(const RowArgs& a, int64_t row, i
     }
   }
   const float total = row_total<T, K>(part, b0, tid);
-  after_first_sum();  // every thread of the row group has read its chunks
   float rstd, mean = 0.0f;
   if constexpr (OP == kOpLnStaticFp8) {
     mean = __fdiv_rn(total, fd);
@@ -1190,68 +1167,6 @@ __global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel
   process_raw_rows_n<OP, T, K, OUT, NR, NARROW>(a, row, tid, xr, s_sum[0], s_sum[1], scale_in, inv_static);
 }
 
-// NR rows per CTA as row_kernel_rows_n, with persistent CTAs that keep the
-// next group of NR rows in flight: CTA b takes groups b, b + G, b + 2G, ...
-// (G = grid size).  Each thread copies its own chunks of the next group into
-// its own slots of a two-stage shared-memory buffer with cp.async while it
-// processes the current group, so the prefetch holds no registers (the
-// register-prefetching raw kernel gives a quarter of its registers to it).
-// Thread t's 16-byte slot for (stage, row r, chunk k) is ((stage * NR + r) *
-// K + k) * T + t: consecutive threads, consecutive slots, no bank conflicts.
-template <int OP, int T, int K, int OUT, int NR>
-__global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel_rows_n_async(const RowArgs a) {
-  static_assert(T >= 64, "multi-row form: one CTA per group of NR rows");
-  constexpr int W = T / 32;
-  __shared__ __align__(16) float s_sum[2][NR * W * 32];
-  extern __shared__ __align__(16) uint4 s_stage[];  // [2][NR][K][T]
-  const int tid = int(threadIdx.x);
-  const int C = a.d >> 3;
-  const int64_t G = gridDim.x;
-  const int64_t n_groups = (a.M + NR - 1) / NR;
-  griddep_wait();
-  const float scale_in = __ldg(a.scale);
-  const float inv_static = __frcp_rn(scale_in);
-  // Issue group p's copies into stage st and commit them (an empty group past
-  // the last one, so that one wait count serves every step).
-  auto issue = [&](int64_t p, int st) {
-    if (p < n_groups) {
-#pragma unroll
-      for (int r = 0; r < NR; ++r) {
-        const int64_t row = p * NR + r;
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-          const int c = tid + k * T;
-          const bool ok = row < a.M && c < C;
-          const uint16_t* src = ok ? a.x + row * a.ld_x + 8 * c : a.x;
-          cp_async16(&s_stage[((st * NR + r) * K + k) * T + tid], src, ok);
-        }
-      }
-    }
-    cp_async_commit();
-  };
-  int64_t p = blockIdx.x;
-  issue(p, 0);
-  for (int j = 0; p < n_groups; ++j, p += G) {
-    const int64_t next = p + G;
-    issue(next, (j + 1) & 1);
-    if (next >= n_groups) griddep_launch_dependents();  // every load of this CTA is issued
-    cp_async_wait<1>();                                  // group p has landed
-    uint4 xr[NR][K];
-    int64_t row[NR];
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      row[r] = p * NR + r;
-#pragma unroll
-      for (int k = 0; k < K; ++k) xr[r][k] = s_stage[(((j & 1) * NR + r) * K + k) * T + tid];
-    }
-    // LayerNorm's two sums use both buffers (each separated from its next
-    // use by the other sum's barrier); a single sum alternates by step.
-    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
-    process_raw_rows_n<OP, T, K, OUT, NR>(a, row, tid, xr, b0, s_sum[1], scale_in, inv_static);
-  }
-  if (blockIdx.x >= n_groups) griddep_launch_dependents();
-}
-
 // Rows without a residual (static RMSNorm, LayerNorm, NVFP4 without
 // residual), 16-byte rows, T > 32.  Only the raw bf16 chunks are kept (half
 // the registers of float32); each pass unpacks them again.  With PERSIST the
@@ -1314,10 +1229,10 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
     if constexpr (GSMEM)
       process_raw_row<OP, T, K, OUT, NARROW>(a, row, tid, [&](int k) { return xr[k]; },
                                              GammaSmem<T, K>{s_gamma, s_gamma + C, tid, C}, b0, b1, scale_in,
-                                             inv_static, [] {});
+                                             inv_static);
     else
       process_raw_row<OP, T, K, OUT, NARROW>(a, row, tid, [&](int k) { return xr[k]; }, GammaLoads<T>{a, tid, C}, b0,
-                                             b1, scale_in, inv_static, [] {});
+                                             b1, scale_in, inv_static);
   };
 
   if constexpr (!PERSIST) {
@@ -1349,148 +1264,6 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
   }
 }
 
-// Rows without a residual, staged in shared memory: one thread per row issues
-// a single bulk asynchronous copy of the whole row (the TMA engine) that
-// completes on an mbarrier, and every pass re-reads the row from shared memory.
-// The row costs no registers while it is in flight or being processed, so
-// many more rows fit on an SM than with register rows (whose occupancy the row
-// data limits); the launch bound asks for at most 40 registers per thread.
-template <int T>
-constexpr int staged_min_blocks() {
-  constexpr int threads = (T == 32) ? 256 : T;
-  constexpr int blocks = 65536 / (threads * 40);
-  return blocks < 1 ? 1 : (blocks > 16 ? 16 : blocks);
-}
-
-template <int OP, int T, int K, int OUT>
-__global__ void __launch_bounds__(T == 32 ? 256 : T, (staged_min_blocks<T>())) row_kernel_staged(const RowArgs a) {
-  static_assert(OP != kOpRmsDynFp8, "staged rows: no residual");
-  constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
-  constexpr int W = T / 32;
-  extern __shared__ __align__(128) uint4 s_rows[];  // R rows of d / 8 chunks
-  __shared__ __align__(16) float s_sum[2][W > 1 ? W * 32 : 1];
-  __shared__ __align__(8) uint64_t s_bar[R];
-  const int tid = (T == 32) ? int(threadIdx.x & 31u) : int(threadIdx.x);
-  const int rsel = (T == 32) ? int(threadIdx.x >> 5) : 0;
-  const int64_t row = int64_t(blockIdx.x) * R + rsel;
-  const int C = a.d >> 3;
-  const uint4* xs = s_rows + int64_t(rsel) * C;
-
-  if (int(threadIdx.x) < R) mbar_init(&s_bar[threadIdx.x], 1);
-  fence_mbar_init();
-  __syncthreads();
-  griddep_wait();
-  const bool live = row < a.M;
-  if (live && tid == 0) {
-    const uint32_t bytes = uint32_t(a.d) * 2u;
-    mbar_arrive_expect_tx(&s_bar[rsel], bytes);
-    bulk_g2s(s_rows + int64_t(rsel) * C, a.x + row * a.ld_x, bytes, &s_bar[rsel]);
-  }
-  griddep_launch_dependents();
-  if (!live) return;  // a whole warp of a warp-per-row CTA: it takes part in no later barrier
-  const float scale_in = (OP == kOpRmsGroupFp8) ? 1.0f : __ldg(a.scale);
-  const float inv_static = __frcp_rn(scale_in);
-  if (!mbar_wait_bounded(&s_bar[rsel], 0)) {
-    // The copy did not land in time: record it, give the copy one more bounded
-    // wait, and finish the row anyway so that every thread meets the same
-    // barriers (its outputs are then not meaningful).
-    atomicOr(a.err, 1u);
-    (void)mbar_wait_bounded(&s_bar[rsel], 0);
-  }
-  process_raw_row<OP, T, K, OUT, true>(
-      a, row, tid,
-      [&](int k) {
-        const int c = tid + k * T;
-        return c < C ? xs[c] : make_uint4(0u, 0u, 0u, 0u);
-      },
-      GammaLoads<T>{a, tid, C}, s_sum[0], s_sum[1], scale_in, inv_static, [] {});
-}
-
-// Persistent rows without a residual through a ring of S row buffers in
-// shared memory.  CTA b walks rows b, b + G, b + 2G, ... (G = grid size).
-// Thread 0 keeps S bulk copies in flight: each lands one whole row and
-// completes on that stage's mbarrier.  A row is copied once from shared
-// memory into registers (raw bf16); after the row's first reduction barrier,
-// no thread reads the stage any more, so thread 0 refills it with the row S
-// steps ahead.  Gamma (and beta) of the thread's fixed columns stay in
-// registers for the whole kernel, so per row the L1 carries only the row
-// itself and its outputs.  Waits are bounded as in row_kernel_staged.
-template <int OP, int T, int K>
-constexpr int ring_min_blocks() {
-  // registers: gamma / beta (RMSNorm 4, LayerNorm 16 per chunk), the raw row
-  // (4 per chunk), ~48 working
-  constexpr int regs = (OP == kOpLnStaticFp8 ? 16 : 4) * K + 4 * K + 48;
-  constexpr int blocks = 65536 / (T * regs);
-  return blocks < 1 ? 1 : blocks;
-}
-
-template <int OP, int T, int K, int S, int OUT>
-__global__ void __launch_bounds__(T, (ring_min_blocks<OP, T, K>())) row_kernel_ring(const RowArgs a) {
-  static_assert(OP != kOpRmsDynFp8, "ring rows: no residual");
-  static_assert(T >= 64, "ring rows: one row per CTA");
-  constexpr int W = T / 32;
-  extern __shared__ __align__(128) uint4 s_ring[];  // S stages of d / 8 chunks
-  __shared__ __align__(16) float s_sum[2][W * 32];
-  __shared__ __align__(8) uint64_t s_full[S];
-  const int tid = int(threadIdx.x);
-  const int C = a.d >> 3;
-  const int64_t G = gridDim.x;
-  const uint32_t bytes = uint32_t(a.d) * 2u;
-
-  if (tid < S) mbar_init(&s_full[tid], 1);
-  fence_mbar_init();
-  __syncthreads();
-  griddep_wait();
-  if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < S; ++i) {
-      const int64_t r = int64_t(blockIdx.x) + int64_t(i) * G;
-      if (r < a.M) {
-        mbar_arrive_expect_tx(&s_full[i], bytes);
-        bulk_g2s(s_ring + int64_t(i) * C, a.x + r * a.ld_x, bytes, &s_full[i]);
-      }
-    }
-  }
-  GammaRegs<OP == kOpLnStaticFp8, T, K> gam;
-  gam.load(a, tid, C);
-  const float scale_in = (OP == kOpRmsGroupFp8) ? 1.0f : __ldg(a.scale);
-  const float inv_static = __frcp_rn(scale_in);
-  bool released = false;
-  int j = 0;
-  for (int64_t row = blockIdx.x; row < a.M; row += G, ++j) {
-    const int st = j % S;
-    const uint32_t parity = uint32_t(j / S) & 1u;
-    const int64_t refill = row + int64_t(S) * G;  // the row this stage takes next
-    if (!released && refill >= a.M) {
-      griddep_launch_dependents();  // every load of this CTA is issued
-      released = true;
-    }
-    if (!mbar_wait_bounded(&s_full[st], parity)) {
-      atomicOr(a.err, 1u);  // see row_kernel_staged
-      (void)mbar_wait_bounded(&s_full[st], parity);
-    }
-    const uint4* xs = s_ring + int64_t(st) * C;
-    uint4 xr[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
-      xr[k] = c < C ? xs[c] : make_uint4(0u, 0u, 0u, 0u);
-    }
-    // Reduction buffers: LayerNorm's two sums use both (each separated from
-    // its next use by the other sum's barrier); single sums alternate by row.
-    float* b0 = (OP == kOpLnStaticFp8) ? s_sum[0] : s_sum[j & 1];
-    process_raw_row<OP, T, K, OUT, true>(
-        a, row, tid, [&](int k) { return xr[k]; }, gam, b0, s_sum[1], scale_in, inv_static, [&] {
-          if (tid == 0 && refill < a.M) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive_expect_tx(&s_full[st], bytes);
-            bulk_g2s(s_ring + int64_t(st) * C, a.x + refill * a.ld_x, bytes, &s_full[st]);
-          }
-        });
-  }
-  if (!released) griddep_launch_dependents();
-}
-
 // Kernel table of one operation and output form (OUT bits): every built
 // (threads, chunks, vec) schedule.
 template <int OP, int OUT>
@@ -1504,14 +1277,7 @@ struct RowTable {
       for (auto& y : x)
         for (auto& z : y)
           for (auto& w : z) w = nullptr;
-    for (auto& x : k.staged)
-      for (auto& y : x) y = nullptr;
     for (auto& x : k.rows2)
-      for (auto& y : x)
-        for (auto& z : y) z = nullptr;
-    for (auto& x : k.rows2p)
-      for (auto& y : x) y = nullptr;
-    for (auto& x : k.ring)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
 #define NQ_RAW(LT, LK)                                                                                         \
@@ -1520,13 +1286,11 @@ struct RowTable {
     k.raw[LT - kMinLogT][LK][1][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT, false>);  \
     k.raw[LT - kMinLogT][LK][0][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT, true>);  \
     k.raw[LT - kMinLogT][LK][1][1] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), true, OUT, true>);   \
-    k.staged[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_staged<OP, (1 << LT), (1 << LK), OUT>);     \
   }                                                                                                            \
   if constexpr (OP == kOpRmsStaticFp8 || OP == kOpLnStaticFp8) {                                               \
     if constexpr (LT > 5 && LK <= 3) {                                                                         \
       k.rows2[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2, false>); \
       k.rows2[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_rows_n<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2, true>); \
-      k.rows2p[LT - kMinLogT][LK] = reinterpret_cast<const void*>(&row_kernel_rows_n_async<OP, (1 << LT), (1 << (LK > 3 ? 3 : LK)), OUT, 2>); \
     }                                                                                                          \
   }
 #define NQ_DIRECT(LT, LK)                                                                                 \
@@ -1542,17 +1306,6 @@ struct RowTable {
     NQ_DIRECT(9, 0) NQ_DIRECT(9, 1) NQ_DIRECT(9, 2)
     NQ_DIRECT(10, 0) NQ_DIRECT(10, 1)
     NQ_RAW(5, 4)  // one warp per row, 16 chunks per lane (rows of up to 4096 elements)
-#define NQ_RING(LT, LK)                                                                                           \
-  if constexpr (OP != kOpRmsDynFp8 && !(OUT & kOutScatter)) {                                                     \
-    k.ring[LT - kMinLogT][LK][0] = reinterpret_cast<const void*>(&row_kernel_ring<OP, (1 << LT), (1 << LK), 2, OUT>); \
-    k.ring[LT - kMinLogT][LK][1] = reinterpret_cast<const void*>(&row_kernel_ring<OP, (1 << LT), (1 << LK), 4, OUT>); \
-  }
-    NQ_RING(6, 0) NQ_RING(6, 1) NQ_RING(6, 2)
-    NQ_RING(7, 0) NQ_RING(7, 1) NQ_RING(7, 2)
-    NQ_RING(8, 0) NQ_RING(8, 1) NQ_RING(8, 2)
-    NQ_RING(9, 0) NQ_RING(9, 1) NQ_RING(9, 2)
-    NQ_RING(10, 0) NQ_RING(10, 1)
-#undef NQ_RING
 #undef NQ_DIRECT
 #undef NQ_RAW
   }

@@ -13,8 +13,8 @@
  * --------------------------------
  * Status. Every call returns an nq_status. NQ_OK = 0. On any other value
  *   nothing was launched and nq_last_error() (thread-local) says why. No call
- *   throws across the ABI, traps on the device, synchronizes the stream or the
- *   device, or allocates memory.
+ *   throws across the ABI, traps on the device or allocates memory, and no
+ *   call but nq_check_device_errors synchronizes a stream or the device.
  * Memory. Every pointer is caller-owned DEVICE memory on the current CUDA
  *   device (the "scale" arguments too: they are read by the kernel at execution
  *   time, so a captured CUDA graph sees scale updates made between replays).
@@ -139,30 +139,25 @@ typedef enum nq_status {
 /* Force a kernel variant (tests and tuning; same bits either way): n = 1 keeps
  * the row in float32 registers; n = 2 keeps only the raw bf16 row and unpacks
  * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row;
- * n = 4 stages the row in shared memory with one bulk asynchronous copy and
- * re-reads it there on every pass; n = 5 runs persistent CTAs that keep a ring
- * of bulk copies of upcoming rows in flight and hold gamma (and beta) in
- * registers (t >= 6, k <= 2 with NQ_FLAG_SCHEDULE); n = 6 (static RMSNorm
- * and LayerNorm, t >= 6) gives each CTA two rows on the same columns, so each
- * thread loads its gamma / beta once for both; n = 7 is n = 6 with persistent
- * CTAs, each thread copying its chunks of the CTA's next two rows into shared
- * memory (cp.async) while it processes the current two.  n = 2..7 apply to
- * 16-byte-aligned rows without a residual and are ignored otherwise; with
- * n = 2..4, NQ_FLAG_SCHEDULE also accepts t = 5, k = 4 (one warp per row, 16
- * chunks per lane, rows of up to 4096 elements).  0 = automatic. */
+ * n = 6 (static RMSNorm and LayerNorm, t >= 6) gives each CTA two rows on the
+ * same columns, so each thread loads its gamma / beta once for both.  n = 2, 3
+ * and 6 apply to 16-byte-aligned rows without a residual and are ignored
+ * otherwise; with n = 2 or 3, NQ_FLAG_SCHEDULE also accepts t = 5, k = 4 (one
+ * warp per row, 16 chunks per lane, rows of up to 4096 elements).  n = 4, 5
+ * and 7 are not built (NQ_ERR_UNSUPPORTED).  0 = automatic. */
 #define NQ_FLAG_VARIANT(n) ((((uint32_t)(n)) & 0x7u) << 24)
 #define NQ_FLAG_VARIANT_MASK (0x7u << 24)
 /* Library version (major * 10000 + minor * 100 + patch). */
 int nq_version(void);
 /* Static text of a status code. */
 const char* nq_status_string(nq_status status);
-/* Synchronous: read and clear this library's device error word on the current
- * device.  NQ_OK if no kernel recorded an error since the last check;
- * NQ_ERR_CUDA (message in nq_last_error) if a kernel's bounded wait for its
- * own bulk copy into shared memory gave up (about one second; bit 0), in which
- * case that launch's outputs are not meaningful, or if a MoE destination row
- * was out of range (bit 1; the store was skipped).  Kernels never trap or
- * hang. */
+/* Synchronous: waits for all work on the current device (every stream), then
+ * reads and clears this library's device error word in one atomic step.
+ * NQ_OK if no kernel recorded an error since the last check; NQ_ERR_CUDA
+ * (message in nq_last_error) if a MoE destination row was out of range (bit 1:
+ * that store was skipped, the other rows are written), or if the device
+ * reported an error while synchronizing.  Kernels never trap or hang, and no
+ * kernel of this library waits on anything. */
 nq_status nq_check_device_errors(void);
 /* Diagnostic (tests): checks, on the device, the bounded division the dynamic
  * FP8 path uses for RN(y / s) (a correctly rounded reciprocal r = RN(1 / s),

@@ -85,6 +85,11 @@ def test_validation_without_gpu(nq):
     assert call_fused(nq, d=1024, flags=nq.flag_schedule(5, 0)) == INV
     # static: residual pair must be both or neither
     L = nq.lib
+    # variants 4, 5 and 7 are not built: rejected on the host, nothing launched
+    for v in (4, 5, 7):
+        assert L.nq_rmsnorm_quant_fp8_static(FAKE, 64, None, None, 64, FAKE, FAKE, FAKE, 64, None, 64, 4, 64,
+                                             1e-6, nq.flag_variant(v), None) == UNS, v
+        assert b"not built" in L.nq_last_error()
     assert L.nq_rmsnorm_quant_fp8_static(FAKE, 64, FAKE, None, 64, FAKE, FAKE, FAKE, 64, None, 64, 4, 64,
                                          1e-6, 0, None) == INV
     # NVFP4 needs d % 16 == 0, and has no e5m2 form

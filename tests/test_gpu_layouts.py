@@ -68,7 +68,7 @@ def test_nvfp4_swizzled_every_schedule_and_variant(nq, d):
     gn = oracle.nvfp4_global_scale(w["x"], w["gamma"])
     eq, esf, _, _ = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn)
     esw = oracle.sf_swizzle(esf)
-    flags = [0] + [nq.flag_schedule(*s_) for s_ in all_schedules(d)] + [nq.flag_variant(v) for v in (1, 2, 3, 4)]
+    flags = [0] + [nq.flag_schedule(*s_) for s_ in all_schedules(d)] + [nq.flag_variant(v) for v in (1, 2, 3)]
     if (d + 7) // 8 <= 512:
         flags.append(nq.flag_variant(2) | nq.flag_schedule(5, 4))
     for f in flags:
@@ -169,7 +169,7 @@ def test_group_scale_layouts_fused(nq, name, col, packed, residual, d, M):
         flags |= nq.FLAG_E5M2 if e5 else 0
         variants = [0] + [nq.flag_schedule(*s_) for s_ in all_schedules(d)]
         if not residual:
-            variants += [nq.flag_variant(v) for v in (2, 3, 4)]
+            variants += [nq.flag_variant(v) for v in (2, 3)]
         for v in variants:
             buf, view, ld = scales_buffer(nq, M, G, col, packed, pad=2)
             q, s, ro, _ = nq.nq_rmsnorm_quant_fp8_group(x, g, 1e-6, group=group, residual=res, scales_out=view,

@@ -103,6 +103,30 @@ def test_moe_out_of_range_destination_is_skipped_and_reported(nq):
     assert np.all(got_q[~ok] == SENT)
 
 
+def test_error_word_seen_from_a_side_stream(nq):
+    """A dispatch with an out-of-range destination launched on a non-default
+    torch stream, with no synchronization before the check: the check waits
+    for every stream of the device, reports bit 1 once, and leaves the word
+    clear (the next check passes)."""
+    M, d, E, topk = 256, 2048, 16, 4
+    w = S.make_rms_inputs(M, d, seed=9, residual=True)
+    r = S.make_moe_routing(M, E, topk, seed=9)
+    bad = torch.from_numpy(r["dest"].copy())
+    bad[M - 1, 0] = r["rows"] + 7
+    nq.nq_check_device_errors()
+    x, g, res = dev_bf16(w["x"]), dev_bf16(w["gamma"]), dev_bf16(w["residual"])
+    dest = bad.cuda()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        for _ in range(20):  # queue work ahead of the reported launch
+            nq.nq_fused_add_rmsnorm_quant_fp8(x, res, g, 1e-6)
+        nq.nq_fused_add_rmsnorm_quant_fp8_moe(x, g, dest, r["rows"], 1e-6, residual=res)
+    with pytest.raises(nq.NQError, match="bit 1"):
+        nq.nq_check_device_errors()
+    nq.nq_check_device_errors()
+
+
 def test_moe_ue8m0_and_forced_schedules(nq):
     M, d, E, topk = 129, 4096, 64, 8
     w = S.make_rms_inputs(M, d, seed=5, residual=True)
