@@ -35,7 +35,7 @@ __all__ = [
 ]
 
 NQ_OK, NQ_ERR_INVALID_ARGUMENT, NQ_ERR_UNSUPPORTED, NQ_ERR_CUDA = 0, 1, 2, 3
-NQ_MAX_D = 16384
+NQ_MAX_D = 65536
 FLAG_PDL = 1 << 0
 FLAG_SCALE_DIV = 1 << 1
 FLAG_SCALE_RECIP = 1 << 2

@@ -9,6 +9,7 @@
 // every schedule and reproducible on the CPU.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -263,6 +264,63 @@ __device__ __forceinline__ float row_max_nonneg(float v, uint32_t* red, int tid)
     for (int i = 0; i < W; ++i) u = max(u, red[i]);
   }
   return __uint_as_float(u);
+}
+
+// ------------------------------------------------- rows over a cluster ----
+// A row wider than one CTA can hold in registers is split over a cluster of NC
+// CTAs (thread-block cluster; each CTA on its own SM).  CTA rank j of the
+// cluster owns, in thread t, the chunks k * NC * T + j * T + t, so the chunk
+// index's bits are, from the top: k (the thread's own slots), j (the CTA),
+// the warp, the lane.  The canonical tree combines them in that order; the
+// level over j runs here, through distributed shared memory: every CTA
+// publishes its per-thread partial, and each CTA combines the NC partials of
+// its thread index (CTA j absorbs CTA j + NC/2, ..., highest bit first), so
+// every CTA holds the same values afterwards.  `xred` holds T floats and is
+// used by one reduction only (no reuse, so no barrier is needed before it is
+// written).  The cluster barrier is a hardware barrier that every thread of
+// the cluster reaches on the same path; nothing here spins.
+template <int T, int NC>
+__device__ __forceinline__ float cluster_tree_sum(float v, float* xred, int tid) {
+  if constexpr (NC == 1) {
+    return v;
+  } else {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    xred[tid] = v;
+    cl.sync();
+    float p[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) p[j] = *cl.map_shared_rank(xred + tid, j);
+#pragma unroll
+    for (int h = NC / 2; h >= 1; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) p[i] = __fadd_rn(p[i], p[i + h]);
+    return p[0];
+  }
+}
+
+// Largest of the cluster's per-CTA values (non-negative floats as bits; order-free).
+template <int NC>
+__device__ __forceinline__ uint32_t cluster_max_u32(uint32_t u, uint32_t* xred, int tid) {
+  if constexpr (NC == 1) {
+    return u;
+  } else {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    if (tid == 0) xred[0] = u;
+    cl.sync();
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) m = max(m, *cl.map_shared_rank(xred, j));
+    return m;
+  }
+}
+
+// Rank of this CTA in its cluster (0 without a cluster).
+template <int NC>
+__device__ __forceinline__ int cluster_rank() {
+  if constexpr (NC == 1) return 0;
+  else return int(cooperative_groups::this_cluster().block_rank());
 }
 
 }  // namespace nq

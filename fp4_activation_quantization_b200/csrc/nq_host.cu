@@ -378,11 +378,49 @@ int64_t resident_ctas(const void* k, int block, size_t smem = 0) {
 // persistent (one CTA per resident slot, next row prefetched), and two rows
 // per CTA (row_kernel_rows_n: static RMSNorm / LayerNorm).  NQ_FLAG_VARIANT
 // forces one where it applies.
+// Clusters per row of a row wider than 16384 elements (2048 chunks): 2 up to
+// 32768 elements, 4 up to 65536; 0 for rows one CTA holds.
+int cluster_ctas(int64_t d) {
+  const int64_t C = (d + 7) / 8;
+  return C <= 2048 ? 0 : (C <= 4096 ? 2 : 4);
+}
+
+// Rows wider than 16384 elements: one row per thread-block cluster of 2 or 4
+// CTAs of 1024 threads (register rows; the variants do not apply).
+nq_status run_cluster_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
+  if (flags & NQ_FLAG_SCHEDULE_MASK)
+    return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE covers at most 2048 chunks; d = %lld takes a cluster "
+                "per row", fn, (long long)a.d);
+  const int nc = cluster_ctas(a.d);
+  const int64_t grid = a.M * nc;
+  if (grid > int64_t(0x7fffffff)) return fail(NQ_ERR_UNSUPPORTED, "%s: M = %lld too large for rows of d = %lld", fn,
+                                              (long long)a.M, (long long)a.d);
+  const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0,
+                                        (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0,
+                                        a.dest != nullptr);
+  const auto& tab = table.cluster[nc == 4 ? 1 : 0];
+  const int64_t span = int64_t(8) * nq::kClusterThreads * nq::kClusterChunks * nc;  // elements a cluster covers
+  const void* k = tab[vec ? 1 : 0];
+  // As for one CTA per row: the predicate-free copy for rows that fill the
+  // cluster, the copy that skips dead chunk slots for narrower rows, each when
+  // it needs no more registers.
+  const int mode = !vec ? 0 : (a.d == span ? 2 : 3);
+  if (mode >= 2 && tab[mode] != nullptr) {
+    const int r_m = kernel_regs(tab[mode]), r_vec = kernel_regs(tab[1]);
+    if (r_m > 0 && r_vec > 0 && r_m <= r_vec) k = tab[mode];
+  }
+  a.err = device_error_word();
+  if (a.err == nullptr) return fail(NQ_ERR_CUDA, "%s: no CUDA device", fn);
+  void* args[] = {&a};
+  return launch(fn, k, unsigned(grid), unsigned(nq::kClusterThreads), 0, args, (flags & NQ_FLAG_PDL) != 0, stream);
+}
+
 nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   const bool has_res = a.res_in != nullptr;
   uint32_t variant = (flags & NQ_FLAG_VARIANT_MASK) >> 24;
   if (variant == 4 || variant == 5 || variant == 7)
     return fail(NQ_ERR_UNSUPPORTED, "%s: NQ_FLAG_VARIANT(%u) is not built (variants 1, 2, 3 and 6 are)", fn, variant);
+  if (cluster_ctas(a.d) > 0) return run_cluster_rows(fn, op, a, vec, flags, stream);
   if (a.dest != nullptr) variant = 1;  // MoE scatter: register rows only
   const bool raw_forced = variant >= 2 && vec && !has_res && op != nq::kOpRmsDynFp8;
   Schedule s;
@@ -538,6 +576,14 @@ nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* t
   NQ_REQUIRE(threads_per_row && chunks_per_thread && rows_per_cta, "%s: null output pointer", fn);
   nq_status st = check_common(fn, M, d, 1.0f);
   if (st != NQ_OK) return st;
+  if (const int nc = cluster_ctas(d)) {
+    // One row per cluster of nc CTAs: threads_per_row counts the cluster's threads.
+    NQ_REQUIRE(!(flags & NQ_FLAG_SCHEDULE_MASK), "%s: NQ_FLAG_SCHEDULE does not cover d = %lld", fn, (long long)d);
+    *threads_per_row = nq::kClusterThreads * nc;
+    *chunks_per_thread = nq::kClusterChunks;
+    *rows_per_cta = 1;
+    return NQ_OK;
+  }
   Schedule s;
   st = plan_rows(fn, op, M, d, flags, &s);
   if (st != NQ_OK) return st;

@@ -81,7 +81,8 @@ struct GroupArgs {
 
 // Schedules: 2^t threads per row (t = 5..10), 2^k chunks of 8 elements per
 // thread (k = 0..3, with t + k <= 11, i.e. up to 2048 chunks = 16384
-// elements).  Rows per CTA: 8 when t == 5 (one warp per row), else 1.
+// elements).  Rows per CTA: 8 when t == 5 (one warp per row), else 1.  Wider
+// rows take a cluster of CTAs (ClusterTable).
 constexpr int kMinLogT = 5, kMaxLogT = 10, kMaxLogK = 3;
 inline int rows_per_cta(int threads) { return threads == 32 ? 8 : 1; }
 inline bool schedule_built(int log_t, int log_k) {
@@ -100,10 +101,16 @@ inline bool raw_schedule_built(int log_t, int log_k) {
 }
 using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2][2];
 using Rows2Table = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
+// Rows wider than 16384 elements: one row per cluster of 2 (rows of up to
+// 32768 elements) or 4 (up to 65536) CTAs of 1024 threads, 2 chunks per
+// thread: [clusters of 2, 4][mode as KernelTable].
+constexpr int kClusterThreads = 1024, kClusterChunks = 2;
+using ClusterTable = const void* [2][4];
 struct RowKernels {
-  KernelTable direct;  // one row per thread group
-  RawTable raw;        // rows without residual, raw bf16 in registers: [.][.][persistent][row narrower than T * K * 8]
-  Rows2Table rows2;    // two rows per CTA on the same columns (static RMSNorm / LayerNorm): [.][.][narrow row]
+  KernelTable direct;    // one row per thread group
+  RawTable raw;          // rows without residual, raw bf16 in registers: [.][.][persistent][row narrower than T * K * 8]
+  Rows2Table rows2;      // two rows per CTA on the same columns (static RMSNorm / LayerNorm): [.][.][narrow row]
+  ClusterTable cluster;  // one row per thread-block cluster
 };
 // Dynamic shared memory of a persistent raw-row kernel: gamma as fp32 for the
 // RMSNorm-type operations (LayerNorm reads gamma / beta through L1).

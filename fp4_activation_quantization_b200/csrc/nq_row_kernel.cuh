@@ -152,29 +152,33 @@ __device__ __forceinline__ float chunk_partial(const float2 (&v)[4]) {
 }
 
 // Row sum of the K chunk partials held by each thread of the group (highest
-// chunk-index bit first: the thread's own chunks, then across threads).
-template <int T, int K>
-__device__ __forceinline__ float row_total(float (&part)[K], float* red, int tid) {
+// chunk-index bit first: the thread's own chunks, then across the CTAs of a
+// cluster (NC > 1, through xred), then across threads).
+template <int T, int K, int NC = 1>
+__device__ __forceinline__ float row_total(float (&part)[K], float* red, int tid, float* xred = nullptr) {
 #pragma unroll
   for (int h = K / 2; h >= 1; h >>= 1)
 #pragma unroll
     for (int i = 0; i < h; ++i) part[i] = __fadd_rn(part[i], part[i + h]);
-  return row_sum<T>(part[0], red, tid);
+  return row_sum<T>(cluster_tree_sum<T, NC>(part[0], xred, tid), red, tid);
 }
 
 // a1: raw bf16 chunks of one row (zeros past the row or for dead rows).
 // FULL: every chunk slot of the schedule is a real chunk of a live row (d ==
-// 8 * T * K, one row per CTA), so no predicate or zero fill is needed.
-template <int T, int K, bool VEC, bool FULL>
+// 8 * T * K * NC, one row per CTA or cluster), so no predicate or zero fill is
+// needed.  With a cluster of NC CTAs, CTA `rank` owns chunks
+// tid + rank * T + k * T * NC.
+template <int T, int K, bool VEC, bool FULL, int NC = 1>
 __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool live, bool has_res, int tid,
-                                         uint4 (&xr)[K], uint4 (&rr)[K]) {
+                                         uint4 (&xr)[K], uint4 (&rr)[K], int rank = 0) {
   const int d = a.d;
   const int C = (d + 7) >> 3;
   const uint16_t* xrow = a.x + row * a.ld_x;
   const uint16_t* rrow = a.res_in + row * a.ld_res;
+  const int cb = tid + (NC > 1 ? rank * T : 0);
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
+    const int c = cb + k * T * NC;
     const bool ok = FULL || (live && c < C);
     if constexpr (VEC) {
       xr[k] = ok ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
@@ -197,17 +201,18 @@ __device__ __forceinline__ void load_raw(const RowArgs& a, int64_t row, bool liv
 
 // The FP8 codes of a row's K chunk slots, stored to each of its destination
 // rows (MoE dispatch).
-template <int T, int K, bool VEC, bool FULL>
+template <int T, int K, bool VEC, bool FULL, int NC = 1>
 __device__ __forceinline__ void scatter_codes(const RowArgs& a, int64_t row, bool live, int tid,
-                                              const uint2 (&codes)[K]) {
+                                              const uint2 (&codes)[K], int rank = 0) {
   if (!live) return;
   const int d = a.d;
-  const int C = FULL ? T * K : (d + 7) >> 3;
+  const int C = FULL ? T * K * NC : (d + 7) >> 3;
+  const int cb = tid + (NC > 1 ? rank * T : 0);
   for_each_dest(a, row, [&](int64_t r) {
     uint8_t* qrow = a.q + r * a.ld_q;
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-      const int c = tid + k * T;
+      const int c = cb + k * T * NC;
       if (FULL || c < C) {
         if constexpr (VEC) {
           *reinterpret_cast<uint2*>(qrow + 8 * c) = codes[k];
@@ -228,11 +233,12 @@ __device__ __forceinline__ void scatter_codes(const RowArgs& a, int64_t row, boo
 // (max 448, or 57344 for e5m2; UE8M0: next power of two), one reciprocal,
 // q = fp8(RN(y * RN(1 / s))).  K <= 8, so a warp's K slots hold at most 32
 // groups (one per lane).
-template <bool E5, bool LAYOUT, int T, int K, bool VEC, bool FULL, bool SCATTER = false>
+template <bool E5, bool LAYOUT, int T, int K, bool VEC, bool FULL, bool SCATTER = false, int NC = 1>
 __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, bool live, int tid,
-                                                const float2 (&v)[K][4], bool div) {
+                                                const float2 (&v)[K][4], bool div, int rank = 0) {
   const int d = a.d;
-  const int C = FULL ? T * K : (d + 7) >> 3;
+  const int C = FULL ? T * K * NC : (d + 7) >> 3;
+  const int cb = tid + (NC > 1 ? rank * T : 0);  // this thread's chunk in slot 0
   const int lcpg = (a.group == 128) ? 4 : 3;  // log2(chunks per group): groups are 64 or 128
   const int cpg = 1 << lcpg;                   // chunks per group: 8 or 16
   const int gpw = 32 >> lcpg;                  // groups per warp per chunk slot
@@ -263,7 +269,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
   const float inv = (s == 0.0f) ? 0.0f : __frcp_rn(s);
   {
     const int kj = lane >> (5 - lcpg), part = lane & (gpw - 1);
-    const int c0 = (tid & ~31) + (part << lcpg) + kj * T;  // first chunk of lane j's group
+    const int c0 = (cb & ~31) + (part << lcpg) + kj * T * NC;  // first chunk of lane j's group
     if (kj < K && (FULL || (live && c0 < C))) {
       if constexpr (SCATTER)
         for_each_dest(a, row, [&](int64_t r) { a.scale_out[r * a.ld_scale + (c0 >> lcpg)] = s; });
@@ -278,7 +284,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
   uint2 kept[SCATTER ? K : 1];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
+    const int c = cb + k * T * NC;
     const int src = k * gpw + (lane >> lcpg);
     const float ik = __shfl_sync(kFull, inv, src);
     const float sk = div ? __shfl_sync(kFull, s, src) : 0.0f;
@@ -299,22 +305,27 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
       }
     }
   }
-  if constexpr (SCATTER) scatter_codes<T, K, VEC, FULL>(a, row, live, tid, kept);
+  if constexpr (SCATTER) scatter_codes<T, K, VEC, FULL, NC>(a, row, live, tid, kept, rank);
 }
 
 // a2..a6 of one row whose raw chunks are in registers.  Contains the row
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
-// reduction buffers.
-template <int OP, int T, int K, bool VEC, bool FULL, int OUT, bool NARROW = false>
+// reduction buffers.  A row split over a cluster of NC CTAs (this one of rank
+// `rank`) also takes the cluster's barriers and its distributed buffers
+// x_sum0 / x_sum1 (T floats each) and x_max (one word).
+template <int OP, int T, int K, bool VEC, bool FULL, int OUT, bool NARROW = false, int NC = 1>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
-                                            float* s_sum1, uint32_t* s_max) {
+                                            float* s_sum1, uint32_t* s_max, int rank = 0, float* x_sum0 = nullptr,
+                                            float* x_sum1 = nullptr, uint32_t* x_max = nullptr) {
   constexpr bool E5 = (OUT & kOutAlt) && OP != kOpRmsNvfp4;   // e5m2 codes
   constexpr bool SWZ = (OUT & kOutAlt) && OP == kOpRmsNvfp4;  // swizzled block scales
   constexpr bool LAYOUT = (OUT & kOutScaleLayout) != 0;       // strided / packed group scales
   constexpr bool SCATTER = (OUT & kOutScatter) != 0;          // MoE destination rows
   const int d = a.d;
-  const int C = FULL ? T * K : (d + 7) >> 3;
+  const int C = FULL ? T * K * NC : (d + 7) >> 3;
+  constexpr int CS = T * NC;                      // chunk stride between a thread's slots
+  const int cb = tid + (NC > 1 ? rank * T : 0);  // this thread's chunk in slot 0
   const bool live = FULL || live_in;
   const bool div_flag = (a.flags & kFlagDiv) != 0;
   const bool bf16_flag = (a.flags & kFlagNormBf16) != 0;
@@ -323,14 +334,14 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
   // except the NVFP4 and group quantization (which run on its zeros); its
   // sums are +0, as zero chunks give.  Only the upper half of the slots can
   // be dead for a planned schedule (see process_raw_row).
-  const int wbase = tid & ~31;
-  auto slot_live = [&](int k) { return !NARROW || k < K / 2 || wbase + k * T < C; };
+  const int wbase = cb & ~31;
+  auto slot_live = [&](int k) { return !NARROW || k < K / 2 || wbase + k * CS < C; };
   // ---- a2: r = x + residual, residual_out; a3: chunk partials
   float2 v[K][4];
   float part[K];
 #pragma unroll
   for (int k = 0; k < K; ++k) {
-    const int c = tid + k * T;
+    const int c = cb + k * CS;
     if (!slot_live(k)) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) v[k][i] = f2(0.0f);
@@ -358,7 +369,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     }
     part[k] = chunk_partial<OP != kOpLnStaticFp8>(v[k]);
   }
-  const float total = row_total<T, K>(part, s_sum0, tid);
+  const float total = row_total<T, K, NC>(part, s_sum0, tid, x_sum0);
 
   const float fd = float(d);
   float rstd;
@@ -369,7 +380,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
     for (int k = 0; k < K; ++k) {
       if (!slot_live(k)) continue;  // part[k] is +0 already
-      const int c = tid + k * T;
+      const int c = cb + k * CS;
       const bool ok = FULL || (live && c < C);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -383,7 +394,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       // a chunk slot past the row adds +0 (its values are never stored)
       part[k] = ok ? chunk_partial<true>(v[k]) : 0.0f;
     }
-    const float sq = row_total<T, K>(part, s_sum1, tid);
+    const float sq = row_total<T, K, NC>(part, s_sum1, tid, x_sum1);
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(sq, fd), a.eps)));
   } else {
     rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(total, fd), a.eps)));
@@ -402,7 +413,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
   for (int k = 0; k < K; ++k) {
     if (!slot_live(k)) continue;  // y stays 0
-    const int c = tid + k * T;
+    const int c = cb + k * CS;
     const bool gok = FULL || c < C;
     if constexpr (OP == kOpLnStaticFp8) {
       const float* gp = static_cast<const float*>(a.gamma) + 8 * c;
@@ -460,7 +471,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       uint16_t* nrow = norm_out + row * a.ld_norm;
 #pragma unroll
       for (int k = 0; k < K; ++k) {
-        const int c = tid + k * T;
+        const int c = cb + k * CS;
         if (FULL || (live && c < C)) {
           if constexpr (VEC) {
             *reinterpret_cast<uint4*>(nrow + 8 * c) = pack_pairs_bf16(v[k]);
@@ -489,7 +500,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       return fmaxf(m8, __shfl_xor_sync(kFull, m8, 1));
     };
     auto quant_store = [&](int k, const Nvfp4Scale& sc, bool sf_here) {
-      const int c = tid + k * T;
+      const int c = cb + k * CS;
       const bool ok = FULL || (live && c < C);
       float t[8];
       const float S = div ? __fmul_rn(e4m3_to_f32(sc.code), g) : 0.0f;
@@ -535,10 +546,10 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
       quant_store(0, nvfp4_block_scale<false>(block_amax(0), g, ngr, g_fast), true);
     }
     if constexpr (SWZ) {
-      if (live) sf_zero_padding_rows<T>(a, row, tid);
+      if (live && cb < T) sf_zero_padding_rows<T>(a, row, tid);  // rank 0 of a cluster
     }
   } else if constexpr (OP == kOpRmsGroupFp8) {
-    quantize_groups<E5, LAYOUT, T, K, VEC, FULL, SCATTER>(a, row, live, tid, v, div);
+    quantize_groups<E5, LAYOUT, T, K, VEC, FULL, SCATTER, NC>(a, row, live, tid, v, div, rank);
   } else {
     float s_div, s_inv;
     bool passthrough = false;
@@ -547,12 +558,13 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
 #pragma unroll
       for (int k = 0; k < K; ++k)
         if (slot_live(k)) m = absmax8(v[k], m);
-      const float amax = row_max_nonneg<T>(m, s_max, tid);
+      const float amax = __uint_as_float(
+          cluster_max_u32<NC>(__float_as_uint(row_max_nonneg<T>(m, s_max, tid)), x_max, tid));
       const float s = fp8_scale_of<E5>(amax);
       if constexpr (SCATTER) {
-        if (live && tid == 0) for_each_dest(a, row, [&](int64_t r) { a.scale_out[r] = s; });
+        if (live && cb == 0) for_each_dest(a, row, [&](int64_t r) { a.scale_out[r] = s; });
       } else {
-        if (live && tid == 0) a.scale_out[row] = s;
+        if (live && cb == 0) a.scale_out[row] = s;
       }
       s_div = s;
       s_inv = __frcp_rn(s);
@@ -564,7 +576,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
     uint8_t* qrow = a.q + row * a.ld_q;
     uint2 kept[SCATTER ? K : 1];
     auto store_codes = [&](int k, const float2 (&t)[4]) {
-      const int c = tid + k * T;
+      const int c = cb + k * CS;
       const uint2 codes = pack_pairs_fp8<E5>(t);
       if constexpr (SCATTER) {
         kept[k] = codes;
@@ -618,7 +630,7 @@ __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool 
         store_codes(k, t);
       }
     }
-    if constexpr (SCATTER) scatter_codes<T, K, VEC, FULL>(a, row, live, tid, kept);
+    if constexpr (SCATTER) scatter_codes<T, K, VEC, FULL, NC>(a, row, live, tid, kept, rank);
   }
   };
   // Measured on B200: the second copy pays with four chunks per thread
@@ -663,6 +675,40 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
   load_raw<T, K, VEC, FULL>(a, row, live, has_res, tid, xr, rr);
   griddep_launch_dependents();  // the next kernel on the stream may start its prologue
   process_row<OP, T, K, VEC, FULL, OUT, NARROW>(a, row, live, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max);
+}
+
+// Rows wider than one CTA can hold in registers (d > 16384 elements): one row
+// per thread-block cluster of NC CTAs of 1024 threads, each on its own SM,
+// each holding K chunks per thread in registers, so the row is still read
+// once and every output written once.  The row sums cross the cluster through
+// distributed shared memory in the canonical order (cluster_tree_sum); the
+// absmax of the dynamic scale likewise.  MODE as for row_kernel.
+template <int OP, int K, int MODE, int OUT, int NC>
+__global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(1024) row_kernel_cluster(const RowArgs a) {
+  constexpr int T = 1024;
+  constexpr bool VEC = MODE >= 1;
+  constexpr bool FULL = MODE == 2;
+  constexpr bool NARROW = MODE == 3;
+  constexpr int W = T / 32;
+  static_assert(NC == 2 || NC == 4, "CTAs per row");
+  __shared__ __align__(16) float s_sum[2][W * 32];
+  __shared__ uint32_t s_max[W];
+  __shared__ __align__(16) float x_sum[2][T];  // read by the other CTAs of the cluster
+  __shared__ uint32_t x_max[1];
+
+  const int tid = int(threadIdx.x);
+  const int rank = cluster_rank<NC>();
+  const int64_t row = int64_t(blockIdx.x) / NC;  // one row per cluster (clusters are consecutive blocks)
+  const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
+
+  griddep_wait();
+  uint4 xr[K], rr[K];
+  load_raw<T, K, VEC, FULL, NC>(a, row, true, has_res, tid, xr, rr, rank);
+  griddep_launch_dependents();
+  process_row<OP, T, K, VEC, FULL, OUT, NARROW, NC>(a, row, true, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max,
+                                                    rank, x_sum[0], x_sum[1], x_max);
+  // No CTA leaves while another may still read its distributed buffers.
+  cooperative_groups::this_cluster().sync();
 }
 
 // Per-chunk gamma (RMSNorm: bf16) or gamma and beta (LayerNorm: float32) of
@@ -1280,6 +1326,16 @@ struct RowTable {
     for (auto& x : k.rows2)
       for (auto& y : x)
         for (auto& z : y) z = nullptr;
+    for (auto& x : k.cluster)
+      for (auto& y : x) y = nullptr;
+    // Rows of 16385 ... 32768 elements: clusters of two CTAs; up to 65536: four.
+#define NQ_CLUSTER(NCI, NC)                                                                                   \
+  k.cluster[NCI][0] = reinterpret_cast<const void*>(&row_kernel_cluster<OP, 2, 0, OUT, NC>);                  \
+  k.cluster[NCI][1] = reinterpret_cast<const void*>(&row_kernel_cluster<OP, 2, 1, OUT, NC>);                  \
+  k.cluster[NCI][2] = reinterpret_cast<const void*>(&row_kernel_cluster<OP, 2, 2, OUT, NC>);                  \
+  k.cluster[NCI][3] = reinterpret_cast<const void*>(&row_kernel_cluster<OP, 2, 3, OUT, NC>);
+    NQ_CLUSTER(0, 2) NQ_CLUSTER(1, 4)
+#undef NQ_CLUSTER
 #define NQ_RAW(LT, LK)                                                                                         \
   if constexpr (OP != kOpRmsDynFp8 && !(OUT & kOutScatter)) {                                                  \
     k.raw[LT - kMinLogT][LK][0][0] = reinterpret_cast<const void*>(&row_kernel_raw<OP, (1 << LT), (1 << LK), false, OUT, false>); \

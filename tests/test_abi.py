@@ -43,7 +43,7 @@ def test_version_and_strings(nq):
 
 def test_flag_values_match_header(nq):
     text = open(HEADER).read()
-    assert "#define NQ_MAX_D 16384" in text and nq.NQ_MAX_D == 16384
+    assert "#define NQ_MAX_D 65536" in text and nq.NQ_MAX_D == 65536
     for name, val in [("NQ_FLAG_PDL", nq.FLAG_PDL), ("NQ_FLAG_SCALE_DIV", nq.FLAG_SCALE_DIV),
                       ("NQ_FLAG_SCALE_RECIP", nq.FLAG_SCALE_RECIP), ("NQ_FLAG_UE8M0", nq.FLAG_UE8M0),
                       ("NQ_FLAG_NORM_BF16_ROUND", nq.FLAG_NORM_BF16_ROUND), ("NQ_FLAG_E5M2", nq.FLAG_E5M2),
@@ -72,7 +72,9 @@ def test_validation_without_gpu(nq):
     assert call_fused(nq, s=None) == INV
     assert call_fused(nq, M=-1) == INV
     assert call_fused(nq, d=0) == INV
-    assert call_fused(nq, d=16385) == UNS
+    assert call_fused(nq, d=65537) == UNS and b"NQ_MAX_D" in nq.lib.nq_last_error()
+    # rows wider than 16384 take a cluster per row: a forced schedule cannot cover them
+    assert call_fused(nq, d=16392, flags=nq.flag_schedule(10, 1)) == INV
     assert call_fused(nq, ld_x=32) == INV
     assert call_fused(nq, eps=float("nan")) == INV
     assert call_fused(nq, eps=-1.0) == INV
@@ -175,6 +177,22 @@ def test_planner_forced_schedules(nq):
     with pytest.raises(nq.NQError):
         nq.nq_query_schedule(0, 100, 64, nq.flag_schedule(10, 2))    # not built (t + k > 11)
     assert nq.nq_query_schedule(0, 100, 8192, nq.flag_schedule(7, 3)) == (128, 8, 1)
+
+
+def test_planner_cluster_rows(nq):
+    """Rows wider than 16384 elements: one cluster of 2 CTAs (up to 32768 elements) or 4 (up to
+    65536) of 1024 threads with 2 chunks each; the cluster covers the next power of two of chunks.
+    A forced schedule cannot cover them."""
+    for op in range(5):
+        for d in (16400, 20480, 32768, 32784, 49152, 65536):
+            T, K, R = nq.nq_query_schedule(op, 4096, d)
+            C = (d + 7) // 8
+            P = 1 << (C - 1).bit_length()
+            assert (T, K, R) == (P // 2, 2, 1) and T in (2048, 4096), (op, d, T, K, R)
+    with pytest.raises(nq.NQError):
+        nq.nq_query_schedule(0, 100, 20000, nq.flag_schedule(10, 1))
+    with pytest.raises(nq.NQError):
+        nq.nq_query_schedule(0, 100, 65537)
 
 
 def test_planner_properties(nq):
