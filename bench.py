@@ -1,27 +1,42 @@
 #!/usr/bin/env python
-"""Benchmark of the fused norm + FP8 quantization hot path on B200.
+"""Benchmark of the fused norm + activation-quantization hot path on B200.
 
-Workload (one "step"): RMSNorm -> e4m3 with a static device scale (0.05) and
-LayerNorm(gamma, beta) -> e4m3 with the same static scale, each over a batch
-of M = 4096 tokens x d = 4096 bf16 activations (eps 1e-5).  The metric is
-achieved HBM bandwidth of the whole step: algorithmic bytes (every input read
-once, every output written once, gamma/beta/scale once per call) divided by
-device time.
+Metric: achieved HBM bandwidth of the fused norm + quantization calls (GB/s,
+and as a fraction of the measured device copy bandwidth), with µs per call and
+tokens/s, for M = 1 ... 65536 tokens.  Bytes are algorithmic: every input read
+once, every output written once, gamma / beta / scales once per call.
 
-Timing: inputs are generated on the device (seeded), and a step uses one of S
-rotating input/output sets whose total (S x 96 MiB) is several times the
-126 MB L2, so no step finds its inputs in L2.  Calls are captured into CUDA
-graphs of S launches (with programmatic dependent launch; ``--no-pdl``
-without) and replayed back to back; CUDA events on the launching
-stream bracket the whole timed region (exactly K steps) and every graph, which
-gives each kernel's mean launch duration for the roofline.  Multi-GPU runs
-(torchrun, one process per GPU) give every rank the same per-GPU workload
+Headline workload (one "step" = one call over one batch): fused residual-add +
+RMSNorm + dynamic per-token e4m3 (division quantization, eps 1e-6) at
+M = 65536 tokens x d = 8192, the largest cell of the sweep configuration: bf16
+x ~ N(0, 1) with four channels scaled x100 (activation outliers), residual
+~ N(0, 1), gamma = 1 + 0.1 N(0, 1); residual_out is written to its own buffer so
+the inputs stay the same from step to step.  One call moves 3.76 GB, far more
+than the 126 MB L2, so no step finds its inputs in L2.  W untimed warm-up
+calls, then exactly K timed calls bracketed by CUDA events on the launching
+stream (with a barrier and a device synchronize on both sides); each call's
+own duration comes from events between calls, for the roofline.  Multi-GPU
+runs (torchrun, one process per GPU) give every rank the same per-GPU workload
 (weak scaling, no data-path collective); the time is the max over ranks.
 
+Every default run also times each configuration's cells ("configs" in the
+JSON line): the sweep (d in {2816, 4096, 7168, 8192} x M in {1, 16, 256, 4096,
+65536}), the small dynamic case (64 x 2816), the static RMSNorm and LayerNorm
+calls (4096 x 4096), per-token-group FP8 (32768 x 4096 and M = 1, fp32 and
+UE8M0 scales) and NVFP4 (d in {7168, 1536 of a [M, 2112] tensor, 512} x M in
+{1, 64, 8192}, with and without residual), plus the fused RMSNorm + group FP8
+and MoE-dispatch calls.  A cell is timed as CUDA graphs of S launches over S
+rotating input / output sets (S x bytes >= 3 x L2 where that fits), launched
+with programmatic dependent launch; each graph is replayed once before its
+timed replays.
+
+``e2e`` is the headline measured through the Python API with the inputs in
+pinned host memory: per step the host -> device copy of x and residual, the
+call, and the device -> host copy of q, the scales and residual_out, pipelined
+over two buffer sets on three streams.
+
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
-instead, on a bounded sample per step.  ``--sweep`` adds a per-configuration
-table (fused add+RMSNorm+dynamic FP8 sweep, group FP8, fused RMSNorm + group
-FP8, NVFP4) under "sweep".
+instead, on a bounded sample of the headline workload per step.
 """
 from __future__ import annotations
 
@@ -40,10 +55,20 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-M_TOK, D_HID, SCALE, EPS = 4096, 4096, 0.05, 1e-5
+METRIC = "fused norm+quant HBM GB/s (% of B200 peak) and µs/call, M=1..65536"
+HEAD_M, HEAD_D, HEAD_EPS = 65536, 8192, 1e-6
+HEAD_WORKLOAD = ("fused residual-add + RMSNorm + dynamic per-token e4m3 (division), "
+                 "M=65536 tokens x d=8192, x with 4 channels x100")
+HEAD_KERNEL = "nq_fused_add_rmsnorm_quant_fp8"
+STATIC_SCALE, STATIC_EPS = 0.05, 1e-5
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
+
+
+# ------------------------------------------------- algorithmic bytes ----
+def fused_dyn_bytes(M, d):
+    return M * (7 * d + 4) + 2 * d         # x, residual read; residual, e4m3, scale write; gamma
 
 
 def rms_static_bytes(M, d):
@@ -52,10 +77,6 @@ def rms_static_bytes(M, d):
 
 def ln_static_bytes(M, d):
     return M * 3 * d + 8 * d + 4           # x read, e4m3 write; fp32 gamma + beta; scale
-
-
-def fused_dyn_bytes(M, d):
-    return M * (7 * d + 4) + 2 * d         # x, residual read; residual, e4m3, scale write; gamma
 
 
 def group_bytes(M, K, g=128):
@@ -102,15 +123,19 @@ def measured_peak():
 
 
 def profiled_traffic(kernel_tag: str):
-    """dram read+write bytes per launch from a committed ncu summary, if it is
-    for the current kernel sources (else None)."""
+    """DRAM bytes read and written per launch of the headline kernel, from a
+    committed ncu summary of the same workload, if that summary was taken on the
+    current kernel sources (else None)."""
     for p in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         text = open(p).read()
-        m_tag = re.search(r"^bench_kernel:\s*(\S+)", text, re.M)
-        m_b = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
-        m_h = re.search(r"^kernel_source_hash:\s*(\S+)", text, re.M)
-        if m_tag and m_b and m_h and m_tag.group(1) == kernel_tag:
-            return int(m_b.group(1)) if m_h.group(1) == kernel_source_hash() else None
+        tag = re.search(r"^bench_kernel:\s*(\S+)", text, re.M)
+        rd = re.search(r"^dram_read_bytes_per_launch:\s*(\d+)", text, re.M)
+        wr = re.search(r"^dram_write_bytes_per_launch:\s*(\d+)", text, re.M)
+        hs = re.search(r"^kernel_source_hash:\s*(\S+)", text, re.M)
+        if tag and rd and wr and hs and tag.group(1) == kernel_tag:
+            if hs.group(1) != kernel_source_hash():
+                return None
+            return {"read": int(rd.group(1)), "write": int(wr.group(1)), "source": os.path.relpath(p, ROOT)}
     return None
 
 
@@ -237,46 +262,34 @@ def job_throughput(world: int, steps: int, step_bytes: int, elapsed_ms: float) -
     return world * steps * step_bytes / (elapsed_ms * 1e-3) / 1e9
 
 
-# ------------------------------------------------------------ GPU arm ----
-class Workload:
-    """S rotating sets of RMSNorm / LayerNorm inputs and outputs on the device."""
+# ------------------------------------------------------- GPU inputs ----
+def outlier_x(M, d, gen, scale=100.0):
+    """bf16 x ~ N(0, 1) with the sweep's four outlier channels scaled (device-seeded)."""
+    import torch
+    import synthetic as S
+    x = torch.randn(M, d, device="cuda", generator=gen)
+    for c in S.outlier_channels(d):
+        x[:, c] *= scale
+    return x.to(torch.bfloat16)
 
-    def __init__(self, nq, M, d, sets, seed=0):
+
+class Headline:
+    """The headline call's device buffers (one set: every call moves more than L2)."""
+
+    def __init__(self, nq, M, d, seed):
         import torch
-        self.nq, self.M, self.d, self.S = nq, M, d, sets
         gen = torch.Generator(device="cuda").manual_seed(seed)
-        bf = torch.bfloat16
-        self.x_rms = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(sets)]
-        self.x_ln = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(sets)]
-        self.q_rms = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(sets)]
-        self.q_ln = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(sets)]
-        self.g_rms = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
-        self.g_ln = 1 + 0.1 * torch.randn(d, device="cuda", generator=gen)
-        self.b_ln = 0.02 * torch.randn(d, device="cuda", generator=gen)
-        self.scale = torch.tensor([SCALE], dtype=torch.float32, device="cuda")
+        self.nq, self.M, self.d = nq, M, d
+        self.x = outlier_x(M, d, gen)
+        self.res = torch.randn(M, d, device="cuda", generator=gen).to(torch.bfloat16)
+        self.gamma = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(torch.bfloat16)
+        self.res_out = torch.empty_like(self.res)
+        self.q = torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda")
+        self.s = torch.empty(M, dtype=torch.float32, device="cuda")
 
-    def rms(self, i, flags=0):
-        self.nq.nq_rmsnorm_quant_fp8_static(self.x_rms[i], self.g_rms, self.scale, EPS, q_out=self.q_rms[i],
-                                            flags=flags)
-
-    def ln(self, i, flags=0):
-        self.nq.nq_layernorm_quant_fp8(self.x_ln[i], self.g_ln, self.b_ln, self.scale, EPS, q_out=self.q_ln[i],
-                                       flags=flags)
-
-    def capture(self, fn, n, flags=0):
-        import torch
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            for i in range(n):
-                fn(i, flags)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(n):
-                fn(i, flags)
-        return g
+    def call(self, flags=0, stream=None):
+        self.nq.nq_fused_add_rmsnorm_quant_fp8(self.x, self.res, self.gamma, HEAD_EPS, residual_out=self.res_out,
+                                               q_out=self.q, scale_out=self.s, flags=flags, stream=stream)
 
 
 def run_gpu_arm(args):
@@ -284,109 +297,50 @@ def run_gpu_arm(args):
     import fp4_activation_quantization_b200 as nq
 
     world, rank, local = dist_setup(args.gpus)
-    M, d = M_TOK, D_HID
-    set_bytes = M * d * 2 * 2 + M * d * 2          # two bf16 inputs + two e4m3 outputs
-    S = max(8, -(-4 * L2_BYTES // set_bytes))      # > 4x L2 in flight between reuses
-    wl = Workload(nq, M, d, S, seed=1234 + rank)
-    # Programmatic dependent launch: each kernel waits (griddepcontrol.wait)
-    # for the previous one before its first read, so no work is skipped; its
-    # CTAs are resident earlier, as when these kernels follow a GEMM.
+    M, d = HEAD_M, HEAD_D
     flags = 0 if args.no_pdl else nq.FLAG_PDL
-    g_rms, g_ln = wl.capture(wl.rms, S, flags), wl.capture(wl.ln, S, flags)
+    hl = Headline(nq, M, d, seed=1234 + rank)
     K, W = args.steps, max(3, args.warmup)
-    q_full, r = divmod(K, S)
-    g_rms_r = wl.capture(wl.rms, r, flags) if r else None
-    g_ln_r = wl.capture(wl.ln, r, flags) if r else None
-
-    def run_steps(n, events=None):
-        full, rem = divmod(n, S)
-        chunks = [(g_rms, g_ln)] * full
-        if rem:
-            chunks.append((wl.capture(wl.rms, rem, flags), wl.capture(wl.ln, rem, flags)) if rem != r
-                          else (g_rms_r, g_ln_r))
-        for ci, (ga, gb) in enumerate(chunks):
-            if events is not None:
-                events[ci][0].record()
-            ga.replay()
-            if events is not None:
-                events[ci][1].record()
-            gb.replay()
-            if events is not None:
-                events[ci][2].record()
-
-    # warm-up: exactly W steps
-    run_steps(W)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
     torch.cuda.synchronize()
 
-    n_chunks = q_full + (1 if r else 0)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_chunks)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # warm-up: exactly W calls, the same launches as the timed region
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            hl.call(flags)
+    torch.cuda.synchronize()
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
     sampler = ClockSampler(gpu_id_for(torch.cuda.current_device()))
     sampler.start()
     time.sleep(0.3)
-
     barrier(world)
     torch.cuda.synchronize()
     t0 = time.time()
-    e0.record()
-    run_steps(K, ev)
-    e1.record()
+    with torch.cuda.stream(stream):
+        ev[0].record()
+        for i in range(K):
+            hl.call(flags)
+            ev[i + 1].record()
     torch.cuda.synchronize()
     t1 = time.time()
     barrier(world)
     time.sleep(0.15)
     sampler.stop()
 
-    elapsed_ms = e0.elapsed_time(e1)
-    rms_ms = sum(c[0].elapsed_time(c[1]) for c in ev)
-    ln_ms = sum(c[1].elapsed_time(c[2]) for c in ev)
-    elapsed_ms = max_over_ranks(world, elapsed_ms)
-
-    step_bytes = rms_static_bytes(M, d) + ln_static_bytes(M, d)
+    per_call_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    elapsed_ms = max_over_ranks(world, ev[0].elapsed_time(ev[K]))
+    step_bytes = fused_dyn_bytes(M, d)
     value = job_throughput(world, K, step_bytes, elapsed_ms)
     peak, peak_src = measured_peak()
-    rms_us, ln_us = rms_ms * 1e3 / K, ln_ms * 1e3 / K
-    dom = ("nq_rmsnorm_quant_fp8_static", rms_us, rms_static_bytes(M, d)) if rms_us >= ln_us else \
-        ("nq_layernorm_quant_fp8", ln_us, ln_static_bytes(M, d))
-    achieved = dom[2] / (dom[1] * 1e-6) / 1e9
+    call_us = sum(per_call_ms) * 1e3 / K
+    achieved = step_bytes / (call_us * 1e-6) / 1e9
     clocks = sampler.summary(t0, t1)
 
-    # ---- end to end through the public API: pinned host buffers, copies in the timed region
-    e2e = None
-    if not args.no_e2e:
-        ke = min(K, args.e2e_steps)
-        xh_r = [wl.x_rms[i % S].cpu().pin_memory() for i in range(2)]
-        xh_l = [wl.x_ln[i % S].cpu().pin_memory() for i in range(2)]
-        qh_r = torch.empty(M, d, dtype=torch.float8_e4m3fn).pin_memory()
-        qh_l = torch.empty(M, d, dtype=torch.float8_e4m3fn).pin_memory()
-        xd_r, xd_l = torch.empty_like(wl.x_rms[0]), torch.empty_like(wl.x_ln[0])
-        qd_r, qd_l = wl.q_rms[0], wl.q_ln[0]
+    e2e = None if args.no_e2e else run_e2e(nq, hl, world, min(K, args.e2e_steps), flags)
 
-        def e2e_step(i):
-            xd_r.copy_(xh_r[i % 2], non_blocking=True)
-            xd_l.copy_(xh_l[i % 2], non_blocking=True)
-            nq.nq_rmsnorm_quant_fp8_static(xd_r, wl.g_rms, wl.scale, EPS, q_out=qd_r)
-            nq.nq_layernorm_quant_fp8(xd_l, wl.g_ln, wl.b_ln, wl.scale, EPS, q_out=qd_l)
-            qh_r.copy_(qd_r, non_blocking=True)
-            qh_l.copy_(qd_l, non_blocking=True)
-
-        for i in range(3):
-            e2e_step(i)
-        torch.cuda.synchronize()
-        barrier(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for i in range(ke):
-            e2e_step(i)
-        b.record()
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(world, a.elapsed_time(b))
-        barrier(world)
-        e2e = {"value": round(job_throughput(world, ke, step_bytes, e2e_ms), 3), "unit": "GB/s",
-               "h2d_bytes_per_step": 2 * M * d * 2, "d2h_bytes_per_step": 2 * M * d, "steps": ke,
-               "ms_per_step": round(e2e_ms / ke, 4)}
-
-    sweep = run_sweep(nq) if args.sweep and rank == 0 else None
+    configs = run_configs(nq, flags) if rank == 0 and not args.no_configs else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -394,45 +348,111 @@ def run_gpu_arm(args):
 
     if world > 1:
         import torch.distributed as dist
-        del g_rms, g_ln, g_rms_r, g_ln_r
         dist.destroy_process_group()
 
     if rank != 0:
         return
+    traffic = profiled_traffic(HEAD_KERNEL)
     out = {
-        "metric": "fused norm+quant HBM GB/s (% of B200 peak) and µs/call, M=1..65536",
+        "metric": METRIC,
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(elapsed_ms / K, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic (device-seeded: x bf16 N(0,1); RMS gamma bf16 1+0.1N; LN gamma f32 1+0.1N, beta f32 0.02N)",
-        "config": {"workload": "RMSNorm->e4m3 static + LayerNorm->e4m3 static, M=4096 tokens, d=4096",
-                   "M": M, "d": d, "scale": SCALE, "eps": EPS, "io": "bf16 in, e4m3 out, fp32 math",
-                   "l2": f"inputs rotate over {S} sets ({S * set_bytes / 2**20:.0f} MiB, > L2 126 MB)",
-                   "graphs": f"CUDA graphs of {S} launches replayed back to back", "pdl": not args.no_pdl,
+        "data": "synthetic (device-seeded: x bf16 N(0,1) with 4 channels x100; residual bf16 N(0,1); "
+                "gamma bf16 1+0.1N)",
+        "config": {"workload": HEAD_WORKLOAD, "M": M, "d": d, "eps": HEAD_EPS,
+                   "io": "bf16 x, residual, gamma in; bf16 residual_out, e4m3 codes, fp32 scales out; fp32 math",
+                   "l2": f"inputs larger than L2 ({2 * M * d * 2 / 2**30:.1f} GiB read per call, L2 126 MB)",
+                   "launch": "one launch per step, CUDA events between launches",
+                   "pdl": not args.no_pdl,
                    "parallelism": f"replicas x{world} (rows shard, no collective)"},
-        "per_call": {"nq_rmsnorm_quant_fp8_static": {"us": round(rms_us, 3),
-                                                     "GBps": round(rms_static_bytes(M, d) / rms_us / 1e3, 1)},
-                     "nq_layernorm_quant_fp8": {"us": round(ln_us, 3),
-                                                "GBps": round(ln_static_bytes(M, d) / ln_us / 1e3, 1)},
-                     "tokens_per_s_per_gpu": round(M * 2 / ((rms_us + ln_us) * 1e-6), 1)},
-        "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
+        "per_call": {HEAD_KERNEL: {"us": round(call_us, 3), "GBps": round(achieved, 1),
+                                   "tokens_per_s": round(M / (call_us * 1e-6), 1)}},
+        "roofline": {"bound": "hbm", "kernel": HEAD_KERNEL, "achieved": round(achieved, 1), "peak": peak,
                      "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "frac_of_nominal_8000": round(achieved / NOMINAL_HBM_GBS, 4),
-                     "algorithmic_bytes_per_launch": dom[2],
-                     "traffic": profiled_traffic(dom[0])},
+                     "algorithmic_bytes_per_launch": step_bytes,
+                     "traffic": None if traffic is None else traffic["read"] + traffic["write"],
+                     "traffic_read": None if traffic is None else traffic["read"],
+                     "traffic_write": None if traffic is None else traffic["write"],
+                     "traffic_source": None if traffic is None else traffic["source"]},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clocks,
         "kernel_source_hash": kernel_source_hash(),
     }
-    if sweep is not None:
-        out["sweep"] = sweep
+    if configs is not None:
+        out["configs"] = configs
     print(json.dumps(out), flush=True)
 
 
-# ------------------------------------------------------ sweep table ----
-def _time_graph(fn, n_sets, reps=20):
+def run_e2e(nq, hl, world, steps, flags):
+    """The headline through the public API with host buffers: H2D of x and the
+    residual, the call, D2H of q, the scales and residual_out, pipelined over two
+    device buffer sets (copy-in, compute and copy-out streams)."""
+    import torch
+    M, d = hl.M, hl.d
+    xh = hl.x.cpu().pin_memory()
+    rh = hl.res.cpu().pin_memory()
+    qh = torch.empty(M, d, dtype=torch.float8_e4m3fn).pin_memory()
+    sh = torch.empty(M, dtype=torch.float32).pin_memory()
+    roh = torch.empty(M, d, dtype=torch.bfloat16).pin_memory()
+    sets = [dict(x=torch.empty_like(hl.x), r=torch.empty_like(hl.res), q=torch.empty_like(hl.q),
+                 s=torch.empty_like(hl.s), ro=torch.empty_like(hl.res_out)) for _ in range(2)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def step(i):
+        b = i & 1
+        B = sets[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[b])      # the call of step i - 2 has read this set's inputs
+            B["x"].copy_(xh, non_blocking=True)
+            B["r"].copy_(rh, non_blocking=True)
+            ev_in[b].record()
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            if i >= 2:
+                s_comp.wait_event(ev_out[b])     # step i - 2's outputs have left this set
+            nq.nq_fused_add_rmsnorm_quant_fp8(B["x"], B["r"], hl.gamma, HEAD_EPS, residual_out=B["ro"],
+                                              q_out=B["q"], scale_out=B["s"], flags=flags)
+            ev_comp[b].record()
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            qh.copy_(B["q"], non_blocking=True)
+            sh.copy_(B["s"], non_blocking=True)
+            roh.copy_(B["ro"], non_blocking=True)
+            ev_out[b].record()
+
+    for i in range(2):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s_in):
+        a.record()
+    for i in range(steps):
+        step(i)
+    with torch.cuda.stream(s_out):
+        b_.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, a.elapsed_time(b_))
+    barrier(world)
+    return {"value": round(job_throughput(world, steps, fused_dyn_bytes(M, d), e2e_ms), 3), "unit": "GB/s",
+            "h2d_bytes_per_step": 2 * M * d * 2, "d2h_bytes_per_step": M * d + 4 * M + 2 * M * d,
+            "steps": steps, "ms_per_step": round(e2e_ms / steps, 4),
+            "how": "pinned host buffers; H2D of x and residual, the call, D2H of codes, scales and residual_out "
+                   "each step, pipelined over two device buffer sets on three streams"}
+
+
+# ------------------------------------------------------ config cells ----
+def time_calls(fn, n_sets, reps):
+    """µs per call of fn(i) (i = set index), captured as one CUDA graph of n_sets
+    launches; the graph is replayed once untimed, then reps times under events."""
     import torch
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -453,66 +473,140 @@ def _time_graph(fn, n_sets, reps=20):
         g.replay()
     b.record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) * 1e3 / (reps * n_sets)  # us per call
+    us = a.elapsed_time(b) * 1e3 / (reps * n_sets)
+    del g
+    return us
 
 
-def run_sweep(nq):
-    """Per-configuration µs/call and GB/s (rotating sets > L2 where they fit, graphs)."""
+def sets_for(nbytes):
+    """Rotating sets so that a set is reused only after >= 3 x L2 of other traffic (2 .. 16)."""
+    return int(max(2, min(16, -(-3 * L2_BYTES // max(1, nbytes)))))
+
+
+def reps_for(nbytes, n_sets):
+    return max(3, min(200, int(4e8 // max(nbytes * n_sets, 1))))
+
+
+def cell(peak, tokens, nbytes, us, **kw):
+    gbs = nbytes / us / 1e3
+    return dict(kw, us=round(us, 3), GBps=round(gbs, 1), frac=round(gbs / peak, 4),
+                tokens_per_s=round(tokens / (us * 1e-6), 1), bytes=nbytes)
+
+
+def run_configs(nq, flags):
+    """µs per call, GB/s, fraction of the measured copy bandwidth and tokens/s of
+    every configuration's cells."""
     import torch
+    import synthetic as S
     gen = torch.Generator(device="cuda").manual_seed(7)
     bf = torch.bfloat16
-    rows = []
     peak, _ = measured_peak()
+    out = {}
 
-    def sets_for(nbytes):
-        return int(max(2, min(16, -(-3 * L2_BYTES // max(1, nbytes)))))
-
-    for d in (2816, 4096, 7168, 8192):
+    def dyn_cell(M, d, outliers):
+        nb = fused_dyn_bytes(M, d)
+        n = sets_for(nb)
+        xs = [outlier_x(M, d, gen, 100.0 if outliers else 1.0) for _ in range(n)]
+        rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)]
+        ro = [torch.empty(M, d, dtype=bf, device="cuda") for _ in range(n)]
+        qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
+        ss = [torch.empty(M, dtype=torch.float32, device="cuda") for _ in range(n)]
         g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
-        for M in (1, 16, 256, 4096, 65536):
-            nb = fused_dyn_bytes(M, d)
-            S = sets_for(nb)
-            xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)]
-            rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)]
-            qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S)]
-            ss = [torch.empty(M, dtype=torch.float32, device="cuda") for _ in range(S)]
-            us = _time_graph(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8(
-                xs[i], rs[i], g, 1e-6, residual_out=rs[i], q_out=qs[i], scale_out=ss[i]), S,
-                reps=max(3, min(200, int(2e8 // max(nb * S, 1)))))
-            rows.append({"op": "fused_add_rmsnorm_quant_fp8", "M": M, "d": d, "us": round(us, 3),
-                         "GBps": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4)})
-            del xs, rs, qs, ss
-    for M in (1, 32768):
-        for flags, tag in ((0, "fp32"), (nq.FLAG_UE8M0, "ue8m0")):
-            K = 4096
+        us = time_calls(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8(
+            xs[i], rs[i], g, 1e-6, residual_out=ro[i], q_out=qs[i], scale_out=ss[i], flags=flags), n,
+            reps_for(nb, n))
+        return cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8", M=M, d=d, sets=n)
+
+    out["1_fused_dynamic_small"] = [dyn_cell(64, 2816, False)]
+    out["5_fused_dynamic_sweep"] = [dyn_cell(M, d, True) for d in (2816, 4096, 7168, 8192)
+                                    for M in (1, 16, 256, 4096, 65536)]
+
+    # config 2: static RMSNorm and LayerNorm, 4096 x 4096, scale 0.05 in device memory, eps 1e-5
+    M, d = 4096, 4096
+    n = 8
+    sc = torch.tensor([STATIC_SCALE], dtype=torch.float32, device="cuda")
+    xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)]
+    qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
+    g_rms = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
+    g_ln = 1 + 0.1 * torch.randn(d, device="cuda", generator=gen)
+    b_ln = 0.02 * torch.randn(d, device="cuda", generator=gen)
+    reps = 100
+    us_rms = time_calls(lambda i: nq.nq_rmsnorm_quant_fp8_static(xs[i], g_rms, sc, STATIC_EPS, q_out=qs[i],
+                                                                 flags=flags), n, reps)
+    us_ln = time_calls(lambda i: nq.nq_layernorm_quant_fp8(xs[i], g_ln, b_ln, sc, STATIC_EPS, q_out=qs[i],
+                                                           flags=flags), n, reps)
+    out["2_static"] = [cell(peak, M, rms_static_bytes(M, d), us_rms, call="nq_rmsnorm_quant_fp8_static", M=M, d=d,
+                            sets=n),
+                       cell(peak, M, ln_static_bytes(M, d), us_ln, call="nq_layernorm_quant_fp8", M=M, d=d, sets=n)]
+    # the same bytes moved by a device copy (reads 2 bytes and writes 1 per element, as a copy of
+    # 2/3 of the bytes each way): the ceiling at this size for a kernel that only moves data
+    nel = M * d * 3 // 4
+    src = [torch.empty(nel, dtype=bf, device="cuda") for _ in range(n)]
+    dst = [torch.empty(nel, dtype=bf, device="cuda") for _ in range(n)]
+    us_cp = time_calls(lambda i: dst[i].copy_(src[i]), n, reps)
+    out["2_static"].append(cell(peak, M, 4 * nel, us_cp, call="device copy of the same bytes (context)",
+                                elements=nel, sets=n))
+    del xs, qs, src, dst
+
+    rows = []
+    for M in (32768, 1):
+        K = 4096
+        for fl, tag in ((0, "fp32"), (nq.FLAG_UE8M0, "ue8m0")):
             nb = group_bytes(M, K)
-            S = sets_for(nb)
-            xs = [torch.randn(M, K, device="cuda", generator=gen).to(bf) for _ in range(S)]
-            qs = [torch.empty(M, K, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S)]
-            sc = [torch.empty(M, K // 128, dtype=torch.float32, device="cuda") for _ in range(S)]
-            us = _time_graph(lambda i: nq.nq_per_token_group_quant_fp8(xs[i], 128, q_out=qs[i], scales_out=sc[i],
-                                                                       flags=flags), S)
-            rows.append({"op": f"per_token_group_quant_fp8[{tag}]", "M": M, "K": K, "us": round(us, 3),
-                         "GBps": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4)})
-            del xs, qs, sc
+            n = sets_for(nb)
+            xs = [torch.randn(M, K, device="cuda", generator=gen).to(bf) for _ in range(n)]
+            for x in xs:  # 0.1 % of elements x50
+                x.mul_(torch.where(torch.rand(M, K, device="cuda", generator=gen) < 1e-3, 50.0, 1.0).to(bf))
+            qs = [torch.empty(M, K, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
+            sc_ = [torch.empty(M, K // 128, dtype=torch.float32, device="cuda") for _ in range(n)]
+            us = time_calls(lambda i: nq.nq_per_token_group_quant_fp8(xs[i], 128, q_out=qs[i], scales_out=sc_[i],
+                                                                      flags=fl | flags), n, reps_for(nb, n))
+            rows.append(cell(peak, M, nb, us, call="nq_per_token_group_quant_fp8", scales=tag, M=M, K=K, sets=n))
+            del xs, qs, sc_
+    out["3_group"] = rows
+
+    rows = []
+    gs = torch.tensor([0.004], dtype=torch.float32, device="cuda")
+    for d, ld in ((7168, 7168), (1536, 2112), (512, 512)):
+        g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
+        for M in (1, 64, 8192):
+            for residual in (False, True):
+                nb = nvfp4_bytes(M, d, residual)
+                n = sets_for(nb)
+                xs = [torch.randn(M, ld, device="cuda", generator=gen).to(bf)[:, :d] for _ in range(n)]
+                rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)] if residual else None
+                qs = [torch.empty(M, d // 2, dtype=torch.uint8, device="cuda") for _ in range(n)]
+                sf = [torch.empty(M, d // 16, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
+                us = time_calls(lambda i: nq.nq_rmsnorm_quant_nvfp4(
+                    xs[i], g, gs, 1e-6, residual=rs[i] if residual else None,
+                    residual_out=rs[i] if residual else None, q_out=qs[i], sf_out=sf[i], flags=flags), n,
+                    reps_for(nb, n))
+                rows.append(cell(peak, M, nb, us, call="nq_rmsnorm_quant_nvfp4", residual=residual, M=M, d=d,
+                                 ld_x=ld, sets=n))
+                del xs, rs, qs, sf
+    out["4_nvfp4"] = rows
+
+    rows = []
     for d in (4096, 7168):
         g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
         for M in (1, 256, 8192, 32768):
             for residual in (False, True):
                 nb = rms_group_bytes(M, d, residual)
-                S = sets_for(nb)
-                xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)]
-                rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)] if residual else None
-                qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S)]
-                sc = [torch.empty(M, d // 128, dtype=torch.float32, device="cuda") for _ in range(S)]
-                us = _time_graph(lambda i: nq.nq_rmsnorm_quant_fp8_group(
+                n = sets_for(nb)
+                xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)]
+                rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)] if residual else None
+                qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
+                sc_ = [torch.empty(M, d // 128, dtype=torch.float32, device="cuda") for _ in range(n)]
+                us = time_calls(lambda i: nq.nq_rmsnorm_quant_fp8_group(
                     xs[i], g, 1e-6, residual=rs[i] if residual else None,
-                    residual_out=rs[i] if residual else None, q_out=qs[i], scales_out=sc[i]), S)
-                rows.append({"op": "rmsnorm_quant_fp8_group" + ("+res" if residual else ""), "M": M, "d": d,
-                             "us": round(us, 3), "GBps": round(nb / us / 1e3, 1),
-                             "frac": round(nb / us / 1e3 / peak, 4)})
-                del xs, rs, qs, sc
-    import synthetic as S
+                    residual_out=rs[i] if residual else None, q_out=qs[i], scales_out=sc_[i], flags=flags), n,
+                    reps_for(nb, n))
+                rows.append(cell(peak, M, nb, us, call="nq_rmsnorm_quant_fp8_group", residual=residual, M=M, d=d,
+                                 sets=n))
+                del xs, rs, qs, sc_
+    out["next_fused_group"] = rows
+
+    rows = []
     d, E, topk = 7168, 256, 8
     g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
     for M in (256, 4096, 32768):
@@ -521,61 +615,49 @@ def run_sweep(nq):
         n_rows = route["rows"]
         for group in (0, 128):
             nb = moe_bytes(M, d, topk, group)
-            S_ = sets_for(nb)
-            xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S_)]
-            rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S_)]
-            qs = [torch.empty(n_rows, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S_)]
-            sc = [torch.empty((n_rows, d // 128) if group else (n_rows,), dtype=torch.float32, device="cuda")
-                  for _ in range(S_)]
-            us = _time_graph(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8_moe(
+            n = sets_for(nb)
+            xs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)]
+            rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)]
+            qs = [torch.empty(n_rows, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
+            sc_ = [torch.empty((n_rows, d // 128) if group else (n_rows,), dtype=torch.float32, device="cuda")
+                   for _ in range(n)]
+            us = time_calls(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8_moe(
                 xs[i], g, dest, n_rows, 1e-6, group=group, residual=rs[i], residual_out=rs[i], q_out=qs[i],
-                scales_out=sc[i]), S_)
-            rows.append({"op": "fused_add_rmsnorm_quant_fp8_moe" + ("[group128]" if group else "[per-token]"),
-                         "M": M, "d": d, "experts": E, "topk": topk, "us": round(us, 3),
-                         "GBps": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4)})
-            del xs, rs, qs, sc
-    gs = torch.tensor([0.004], dtype=torch.float32, device="cuda")
-    for d, ld in ((7168, 7168), (1536, 2112), (512, 512)):
-        g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
-        for M in (1, 64, 8192):
-            for residual in (False, True):
-                nb = nvfp4_bytes(M, d, residual)
-                S = sets_for(nb)
-                xs = [torch.randn(M, ld, device="cuda", generator=gen).to(bf)[:, :d] for _ in range(S)]
-                rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(S)] if residual else None
-                qs = [torch.empty(M, d // 2, dtype=torch.uint8, device="cuda") for _ in range(S)]
-                sf = [torch.empty(M, d // 16, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(S)]
-                us = _time_graph(lambda i: nq.nq_rmsnorm_quant_nvfp4(
-                    xs[i], g, gs, 1e-6, residual=rs[i] if residual else None,
-                    residual_out=rs[i] if residual else None, q_out=qs[i], sf_out=sf[i]), S)
-                rows.append({"op": "rmsnorm_quant_nvfp4" + ("+res" if residual else ""), "M": M, "d": d,
-                             "ld_x": ld, "us": round(us, 3), "GBps": round(nb / us / 1e3, 1),
-                             "frac": round(nb / us / 1e3 / peak, 4)})
-                del xs, rs, qs, sf
+                scales_out=sc_[i], flags=flags), n, reps_for(nb, n))
+            rows.append(cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8_moe", group=group, M=M, d=d,
+                             experts=E, topk=topk, sets=n))
+            del xs, rs, qs, sc_
+    out["next_moe_dispatch"] = rows
+    torch.cuda.synchronize()
     torch.cuda.empty_cache()
-    return rows
+    return out
 
 
 # ----------------------------------------------------- CPU baseline ----
-def cpu_baseline(seconds: float = 15.0):
-    """The oracle as it stands (single-threaded C++), on the host cores, on the
-    same workload (full M x d calls, repeated until ~`seconds` have passed)."""
-    import oracle
+def _oracle_sample(rows: int, seed: int = 0):
+    """A bounded sample of the headline workload for the oracle: `rows` tokens of
+    the same width and input distribution, from the seeded host generator."""
     import synthetic as S
-    w = S.make_rms_inputs(M_TOK, D_HID, seed=0, residual=False)
-    lw = S.make_ln_inputs(M_TOK, D_HID, seed=0)
+    return S.make_rms_inputs(rows, HEAD_D, seed=seed, x_outlier_channels=True)
+
+
+def cpu_baseline(seconds: float = 15.0, rows: int = 256):
+    """The oracle as it stands (single-threaded C++) on the host cores, on
+    samples of the headline workload, repeated until ~`seconds` have passed."""
+    import oracle
+    w = _oracle_sample(rows)
     oracle.build()
-    steps, t0 = 0, time.perf_counter()
+    calls, t0 = 0, time.perf_counter()
     while True:
-        oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], SCALE, eps=EPS)
-        oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], SCALE, eps=EPS)
-        steps += 1
+        oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"], eps=HEAD_EPS)
+        calls += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    step_bytes = rms_static_bytes(M_TOK, D_HID) + ln_static_bytes(M_TOK, D_HID)
-    return {"value": round(steps * step_bytes / el / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps} full steps (RMSNorm + LayerNorm static e4m3, 4096x4096) in {el:.1f} s",
+    nb = fused_dyn_bytes(rows, HEAD_D)
+    return {"value": round(calls * nb / el / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{calls} calls of {rows} of the 65536 tokens (d = 8192, same input distribution) "
+                      f"in {el:.1f} s",
             "cpu": _cpu_model(), "host_cores": os.cpu_count()}
 
 
@@ -590,35 +672,31 @@ def _cpu_model():
 
 
 def run_reference_arm(args):
-    """The oracle timed on host cores on a bounded sample per step (rank 0 only)."""
+    """The oracle timed on host cores, each step a bounded sample of the headline
+    workload (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
-    import synthetic as S
     rows = args.ref_rows
-    w = S.make_rms_inputs(rows, D_HID, seed=0, residual=False)
-    lw = S.make_ln_inputs(rows, D_HID, seed=0)
+    w = _oracle_sample(rows)
     oracle.build()
     K, W = args.steps, max(3, args.warmup)
     for _ in range(W):
-        oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], SCALE, eps=EPS)
-        oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], SCALE, eps=EPS)
+        oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"], eps=HEAD_EPS)
     t0 = time.perf_counter()
     for _ in range(K):
-        oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], SCALE, eps=EPS)
-        oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], SCALE, eps=EPS)
+        oracle.fused_add_rmsnorm_quant_fp8(w["x"], w["residual"], w["gamma"], eps=HEAD_EPS)
     el = time.perf_counter() - t0
-    step_bytes = rms_static_bytes(rows, D_HID) + ln_static_bytes(rows, D_HID)
-    value = K * step_bytes / el / 1e9
-    sample = f"{rows} of 4096 tokens per step (RMSNorm + LayerNorm static e4m3, d=4096)"
+    nb = fused_dyn_bytes(rows, HEAD_D)
+    value = K * nb / el / 1e9
+    sample = f"{rows} of the 65536 tokens per step (d = 8192, same input distribution)"
     print(json.dumps({
-        "impl": "reference", "metric": "fused norm+quant HBM GB/s (% of B200 peak) and µs/call, M=1..65536",
+        "impl": "reference", "metric": METRIC,
         "value": round(value, 4), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": K,
         "warmup": W, "ms_per_step": round(el * 1e3 / K, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded host generator)",
-        "config": {"workload": "RMSNorm->e4m3 static + LayerNorm->e4m3 static, M=4096 tokens, d=4096",
-                   "M": M_TOK, "d": D_HID, "scale": SCALE, "eps": EPS, "sample_rows": rows},
+        "config": {"workload": HEAD_WORKLOAD, "M": HEAD_M, "d": HEAD_D, "eps": HEAD_EPS, "sample_rows": rows},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
                          "cpu": _cpu_model()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -627,32 +705,34 @@ def run_reference_arm(args):
 
 def run_case(args):
     """Run one call a few times on a device-seeded input (for ncu captures of a
-    single kernel on a small case); prints nothing but 'ok'."""
+    single kernel); prints nothing but 'ok'."""
     import torch
     import fp4_activation_quantization_b200 as nq
     M, d, op = args.M, args.d, args.case
     bf = torch.bfloat16
     g = torch.Generator(device="cuda").manual_seed(0)
-    x = torch.randn(M, d, device="cuda", generator=g).to(bf)
+    x = outlier_x(M, d, g) if op == "fused_add_rmsnorm_quant_fp8" else \
+        torch.randn(M, d, device="cuda", generator=g).to(bf)
     res = (torch.randn(M, d, device="cuda", generator=g).to(bf)
            if op in ("fused_add_rmsnorm_quant_fp8", "nvfp4_res", "rmsnorm_quant_fp8_group_res") else None)
     gam = (1 + 0.1 * torch.randn(d, device="cuda", generator=g)).to(bf)
     gl = 1 + 0.1 * torch.randn(d, device="cuda", generator=g)
     bl = 0.02 * torch.randn(d, device="cuda", generator=g)
-    sc = torch.tensor([SCALE], device="cuda")
+    sc = torch.tensor([STATIC_SCALE], device="cuda")
+    ro = torch.empty_like(res) if res is not None else None
     for _ in range(args.iters):
         if op == "rmsnorm_quant_fp8_static":
-            nq.nq_rmsnorm_quant_fp8_static(x, gam, sc, EPS)
+            nq.nq_rmsnorm_quant_fp8_static(x, gam, sc, STATIC_EPS)
         elif op == "layernorm_quant_fp8":
-            nq.nq_layernorm_quant_fp8(x, gl, bl, sc, EPS)
+            nq.nq_layernorm_quant_fp8(x, gl, bl, sc, STATIC_EPS)
         elif op == "fused_add_rmsnorm_quant_fp8":
-            nq.nq_fused_add_rmsnorm_quant_fp8(x, res, gam, 1e-6, residual_out=res)
+            nq.nq_fused_add_rmsnorm_quant_fp8(x, res, gam, HEAD_EPS, residual_out=ro)
         elif op in ("nvfp4", "nvfp4_res"):
-            nq.nq_rmsnorm_quant_nvfp4(x, gam, sc, 1e-6, residual=res, residual_out=res)
+            nq.nq_rmsnorm_quant_nvfp4(x, gam, sc, 1e-6, residual=res, residual_out=ro)
         elif op == "per_token_group_quant_fp8":
             nq.nq_per_token_group_quant_fp8(x, 128)
         elif op in ("rmsnorm_quant_fp8_group", "rmsnorm_quant_fp8_group_res"):
-            nq.nq_rmsnorm_quant_fp8_group(x, gam, 1e-6, residual=res, residual_out=res)
+            nq.nq_rmsnorm_quant_fp8_group(x, gam, 1e-6, residual=res, residual_out=ro)
     torch.cuda.synchronize()
     print("ok")
 
@@ -660,14 +740,14 @@ def run_case(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["nq", "reference"], default="nq")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (default: with)")
-    ap.add_argument("--sweep", action="store_true", help="add the per-configuration table")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration cells")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=64)
