@@ -173,3 +173,29 @@ def test_wide_plain_order_tolerance(nq):
     assert np.all(np.abs(s.cpu().numpy().astype(np.float64) / es - 1) <= 1e-6)
     diff = np.abs(e4m3_rank(host_u8(q)) - e4m3_rank(eq))
     assert diff.max() <= 1 and (diff > 0).mean() <= 1e-3
+
+
+def test_wide_rows_in_a_cuda_graph(nq):
+    """Cluster launches captured in a CUDA graph (with programmatic dependent launch) and
+    replayed: the static scale is read at execution time, so updating it between replays
+    changes the codes, and each replay matches the oracle for the scale it saw."""
+    M, d = 7, 30000
+    w = S.make_rms_inputs(M, d, seed=31, residual=False)
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    q = torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, q_out=q, flags=nq.FLAG_PDL)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, q_out=q, flags=nq.FLAG_PDL)
+    for scale in (0.05, 0.2, 0.01):
+        sc.fill_(scale)
+        graph.replay()
+        torch.cuda.synchronize()
+        eq, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], scale)
+        assert np.array_equal(host_u8(q), eq), scale
