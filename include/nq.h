@@ -132,7 +132,9 @@ typedef enum nq_status {
 #define NQ_FLAG_SCALES_PACKED_UE8M0 (1u << 8)
 /* Force a schedule: 2^t threads per row (t = 5..10) and 2^k 16-byte chunks per
  * thread (k = 0..3, t + k <= 11), with 2^(t+k) * 8 >= d.  Every schedule gives
- * bitwise identical results; this exists for tests and tuning.  0 = automatic. */
+ * bitwise identical results; this exists for tests and tuning.  0 = automatic.
+ * Rows wider than 16384 elements always take a cluster of CTAs; a forced
+ * schedule is rejected there (NQ_ERR_INVALID_ARGUMENT). */
 #define NQ_FLAG_SCHEDULE(t, k) ((((uint32_t)(t) - 4u) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 #define NQ_FLAG_SCHEDULE_MASK (0x7Fu << 16)
 /* Group quantization's schedule (same bit field): 2^t lanes per group, 2^k
