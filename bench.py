@@ -28,7 +28,8 @@ UE8M0 scales) and NVFP4 (d in {7168, 1536 of a [M, 2112] tensor, 512} x M in
 and MoE-dispatch calls.  A cell is timed as CUDA graphs of S launches over S
 rotating input / output sets (S x bytes >= 3 x L2 where that fits), launched
 with programmatic dependent launch; each graph is replayed once before its
-timed replays.
+timed replays.  Cells of M <= 64 also give the median host-to-completion
+latency of one call through the Python API (``host_latency_us``).
 
 ``e2e`` is the headline measured through the Python API with the inputs in
 pinned host memory: per step the host -> device copy of x and residual, the
@@ -487,6 +488,21 @@ def reps_for(nbytes, n_sets):
     return max(3, min(200, int(4e8 // max(nbytes * n_sets, 1))))
 
 
+def host_latency_us(fn, reps=50):
+    """Median wall time of one call from the host to its completion (the Python API's
+    call, the launch and a device synchronize): the latency a decode step sees."""
+    import torch
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        fn(0)
+        torch.cuda.synchronize()
+        ts.append(time.perf_counter() - t0)
+    ts.sort()
+    return round(ts[len(ts) // 2] * 1e6, 2)
+
+
 def cell(peak, tokens, nbytes, us, **kw):
     gbs = nbytes / us / 1e3
     return dict(kw, us=round(us, 3), GBps=round(gbs, 1), frac=round(gbs / peak, 4),
@@ -512,10 +528,11 @@ def run_configs(nq, flags):
         qs = [torch.empty(M, d, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
         ss = [torch.empty(M, dtype=torch.float32, device="cuda") for _ in range(n)]
         g = (1 + 0.1 * torch.randn(d, device="cuda", generator=gen)).to(bf)
-        us = time_calls(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8(
-            xs[i], rs[i], g, 1e-6, residual_out=ro[i], q_out=qs[i], scale_out=ss[i], flags=flags), n,
-            reps_for(nb, n))
-        return cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8", M=M, d=d, sets=n)
+        fn = lambda i: nq.nq_fused_add_rmsnorm_quant_fp8(xs[i], rs[i], g, 1e-6, residual_out=ro[i], q_out=qs[i],
+                                                         scale_out=ss[i], flags=flags)
+        us = time_calls(fn, n, reps_for(nb, n))
+        extra = {"host_latency_us": host_latency_us(fn)} if M <= 64 else {}
+        return cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8", M=M, d=d, sets=n, **extra)
 
     out["1_fused_dynamic_small"] = [dyn_cell(64, 2816, False)]
     out["5_fused_dynamic_sweep"] = [dyn_cell(M, d, True) for d in (2816, 4096, 7168, 8192)
@@ -559,9 +576,12 @@ def run_configs(nq, flags):
                 x.mul_(torch.where(torch.rand(M, K, device="cuda", generator=gen) < 1e-3, 50.0, 1.0).to(bf))
             qs = [torch.empty(M, K, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
             sc_ = [torch.empty(M, K // 128, dtype=torch.float32, device="cuda") for _ in range(n)]
-            us = time_calls(lambda i: nq.nq_per_token_group_quant_fp8(xs[i], 128, q_out=qs[i], scales_out=sc_[i],
-                                                                      flags=fl | flags), n, reps_for(nb, n))
-            rows.append(cell(peak, M, nb, us, call="nq_per_token_group_quant_fp8", scales=tag, M=M, K=K, sets=n))
+            fn = lambda i: nq.nq_per_token_group_quant_fp8(xs[i], 128, q_out=qs[i], scales_out=sc_[i],
+                                                           flags=fl | flags)
+            us = time_calls(fn, n, reps_for(nb, n))
+            extra = {"host_latency_us": host_latency_us(fn)} if M <= 64 else {}
+            rows.append(cell(peak, M, nb, us, call="nq_per_token_group_quant_fp8", scales=tag, M=M, K=K, sets=n,
+                             **extra))
             del xs, qs, sc_
     out["3_group"] = rows
 
@@ -577,12 +597,13 @@ def run_configs(nq, flags):
                 rs = [torch.randn(M, d, device="cuda", generator=gen).to(bf) for _ in range(n)] if residual else None
                 qs = [torch.empty(M, d // 2, dtype=torch.uint8, device="cuda") for _ in range(n)]
                 sf = [torch.empty(M, d // 16, dtype=torch.float8_e4m3fn, device="cuda") for _ in range(n)]
-                us = time_calls(lambda i: nq.nq_rmsnorm_quant_nvfp4(
+                fn = lambda i: nq.nq_rmsnorm_quant_nvfp4(
                     xs[i], g, gs, 1e-6, residual=rs[i] if residual else None,
-                    residual_out=rs[i] if residual else None, q_out=qs[i], sf_out=sf[i], flags=flags), n,
-                    reps_for(nb, n))
+                    residual_out=rs[i] if residual else None, q_out=qs[i], sf_out=sf[i], flags=flags)
+                us = time_calls(fn, n, reps_for(nb, n))
+                extra = {"host_latency_us": host_latency_us(fn)} if M <= 64 else {}
                 rows.append(cell(peak, M, nb, us, call="nq_rmsnorm_quant_nvfp4", residual=residual, M=M, d=d,
-                                 ld_x=ld, sets=n))
+                                 ld_x=ld, sets=n, **extra))
                 del xs, rs, qs, sf
     out["4_nvfp4"] = rows
 
