@@ -349,6 +349,7 @@ def run_gpu_arm(args):
 
     if world > 1:
         import torch.distributed as dist
+        barrier(world)  # every rank waits for rank 0's configuration cells before leaving the group
         dist.destroy_process_group()
 
     if rank != 0:

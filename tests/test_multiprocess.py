@@ -54,3 +54,5 @@ def test_bytes_models():
     assert bench.group_bytes(32768, 4096) == 406_847_488
     assert bench.nvfp4_bytes(8192, 7168, False) == 150_484_996
     assert bench.nvfp4_bytes(8192, 7168, True) == 385_366_020
+    # the headline: fused add + RMSNorm + dynamic e4m3 at 65536 x 8192
+    assert bench.fused_dyn_bytes(bench.HEAD_M, bench.HEAD_D) == 65536 * (7 * 8192 + 4) + 2 * 8192 == 3_758_374_912
