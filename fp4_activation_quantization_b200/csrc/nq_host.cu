@@ -378,15 +378,15 @@ int64_t resident_ctas(const void* k, int block, size_t smem = 0) {
 // persistent (one CTA per resident slot, next row prefetched), and two rows
 // per CTA (row_kernel_rows_n: static RMSNorm / LayerNorm).  NQ_FLAG_VARIANT
 // forces one where it applies.
-// Clusters per row of a row wider than 16384 elements (2048 chunks): 2 up to
-// 32768 elements, 4 up to 65536; 0 for rows one CTA holds.
+// CTAs per row of a row wider than 16384 elements (2048 chunks): 4 up to
+// 32768 elements, 8 up to 65536; 0 for rows one CTA holds.
 int cluster_ctas(int64_t d) {
   const int64_t C = (d + 7) / 8;
-  return C <= 2048 ? 0 : (C <= 4096 ? 2 : 4);
+  return C <= 2048 ? 0 : (C <= 4096 ? 4 : 8);
 }
 
-// Rows wider than 16384 elements: one row per thread-block cluster of 2 or 4
-// CTAs of 1024 threads (register rows; the variants do not apply).
+// Rows wider than 16384 elements: one row per thread-block cluster of 4 or 8
+// CTAs of 256 threads (register rows; the variants do not apply).
 nq_status run_cluster_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags, cudaStream_t stream) {
   if (flags & NQ_FLAG_SCHEDULE_MASK)
     return fail(NQ_ERR_INVALID_ARGUMENT, "%s: NQ_FLAG_SCHEDULE covers at most 2048 chunks; d = %lld takes a cluster "
@@ -398,7 +398,7 @@ nq_status run_cluster_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_
   const nq::RowKernels& table = table_of(op, (flags & (NQ_FLAG_E5M2 | NQ_FLAG_SF_SWIZZLED)) != 0,
                                         (flags & (NQ_FLAG_SCALES_COL_MAJOR | NQ_FLAG_SCALES_PACKED_UE8M0)) != 0,
                                         a.dest != nullptr);
-  const auto& tab = table.cluster[nc == 4 ? 1 : 0];
+  const auto& tab = table.cluster[nc == 8 ? 1 : 0];
   const int64_t span = int64_t(8) * nq::kClusterThreads * nq::kClusterChunks * nc;  // elements a cluster covers
   const void* k = tab[vec ? 1 : 0];
   // As for one CTA per row: the predicate-free copy for rows that fill the

@@ -101,10 +101,10 @@ inline bool raw_schedule_built(int log_t, int log_k) {
 }
 using RawTable = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2][2];
 using Rows2Table = const void* [kMaxLogT - kMinLogT + 1][kMaxLogK + 2][2];
-// Rows wider than 16384 elements: one row per cluster of 2 (rows of up to
-// 32768 elements) or 4 (up to 65536) CTAs of 1024 threads, 2 chunks per
-// thread: [clusters of 2, 4][mode as KernelTable].
-constexpr int kClusterThreads = 1024, kClusterChunks = 2;
+// Rows wider than 16384 elements: one row per cluster of 4 (rows of up to
+// 32768 elements) or 8 (up to 65536) CTAs of 256 threads, 4 chunks per
+// thread: [clusters of 4, 8][mode as KernelTable].
+constexpr int kClusterThreads = 256, kClusterChunks = 4;
 using ClusterTable = const void* [2][4];
 struct RowKernels {
   KernelTable direct;    // one row per thread group

@@ -83,8 +83,9 @@ typedef enum nq_status {
 } nq_status;
 
 /* Widest row the norm calls accept (elements).  Rows of up to 16384 elements
- * take one CTA (or one warp) per row; wider rows one thread-block cluster of 2
- * (up to 32768) or 4 (up to 65536) CTAs per row, with identical numerics. */
+ * take one CTA (or one warp) per row; wider rows one thread-block cluster of 4
+ * (up to 32768) or 8 (up to 65536) CTAs of 256 threads per row, with identical
+ * numerics. */
 #define NQ_MAX_D 65536
 
 /* ---- flags (bitwise OR) ---- */
@@ -185,7 +186,8 @@ const char* nq_last_error(void);
  * NVFP4, 4 = RMSNorm group FP8) at (M, d, flags): threads per row, 16-byte
  * chunks per thread and rows per CTA; for op 3, the call without a residual.
  * A row of more than 16384 elements is split over a cluster of CTAs:
- * threads_per_row then counts the cluster's threads (2048 or 4096).
+ * threads_per_row then counts the cluster's threads (1024 or 2048) and
+ * chunks_per_thread is 4.
  * Pure host function; launches nothing.
  */
 nq_status nq_query_schedule(int op, int64_t M, int64_t d, uint32_t flags, int* threads_per_row,

@@ -180,15 +180,15 @@ def test_planner_forced_schedules(nq):
 
 
 def test_planner_cluster_rows(nq):
-    """Rows wider than 16384 elements: one cluster of 2 CTAs (up to 32768 elements) or 4 (up to
-    65536) of 1024 threads with 2 chunks each; the cluster covers the next power of two of chunks.
+    """Rows wider than 16384 elements: one cluster of 4 CTAs (up to 32768 elements) or 8 (up to
+    65536) of 256 threads with 4 chunks each; the cluster covers the next power of two of chunks.
     A forced schedule cannot cover them."""
     for op in range(5):
         for d in (16400, 20480, 32768, 32784, 49152, 65536):
             T, K, R = nq.nq_query_schedule(op, 4096, d)
             C = (d + 7) // 8
             P = 1 << (C - 1).bit_length()
-            assert (T, K, R) == (P // 2, 2, 1) and T in (2048, 4096), (op, d, T, K, R)
+            assert (T, K, R) == (P // 4, 4, 1) and T in (1024, 2048), (op, d, T, K, R)
     with pytest.raises(nq.NQError):
         nq.nq_query_schedule(0, 100, 20000, nq.flag_schedule(10, 1))
     with pytest.raises(nq.NQError):

@@ -1,5 +1,5 @@
 """Rows wider than 16384 elements (up to NQ_MAX_D = 65536), split over a
-thread-block cluster of 2 or 4 CTAs per row, against the oracle (needs a B200).
+thread-block cluster of 4 or 8 CTAs per row, against the oracle (needs a B200).
 
 The row sums cross the cluster through distributed shared memory in the same
 canonical order as one CTA would use, so every output is bit-exact with the
@@ -31,9 +31,9 @@ def nq():
 
 
 def test_query_reports_clusters(nq):
-    for d, n in ((16384, 0), (16392, 2), (32768, 2), (32776, 4), (65536, 4)):
+    for d, n in ((16384, 0), (16392, 4), (32768, 4), (32776, 8), (65536, 8)):
         t, k, r = nq.nq_query_schedule(nq.OP_RMS_DYN_FP8, 64, d)
-        assert (t == 1024 * n and k == 2 and r == 1) if n else t <= 1024, (d, t, k, r)
+        assert (t == 256 * n and k == 4 and r == 1) if n else t <= 1024, (d, t, k, r)
 
 
 @pytest.mark.parametrize("d", WIDTHS + [65535])
