@@ -100,16 +100,23 @@ def nvfp4_bytes(M, d, residual):
     return M * per + 2 * d + 4
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without // and /* */ comments (string literals left alone)."""
+    return re.sub(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"',
+                  lambda m: m.group(0) if m.group(0).startswith('"') else "", src, flags=re.S)
+
+
 def kernel_source_hash() -> str:
-    """Hash of the device-code sources (every csrc file except the host-side
-    launcher nq_host.cu): a profile's counters stay valid while it matches."""
+    """Hash of the device code (every csrc file except the host-side launcher
+    nq_host.cu, comments stripped and whitespace collapsed): a profile's
+    counters stay valid while it matches."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "fp4_activation_quantization_b200", "csrc", "*"))):
         if os.path.basename(p) == "nq_host.cu":
             continue
-        with open(p, "rb") as f:
+        with open(p, encoding="utf-8") as f:
             h.update(os.path.basename(p).encode())
-            h.update(f.read())
+            h.update(" ".join(_strip_comments(f.read()).split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,10 +1,12 @@
 // nq_row_kernel.cuh — the fused residual-add + norm + quantize row kernel.
 //
 // One row (token) is owned by a group of T threads: a single warp (T = 32,
-// eight rows per CTA) or the whole CTA (T = 64..1024).  Thread t of the group
-// owns the 16-byte chunks c = t + k*T, k = 0..K-1, of the row (8 bf16 values
-// each), so every load and store instruction of a warp touches one contiguous
-// 512-byte span.  The row stays in float32 registers from load to quantized
+// eight rows per CTA), the whole CTA (T = 64..1024), or, for rows wider than
+// 16384 elements, a thread-block cluster of NC CTAs (row_kernel_cluster).
+// Thread t of the group owns the 16-byte chunks c = t + k*T, k = 0..K-1, of
+// the row (8 bf16 values each; c = t + j*T + k*T*NC in CTA j of a cluster), so
+// every load and store instruction of a warp touches one contiguous 512-byte
+// span.  The row stays in float32 registers from load to quantized
 // store: the row is read once, and each output is written once.
 //
 // Steps, per row (netraruntime blog "Fusing RMSNorm and FP8 Quantization
