@@ -272,13 +272,17 @@ __device__ __forceinline__ float row_max_nonneg(float v, uint32_t* red, int tid)
 // cluster owns, in thread t, the chunks k * NC * T + j * T + t, so the chunk
 // index's bits are, from the top: k (the thread's own slots), j (the CTA),
 // the warp, the lane.  The canonical tree combines them in that order; the
-// level over j runs here, through distributed shared memory: every CTA
-// publishes its per-thread partial, and each CTA combines the NC partials of
-// its thread index (CTA j absorbs CTA j + NC/2, ..., highest bit first), so
-// every CTA holds the same values afterwards.  `xred` holds T floats and is
-// used by one reduction only (no reuse, so no barrier is needed before it is
-// written).  The cluster barrier is a hardware barrier that every thread of
-// the cluster reaches on the same path; nothing here spins.
+// level over j runs here, through distributed shared memory: each CTA writes
+// its partial into slot `rank` of every CTA's xred (NC x T floats), and after
+// the cluster barrier combines the NC partials of its thread index from its
+// own buffer (CTA j absorbs CTA j + NC/2, ..., highest bit first), so every
+// CTA holds the same values afterwards.  Nothing remote is touched after the
+// barrier.  The remote buffers must exist before the first remote write,
+// which the kernel ensures (every CTA arrives on the cluster barrier at entry
+// and waits on it before its first reduction).  Each xred is used by one
+// reduction only (no reuse, so no barrier is needed before it is written).
+// The cluster barrier is a hardware barrier that every thread of the cluster
+// reaches on the same path; nothing here spins.
 template <int T, int NC>
 __device__ __forceinline__ float cluster_tree_sum(float v, float* xred, int tid) {
   if constexpr (NC == 1) {
@@ -286,11 +290,13 @@ __device__ __forceinline__ float cluster_tree_sum(float v, float* xred, int tid)
   } else {
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
-    xred[tid] = v;
+    const int rank = int(cl.block_rank());
+#pragma unroll
+    for (int j = 0; j < NC; ++j) *cl.map_shared_rank(xred + rank * T + tid, j) = v;
     cl.sync();
     float p[NC];
 #pragma unroll
-    for (int j = 0; j < NC; ++j) p[j] = *cl.map_shared_rank(xred + tid, j);
+    for (int j = 0; j < NC; ++j) p[j] = xred[j * T + tid];
 #pragma unroll
     for (int h = NC / 2; h >= 1; h >>= 1)
 #pragma unroll
@@ -299,7 +305,13 @@ __device__ __forceinline__ float cluster_tree_sum(float v, float* xred, int tid)
   }
 }
 
-// Largest of the cluster's per-CTA values (non-negative floats as bits; order-free).
+// Largest of the cluster's per-CTA values (non-negative floats as bits;
+// order-free).  Pull form: each CTA publishes its value in its own xred[0]
+// and after the barrier reads the NC values from the CTAs' buffers, so a
+// kernel that calls it ends with one more cluster barrier before any CTA
+// exits.  (Measured on B200 for the dynamic path, 2048 x 65536 ... 8192 x
+// 20480: pushing the absmax into every CTA as well and leaving without that
+// barrier was 5-7 % slower.)
 template <int NC>
 __device__ __forceinline__ uint32_t cluster_max_u32(uint32_t u, uint32_t* xred, int tid) {
   if constexpr (NC == 1) {

@@ -439,9 +439,14 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     // would hold twice the registers); the fused group quantization from raw
     // rows at every width (1.13x - 1.26x).  LayerNorm rows wider than a warp
     // take two rows per CTA (gamma / beta loaded once for both: 1.27x at
-    // 65536 x 4096).
+    // 65536 x 4096); rows wider than 8192 elements (one CTA per SM, bound by
+    // the 8 d bytes of shared memory) from persistent CTAs that prefetch the
+    // next row and keep gamma / beta in shared memory (1.2x - 1.3x at d =
+    // 10240 ... 16384, M >= 1024), and from raw rows where persistence does
+    // not pay (100 x 16384: 7.0 -> 5.4 us).
     if (op == nq::kOpRmsStaticFp8) variant = 3;
     else if (op == nq::kOpRmsNvfp4 && threads > 32) variant = 2;
+    else if (op == nq::kOpLnStaticFp8 && a.d > 8192) variant = 3;
     else if (op == nq::kOpLnStaticFp8 && threads > 32) variant = 6;
     else if (op == nq::kOpLnStaticFp8 && a.d >= 1024) variant = 2;
     else if (op == nq::kOpRmsGroupFp8) variant = 2;
@@ -463,7 +468,7 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     const int narrow = a.d == (8 * int64_t(threads)) << s.log_k ? 0 : 1;
     const auto& raw = table.raw[s.log_t - nq::kMinLogT][s.log_k];
     if (variant == 3 && raw[1][narrow] != nullptr) {
-      // Persistent CTAs of the RMSNorm-type operations hold gamma as fp32 in
+      // Persistent CTAs hold gamma (LayerNorm: gamma and beta) as fp32 in
       // shared memory.
       const size_t gsmem = nq::raw_gamma_smem_bytes(op, a.d);
       if (!allow_smem(raw[1][narrow], gsmem))

@@ -112,9 +112,9 @@ struct RowKernels {
   Rows2Table rows2;      // two rows per CTA on the same columns (static RMSNorm / LayerNorm): [.][.][narrow row]
   ClusterTable cluster;  // one row per thread-block cluster
 };
-// Dynamic shared memory of a persistent raw-row kernel: gamma as fp32 for the
-// RMSNorm-type operations (LayerNorm reads gamma / beta through L1).
-inline size_t raw_gamma_smem_bytes(int op, int64_t d) { return op == kOpLnStaticFp8 ? 0 : size_t(d) * 4u; }
+// Dynamic shared memory of a persistent raw-row kernel: gamma as fp32 (the
+// RMSNorm-type operations), or LayerNorm's fp32 gamma and beta.
+inline size_t raw_gamma_smem_bytes(int op, int64_t d) { return size_t(d) * (op == kOpLnStaticFp8 ? 8u : 4u); }
 const RowKernels& row_kernels_rms_dyn();
 const RowKernels& row_kernels_rms_static();
 const RowKernels& row_kernels_ln_static();

@@ -314,7 +314,7 @@ __device__ __forceinline__ void quantize_groups(const RowArgs& a, int64_t row, b
 // group's barriers (T > 32).  s_sum0 / s_sum1 / s_max are the group's
 // reduction buffers.  A row split over a cluster of NC CTAs (this one of rank
 // `rank`) also takes the cluster's barriers and its distributed buffers
-// x_sum0 / x_sum1 (T floats each) and x_max (one word).
+// x_sum0 / x_sum1 (NC x T floats each) and x_max (one word).
 template <int OP, int T, int K, bool VEC, bool FULL, int OUT, bool NARROW = false, int NC = 1>
 __device__ __forceinline__ void process_row(const RowArgs& a, int64_t row, bool live_in, bool has_res, int tid,
                                             const uint4 (&xr)[K], const uint4 (&rr)[K], float* s_sum0,
@@ -686,7 +686,8 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T) row_kernel(const RowArgs a)
 // chunks each, in clusters of 4 or 8, runs 1.5x faster than 1024 threads with
 // two chunks in clusters of 2 or 4; 512 x 4 and 128 x 8 land in between.)  The row sums cross the cluster through
 // distributed shared memory in the canonical order (cluster_tree_sum); the
-// absmax of the dynamic scale likewise.  MODE as for row_kernel.
+// absmax of the dynamic scale likewise (cluster_max_u32).  MODE as for
+// row_kernel.
 template <int OP, int K, int MODE, int OUT, int NC>
 __global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(kClusterThreads) row_kernel_cluster(const RowArgs a) {
   constexpr int T = kClusterThreads;
@@ -697,22 +698,28 @@ __global__ void __cluster_dims__(NC, 1, 1) __launch_bounds__(kClusterThreads) ro
   static_assert(NC == 2 || NC == 4 || NC == 8, "CTAs per row (8: the portable cluster size limit)");
   __shared__ __align__(16) float s_sum[2][W * 32];
   __shared__ uint32_t s_max[W];
-  __shared__ __align__(16) float x_sum[2][T];  // read by the other CTAs of the cluster
-  __shared__ uint32_t x_max[1];
+  __shared__ __align__(16) float x_sum[2][NC * T];  // written by every CTA of the cluster
+  __shared__ uint32_t x_max[1];                     // read by every CTA of the cluster
 
   const int tid = int(threadIdx.x);
   const int rank = cluster_rank<NC>();
   const int64_t row = int64_t(blockIdx.x) / NC;  // one row per cluster (clusters are consecutive blocks)
   const bool has_res = (OP != kOpLnStaticFp8) && (a.res_in != nullptr);
 
+  // Every CTA of the cluster has started (its shared memory exists) before
+  // any CTA writes to it: the arrive costs nothing here, and the wait, after
+  // the row's loads are issued, finds every CTA arrived.
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   griddep_wait();
   uint4 xr[K], rr[K];
   load_raw<T, K, VEC, FULL, NC>(a, row, true, has_res, tid, xr, rr, rank);
   griddep_launch_dependents();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   process_row<OP, T, K, VEC, FULL, OUT, NARROW, NC>(a, row, true, has_res, tid, xr, rr, s_sum[0], s_sum[1], s_max,
                                                     rank, x_sum[0], x_sum[1], x_max);
-  // No CTA leaves while another may still read its distributed buffers.
-  cooperative_groups::this_cluster().sync();
+  // The absmax (dynamic path only) is read from the other CTAs' buffers: no
+  // CTA leaves while another may still read them.
+  if constexpr (OP == kOpRmsDynFp8) cooperative_groups::this_cluster().sync();
 }
 
 // Per-chunk gamma (RMSNorm: bf16) or gamma and beta (LayerNorm: float32) of
@@ -745,12 +752,18 @@ struct GammaLoads {
 // RMSNorm gamma (bf16) widened to fp32 once per persistent CTA and kept in
 // shared memory: per chunk two conflict-free 16-byte loads replace a load and
 // eight integer unpack instructions on every row.  Chunk c's first four
-// values are lo[c], the last four hi[c].
+// values are lo[c], the last four hi[c]; LayerNorm's fp32 beta follows as
+// lo[2 C + c] and lo[3 C + c].
 template <int T, int K>
 struct GammaSmem {
   const float4* lo;
   const float4* hi;
   int tid, C;
+  __device__ __forceinline__ void ln(int k, float4& g0, float4& g1, float4& e0, float4& e1) const {
+    const int c = tid + k * T;
+    g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0, e0 = g0, e1 = g0;
+    if (c < C) g0 = lo[c], g1 = hi[c], e0 = lo[2 * C + c], e1 = lo[3 * C + c];
+  }
   __device__ __forceinline__ void rms2(int k, float2 (&g)[4]) const {
     const int c = tid + k * T;
     float4 l = make_float4(0.f, 0.f, 0.f, 0.f), h = l;
@@ -1259,18 +1272,25 @@ __global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSI
       xr[k] = (row < a.M && c < C) ? __ldcs(reinterpret_cast<const uint4*>(xrow + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
     }
   };
-  // Persistent CTAs of the RMSNorm-type operations keep gamma as fp32 in
-  // (dynamic) shared memory, widened once by the whole CTA (raw_gamma_smem_bytes)
-  // while the first row's load is in flight.
-  constexpr bool GSMEM = PERSIST && OP != kOpLnStaticFp8;
-  extern __shared__ __align__(16) float4 s_gamma[];  // [2][C]: GSMEM only
+  // Persistent CTAs keep gamma as fp32 in (dynamic) shared memory, widened
+  // once by the whole CTA (raw_gamma_smem_bytes) while the first row's load
+  // is in flight; LayerNorm keeps its fp32 gamma and beta there.
+  constexpr bool GSMEM = PERSIST;
+  extern __shared__ __align__(16) float4 s_gamma[];  // [2][C], LayerNorm [4][C]: GSMEM only
   auto stage_gamma = [&] {
     if constexpr (GSMEM) {
       for (int c = int(threadIdx.x); c < C; c += int(blockDim.x)) {
-        float2 g[4];
-        unpack_pairs(__ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c)), g);
-        s_gamma[c] = make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
-        s_gamma[C + c] = make_float4(g[2].x, g[2].y, g[3].x, g[3].y);
+        if constexpr (OP == kOpLnStaticFp8) {
+          const float4* gp = reinterpret_cast<const float4*>(static_cast<const float*>(a.gamma) + 8 * c);
+          const float4* bp = reinterpret_cast<const float4*>(a.beta + 8 * c);
+          s_gamma[c] = __ldg(gp), s_gamma[C + c] = __ldg(gp + 1);
+          s_gamma[2 * C + c] = __ldg(bp), s_gamma[3 * C + c] = __ldg(bp + 1);
+        } else {
+          float2 g[4];
+          unpack_pairs(__ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.gamma) + 8 * c)), g);
+          s_gamma[c] = make_float4(g[0].x, g[0].y, g[1].x, g[1].y);
+          s_gamma[C + c] = make_float4(g[2].x, g[2].y, g[3].x, g[3].y);
+        }
       }
       __syncthreads();
     }

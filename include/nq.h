@@ -143,7 +143,8 @@ typedef enum nq_status {
 #define NQ_FLAG_GROUP_SCHEDULE(t, k) ((((uint32_t)(t)) & 0xFu) << 16 | (((uint32_t)(k) + 1u) & 0x7u) << 20)
 /* Force a kernel variant (tests and tuning; same bits either way): n = 1 keeps
  * the row in float32 registers; n = 2 keeps only the raw bf16 row and unpacks
- * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row;
+ * it per pass; n = 3 is n = 2 with persistent CTAs that prefetch the next row
+ * and keep gamma (LayerNorm: gamma and beta) as fp32 in shared memory;
  * n = 6 (static RMSNorm and LayerNorm, t >= 6) gives each CTA two rows on the
  * same columns, so each thread loads its gamma / beta once for both.  n = 2, 3
  * and 6 apply to 16-byte-aligned rows without a residual and are ignored

@@ -574,3 +574,22 @@ def test_static_persistent_wide_rows(nq, d):
         assert np.array_equal(host_u8(q), eq), f
         q4, sf, _, _ = nq.nq_rmsnorm_quant_nvfp4(x, gam, gs, 1e-6, flags=f)
         assert np.array_equal(host_u8(q4), e4) and np.array_equal(host_u8(sf), esf), f
+
+
+@pytest.mark.parametrize("M", [100, 700])
+@pytest.mark.parametrize("d", [8200, 11264, 16384])
+def test_layernorm_persistent_wide_rows(nq, d, M):
+    """LayerNorm rows wider than 8192 elements run on persistent CTAs that keep the fp32 gamma
+    and beta in dynamic shared memory (8 d bytes: up to 128 KB) once each CTA walks two or
+    more rows (700 rows), else on raw rows (100 rows).  Automatic and forced persistent, e4m3
+    and e5m2, bit-exact; d = 8200 leaves most chunk slots of the last warps past the row."""
+    lw = S.make_ln_inputs(M, d, seed=d + 17)
+    x, gl, bl = dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    e4 = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-5)
+    e5 = oracle.layernorm_quant_fp8(lw["x"], lw["gamma"], lw["beta"], 0.05, eps=1e-5, flags=oracle.E5M2)
+    for f in (0, nq.flag_variant(3), nq.flag_variant(3) | nq.FLAG_PDL):
+        q = nq.nq_layernorm_quant_fp8(x, gl, bl, sc, 1e-5, flags=f)
+        assert np.array_equal(host_u8(q), e4), f
+        q = nq.nq_layernorm_quant_fp8(x, gl, bl, sc, 1e-5, flags=f | nq.FLAG_E5M2)
+        assert np.array_equal(host_u8(q), e5), f
