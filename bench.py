@@ -519,13 +519,31 @@ def cell(peak, tokens, nbytes, us, **kw):
 
 def run_configs(nq, flags):
     """µs per call, GB/s, fraction of the measured copy bandwidth and tokens/s of
-    every configuration's cells."""
+    every configuration's cells.  Cells of M >= 4096 also carry `copy_frac`: the
+    fraction of the measured copy bandwidth that a device copy moving the same
+    bytes reaches, timed the same way (the ceiling at that size for a kernel
+    that only moves data)."""
     import torch
     import synthetic as S
     gen = torch.Generator(device="cuda").manual_seed(7)
     bf = torch.bfloat16
     peak, _ = measured_peak()
     out = {}
+    copy_us = {}
+
+    def with_copy(c):
+        if c["M"] < 4096:
+            return c
+        nb = c["bytes"]
+        if nb not in copy_us:
+            nel = nb // 4  # bf16 elements each way: 2 bytes read and 2 written per element
+            n = sets_for(nb)
+            src = [torch.empty(nel, dtype=bf, device="cuda") for _ in range(n)]
+            dst = [torch.empty(nel, dtype=bf, device="cuda") for _ in range(n)]
+            copy_us[nb] = time_calls(lambda i: dst[i].copy_(src[i]), n, reps_for(nb, n))
+            del src, dst
+        c["copy_frac"] = round(nb / copy_us[nb] / 1e3 / peak, 4)
+        return c
 
     def dyn_cell(M, d, outliers):
         nb = fused_dyn_bytes(M, d)
@@ -540,7 +558,9 @@ def run_configs(nq, flags):
                                                          scale_out=ss[i], flags=flags)
         us = time_calls(fn, n, reps_for(nb, n))
         extra = {"host_latency_us": host_latency_us(fn)} if M <= 64 else {}
-        return cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8", M=M, d=d, sets=n, **extra)
+        c = cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8", M=M, d=d, sets=n, **extra)
+        del xs, rs, ro, qs, ss
+        return with_copy(c)
 
     out["1_fused_dynamic_small"] = [dyn_cell(64, 2816, False)]
     out["5_fused_dynamic_sweep"] = [dyn_cell(M, d, True) for d in (2816, 4096, 7168, 8192)
@@ -571,6 +591,8 @@ def run_configs(nq, flags):
     us_cp = time_calls(lambda i: dst[i].copy_(src[i]), n, reps)
     out["2_static"].append(cell(peak, M, 4 * nel, us_cp, call="device copy of the same bytes (context)",
                                 elements=nel, sets=n))
+    for c in out["2_static"][:2]:
+        c["copy_frac"] = out["2_static"][2]["frac"]
     del xs, qs, src, dst
 
     rows = []
@@ -588,9 +610,9 @@ def run_configs(nq, flags):
                                                            flags=fl | flags)
             us = time_calls(fn, n, reps_for(nb, n))
             extra = {"host_latency_us": host_latency_us(fn)} if M <= 64 else {}
-            rows.append(cell(peak, M, nb, us, call="nq_per_token_group_quant_fp8", scales=tag, M=M, K=K, sets=n,
-                             **extra))
             del xs, qs, sc_
+            rows.append(with_copy(cell(peak, M, nb, us, call="nq_per_token_group_quant_fp8", scales=tag, M=M, K=K,
+                                       sets=n, **extra)))
     out["3_group"] = rows
 
     rows = []
@@ -610,9 +632,9 @@ def run_configs(nq, flags):
                     residual_out=rs[i] if residual else None, q_out=qs[i], sf_out=sf[i], flags=flags)
                 us = time_calls(fn, n, reps_for(nb, n))
                 extra = {"host_latency_us": host_latency_us(fn)} if M <= 64 else {}
-                rows.append(cell(peak, M, nb, us, call="nq_rmsnorm_quant_nvfp4", residual=residual, M=M, d=d,
-                                 ld_x=ld, sets=n, **extra))
                 del xs, rs, qs, sf
+                rows.append(with_copy(cell(peak, M, nb, us, call="nq_rmsnorm_quant_nvfp4", residual=residual, M=M,
+                                           d=d, ld_x=ld, sets=n, **extra)))
     out["4_nvfp4"] = rows
 
     rows = []
@@ -630,9 +652,9 @@ def run_configs(nq, flags):
                     xs[i], g, 1e-6, residual=rs[i] if residual else None,
                     residual_out=rs[i] if residual else None, q_out=qs[i], scales_out=sc_[i], flags=flags), n,
                     reps_for(nb, n))
-                rows.append(cell(peak, M, nb, us, call="nq_rmsnorm_quant_fp8_group", residual=residual, M=M, d=d,
-                                 sets=n))
                 del xs, rs, qs, sc_
+                rows.append(with_copy(cell(peak, M, nb, us, call="nq_rmsnorm_quant_fp8_group", residual=residual,
+                                           M=M, d=d, sets=n)))
     out["next_fused_group"] = rows
 
     rows = []
@@ -653,9 +675,9 @@ def run_configs(nq, flags):
             us = time_calls(lambda i: nq.nq_fused_add_rmsnorm_quant_fp8_moe(
                 xs[i], g, dest, n_rows, 1e-6, group=group, residual=rs[i], residual_out=rs[i], q_out=qs[i],
                 scales_out=sc_[i], flags=flags), n, reps_for(nb, n))
-            rows.append(cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8_moe", group=group, M=M, d=d,
-                             experts=E, topk=topk, sets=n))
             del xs, rs, qs, sc_
+            rows.append(with_copy(cell(peak, M, nb, us, call="nq_fused_add_rmsnorm_quant_fp8_moe", group=group, M=M,
+                                       d=d, experts=E, topk=topk, sets=n)))
     out["next_moe_dispatch"] = rows
     torch.cuda.synchronize()
     torch.cuda.empty_cache()

@@ -190,6 +190,18 @@ nq_status plan_rows(const char* fn, int op, int64_t M, int64_t d, uint32_t flags
     // upper slots then whole slots of every warp) and for rows narrower than
     // P = 512 (65536 x 2816: 142.5 -> 130.2 us); at d = 4096 four stay faster.
     if (op == nq::kOpRmsNvfp4 && !has_res && M >= 768 && (lp == 10 || (lp == 9 && C < (int64_t(1) << lp)))) lk = 3;
+    // Rows of 8193 ... 16384 elements without residual: eight chunks per
+    // thread (256 threads) on rows narrower than P = 2048 (16384 x 10240:
+    // static RMSNorm 120.7 -> 94.3 us, NVFP4 164.1 -> 130.3, group 177.3 ->
+    // 152.8, LayerNorm 180.3 -> 143.6), and on full rows for static RMSNorm
+    // (16384 x 16384: 150.2 -> 133.4 us) and, from 4096 rows, NVFP4 (185.5 ->
+    // 172.7 us) and the fused group (217.5 -> 208.6 us); LayerNorm keeps four
+    // on full rows.
+    if (!has_res && lp == 11 && M >= 768 &&
+        (C < 2048 ? op != nq::kOpRmsDynFp8
+                  : (op == nq::kOpRmsStaticFp8 ||
+                     ((op == nq::kOpRmsNvfp4 || op == nq::kOpRmsGroupFp8) && M >= 4096))))
+      lk = 3;
     int lt = lp - lk;
     if (lt > 10) lt = 10;
     s->log_t = lt;
@@ -443,10 +455,12 @@ nq_status run_rows(const char* fn, int op, RowArgs& a, bool vec, uint32_t flags,
     // the 8 d bytes of shared memory) from persistent CTAs that prefetch the
     // next row and keep gamma / beta in shared memory (1.2x - 1.3x at d =
     // 10240 ... 16384, M >= 1024), and from raw rows where persistence does
-    // not pay (100 x 16384: 7.0 -> 5.4 us).
+    // not pay (100 x 16384: 7.0 -> 5.4 us); with eight chunks per thread
+    // (rows narrower than 16384 elements, M >= 768) two rows per CTA again
+    // (16384 x 12288: 178.3 -> 160.8 us).
     if (op == nq::kOpRmsStaticFp8) variant = 3;
     else if (op == nq::kOpRmsNvfp4 && threads > 32) variant = 2;
-    else if (op == nq::kOpLnStaticFp8 && a.d > 8192) variant = 3;
+    else if (op == nq::kOpLnStaticFp8 && a.d > 8192) variant = s.log_k == 3 ? 6 : 3;
     else if (op == nq::kOpLnStaticFp8 && threads > 32) variant = 6;
     else if (op == nq::kOpLnStaticFp8 && a.d >= 1024) variant = 2;
     else if (op == nq::kOpRmsGroupFp8) variant = 2;

@@ -185,7 +185,8 @@ const char* nq_last_error(void);
  * Schedule the planner picks for a norm call (op: 0 = fused add+RMSNorm+
  * dynamic FP8, 1 = RMSNorm static FP8, 2 = LayerNorm static FP8, 3 = RMSNorm
  * NVFP4, 4 = RMSNorm group FP8) at (M, d, flags): threads per row, 16-byte
- * chunks per thread and rows per CTA; for op 3, the call without a residual.
+ * chunks per thread and rows per CTA; for ops 1, 3 and 4, the call without a
+ * residual.
  * A row of more than 16384 elements is split over a cluster of CTAs:
  * threads_per_row then counts the cluster's threads (1024 or 2048) and
  * chunks_per_thread is 4.

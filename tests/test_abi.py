@@ -164,6 +164,19 @@ def test_validation_without_gpu(nq):
     (3, 8192, 8192, (128, 8, 1)),    # ... and at P = 1024 whatever the width
     (3, 8192, 4096, (128, 4, 1)),    # ... but four on rows that fill P = 512
     (3, 8192, 1536, (64, 4, 1)),
+    # rows of 8193 ... 16384 elements without residual: eight chunks per thread from 768 rows
+    (1, 4096, 10240, (256, 8, 1)),
+    (2, 4096, 12288, (256, 8, 1)),
+    (3, 4096, 12288, (256, 8, 1)),
+    (4, 4096, 10240, (256, 8, 1)),
+    (2, 700, 12288, (512, 4, 1)),
+    (1, 4096, 16384, (256, 8, 1)),   # ... on full rows too for static RMSNorm,
+    (3, 4096, 16384, (256, 8, 1)),   # ... and NVFP4 and the fused group from 4096 rows
+    (4, 4096, 16384, (256, 8, 1)),
+    (3, 1024, 16384, (512, 4, 1)),
+    (4, 1024, 16384, (512, 4, 1)),
+    (2, 4096, 16384, (512, 4, 1)),
+    (0, 4096, 12288, (512, 4, 1)),   # the residual-add path keeps four
 ])
 def test_planner(nq, op, M, d, exp):
     assert nq.nq_query_schedule(op, M, d) == exp

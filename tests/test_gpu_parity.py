@@ -556,33 +556,39 @@ def test_narrow_rows_partial_warps_every_schedule(nq, residual):
                 assert np.array_equal(host_u16(ro), er), (d, sched, "residual_out")
 
 
+@pytest.mark.parametrize("M", [700, 1000])
 @pytest.mark.parametrize("d", [11264, 12288, 16384])
-def test_static_persistent_wide_rows(nq, d):
+def test_static_persistent_wide_rows(nq, d, M):
     """Persistent raw rows keep gamma as fp32 in dynamic shared memory (4 d bytes: 44, 48 and
-    64 KB here, on top of the kernel's static buffers).  Static RMSNorm and NVFP4, automatic and
-    forced persistent variant, bit-exact with the oracle."""
-    M = 700
-    w = S.make_rms_inputs(M, d, seed=d, residual=False)
+    64 KB here, on top of the kernel's static buffers).  Static RMSNorm, NVFP4 and the fused
+    group path without residual, automatic (512 threads x 4 chunks at 700 rows, 256 x 8 at
+    1000 rows below 16384 elements) and forced persistent variant, bit-exact with the oracle."""
+    w = S.make_rms_inputs(M, d, seed=d + M, residual=False)
     x, gam = dev_bf16(w["x"]), dev_bf16(w["gamma"])
     sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
     eq, _, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05)
     g = oracle.nvfp4_global_scale(w["x"], w["gamma"], d=d)
     e4, esf, _, _ = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], g, d=d)
+    eg, esg, _, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"])
     gs = torch.tensor([g], dtype=torch.float32, device="cuda")
     for f in (0, nq.flag_variant(3)):
         q, _, _ = nq.nq_rmsnorm_quant_fp8_static(x, gam, sc, 1e-6, flags=f)
         assert np.array_equal(host_u8(q), eq), f
         q4, sf, _, _ = nq.nq_rmsnorm_quant_nvfp4(x, gam, gs, 1e-6, flags=f)
         assert np.array_equal(host_u8(q4), e4) and np.array_equal(host_u8(sf), esf), f
+        qg, sg, _, _ = nq.nq_rmsnorm_quant_fp8_group(x, gam, 1e-6, flags=f)
+        assert np.array_equal(host_u8(qg), eg) and np.array_equal(sg.cpu().numpy().view(np.uint32),
+                                                                 esg.view(np.uint32)), f
 
 
-@pytest.mark.parametrize("M", [100, 700])
+@pytest.mark.parametrize("M", [100, 700, 1000])
 @pytest.mark.parametrize("d", [8200, 11264, 16384])
-def test_layernorm_persistent_wide_rows(nq, d, M):
-    """LayerNorm rows wider than 8192 elements run on persistent CTAs that keep the fp32 gamma
-    and beta in dynamic shared memory (8 d bytes: up to 128 KB) once each CTA walks two or
-    more rows (700 rows), else on raw rows (100 rows).  Automatic and forced persistent, e4m3
-    and e5m2, bit-exact; d = 8200 leaves most chunk slots of the last warps past the row."""
+def test_layernorm_wide_rows(nq, d, M):
+    """LayerNorm rows wider than 8192 elements: raw rows (100 rows); persistent CTAs that keep
+    the fp32 gamma and beta in dynamic shared memory (8 d bytes: up to 128 KB) once each CTA
+    walks two or more rows (700 rows; 1000 rows of 16384); two rows per CTA at 256 threads x 8
+    chunks (1000 rows narrower than 16384).  Automatic and forced persistent, e4m3 and e5m2,
+    bit-exact; d = 8200 leaves most chunk slots of the last warps past the row."""
     lw = S.make_ln_inputs(M, d, seed=d + 17)
     x, gl, bl = dev_bf16(lw["x"]), dev_f32(lw["gamma"]), dev_f32(lw["beta"])
     sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
