@@ -1237,19 +1237,27 @@ __global__ void __launch_bounds__(T, (rows_n_min_blocks<T, K, NR>())) row_kernel
 // processes the current one, so a load is always in flight; the static scale's
 // reciprocal is then computed once per CTA.
 // Register budget of the raw kernel: the raw row (4 registers per chunk, 8
-// when the next row is prefetched) plus ~48 working registers; the launch
-// bound asks ptxas to fit it, which stops it from hoisting every chunk's
-// gamma / beta loads at once (more CTAs per SM matter more here).
-template <int T, int K, bool PERSIST>
+// when the next row is prefetched) plus ~48 working registers, at least 64;
+// the launch bound asks ptxas to fit it, which stops it from hoisting every
+// chunk's gamma / beta loads at once (more CTAs per SM matter more here).
+// NVFP4 and the fused group without prefetch take 32 working registers, at
+// least 56, even where ptxas then spills a few words: measured on B200,
+// NVFP4 128 x 8 chunks at 64 registers (8 CTAs per SM, was 80 and 6) 8192 x
+// 7168 42.7 -> 40.2 us and 65536 x 7168 298.4 -> 277.8 us, 128 x 4 at 56 (9
+// CTAs) 65536 x 4096 161.3 -> 156.3 us; the fused group 128 x 4 at 56 32768
+// x 4096 99.2 -> 95.3 us.
+template <int OP, int T, int K, bool PERSIST>
 constexpr int raw_min_blocks() {
   constexpr int threads = (T == 32) ? 256 : T;
-  constexpr int cap = (PERSIST ? 8 * K : 4 * K) + 48;
-  constexpr int blocks = 65536 / (threads * (cap < 64 ? 64 : cap));
+  constexpr bool LEAN = (OP == kOpRmsNvfp4 || OP == kOpRmsGroupFp8) && !PERSIST;
+  constexpr int cap = (PERSIST ? 8 * K : 4 * K) + (LEAN ? 32 : 48);
+  constexpr int lo = LEAN ? 56 : 64;
+  constexpr int blocks = 65536 / (threads * (cap < lo ? lo : cap));
   return blocks < 1 ? 1 : blocks;
 }
 
 template <int OP, int T, int K, bool PERSIST, int OUT, bool NARROW>
-__global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<T, K, PERSIST>()))
+__global__ void __launch_bounds__(T == 32 ? 256 : T, (raw_min_blocks<OP, T, K, PERSIST>()))
     row_kernel_raw(const RowArgs a) {
   static_assert(OP != kOpRmsDynFp8, "raw rows: no residual");
   constexpr int R = (T == 32) ? 8 : 1;  // rows per CTA (one warp per row when T == 32)
