@@ -442,6 +442,24 @@ def test_variants_without_residual_bit_exact(nq, d, M, ld):
             assert np.array_equal(host_u8(q), e_fp4[0]) and np.array_equal(host_u8(sf), e_fp4[1]), (var, sched)
 
 
+@pytest.mark.parametrize("M,d", [(1000, 8192), (800, 2816), (1000, 7168), (1000, 4096)])
+def test_lean_raw_rows_automatic(nq, M, d):
+    """The automatic raw-row kernels of NVFP4 and the fused group path without residual at the
+    shapes where they run on their lean register budget (8 chunks per thread at d = 2816, 7168
+    and 8192, where ptxas spills a few words; 4 chunks at 4096): bit-exact with the oracle."""
+    w = S.make_rms_inputs(M, d, seed=M * 7 + d, residual=False, x_outlier_channels=True)
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    gn = oracle.nvfp4_global_scale(w["x"], w["gamma"])
+    e4, esf, _, _ = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn)
+    q4, sf, _, _ = nq.nq_rmsnorm_quant_nvfp4(x, g, torch.tensor([gn], dtype=torch.float32, device="cuda"), 1e-6)
+    assert np.array_equal(host_u8(q4), e4) and np.array_equal(host_u8(sf), esf)
+    if d % 128 == 0:
+        eg, esg, _, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"])
+        qg, sg, _, _ = nq.nq_rmsnorm_quant_fp8_group(x, g, 1e-6)
+        assert np.array_equal(host_u8(qg), eg)
+        assert np.array_equal(sg.cpu().numpy().view(np.uint32), esg.view(np.uint32))
+
+
 # ------------------------------------- fused RMSNorm + per-token-group FP8 ----
 @pytest.mark.parametrize("group", [64, 128])
 @pytest.mark.parametrize("residual", [False, True])
