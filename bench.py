@@ -106,14 +106,16 @@ def _strip_comments(src: str) -> str:
                   lambda m: m.group(0) if m.group(0).startswith('"') else "", src, flags=re.S)
 
 
+HEAD_KERNEL_SOURCES = ("nq_row_rms_dyn.cu", "nq_row_kernel.cuh", "nq_device.cuh", "nq_internal.h")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the device code (every csrc file except the host-side launcher
-    nq_host.cu, comments stripped and whitespace collapsed): a profile's
-    counters stay valid while it matches."""
+    """Hash of the headline kernel's device code (its translation unit and the
+    headers it includes, comments stripped and whitespace collapsed): the
+    headline profile's counters stay valid while it matches."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "fp4_activation_quantization_b200", "csrc", "*"))):
-        if os.path.basename(p) == "nq_host.cu":
-            continue
+    for name in HEAD_KERNEL_SOURCES:
+        p = os.path.join(ROOT, "fp4_activation_quantization_b200", "csrc", name)
         with open(p, encoding="utf-8") as f:
             h.update(os.path.basename(p).encode())
             h.update(" ".join(_strip_comments(f.read()).split()).encode())

@@ -891,7 +891,8 @@ nq_status nq_per_token_group_quant_fp8(const void* x, int64_t ld_x, void* q_out,
   // Team of 2^t lanes per group, 2^u groups per thread.  Many groups: teams
   // of four lanes, one group per thread (measured best on B200: each lane pays
   // the group's scale once per 32 elements, a team reads 64 contiguous bytes,
-  // 56 registers).  Few groups: a lane per chunk for the shortest latency.
+  // 48 registers, 5 CTAs per SM).  Few groups: a lane per chunk for the
+  // shortest latency.
   // NQ_FLAG_GROUP_SCHEDULE(t, u) forces it.
   int lt = a.G >= int64_t(148) * 64 ? 2 : (group == 128 ? 4 : 3), lu = 0;
   const uint32_t ft = (flags >> 16) & 0xFu, fk = (flags >> 20) & 0x7u;
