@@ -442,6 +442,32 @@ def test_variants_without_residual_bit_exact(nq, d, M, ld):
             assert np.array_equal(host_u8(q), e_fp4[0]) and np.array_equal(host_u8(sf), e_fp4[1]), (var, sched)
 
 
+@pytest.mark.parametrize("d", [10240, 16384])
+def test_residual_rows_512_threads(nq, d):
+    """Rows of 8193 ... 16384 elements with a residual at M >= 384 run on 512 threads x 4 chunks
+    under the two-CTA launch bound (the predicate-free copy at d = 16384, the one that skips
+    dead chunk slots at 10240): dynamic, static RMSNorm, NVFP4 and the fused group path,
+    bit-exact with the oracle, residual_out included."""
+    M = 400
+    w = S.make_rms_inputs(M, d, seed=d + 3, x_outlier_channels=True)
+    assert nq.nq_query_schedule(0, M, d) == (512, 4, 1)
+    assert_fused_equal(run_fused(nq, w), oracle_fused(w))
+    x, g = dev_bf16(w["x"]), dev_bf16(w["gamma"])
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    q, ro, _ = nq.nq_rmsnorm_quant_fp8_static(x, g, sc, 1e-6, residual=dev_bf16(w["residual"]))
+    eq, er, _ = oracle.rmsnorm_quant_fp8_static(w["x"], w["gamma"], 0.05, w["residual"])
+    assert np.array_equal(host_u8(q), eq) and np.array_equal(host_u16(ro), er)
+    gn = oracle.nvfp4_global_scale(w["x"], w["gamma"], w["residual"])
+    q4, sf, ro4, _ = nq.nq_rmsnorm_quant_nvfp4(x, g, torch.tensor([gn], dtype=torch.float32, device="cuda"), 1e-6,
+                                               residual=dev_bf16(w["residual"]))
+    e4, esf, er4, _ = oracle.rmsnorm_quant_nvfp4(w["x"], w["gamma"], gn, w["residual"])
+    assert np.array_equal(host_u8(q4), e4) and np.array_equal(host_u8(sf), esf) and np.array_equal(host_u16(ro4), er4)
+    qg, sg, rog, _ = nq.nq_rmsnorm_quant_fp8_group(x, g, 1e-6, residual=dev_bf16(w["residual"]))
+    eg, esg, erg, _ = oracle.rmsnorm_quant_fp8_group(w["x"], w["gamma"], w["residual"])
+    assert np.array_equal(host_u8(qg), eg) and np.array_equal(host_u16(rog), erg)
+    assert np.array_equal(sg.cpu().numpy().view(np.uint32), esg.view(np.uint32))
+
+
 @pytest.mark.parametrize("M,d", [(1000, 8192), (800, 2816), (1000, 7168), (1000, 4096)])
 def test_lean_raw_rows_automatic(nq, M, d):
     """The automatic raw-row kernels of NVFP4 and the fused group path without residual at the
