@@ -767,8 +767,9 @@ def run_case(args):
     M, d, op = args.M, args.d, args.case
     bf = torch.bfloat16
     g = torch.Generator(device="cuda").manual_seed(0)
+    ld = max(args.ld, d)  # > d: x is the first d columns of an [M, ld] tensor
     x = outlier_x(M, d, g) if op == "fused_add_rmsnorm_quant_fp8" else \
-        torch.randn(M, d, device="cuda", generator=g).to(bf)
+        torch.randn(M, ld, device="cuda", generator=g).to(bf)[:, :d]
     res = (torch.randn(M, d, device="cuda", generator=g).to(bf)
            if op in ("fused_add_rmsnorm_quant_fp8", "nvfp4_res", "rmsnorm_quant_fp8_group_res") else None)
     gam = (1 + 0.1 * torch.randn(d, device="cuda", generator=g)).to(bf)
@@ -815,6 +816,7 @@ def main():
     ap.add_argument("--M", type=int, default=16384)
     ap.add_argument("--d", type=int, default=4096)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--ld", type=int, default=0, help="--case: row stride of x (a column slice when > d)")
     args = ap.parse_args()
     if args.case:
         run_case(args)
